@@ -1,0 +1,240 @@
+/*
+ * libsa - cross-layer shared sparse attention on B200 (sm_100a).
+ *
+ * C ABI of the hot path: a lightweight indexer scores every cached key
+ * against the current query, a top-k over the whole context picks the
+ * tokens to attend to, and that one index is shared by a group of layers
+ * reading one KV cache, each running softmax attention over only the
+ * selected tokens.  A chunked-prefill variant unions the selected KV blocks
+ * per GQA group into a block table and attends to those blocks in place.
+ *
+ * Pages this interface follows (cited per entry below):
+ *   [CLSA] "Le routage partage entre couches accelere l'attention sparse de
+ *          7x sans perte de qualite" - news article on "CLSA: You Only Index
+ *          Once", section "Comment CLSA fonctionne".
+ *   [IC]   "IndexCache: Accelerating Sparse Attention via Cross-Layer Index
+ *          Reuse" - technical summary, sections 1 "Problematique" and
+ *          2 "Methodologie : IndexCache".
+ *   [CA]   "CompactAttention: Accelerating Chunked Prefill with Block-Union
+ *          KV Selection" - technical summary, section "Methodologie :
+ *          CompactAttention" (selection step, execution step).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every tensor pointer is DEVICE memory owned by the caller.  The library
+ *   never allocates, frees or synchronises inside a compute call; each call
+ *   only enqueues work on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and returns.
+ * - bf16 tensors are passed as `const void*` holding IEEE bfloat16 bit
+ *   patterns.  Rows of bf16 tensors must start 16-byte aligned (all the
+ *   shapes below have d or d_I a multiple of 64, so a 16-byte aligned base
+ *   suffices).
+ * - Argument errors are detected on the host before anything is enqueued;
+ *   the call then returns SA_ERR_INVALID_ARG / SA_ERR_UNSUPPORTED /
+ *   SA_ERR_WORKSPACE and sa_last_error() describes the problem.
+ * - Errors only the device can see (an index out of range, a sequence length
+ *   above the stated maximum, a bounded wait that gave up) are recorded in
+ *   the status block at the start of the workspace and read back with
+ *   sa_read_device_status().  The kernel skips the offending element instead
+ *   of touching memory outside the buffers.
+ * - Workspace: `ws` must be 256-byte aligned and at least the size returned
+ *   by the matching *_workspace_size() function.  Its first
+ *   SA_WS_HEADER_BYTES bytes are the status block; zero them once when the
+ *   workspace is allocated (the library only ever writes a non-zero code
+ *   there, so the status is sticky until sa_clear_device_status()).  The
+ *   rest is scratch owned by the call while it runs on `stream`: calls that
+ *   overlap on the GPU must not share one workspace.
+ * - The library keeps no global state between calls apart from a cached
+ *   driver entry point; calls are reentrant and thread-safe.
+ */
+#ifndef CROSS_LAYER_SHARED_SA_H
+#define CROSS_LAYER_SHARED_SA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int sa_status;
+#define SA_OK 0
+#define SA_ERR_INVALID_ARG 1 /* bad pointer, size, shape or alignment          */
+#define SA_ERR_UNSUPPORTED 2 /* valid request this build does not implement    */
+#define SA_ERR_WORKSPACE 3   /* workspace missing, misaligned or too small      */
+#define SA_ERR_CUDA 4        /* a CUDA runtime call failed (launch, attribute)  */
+#define SA_ERR_TIMEOUT 5     /* device: a bounded wait gave up                  */
+#define SA_ERR_DEVICE 6      /* device: an input value was out of range         */
+
+typedef enum { SA_BF16 = 0, SA_F32 = 1 } sa_dtype;
+
+#define SA_WS_HEADER_BYTES 256
+
+/* Human-readable name of a status code (static string). */
+const char* sa_status_string(sa_status status);
+
+/* Detail of the last failing call made by this thread ("" if none). */
+const char* sa_last_error(void);
+
+/* ABI version of this header: 1. */
+int sa_abi_version(void);
+
+/*
+ * Synchronises `stream`, then copies the status block's first word into
+ * *device_status (SA_OK, SA_ERR_TIMEOUT or SA_ERR_DEVICE) and, when
+ * `detail` is not NULL, four detail words (kernel id, element index, value,
+ * bound) into detail[0..3].  Returns SA_ERR_CUDA if the copy failed.
+ */
+sa_status sa_read_device_status(const void* ws, void* stream, int* device_status, int64_t* detail);
+
+/* Enqueues a reset of the status block to zero on `stream`. */
+sa_status sa_clear_device_status(void* ws, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Indexer score, decode form  [IC section 1: the lightning indexer scores
+ * every previous token for the current query; CLSA "Comment CLSA
+ * fonctionne": the shared indexer layer computes the scores once].
+ *
+ * The pages name the DSA lightning indexer but print no formula; this call
+ * computes its DSA form, one key vector per token shared by every indexer
+ * head:
+ *   scores[b*ld + t] = sum_j w[b,j] * max(0, sum_c qI[b,j,c] * KI[seq_off[b]+t, c])
+ * for t in [0, seq_len[b]), with fp32 accumulation; the result is canonical
+ * (+0, never -0).  Entries t >= seq_len[b] are left untouched.
+ *
+ *   qI       bf16 [B, H_I, d_I]       query of sequence b, one row per head
+ *   w        fp32 [B, H_I]            head weights (positive in the method)
+ *   KI       bf16 [n_tokens, d_I]     packed indexer-key cache
+ *   seq_off  int64 [B+1] (device)     first KI row of sequence b
+ *   seq_len  int32 [B]   (device)     visible keys of sequence b (<= S_max)
+ *   S_max    host upper bound on seq_len (sizes the grid); ld >= S_max
+ *   scores   fp32 [B, ld]
+ * Supported: 1 <= H_I <= 64, d_I in {64, 128, 192, 256}.
+ * Device errors: seq_len[b] > S_max or a row past n_tokens -> SA_ERR_DEVICE
+ * (rows past n_tokens read as zero; nothing past column S_max is written).
+ * ---------------------------------------------------------------------- */
+size_t sa_index_score_workspace_size(int B);
+sa_status sa_index_score(const void* qI, const float* w, const void* KI, const int64_t* seq_off,
+                         const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I,
+                         int d_I, float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* ------------------------------------------------------------------------
+ * Indexer score, chunked-prefill form  [same definition, IC section 1;
+ * CA "Enonce du Probleme": queries of the current chunk attend to the
+ * accumulated KV cache].  Nq queries of ONE sequence; query p sees keys
+ * t in [0, q_pos[p]]:
+ *   scores[p*ld + t] = sum_j w[p,j] * max(0, sum_c qI[p,j,c] * KI[t,c])
+ *
+ *   qI bf16 [Nq, H_I, d_I]; w fp32 [Nq, H_I]; KI bf16 [S, d_I];
+ *   q_pos int32 [Nq] (device), each in [0, S); max_pos = host upper bound
+ *   of q_pos (< S); scores fp32 [Nq, ld] with ld >= max_pos + 1.
+ * Supported: H_I * 16 <= 256 ... see sa_index_score; Nq >= 1.
+ * Device errors: q_pos out of [0, max_pos] -> SA_ERR_DEVICE, row skipped.
+ * ---------------------------------------------------------------------- */
+size_t sa_index_score_prefill_workspace_size(int Nq);
+sa_status sa_index_score_prefill(const void* qI, const float* w, const void* KI,
+                                 const int32_t* q_pos, int Nq, int S, int max_pos, int H_I,
+                                 int d_I, float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* ------------------------------------------------------------------------
+ * Top-k  [IC section 1: keep the k most relevant tokens; CLSA: the top-k
+ * selection runs once and its index is reused].
+ *
+ * Row q of `scores` has n_valid[q] valid entries.  Selects the min(k,
+ * n_valid[q]) largest; ties go to the LOWER index; the order on floats is
+ * IEEE with -0 == +0 (NaN inputs give an unspecified, in-range result).
+ *   idx        int32 [Nq, k]  selected indices in ASCENDING order, then -1
+ *   top_scores fp32 [Nq, k]   (nullable) the matching scores, 0 for padding
+ *   n_max      host upper bound of n_valid (<= ld)
+ * Device errors: n_valid[q] outside [0, n_max] -> SA_ERR_DEVICE, clamped.
+ * ---------------------------------------------------------------------- */
+size_t sa_topk_workspace_size(int Nq, int n_max, int k);
+sa_status sa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max,
+                  int k, int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Sparse decode attention for one layer group  [IC section 1: main
+ * attention over the k selected tokens; IC section 2: S layers reuse the
+ * top-k index of the nearest upstream F layer; CLSA "Comment CLSA
+ * fonctionne": the same index is handed to every cross-decoder layer over
+ * the shared KV cache].
+ *
+ * For layer l < L_g, sequence b, query head h (KV head g = h / (Hq/Hkv)):
+ *   z_t = scale * Q[l,b,h,:] . K_b[g,t,:],  t in idx[b,:] (entries < 0 skipped)
+ *   O[l,b,h,:] = sum_t softmax(z)_t * V_b[g,t,:]      (fp32 softmax/accumulate)
+ * A row with no valid index gets O = 0.
+ *
+ *   Q        bf16 [L_g, B, Hq, d]   queries of every layer of the group
+ *   K, V     bf16 packed per sequence: sequence b starts at element
+ *            seq_off[b]*Hkv*d and is laid out [Hkv, seq_len[b], d]
+ *            (KV-head-major); every layer of the group reads this cache
+ *   seq_off  int64 [B+1], seq_len int32 [B] (device)
+ *   idx      int32 [B, k] (device) shared index of the group
+ *   O        [L_g, B, Hq, d], bf16 or fp32 per out_dtype
+ * Each selected K/V row is brought from HBM once per (sequence, KV head)
+ * for the whole group.  Supported: d = 128, Hq % Hkv == 0, Hq/Hkv <= 128.
+ * Device errors: idx entry >= seq_len[b] -> SA_ERR_DEVICE, entry skipped.
+ * ---------------------------------------------------------------------- */
+size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int d, int k);
+sa_status sa_sparse_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
+                                const int32_t* seq_len, const int32_t* idx, int L_g, int B, int Hq,
+                                int Hkv, int d, int k, float scale, void* O, sa_dtype out_dtype,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * One decode step over a layer pattern  [IC section 2: a binary pattern
+ * marks F layers, which run their indexer and overwrite the cached top-k
+ * index, and S layers, which reuse the index of the nearest upstream F
+ * layer - one conditional branch in the inference loop, no extra memory].
+ *
+ * pattern: n_layers characters 'F' / 'S', first one 'F'.  Host arrays of
+ * device pointers, one entry per layer: qI[l], w[l], KI[l] (read for F
+ * layers only, shapes as in sa_index_score) and K[l], V[l] (the cache that
+ * layer reads, layout as in sa_sparse_decode_attn).  Q / O: [n_layers, B,
+ * Hq, d].  idx [B, k] is the index cache (overwritten at every F layer) and
+ * scores [B, ld] the indexer's scratch output.  Consecutive layers that
+ * share one index and one cache run as a single fused group call.
+ * ---------------------------------------------------------------------- */
+size_t sa_decode_step_workspace_size(int n_layers, int B, int S_max, int Hq, int Hkv, int d, int k);
+sa_status sa_decode_step(const char* pattern, int n_layers, const void* const* qI,
+                         const float* const* w, const void* const* KI, const void* const* K,
+                         const void* const* V, const int64_t* seq_off, const int32_t* seq_len,
+                         int B, int64_t n_tokens, int S_max, int H_I, int d_I, int k, const void* Q,
+                         int Hq, int Hkv, int d, float scale, void* O, sa_dtype out_dtype,
+                         int32_t* idx, float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* ------------------------------------------------------------------------
+ * Block union + zero-copy paged causal attention for one prefill chunk
+ * [CA selection step: map each selected token to its KV block, union over
+ * the query blocks of the chunk (Q-block union) and over the query heads
+ * of each GQA group (intra-group union) into a minimal per-group table
+ * T_g that keeps every selected block; CA execution step: the table goes
+ * to a dense paged attention kernel as kv_indptr / kv_indices and the
+ * blocks are read in place from the KV-head-major cache, no copy].
+ *
+ *   idx        int32 [Nq, k]  per-query selected tokens (entries < 0 skipped)
+ *   q_pos      int32 [Nq]     position of each query (causal limit)
+ *   Q          bf16 [Nq, Hq, d];  K, V bf16 [Hkv, S, d]
+ *   kv_indptr  int32 [Hkv + 1]           (output) CSR row pointers
+ *   kv_indices int32 [Hkv * ceil(S/block)] (output) sorted distinct blocks
+ *   O          [Nq, Hq, d] bf16 / fp32: query p, head h attends with
+ *              softmax to every key t in the blocks of T_{h/(Hq/Hkv)} with
+ *              t <= q_pos[p] and t < S.
+ * The selection is shared by all heads, so every group's table is the
+ * same set.  Supported: d = 128, block = 64.
+ * ---------------------------------------------------------------------- */
+size_t sa_block_union_prefill_workspace_size(int S, int Nq, int Hq, int Hkv, int d, int k, int block);
+sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const void* Q,
+                                 const void* K, const void* V, int S, int Nq, int Hq, int Hkv,
+                                 int d, int k, int block, float scale, int32_t* kv_indptr,
+                                 int32_t* kv_indices, void* O, sa_dtype out_dtype, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CROSS_LAYER_SHARED_SA_H */

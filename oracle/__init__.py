@@ -1,0 +1,167 @@
+"""CPU oracle for cross-layer shared sparse attention (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  It shares no code with the CUDA path in
+``cross_layer_shared_b200``: the arithmetic is the plain C in
+``oracle/sa_oracle.c`` (fp64, naive loops, OpenMP over independent
+outputs), loaded here through ctypes; the only Python logic is the layer
+pattern walk of ``decode_step`` (IndexCache's F/S rule) and argument
+marshalling.
+
+Parity pins: tests/test_oracle_pins.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sa_oracle.c")
+_LIB = os.path.join(_HERE, "libsa_oracle.so")
+CFLAGS = ["-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared", "-std=c11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def load(path: str):
+    """Load a compiled oracle library and declare its signatures."""
+    lb = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    I64 = ctypes.c_int64
+    D = ctypes.c_double
+    lb.oracle_index_score.argtypes = [P, P, P, P, P, P, I, I, I, P, I64]
+    lb.oracle_topk.argtypes = [P, I64, P, I, I, P, P]
+    lb.oracle_sparse_decode_attn.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, D, P]
+    lb.oracle_block_union.argtypes = [P, I, I, I, I, I, P, P]
+    lb.oracle_block_union.restype = I
+    lb.oracle_paged_prefill_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, D, P]
+    lb.oracle_num_threads.restype = I
+    return lb
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = load(build())
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+def index_score(qI, w, KI, seq_off, q_seq, q_pos, ld: Optional[int] = None) -> np.ndarray:
+    """scores [Nq, ld] fp32; entries past q_pos are NaN (never written)."""
+    qI = _c(qI, np.uint16)
+    Nq, H_I, d_I = qI.shape
+    w = _c(w, np.float32)
+    KI = _c(KI, np.uint16)
+    seq_off = _c(seq_off, np.int64)
+    q_seq = _c(q_seq, np.int32)
+    q_pos = _c(q_pos, np.int32)
+    ld = int(ld if ld is not None else q_pos.max() + 1)
+    out = np.full((Nq, ld), np.nan, dtype=np.float32)
+    lib().oracle_index_score(_p(qI), _p(w), _p(KI), _p(seq_off), _p(q_seq), _p(q_pos), Nq, H_I, d_I,
+                             _p(out), ld)
+    return out
+
+
+def topk(scores, n_valid, k: int, with_scores: bool = False):
+    scores = _c(scores, np.float32)
+    Nq, ld = scores.shape
+    n_valid = _c(n_valid, np.int32)
+    idx = np.empty((Nq, k), dtype=np.int32)
+    ts = np.empty((Nq, k), dtype=np.float32) if with_scores else None
+    lib().oracle_topk(_p(scores), ld, _p(n_valid), Nq, k, _p(idx), _p(ts))
+    return (idx, ts) if with_scores else idx
+
+
+def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float) -> np.ndarray:
+    Q = _c(Q, np.uint16)
+    L, B, Hq, d = Q.shape
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    idx = _c(idx, np.int32)
+    k = idx.shape[1]
+    out = np.empty((L, B, Hq, d), dtype=np.float64)
+    lib().oracle_sparse_decode_attn(_p(Q), _p(K), _p(V), _p(_c(seq_off, np.int64)),
+                                    _p(_c(seq_len, np.int32)), _p(idx), L, B, Hq, Hkv, d, k,
+                                    float(scale), _p(out))
+    return out
+
+
+def block_union(idx, S: int, block: int, Hkv: int):
+    idx = _c(idx, np.int32)
+    Nq, k = idx.shape
+    nb = (S + block - 1) // block
+    indptr = np.zeros(Hkv + 1, dtype=np.int32)
+    indices = np.zeros(max(1, Hkv * nb), dtype=np.int32)
+    n = lib().oracle_block_union(_p(idx), Nq, k, S, block, Hkv, _p(indptr), _p(indices))
+    return indptr, indices[: Hkv * n].copy()
+
+
+def paged_prefill_attn(Q, q_pos, K, V, block: int, kv_indptr, kv_indices, scale: float) -> np.ndarray:
+    Q = _c(Q, np.uint16)
+    Nq, Hq, d = Q.shape
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    Hkv, S, _ = K.shape
+    out = np.empty((Nq, Hq, d), dtype=np.float64)
+    ind = _c(kv_indices, np.int32)
+    if ind.size == 0:
+        ind = np.zeros(1, np.int32)
+    lib().oracle_paged_prefill_attn(_p(Q), _p(_c(q_pos, np.int32)), _p(K), _p(V), S, Nq, Hq, Hkv, d,
+                                    block, _p(_c(kv_indptr, np.int32)), _p(ind), float(scale),
+                                    _p(out))
+    return out
+
+
+def decode_step(pattern: str, qI: Sequence, w: Sequence, KI: Sequence, seq_off, seq_len, k: int,
+                Q, K: Sequence, V: Sequence, Hkv: int, scale: float):
+    """One decode step over the layers of `pattern` [IndexCache, technical
+    summary section 2: an F layer runs its indexer and overwrites the cached
+    top-k index; an S layer reuses the index of the nearest upstream F
+    layer].  qI/w/KI/K/V are per-layer lists (entries of S layers' indexer
+    inputs are ignored).  Returns (O [L,B,Hq,d] fp64, list of the index used
+    by each layer)."""
+    if not pattern or pattern[0] != "F":
+        raise ValueError("a layer pattern must start with F: an S layer needs an upstream F layer")
+    L = len(pattern)
+    B = len(seq_len)
+    seq_len = np.asarray(seq_len, dtype=np.int32)
+    out = []
+    used = []
+    idx = None
+    for layer in range(L):
+        if pattern[layer] == "F":
+            s = index_score(qI[layer], w[layer], KI[layer], seq_off, np.arange(B), seq_len - 1)
+            idx = topk(s, seq_len, k)
+        elif pattern[layer] != "S":
+            raise ValueError("pattern letters are F or S")
+        used.append(idx)
+        out.append(sparse_decode_attn(np.asarray(Q)[layer:layer + 1], K[layer], V[layer], seq_off,
+                                      seq_len, idx, Hkv, scale)[0])
+    return np.stack(out), used

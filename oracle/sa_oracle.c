@@ -1,0 +1,274 @@
+/*
+ * CPU oracle for cross-layer shared sparse attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, the smoke check and the bench's
+ * CPU-baseline leg may load this library.  It shares no code, header, table
+ * or helper with the CUDA path in cross_layer_shared_b200/csrc.
+ *
+ * Each function is the plain definition of one step, computed naively in
+ * fp64 (inputs are bf16 bit patterns / fp32 values, widened exactly), with
+ * loops in the order the definition is written and OpenMP only over
+ * independent outputs.  No blocking, fusion or reordering.
+ *
+ * Pages followed:
+ *   [CLSA]   "Le routage partage entre couches accelere l'attention sparse
+ *            de 7x sans perte de qualite" (news article on "CLSA: You Only
+ *            Index Once"), section "Comment CLSA fonctionne".
+ *   [IC]     "IndexCache: Accelerating Sparse Attention via Cross-Layer
+ *            Index Reuse", technical summary, sections 1 (Problematique)
+ *            and 2 (Methodologie : IndexCache).
+ *   [CA]     "CompactAttention: Accelerating Chunked Prefill with
+ *            Block-Union KV Selection", technical summary, section
+ *            "Methodologie : CompactAttention" (selection step, execution
+ *            step).
+ *
+ * The pages name the DSA "lightning indexer" but print no formula for its
+ * score; the oracle uses the DSA form score_t = sum_j w_j * ReLU(q_j . k_t)
+ * with one key vector per token shared by all indexer heads, no 1/sqrt(d)
+ * and no softmax.  The score is rounded once to fp32, the precision in
+ * which both sides take the top-k decision.
+ *
+ * Parity pins for every function live in tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/*
+ * Indexer score [IC section 1: the lightning indexer scores every previous
+ * token for the current query; CLSA section "Comment CLSA fonctionne": the
+ * shared indexer layer computes the scores once].
+ *
+ * For query q (sequence q_seq[q], last visible key q_pos[q]) and each key
+ * t in [0, q_pos[q]]:
+ *   dot_j   = sum_c qI[q,j,c] * KI[seq_off[q_seq[q]] + t, c]
+ *   score_t = sum_j w[q,j] * max(dot_j, 0)
+ * written to scores[q*ld + t] as fp32 (+0 when every dot is <= 0).
+ * Entries beyond q_pos are not written.
+ */
+void oracle_index_score(const uint16_t* qI, const float* w, const uint16_t* KI,
+                        const int64_t* seq_off, const int32_t* q_seq, const int32_t* q_pos,
+                        int Nq, int H_I, int d_I, float* scores, int64_t ld) {
+  for (int q = 0; q < Nq; ++q) {
+    const int64_t base = seq_off[q_seq[q]];
+    const int64_t n = (int64_t)q_pos[q] + 1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n; ++t) {
+      const uint16_t* k = KI + (base + t) * d_I;
+      double s = 0.0;
+      for (int j = 0; j < H_I; ++j) {
+        const uint16_t* qj = qI + ((int64_t)q * H_I + j) * d_I;
+        double dot = 0.0;
+        for (int c = 0; c < d_I; ++c) dot += bf(qj[c]) * bf(k[c]);
+        const double relu = dot > 0.0 ? dot : 0.0;
+        s += (double)w[(int64_t)q * H_I + j] * relu;
+      }
+      scores[(int64_t)q * ld + t] = (float)s;
+    }
+  }
+}
+
+typedef struct {
+  float s;
+  int32_t i;
+} scored_t;
+
+/* order: score descending, then index ascending (ties go to the lower index) */
+static int by_score_then_index(const void* a, const void* b) {
+  const scored_t* x = (const scored_t*)a;
+  const scored_t* y = (const scored_t*)b;
+  if (x->s > y->s) return -1;
+  if (x->s < y->s) return 1;
+  return (x->i > y->i) - (x->i < y->i);
+}
+
+static int by_index(const void* a, const void* b) {
+  const int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+  return (x > y) - (x < y);
+}
+
+/*
+ * Top-k [IC section 1: the indexer keeps the k most relevant tokens;
+ * CLSA: the top-k selection runs once and its index is passed on].
+ *
+ * Row q: sort the n_valid[q] scores by (score desc, index asc), keep the
+ * first min(k, n_valid[q]), emit their indices in ascending order, pad the
+ * rest of the row with -1.  top_scores (nullable) gets the matching scores
+ * (0 for padding).
+ */
+void oracle_topk(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int k,
+                 int32_t* idx, float* top_scores) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int q = 0; q < Nq; ++q) {
+    const int n = n_valid[q];
+    scored_t* all = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n > 0 ? n : 1));
+    for (int t = 0; t < n; ++t) {
+      all[t].s = scores[(int64_t)q * ld + t];
+      all[t].i = t;
+    }
+    qsort(all, (size_t)n, sizeof(scored_t), by_score_then_index);
+    const int m = n < k ? n : k;
+    int32_t* row = idx + (int64_t)q * k;
+    for (int j = 0; j < m; ++j) row[j] = all[j].i;
+    qsort(row, (size_t)m, sizeof(int32_t), by_index);
+    for (int j = m; j < k; ++j) row[j] = -1;
+    if (top_scores) {
+      float* ts = top_scores + (int64_t)q * k;
+      for (int j = 0; j < m; ++j) ts[j] = scores[(int64_t)q * ld + row[j]];
+      for (int j = m; j < k; ++j) ts[j] = 0.0f;
+    }
+    free(all);
+  }
+}
+
+/*
+ * Softmax attention of one query row over an explicit key list (helper of
+ * the two attention definitions below).
+ *   z_t = scale * (q . K_t),  o = sum_t exp(z_t - max z) V_t / sum_t exp(z_t - max z)
+ * An empty key list gives o = 0.
+ */
+static void attend_row(const uint16_t* q, const uint16_t* Kb, const uint16_t* Vb, const int64_t* keys,
+                       int64_t n, int d, double scale, double* z, double* o) {
+  for (int c = 0; c < d; ++c) o[c] = 0.0;
+  if (n == 0) return;
+  double m = -INFINITY;
+  for (int64_t j = 0; j < n; ++j) {
+    const uint16_t* kr = Kb + keys[j] * d;
+    double dot = 0.0;
+    for (int c = 0; c < d; ++c) dot += bf(q[c]) * bf(kr[c]);
+    z[j] = scale * dot;
+    if (z[j] > m) m = z[j];
+  }
+  double den = 0.0;
+  for (int64_t j = 0; j < n; ++j) {
+    const double p = exp(z[j] - m);
+    const uint16_t* vr = Vb + keys[j] * d;
+    den += p;
+    for (int c = 0; c < d; ++c) o[c] += p * bf(vr[c]);
+  }
+  for (int c = 0; c < d; ++c) o[c] /= den;
+}
+
+/*
+ * Sparse decode attention for one layer group reading one KV cache
+ * [IC section 1: main attention over the k selected tokens, O(Lk);
+ *  IC section 2: S layers reuse the index of the nearest upstream F layer;
+ *  CLSA "Comment CLSA fonctionne": every cross-decoder layer gets the same
+ *  index over the shared KV cache].
+ *
+ * Q [L,B,Hq,d]; K,V: sequence b at element offset seq_off[b]*Hkv*d, laid
+ * out [Hkv, seq_len[b], d]; idx [B,k] (entries < 0 skipped); query head h
+ * reads KV head h / (Hq/Hkv).  O [L,B,Hq,d] in fp64.
+ */
+void oracle_sparse_decode_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                               const int64_t* seq_off, const int32_t* seq_len, const int32_t* idx,
+                               int L, int B, int Hq, int Hkv, int d, int k, double scale,
+                               double* O) {
+  const int G = Hq / Hkv;
+  const int64_t rows = (int64_t)L * B * Hq;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t r = 0; r < rows; ++r) {
+    const int h = (int)(r % Hq);
+    const int b = (int)((r / Hq) % B);
+    const int g = h / G;
+    const uint16_t* Kb = K + seq_off[b] * Hkv * d + (int64_t)g * seq_len[b] * d;
+    const uint16_t* Vb = V + seq_off[b] * Hkv * d + (int64_t)g * seq_len[b] * d;
+    int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)(k > 0 ? k : 1));
+    double* z = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+    int64_t n = 0;
+    for (int j = 0; j < k; ++j) {
+      const int32_t t = idx[(int64_t)b * k + j];
+      if (t >= 0) keys[n++] = t;
+    }
+    attend_row(Q + r * d, Kb, Vb, keys, n, d, scale, z, O + r * d);
+    free(keys);
+    free(z);
+  }
+}
+
+/*
+ * Block union [CA, selection step]: map every selected token t to its KV
+ * block t / block, take the union over every query of the chunk (Q-block
+ * union) and over the query heads of each KV group (intra-group union; the
+ * index is shared by all heads, so every group gets the same set).  The
+ * per-group table T_g is the sorted list of distinct blocks, emitted as
+ * CSR: kv_indptr[g+1] = kv_indptr[g] + |T_g|, kv_indices holds the blocks.
+ * Returns |T_g|.
+ */
+int oracle_block_union(const int32_t* idx, int Nq, int k, int S, int block, int Hkv,
+                       int32_t* kv_indptr, int32_t* kv_indices) {
+  const int nb = (S + block - 1) / block;
+  unsigned char* mark = (unsigned char*)calloc((size_t)nb, 1);
+  for (int64_t q = 0; q < Nq; ++q)
+    for (int j = 0; j < k; ++j) {
+      const int32_t t = idx[q * k + j];
+      if (t >= 0) mark[t / block] = 1;
+    }
+  int n = 0;
+  for (int bl = 0; bl < nb; ++bl) n += mark[bl];
+  kv_indptr[0] = 0;
+  for (int g = 0; g < Hkv; ++g) {
+    int32_t* out = kv_indices + (int64_t)g * n;
+    int m = 0;
+    for (int bl = 0; bl < nb; ++bl)
+      if (mark[bl]) out[m++] = bl;
+    kv_indptr[g + 1] = kv_indptr[g] + n;
+  }
+  free(mark);
+  return n;
+}
+
+/*
+ * Paged causal attention over the union blocks [CA, execution step: the
+ * per-group block table is handed to a dense paged attention kernel that
+ * reads the selected blocks in place from the KV-head-major cache
+ * [B, H_kv, L, D]].
+ *
+ * Query p (position q_pos[p]) and head h attend, with softmax, to every key
+ * t of the blocks in T_{h/(Hq/Hkv)} with t <= q_pos[p] and t < S.
+ * Q [Nq,Hq,d]; K,V [Hkv,S,d]; O [Nq,Hq,d] in fp64.
+ */
+void oracle_paged_prefill_attn(const uint16_t* Q, const int32_t* q_pos, const uint16_t* K,
+                               const uint16_t* V, int S, int Nq, int Hq, int Hkv, int d, int block,
+                               const int32_t* kv_indptr, const int32_t* kv_indices, double scale,
+                               double* O) {
+  const int G = Hq / Hkv;
+  const int64_t rows = (int64_t)Nq * Hq;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t r = 0; r < rows; ++r) {
+    const int p = (int)(r / Hq);
+    const int h = (int)(r % Hq);
+    const int g = h / G;
+    const int64_t nblk = kv_indptr[g + 1] - kv_indptr[g];
+    int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nblk * block + 1));
+    double* z = (double*)malloc(sizeof(double) * (size_t)(nblk * block + 1));
+    int64_t n = 0;
+    for (int64_t i = 0; i < nblk; ++i) {
+      const int64_t b0 = (int64_t)kv_indices[kv_indptr[g] + i] * block;
+      for (int64_t t = b0; t < b0 + block; ++t)
+        if (t <= q_pos[p] && t < S) keys[n++] = t;
+    }
+    attend_row(Q + r * d, K + (int64_t)g * S * d, V + (int64_t)g * S * d, keys, n, d, scale, z,
+               O + r * d);
+    free(keys);
+    free(z);
+  }
+}
+
+/* threads OpenMP will use (reported next to CPU timings) */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  extern int omp_get_max_threads(void);
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

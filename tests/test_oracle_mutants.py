@@ -1,0 +1,54 @@
+"""The pins catch planted mistakes: each mutant is a copy of the oracle's C
+source with one plausible slip, compiled on the CPU; at least one pin in
+tests/test_oracle_pins.py must fail against it."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "sa_oracle.c")
+
+MUTANTS = {
+    "relu dropped": ("const double relu = dot > 0.0 ? dot : 0.0;", "const double relu = dot;"),
+    "one head weight for all heads": ("s += (double)w[(int64_t)q * H_I + j] * relu;",
+                                      "s += (double)w[(int64_t)q * H_I] * relu;"),
+    "last visible key dropped": ("const int64_t n = (int64_t)q_pos[q] + 1;",
+                                 "const int64_t n = (int64_t)q_pos[q];"),
+    "sequence offset ignored": ("const int64_t base = seq_off[q_seq[q]];", "const int64_t base = 0;"),
+    "ties to the higher index": ("return (x->i > y->i) - (x->i < y->i);",
+                                 "return (x->i < y->i) - (x->i > y->i);"),
+    "output not in index order": ("qsort(row, (size_t)m, sizeof(int32_t), by_index);", ";"),
+    "scale dropped": ("z[j] = scale * dot;", "z[j] = dot;"),
+    "GQA map modulo": ("const int g = h / G;\n    const uint16_t* Kb", "const int g = h % Hkv;\n    const uint16_t* Kb"),
+    "ceil block map": ("if (t >= 0) mark[t / block] = 1;", "if (t >= 0) mark[(t + block - 1) / block] = 1;"),
+    "causal strict": ("if (t <= q_pos[p] && t < S) keys[n++] = t;", "if (t < q_pos[p] && t < S) keys[n++] = t;"),
+    "value row of the wrong token": ("const uint16_t* vr = Vb + keys[j] * d;", "const uint16_t* vr = Vb + keys[0] * d;"),
+}
+
+PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique: {name}"
+    mut = tmp_path / "mutant.c"
+    mut.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", str(so), str(mut), "-lm"])
+    saved = oracle._lib
+    oracle._lib = oracle.load(str(so))
+    failed = []
+    try:
+        for pin in PINS:
+            try:
+                pin()
+            except (AssertionError, ValueError):
+                failed.append(pin.__name__)
+    finally:
+        oracle._lib = saved
+    assert failed, f"no pin catches the mutant '{name}'"

@@ -1,0 +1,418 @@
+"""Pins for the CPU oracle: each test ties it to something other than itself.
+
+The pages print no worked example, so the pins are closed forms, brute force
+on tiny inputs, special cases that reduce to a library routine (torch fp64
+softmax attention), exact rational arithmetic, and invariants that the
+definitions imply.  Each is chosen so that a plausible slip in the oracle
+(dropped ReLU, wrong head weight, transposed operand, wrong GQA map, wrong
+tie rule, off-by-one visibility, wrong block map) fails at least one.
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import bf16_bits_to_f32, f32_to_bf16_bits
+
+
+def bf(x):
+    return f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+# ----------------------------------------------------------------------------
+# indexer score
+# ----------------------------------------------------------------------------
+def test_index_one_hot_closed_form():
+    # q_j = e_{a_j}, k_t = 2 e_{t mod 8}: dot_j = 2 [a_j == t mod 8], score = 2 w_j of that head
+    d_I, H_I, S = 8, 3, 24
+    a = [1, 4, 6]
+    qI = np.zeros((1, H_I, d_I), np.float32)
+    for j, aj in enumerate(a):
+        qI[0, j, aj] = 1.0
+    KI = np.zeros((S, d_I), np.float32)
+    for t in range(S):
+        KI[t, t % 8] = 2.0
+    w = np.array([[0.25, 0.5, 0.875]], np.float32)
+    s = oracle.index_score(bf(qI), w, bf(KI), [0, S], [0], [S - 1])[0]
+    for t in range(S):
+        want = 2.0 * w[0, a.index(t % 8)] if (t % 8) in a else 0.0
+        assert s[t] == np.float32(want), t
+
+
+def test_index_relu_sign_and_positive_zero():
+    # q_0 = +1, q_1 = -1, q_2 = +0.5 (all coords), k_t = (t-3) (all coords)
+    # dot_j = d*s_j*c_t ; score = d*c_t*(w0 + 0.5 w2) for c_t>0, d*|c_t|*w1 for c_t<0, +0 at c_t=0
+    d_I, S = 4, 8
+    sj = [1.0, -1.0, 0.5]
+    qI = np.array([[[v] * d_I for v in sj]], np.float32)
+    KI = np.array([[t - 3.0] * d_I for t in range(S)], np.float32)
+    w = np.array([[0.5, 0.25, 1.0]], np.float32)
+    s = oracle.index_score(bf(qI), w, bf(KI), [0, S], [0], [S - 1])[0]
+    for t in range(S):
+        c = t - 3
+        if c > 0:
+            want = d_I * c * (0.5 + 0.5 * 1.0)
+        elif c < 0:
+            want = d_I * (-c) * 0.25
+        else:
+            want = 0.0
+        assert s[t] == np.float32(want)
+    assert np.float32(s[3]).view(np.uint32) == 0, "score must be +0, not -0"
+
+
+def test_index_visibility_and_sequence_offsets():
+    # two packed sequences with constant keys 1 and 3; query b reads only its own
+    # sequence and only keys t <= q_pos
+    d_I, H_I = 4, 2
+    S0, S1 = 5, 7
+    KI = np.concatenate([np.full((S0, d_I), 1.0), np.full((S1, d_I), 3.0)]).astype(np.float32)
+    qI = np.ones((2, H_I, d_I), np.float32)
+    w = np.array([[1.0, 0.5], [0.25, 0.125]], np.float32)
+    s = oracle.index_score(bf(qI), w, bf(KI), [0, S0, S0 + S1], [0, 1], [2, 6], ld=8)
+    assert np.all(s[0, :3] == np.float32(d_I * 1.0 * 1.5))
+    assert np.all(np.isnan(s[0, 3:])), "keys past q_pos must not be written"
+    assert np.all(s[1, :7] == np.float32(d_I * 3.0 * 0.375))
+    assert np.isnan(s[1, 7])
+
+
+def test_index_exact_rational_arithmetic():
+    # the oracle's fp32 score is the exact real score rounded once (allow one ulp)
+    rng = np.random.default_rng(7)
+    H_I, d_I, S = 4, 16, 32
+    qI = bf(rng.standard_normal((1, H_I, d_I)) / 8)
+    KI = bf(rng.standard_normal((S, d_I)) / 8)
+    w = rng.uniform(0.1, 1.0, (1, H_I)).astype(np.float32)
+    s = oracle.index_score(qI, w, KI, [0, S], [0], [S - 1])[0]
+    qf = bf16_bits_to_f32(qI)[0]
+    kf = bf16_bits_to_f32(KI)
+    for t in range(S):
+        exact = Fraction(0)
+        for j in range(H_I):
+            dot = sum(Fraction(float(qf[j, c])) * Fraction(float(kf[t, c])) for c in range(d_I))
+            exact += Fraction(float(w[0, j])) * max(dot, Fraction(0))
+        ulp = np.spacing(np.float32(float(exact)))
+        assert abs(Fraction(float(s[t])) - exact) <= Fraction(float(ulp)), t
+
+
+def test_index_weight_scaling_and_head_permutation():
+    rng = np.random.default_rng(3)
+    H_I, d_I, S = 5, 32, 40
+    qI = bf(rng.standard_normal((1, H_I, d_I)) / 8)
+    KI = bf(rng.standard_normal((S, d_I)) / 8)
+    w = rng.uniform(0.1, 1.0, (1, H_I)).astype(np.float32)
+    base = oracle.index_score(qI, w, KI, [0, S], [0], [S - 1])[0]
+    doubled = oracle.index_score(qI, 2 * w, KI, [0, S], [0], [S - 1])[0]
+    assert np.array_equal(doubled, 2 * base)
+    perm = rng.permutation(H_I)
+    permuted = oracle.index_score(qI[:, perm], w[:, perm], KI, [0, S], [0], [S - 1])[0]
+    np.testing.assert_allclose(permuted, base, rtol=2 ** -23, atol=0)
+    # a head with a zero weight contributes nothing
+    w0 = w.copy()
+    w0[0, 2] = 0
+    drop = oracle.index_score(np.delete(qI, 2, axis=1), np.delete(w, 2, axis=1), KI, [0, S], [0], [S - 1])[0]
+    np.testing.assert_allclose(oracle.index_score(qI, w0, KI, [0, S], [0], [S - 1])[0], drop,
+                               rtol=2 ** -23)
+
+
+# ----------------------------------------------------------------------------
+# top-k
+# ----------------------------------------------------------------------------
+def _brute_force_topk(s, k):
+    """Unique subset whose members all beat all non-members under
+    (score desc, index asc), found by enumeration."""
+    n = len(s)
+    good = []
+    for sub in itertools.combinations(range(n), k):
+        inside = set(sub)
+        ok = all((s[i] > s[j]) or (s[i] == s[j] and i < j)
+                 for i in inside for j in range(n) if j not in inside)
+        if ok:
+            good.append(sub)
+    assert len(good) == 1
+    return list(good[0])
+
+
+def test_topk_brute_force_with_ties():
+    rng = np.random.default_rng(11)
+    for trial in range(40):
+        n = int(rng.integers(1, 10))
+        s = rng.choice(np.array([0.0, 0.5, 1.0, 1.5], np.float32), size=n)
+        for k in range(1, n + 1):
+            got = oracle.topk(s[None, :], [n], k)[0]
+            assert list(got) == _brute_force_topk(list(s), k)
+
+
+def test_topk_all_equal_takes_lowest_indices():
+    s = np.full((2, 100), 0.75, np.float32)
+    got = oracle.topk(s, [100, 60], 16)
+    assert list(got[0]) == list(range(16))
+    assert list(got[1]) == list(range(16))
+
+
+def test_topk_short_rows_pad_with_minus_one():
+    s = np.array([[3.0, 1.0, 2.0, 9.0]], np.float32)
+    got, ts = oracle.topk(s, [3], 5, with_scores=True)
+    assert list(got[0]) == [0, 1, 2, -1, -1]
+    assert list(ts[0]) == [3.0, 1.0, 2.0, 0.0, 0.0]
+    assert list(oracle.topk(s, [0], 3)[0]) == [-1, -1, -1]
+
+
+def test_topk_distinct_scores_match_argsort():
+    rng = np.random.default_rng(5)
+    s = rng.permutation(5000).astype(np.float32)[None, :] * np.float32(0.001)
+    got = oracle.topk(s, [5000], 300)[0]
+    want = np.sort(np.argsort(-s[0], kind="stable")[:300])
+    assert np.array_equal(got, want)
+
+
+def test_topk_signed_zero_ties_by_index():
+    s = np.array([[-0.0, 0.0, -0.0, 0.0, -1.0]], np.float32)
+    assert list(oracle.topk(s, [5], 3)[0]) == [0, 1, 2]
+
+
+# ----------------------------------------------------------------------------
+# sparse decode attention
+# ----------------------------------------------------------------------------
+def _dense_attention_torch(Q, K, V, scale):
+    """Library routine: softmax(scale*Q K^T) V in fp64 (torch CPU)."""
+    q = torch.from_numpy(bf16_bits_to_f32(Q).astype(np.float64))
+    k = torch.from_numpy(bf16_bits_to_f32(K).astype(np.float64))
+    v = torch.from_numpy(bf16_bits_to_f32(V).astype(np.float64))
+    return (torch.softmax(scale * q @ k.T, dim=-1) @ v).numpy()
+
+
+def _tiny_decode(rng, B=2, S=(9, 13), Hq=4, Hkv=2, d=16, L=2):
+    seq_off = np.concatenate([[0], np.cumsum(S)]).astype(np.int64)
+    T = int(seq_off[-1])
+    Q = bf(rng.standard_normal((L, B, Hq, d)))
+    K = bf(rng.standard_normal(T * Hkv * d))
+    V = bf(rng.standard_normal(T * Hkv * d))
+    return seq_off, np.array(S, np.int32), Q, K, V
+
+
+def _kv(K, seq_off, S, Hkv, d, b, g):
+    base = seq_off[b] * Hkv * d + g * S[b] * d
+    return K[base: base + S[b] * d].reshape(S[b], d)
+
+
+def test_attn_full_selection_equals_dense_attention():
+    rng = np.random.default_rng(1)
+    seq_off, S, Q, K, V = _tiny_decode(rng)
+    L, B, Hq, d = Q.shape
+    Hkv, k = 2, int(S.max())
+    idx = np.full((B, k), -1, np.int32)
+    for b in range(B):
+        idx[b, :S[b]] = np.arange(S[b])
+    scale = 1 / math.sqrt(d)
+    got = oracle.sparse_decode_attn(Q, K, V, seq_off, S, idx, Hkv, scale)
+    for l, b, h in itertools.product(range(L), range(B), range(Hq)):
+        g = h // (Hq // Hkv)
+        want = _dense_attention_torch(Q[l, b, h][None], _kv(K, seq_off, S, Hkv, d, b, g),
+                                      _kv(V, seq_off, S, Hkv, d, b, g), scale)[0]
+        np.testing.assert_allclose(got[l, b, h], want, rtol=0, atol=1e-12)
+
+
+def test_attn_sparse_equals_masked_dense():
+    rng = np.random.default_rng(2)
+    seq_off, S, Q, K, V = _tiny_decode(rng)
+    L, B, Hq, d = Q.shape
+    Hkv, k = 2, 5
+    idx = np.stack([np.sort(rng.choice(S[b], k, replace=False)) for b in range(B)]).astype(np.int32)
+    scale = 1 / math.sqrt(d)
+    got = oracle.sparse_decode_attn(Q, K, V, seq_off, S, idx, Hkv, scale)
+    for l, b, h in itertools.product(range(L), range(B), range(Hq)):
+        g = h // (Hq // Hkv)
+        Kb = _kv(K, seq_off, S, Hkv, d, b, g)
+        Vb = _kv(V, seq_off, S, Hkv, d, b, g)
+        q = torch.from_numpy(bf16_bits_to_f32(Q[l, b, h]).astype(np.float64))
+        z = scale * torch.from_numpy(bf16_bits_to_f32(Kb).astype(np.float64)) @ q
+        mask = torch.full_like(z, -math.inf)
+        mask[torch.from_numpy(idx[b].astype(np.int64))] = 0.0
+        want = torch.softmax(z + mask, 0) @ torch.from_numpy(bf16_bits_to_f32(Vb).astype(np.float64))
+        np.testing.assert_allclose(got[l, b, h], want.numpy(), rtol=0, atol=1e-12)
+
+
+def test_attn_single_token_returns_its_value_row():
+    rng = np.random.default_rng(4)
+    seq_off, S, Q, K, V = _tiny_decode(rng)
+    L, B, Hq, d = Q.shape
+    idx = np.array([[-1, 3, -1], [-1, -1, 12]], np.int32)
+    got = oracle.sparse_decode_attn(Q, K, V, seq_off, S, idx, 2, 0.25)
+    for l, b, h in itertools.product(range(L), range(B), range(Hq)):
+        t = idx[b][idx[b] >= 0][0]
+        want = bf16_bits_to_f32(_kv(V, seq_off, S, 2, d, b, h // 2)[t])
+        assert np.array_equal(got[l, b, h], want.astype(np.float64))
+
+
+def test_attn_two_tokens_closed_form():
+    # q = (1,..,1), K rows = 1 and 2 (all coords) -> logits scale*d*1, scale*d*2
+    d = 8
+    Q = bf(np.ones((1, 1, 1, d)))
+    K = bf(np.concatenate([np.full(d, 1.0), np.full(d, 2.0)]))
+    V = bf(np.concatenate([np.full(d, 3.0), np.full(d, -1.0)]))
+    scale = 0.125
+    got = oracle.sparse_decode_attn(Q, K, V, [0, 2], [2], np.array([[0, 1]], np.int32), 1, scale)
+    z1, z2 = scale * d * 1.0, scale * d * 2.0
+    want = (math.exp(z1) * 3.0 + math.exp(z2) * -1.0) / (math.exp(z1) + math.exp(z2))
+    np.testing.assert_allclose(got[0, 0, 0], np.full(d, want), rtol=0, atol=1e-14)
+
+
+def test_attn_common_key_shift_changes_nothing():
+    # adding a vector e to every key adds q.e to every logit of that query
+    rng = np.random.default_rng(8)
+    d, S = 16, 12
+    Q = bf(rng.integers(-2, 3, (1, 1, 1, d)))
+    Kf = rng.integers(-2, 3, (S, d)).astype(np.float32)
+    e = rng.integers(-2, 3, d).astype(np.float32)
+    V = bf(rng.standard_normal(S * d))
+    idx = np.array([[0, 2, 3, 7, 11]], np.int32)
+    a = oracle.sparse_decode_attn(Q, bf(Kf.ravel()), V, [0, S], [S], idx, 1, 0.1)
+    b = oracle.sparse_decode_attn(Q, bf((Kf + e).ravel()), V, [0, S], [S], idx, 1, 0.1)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+def test_attn_padding_and_index_order_do_not_matter():
+    rng = np.random.default_rng(9)
+    seq_off, S, Q, K, V = _tiny_decode(rng)
+    idx = np.array([[1, 4, 6, -1], [0, 2, 11, 12]], np.int32)
+    shuffled = np.array([[-1, 6, 1, 4], [12, 0, 11, 2]], np.int32)
+    a = oracle.sparse_decode_attn(Q, K, V, seq_off, S, idx, 2, 0.3)
+    b = oracle.sparse_decode_attn(Q, K, V, seq_off, S, shuffled, 2, 0.3)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+def test_attn_gqa_head_to_kv_head_map():
+    # KV head 0 has V = +1 everywhere, KV head 1 has V = -1: heads 0,1 -> +1, heads 2,3 -> -1
+    d, S, Hq, Hkv = 8, 6, 4, 2
+    rng = np.random.default_rng(10)
+    Q = bf(rng.standard_normal((1, 1, Hq, d)))
+    K = bf(rng.standard_normal(Hkv * S * d))
+    V = bf(np.concatenate([np.ones(S * d), -np.ones(S * d)]))
+    got = oracle.sparse_decode_attn(Q, K, V, [0, S], [S], np.array([[0, 1, 5]], np.int32), Hkv, 0.5)
+    np.testing.assert_allclose(got[0, 0, :2], 1.0, atol=1e-15)
+    np.testing.assert_allclose(got[0, 0, 2:], -1.0, atol=1e-15)
+
+
+def test_attn_no_valid_key_gives_zero():
+    Q = bf(np.ones((1, 1, 1, 4)))
+    out = oracle.sparse_decode_attn(Q, bf(np.ones(8)), bf(np.ones(8)), [0, 2], [2],
+                                    np.array([[-1, -1]], np.int32), 1, 1.0)
+    assert np.all(out == 0)
+
+
+# ----------------------------------------------------------------------------
+# index reuse across layers (F/S pattern)
+# ----------------------------------------------------------------------------
+def _decode_inputs(rng, L, same_indexer):
+    B, S, H_I, d_I, Hq, Hkv, d = 2, (20, 31), 2, 8, 4, 2, 8
+    seq_off = np.concatenate([[0], np.cumsum(S)]).astype(np.int64)
+    T = int(seq_off[-1])
+    mk = lambda: (bf(rng.standard_normal((B, H_I, d_I)) / 8),
+                  rng.uniform(0.1, 1, (B, H_I)).astype(np.float32),
+                  bf(rng.standard_normal((T, d_I)) / 8))
+    ix = [mk()] * L if same_indexer else [mk() for _ in range(L)]
+    Q = bf(rng.standard_normal((L, B, Hq, d)))
+    K = bf(rng.standard_normal(T * Hkv * d))
+    V = bf(rng.standard_normal(T * Hkv * d))
+    return ix, seq_off, np.array(S), Q, K, V, Hkv
+
+
+def test_reuse_FFFF_with_identical_indexers_equals_FSSS():
+    rng = np.random.default_rng(12)
+    ix, seq_off, S, Q, K, V, Hkv = _decode_inputs(rng, 4, True)
+    args = ([a[0] for a in ix], [a[1] for a in ix], [a[2] for a in ix], seq_off, S, 6, Q, [K] * 4,
+            [V] * 4, Hkv, 0.35)
+    o1, used1 = oracle.decode_step("FFFF", *args)
+    o2, used2 = oracle.decode_step("FSSS", *args)
+    assert np.array_equal(o1, o2)
+    for a, b in zip(used1, used2):
+        assert np.array_equal(a, b)
+
+
+def test_reuse_takes_nearest_upstream_full_layer():
+    rng = np.random.default_rng(13)
+    ix, seq_off, S, Q, K, V, Hkv = _decode_inputs(rng, 4, False)
+    o, used = oracle.decode_step("FSFS", [a[0] for a in ix], [a[1] for a in ix], [a[2] for a in ix],
+                                 seq_off, S, 6, Q, [K] * 4, [V] * 4, Hkv, 0.35)
+    assert used[1] is used[0] and used[3] is used[2]
+    assert not np.array_equal(used[0], used[2])
+    # the index of layer 2 is its own indexer's top-k
+    s2 = oracle.index_score(ix[2][0], ix[2][1], ix[2][2], seq_off, [0, 1], S - 1)
+    assert np.array_equal(used[2], oracle.topk(s2, S, 6))
+
+
+def test_pattern_must_start_with_full_layer():
+    with pytest.raises(ValueError):
+        oracle.decode_step("SFSS", [None] * 4, [None] * 4, [None] * 4, [0, 1], [1], 1, None, [], [], 1, 1.0)
+
+
+# ----------------------------------------------------------------------------
+# block union + paged causal attention
+# ----------------------------------------------------------------------------
+def test_union_matches_set_union_coverage_and_minimality():
+    rng = np.random.default_rng(14)
+    S, block, Hkv, Nq, k = 1000, 64, 3, 7, 20
+    idx = np.stack([rng.choice(S, k, replace=False) for _ in range(Nq)]).astype(np.int32)
+    idx[2, 5:] = -1
+    indptr, indices = oracle.block_union(idx, S, block, Hkv)
+    want = sorted({int(t) // block for t in idx.ravel() if t >= 0})
+    assert list(indptr) == [g * len(want) for g in range(Hkv + 1)]
+    for g in range(Hkv):
+        T = list(indices[indptr[g]:indptr[g + 1]])
+        assert T == want
+        covered = {t for t in idx.ravel() if t >= 0}
+        assert all(t // block in T for t in covered)                      # coverage
+        assert all(any(bl * block <= t < (bl + 1) * block for t in covered) for bl in T)  # minimal
+
+
+def test_dense_selection_gives_dense_causal_attention():
+    rng = np.random.default_rng(15)
+    S, block, Hq, Hkv, d, Nq = 200, 64, 4, 2, 16, 6
+    q_pos = np.arange(S - Nq, S, dtype=np.int32)
+    idx = np.stack([np.concatenate([np.arange(p + 1), -np.ones(S - p - 1)]) for p in q_pos]).astype(np.int32)
+    indptr, indices = oracle.block_union(idx, S, block, Hkv)
+    assert list(indices[:indptr[1]]) == list(range((S + block - 1) // block))  # partial last block kept
+    Q = bf(rng.standard_normal((Nq, Hq, d)))
+    K = bf(rng.standard_normal((Hkv, S, d)))
+    V = bf(rng.standard_normal((Hkv, S, d)))
+    scale = 1 / math.sqrt(d)
+    got = oracle.paged_prefill_attn(Q, q_pos, K, V, block, indptr, indices, scale)
+    for i, h in itertools.product(range(Nq), range(Hq)):
+        g = h // (Hq // Hkv)
+        p = q_pos[i]
+        want = _dense_attention_torch(Q[i, h][None], K[g, :p + 1], V[g, :p + 1], scale)[0]
+        np.testing.assert_allclose(got[i, h], want, rtol=0, atol=1e-12)
+
+
+def test_paged_attention_only_reads_listed_blocks_and_is_causal():
+    # table {1}; query at position 70 sees keys 64..70 of block 1 only
+    rng = np.random.default_rng(16)
+    S, block, d = 256, 64, 8
+    Q = bf(rng.standard_normal((1, 1, d)))
+    K = bf(rng.standard_normal((1, S, d)))
+    V = bf(rng.standard_normal((1, S, d)))
+    got = oracle.paged_prefill_attn(Q, [70], K, V, block, [0, 1], [1], 0.5)
+    want = _dense_attention_torch(Q[0, 0][None], K[0, 64:71], V[0, 64:71], 0.5)[0]
+    np.testing.assert_allclose(got[0, 0], want, rtol=0, atol=1e-12)
+    # a query before the listed block sees nothing -> zero output
+    assert np.all(oracle.paged_prefill_attn(Q, [10], K, V, block, [0, 1], [1], 0.5) == 0)
+
+
+# ----------------------------------------------------------------------------
+# the synthetic workloads: planted needles are found
+# ----------------------------------------------------------------------------
+def test_c1_needles_are_selected():
+    cfg = synth.workload("c1")
+    g = 0
+    s = oracle.index_score(cfg.qI(g), cfg.w(g), cfg.KI_full(g), cfg.seq_off, [0], [cfg.S_max - 1])
+    idx = oracle.topk(s, cfg.seq_lens, cfg.k)[0]
+    needles = [t for (b, t, _, kr) in cfg.planted(g) if kr is not None]
+    assert len(needles) == 8
+    kth = np.sort(s[0])[::-1][cfg.k - 1]
+    for t in needles:
+        assert s[0, t] > kth and t in set(idx.tolist())
