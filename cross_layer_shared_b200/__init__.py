@@ -1,0 +1,245 @@
+"""Cross-layer shared sparse attention on B200 (sm_100a).
+
+Thin Python binding of libsa (include/sa.h): argument marshalling only.
+Every step of the path runs in the CUDA kernels of ``csrc/``; PyTorch
+provides device memory and streams.  There is no CPU fallback: if the
+library is not built, every call raises.
+
+Build:  python -m cross_layer_shared_b200.build
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsa.so")
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, SA_ERR_TIMEOUT, SA_ERR_DEVICE = range(7)
+SA_BF16, SA_F32 = 0, 1
+WS_HEADER_BYTES = 256
+
+# every symbol include/sa.h declares, with its ctypes signature
+_P, _I, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+_PP = ctypes.POINTER(ctypes.c_void_p)
+SIGNATURES = {
+    "sa_status_string": ([_I], ctypes.c_char_p),
+    "sa_last_error": ([], ctypes.c_char_p),
+    "sa_abi_version": ([], _I),
+    "sa_read_device_status": ([_P, _P, ctypes.POINTER(_I), ctypes.POINTER(_I64)], _I),
+    "sa_clear_device_status": ([_P, _P], _I),
+    "sa_index_score_workspace_size": ([_I], _SZ),
+    "sa_index_score": ([_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _P, _I64, _P, _SZ, _P], _I),
+    "sa_index_score_prefill_workspace_size": ([_I], _SZ),
+    "sa_index_score_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P, _SZ, _P], _I),
+    "sa_topk_workspace_size": ([_I, _I, _I], _SZ),
+    "sa_topk": ([_P, _I64, _P, _I, _I, _I, _P, _P, _P, _SZ, _P], _I),
+    "sa_sparse_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
+    "sa_sparse_decode_attn": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _SZ, _P], _I),
+    "sa_decode_step_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
+    "sa_decode_step": ([ctypes.c_char_p, _I, _PP, _PP, _PP, _PP, _PP, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _I,
+                        _I, _I, _F, _P, _I, _P, _P, _I64, _P, _SZ, _P], _I),
+    "sa_block_union_prefill_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
+    "sa_block_union_prefill": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
+                               _I),
+}
+
+
+class SAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{_STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+_STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_WORKSPACE",
+                 4: "SA_ERR_CUDA", 5: "SA_ERR_TIMEOUT", 6: "SA_ERR_DEVICE"}
+
+_lib = None
+
+
+def lib():
+    """The loaded libsa.  Raises if the CUDA library has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m cross_layer_shared_b200.build`"
+                               " (there is no fallback path)")
+        lb = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(lb, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lb
+    return _lib
+
+
+def _check(code: int) -> None:
+    if code != SA_OK:
+        raise SAError(code, lib().sa_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor of {dtype}")
+    return t
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zeroed workspace (status block included) of at least nbytes."""
+    n = max(int(nbytes), WS_HEADER_BYTES)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def read_status(ws: torch.Tensor, stream=None):
+    """(code, [kernel, element, value, bound]) of the device status block (synchronises)."""
+    code = ctypes.c_int(0)
+    det = (ctypes.c_int64 * 4)()
+    _check(lib().sa_read_device_status(_ptr(ws), _stream(stream), ctypes.byref(code), det))
+    return code.value, list(det)
+
+
+def clear_status(ws: torch.Tensor, stream=None) -> None:
+    _check(lib().sa_clear_device_status(_ptr(ws), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+def index_score(qI, w, KI, seq_off, seq_len, S_max: int, scores=None, ld: Optional[int] = None, ws=None,
+                stream=None) -> torch.Tensor:
+    B, H_I, d_I = qI.shape
+    _dev(qI, torch.bfloat16, "qI"), _dev(w, torch.float32, "w"), _dev(KI, torch.bfloat16, "KI")
+    _dev(seq_off, torch.int64, "seq_off"), _dev(seq_len, torch.int32, "seq_len")
+    ld = int(ld if ld is not None else max(S_max, 1))
+    if scores is None:
+        scores = torch.empty((B, ld), dtype=torch.float32, device=qI.device)
+    if ws is None:
+        ws = workspace(lib().sa_index_score_workspace_size(B), qI.device)
+    _check(lib().sa_index_score(_ptr(qI), _ptr(w), _ptr(KI), _ptr(seq_off), _ptr(seq_len), B, KI.shape[0], S_max,
+                                H_I, d_I, _ptr(scores), ld, _ptr(ws), ws.numel(), _stream(stream)))
+    return scores
+
+
+def index_score_prefill(qI, w, KI, q_pos, max_pos: int, scores=None, ld: Optional[int] = None, ws=None,
+                        stream=None) -> torch.Tensor:
+    Nq, H_I, d_I = qI.shape
+    _dev(qI, torch.bfloat16, "qI"), _dev(w, torch.float32, "w"), _dev(KI, torch.bfloat16, "KI")
+    _dev(q_pos, torch.int32, "q_pos")
+    ld = int(ld if ld is not None else max_pos + 1)
+    if scores is None:
+        scores = torch.empty((Nq, ld), dtype=torch.float32, device=qI.device)
+    if ws is None:
+        ws = workspace(lib().sa_index_score_prefill_workspace_size(Nq), qI.device)
+    _check(lib().sa_index_score_prefill(_ptr(qI), _ptr(w), _ptr(KI), _ptr(q_pos), Nq, KI.shape[0], max_pos, H_I,
+                                        d_I, _ptr(scores), ld, _ptr(ws), ws.numel(), _stream(stream)))
+    return scores
+
+
+def topk(scores, n_valid, n_max: int, k: int, idx=None, top_scores=None, want_scores=False, ws=None, stream=None):
+    Nq, ld = scores.shape
+    _dev(scores, torch.float32, "scores"), _dev(n_valid, torch.int32, "n_valid")
+    if idx is None:
+        idx = torch.empty((Nq, k), dtype=torch.int32, device=scores.device)
+    if want_scores and top_scores is None:
+        top_scores = torch.empty((Nq, k), dtype=torch.float32, device=scores.device)
+    if ws is None:
+        ws = workspace(lib().sa_topk_workspace_size(Nq, n_max, k), scores.device)
+    _check(lib().sa_topk(_ptr(scores), ld, _ptr(n_valid), Nq, n_max, k, _ptr(idx), _ptr(top_scores), _ptr(ws),
+                         ws.numel(), _stream(stream)))
+    return (idx, top_scores) if want_scores else idx
+
+
+def sparse_decode_attn_workspace_size(L_g, B, Hq, Hkv, d, k) -> int:
+    return int(lib().sa_sparse_decode_attn_workspace_size(L_g, B, Hq, Hkv, d, k))
+
+
+def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, out_dtype=torch.bfloat16, O=None,
+                       ws=None, stream=None) -> torch.Tensor:
+    L, B, Hq, d = Q.shape
+    k = idx.shape[1]
+    _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
+    _dev(idx, torch.int32, "idx")
+    if O is None:
+        O = torch.empty((L, B, Hq, d), dtype=out_dtype, device=Q.device)
+    if ws is None:
+        ws = workspace(sparse_decode_attn_workspace_size(L, B, Hq, Hkv, d, k), Q.device)
+    code = SA_F32 if O.dtype == torch.float32 else SA_BF16
+    _check(lib().sa_sparse_decode_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), _ptr(idx), L, B, Hq,
+                                       Hkv, d, k, float(scale), _ptr(O), code, _ptr(ws), ws.numel(),
+                                       _stream(stream)))
+    return O
+
+
+def decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k) -> int:
+    return int(lib().sa_decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k))
+
+
+def _ptr_array(ts: Sequence[Optional[torch.Tensor]]):
+    arr = (ctypes.c_void_p * len(ts))(*[None if t is None else t.data_ptr() for t in ts])
+    return ctypes.cast(arr, _PP), arr
+
+
+def decode_step(pattern: str, qI: Sequence, w: Sequence, KI: Sequence, K: Sequence, V: Sequence, seq_off, seq_len,
+                S_max: int, k: int, Q, Hkv: int, scale: float, out_dtype=torch.bfloat16, O=None, idx=None,
+                scores=None, ws=None, stream=None):
+    """One decode step over `pattern` (per-layer lists; entries of S layers'
+    indexer inputs may be None).  Returns (O, idx of the last F layer)."""
+    L, B, Hq, d = Q.shape
+    n = len(pattern)
+    assert L == n and len(K) == n and len(V) == n
+    f0 = next(t for t in qI if t is not None)
+    H_I, d_I = f0.shape[1], f0.shape[2]
+    n_tokens = next(t for t in KI if t is not None).shape[0]
+    if O is None:
+        O = torch.empty((L, B, Hq, d), dtype=out_dtype, device=Q.device)
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=Q.device)
+    if scores is None:
+        scores = torch.empty((B, max(S_max, 1)), dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws = workspace(decode_step_workspace_size(n, B, S_max, Hq, Hkv, d, k), Q.device)
+    keep = []
+    arrays = []
+    for lst in (qI, w, KI, K, V):
+        p, a = _ptr_array(lst)
+        arrays.append(p)
+        keep.append(a)
+    code = SA_F32 if O.dtype == torch.float32 else SA_BF16
+    _check(lib().sa_decode_step(pattern.encode(), n, *arrays, _ptr(seq_off), _ptr(seq_len), B, n_tokens, S_max, H_I,
+                                d_I, k, _ptr(Q), Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(idx), _ptr(scores),
+                                scores.shape[1], _ptr(ws), ws.numel(), _stream(stream)))
+    return O, idx
+
+
+def block_union_prefill(idx, q_pos, Q, K, V, block: int, scale: float, out_dtype=torch.bfloat16, O=None,
+                        kv_indptr=None, kv_indices=None, ws=None, stream=None):
+    """Returns (kv_indptr [Hkv+1], kv_indices [Hkv*ceil(S/block)], O [Nq,Hq,d])."""
+    Nq, Hq, d = Q.shape
+    Hkv, S, _ = K.shape
+    k = idx.shape[1]
+    _dev(idx, torch.int32, "idx"), _dev(q_pos, torch.int32, "q_pos")
+    _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
+    nb = (S + block - 1) // block
+    if kv_indptr is None:
+        kv_indptr = torch.empty(Hkv + 1, dtype=torch.int32, device=Q.device)
+    if kv_indices is None:
+        kv_indices = torch.empty(Hkv * nb, dtype=torch.int32, device=Q.device)
+    if O is None:
+        O = torch.empty((Nq, Hq, d), dtype=out_dtype, device=Q.device)
+    if ws is None:
+        ws = workspace(lib().sa_block_union_prefill_workspace_size(S, Nq, Hq, Hkv, d, k, block), Q.device)
+    code = SA_F32 if O.dtype == torch.float32 else SA_BF16
+    _check(lib().sa_block_union_prefill(_ptr(idx), _ptr(q_pos), _ptr(Q), _ptr(K), _ptr(V), S, Nq, Hq, Hkv, d, k,
+                                        block, float(scale), _ptr(kv_indptr), _ptr(kv_indices), _ptr(O), code,
+                                        _ptr(ws), ws.numel(), _stream(stream)))
+    return kv_indptr, kv_indices, O

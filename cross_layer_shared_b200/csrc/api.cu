@@ -1,0 +1,488 @@
+// C ABI of libsa (declared in include/sa.h): host-side argument checks,
+// tensor-map encoding, workspace carving and kernel launches.  Every check
+// runs before anything is enqueued; nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/sa.h"
+#include "attn.cuh"
+#include "sm100.cuh"
+#include "indexer.cuh"
+#include "status.cuh"
+#include "topk.cuh"
+#include "union.cuh"
+
+namespace sa {
+
+namespace {
+std::mutex g_attr_mu;
+struct AttrEntry {
+  int dev;
+  const void* fn;
+};
+AttrEntry g_attr[256];
+int g_attr_n = 0;
+}  // namespace
+
+bool smem_attr_done(int dev, const void* fn) {
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  for (int i = 0; i < g_attr_n; ++i)
+    if (g_attr[i].dev == dev && g_attr[i].fn == fn) return true;
+  return false;
+}
+
+void smem_attr_mark(int dev, const void* fn) {
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (g_attr_n < 256) g_attr[g_attr_n++] = {dev, fn};
+}
+
+}  // namespace sa
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sa_status fail(sa_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+sa_status cuda_fail(const char* where, cudaError_t e) {
+  return fail(SA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cache[64] = {0};
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims innermost first (elements),
+// strides in bytes for dims 1.. ; box in elements.
+sa_status make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                    const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  uint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SA_ERR_INVALID_ARG, "tensor map encoding failed (CUresult %d)", (int)r);
+  return SA_OK;
+}
+
+sa::DeviceStatus* status_of(void* ws) { return reinterpret_cast<sa::DeviceStatus*>(ws); }
+
+sa_status check_ws(void* ws, size_t ws_bytes, size_t need, const char* who) {
+  if (ws == nullptr) return fail(SA_ERR_WORKSPACE, "%s: workspace is NULL", who);
+  if (!aligned(ws, 256)) return fail(SA_ERR_WORKSPACE, "%s: workspace must be 256-byte aligned", who);
+  if (ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "%s: workspace of %zu bytes is below the %zu required", who, ws_bytes, need);
+  return SA_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int index_npad(int H_I) { return (H_I + 15) / 16 * 16; }
+
+// ---- sparse attention split choice -----------------------------------------
+struct AttnPlan {
+  int n_mtiles, n_split, keys_per_split, units;
+};
+
+AttnPlan plan_decode_attn(int L_g, int B, int Hq, int Hkv, int k) {
+  AttnPlan p;
+  const int R = L_g * (Hq / Hkv);
+  p.n_mtiles = (R + 127) / 128;
+  const int base = B * Hkv * p.n_mtiles;
+  const int max_split = (k + 127) / 128;
+  int s = num_sms() / (base > 0 ? base : 1);
+  if (s < 1) s = 1;
+  if (s > max_split) s = max_split;
+  p.keys_per_split = (int)round_up((size_t)((k + s - 1) / s), 128);
+  if (p.keys_per_split < 128) p.keys_per_split = 128;
+  p.n_split = (k + p.keys_per_split - 1) / p.keys_per_split;
+  if (p.n_split < 1) p.n_split = 1;
+  p.units = base * p.n_split;
+  return p;
+}
+
+size_t attn_ws_bytes(const AttnPlan& p) {
+  return SA_WS_HEADER_BYTES + (p.n_split > 1 ? round_up(sa::attn_partial_bytes(p.units), 256) : 0);
+}
+
+sa_status validate_index(const void* qI, const float* w, const void* KI, int H_I, int d_I, const char* who) {
+  if (!qI || !w || !KI) return fail(SA_ERR_INVALID_ARG, "%s: NULL tensor pointer", who);
+  if (H_I < 1 || H_I > 64) return fail(SA_ERR_UNSUPPORTED, "%s: H_I=%d outside [1, 64]", who, H_I);
+  if (d_I != 64 && d_I != 128 && d_I != 192 && d_I != 256)
+    return fail(SA_ERR_UNSUPPORTED, "%s: d_I=%d not in {64, 128, 192, 256}", who, d_I);
+  if (!aligned(qI, 16) || !aligned(KI, 16)) return fail(SA_ERR_INVALID_ARG, "%s: qI and KI must be 16-byte aligned", who);
+  if (!aligned(w, 4)) return fail(SA_ERR_INVALID_ARG, "%s: w must be 4-byte aligned", who);
+  return SA_OK;
+}
+
+sa_status run_index_decode(const void* qI, const float* w, const void* KI, const int64_t* seq_off,
+                           const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I,
+                           float* scores, int64_t ld, void* ws, cudaStream_t stream) {
+  CUtensorMap tm_ki, tm_qi;
+  {
+    const uint64_t dims[2] = {(uint64_t)d_I, (uint64_t)n_tokens};
+    const uint64_t str[1] = {(uint64_t)d_I * 2};
+    const uint32_t box[2] = {64, 128};
+    sa_status st = make_tmap(&tm_ki, KI, 2, dims, str, box);
+    if (st != SA_OK) return st;
+  }
+  const int npad = index_npad(H_I);
+  {
+    const uint64_t dims[3] = {(uint64_t)d_I, (uint64_t)H_I, (uint64_t)B};
+    const uint64_t str[2] = {(uint64_t)d_I * 2, (uint64_t)H_I * d_I * 2};
+    const uint32_t box[3] = {64, (uint32_t)npad, 1};
+    sa_status st = make_tmap(&tm_qi, qI, 3, dims, str, box);
+    if (st != SA_OK) return st;
+  }
+  sa::IndexerArgs a{w, seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, status_of(ws)};
+  cudaError_t e = sa::launch_indexer_decode(a, tm_ki, tm_qi, npad, num_sms(), stream);
+  if (e != cudaSuccess) return cuda_fail("sa_index_score launch", e);
+  return SA_OK;
+}
+
+__global__ void prefill_rows_kernel(const int32_t* __restrict__ q_pos, int Nq, int max_pos, int64_t* seq_off,
+                                    int32_t* seq_len, sa::DeviceStatus* status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i <= Nq) seq_off[i] = 0;
+  if (i < Nq) {
+    int p = q_pos[i];
+    if (p < 0 || p > max_pos) {
+      sa::report(status, sa::kErrDevice, sa::kKernIndexerPrefill, i, p, max_pos);
+      p = -1;  // row skipped
+    }
+    seq_len[i] = p + 1;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
+    case SA_ERR_DEVICE: return "SA_ERR_DEVICE";
+    default: return "SA_ERR_UNKNOWN";
+  }
+}
+
+const char* sa_last_error(void) { return g_last_error.c_str(); }
+
+int sa_abi_version(void) { return 1; }
+
+sa_status sa_read_device_status(const void* ws, void* stream, int* device_status, int64_t* detail) {
+  if (!ws || !device_status) return fail(SA_ERR_INVALID_ARG, "sa_read_device_status: NULL argument");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail("sa_read_device_status sync", e);
+  sa::DeviceStatus st;
+  e = cudaMemcpy(&st, ws, sizeof st, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail("sa_read_device_status copy", e);
+  *device_status = st.code;
+  if (detail)
+    for (int i = 0; i < 4; ++i) detail[i] = st.detail[i];
+  return SA_OK;
+}
+
+sa_status sa_clear_device_status(void* ws, void* stream) {
+  if (!ws) return fail(SA_ERR_INVALID_ARG, "sa_clear_device_status: NULL workspace");
+  cudaError_t e = cudaMemsetAsync(ws, 0, SA_WS_HEADER_BYTES, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail("sa_clear_device_status", e);
+  return SA_OK;
+}
+
+// ---------------------------------------------------------------- indexer
+size_t sa_index_score_workspace_size(int B) {
+  (void)B;
+  return SA_WS_HEADER_BYTES;
+}
+
+sa_status sa_index_score(const void* qI, const float* w, const void* KI, const int64_t* seq_off,
+                         const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I, float* scores,
+                         int64_t ld, void* ws, size_t ws_bytes, void* stream) {
+  const char* who = "sa_index_score";
+  if (B < 0 || B > 4096) return fail(SA_ERR_INVALID_ARG, "%s: B=%d outside [0, 4096]", who, B);
+  if (S_max < 0) return fail(SA_ERR_INVALID_ARG, "%s: S_max=%d < 0", who, S_max);
+  if (n_tokens < 1 || n_tokens >= (1ll << 31)) return fail(SA_ERR_INVALID_ARG, "%s: n_tokens=%lld outside [1, 2^31)", who, (long long)n_tokens);
+  if (ld < S_max) return fail(SA_ERR_INVALID_ARG, "%s: ld=%lld < S_max=%d", who, (long long)ld, S_max);
+  sa_status st = validate_index(qI, w, KI, H_I, d_I, who);
+  if (st != SA_OK) return st;
+  if (!seq_off || !seq_len || !scores) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if ((st = check_ws(ws, ws_bytes, sa_index_score_workspace_size(B), who)) != SA_OK) return st;
+  if (B == 0 || S_max == 0) return SA_OK;
+  return run_index_decode(qI, w, KI, seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, ws,
+                          (cudaStream_t)stream);
+}
+
+size_t sa_index_score_prefill_workspace_size(int Nq) {
+  return SA_WS_HEADER_BYTES + round_up(8 * ((size_t)Nq + 1), 256) + round_up(4 * (size_t)Nq, 256);
+}
+
+sa_status sa_index_score_prefill(const void* qI, const float* w, const void* KI, const int32_t* q_pos, int Nq, int S,
+                                 int max_pos, int H_I, int d_I, float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  const char* who = "sa_index_score_prefill";
+  if (Nq < 0 || Nq > 4096) return fail(SA_ERR_INVALID_ARG, "%s: Nq=%d outside [0, 4096]", who, Nq);
+  if (S < 1 || max_pos < 0 || max_pos >= S) return fail(SA_ERR_INVALID_ARG, "%s: need 0 <= max_pos < S", who);
+  if (ld < (int64_t)max_pos + 1) return fail(SA_ERR_INVALID_ARG, "%s: ld below max_pos + 1", who);
+  sa_status st = validate_index(qI, w, KI, H_I, d_I, who);
+  if (st != SA_OK) return st;
+  if (!q_pos || !scores) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if ((st = check_ws(ws, ws_bytes, sa_index_score_prefill_workspace_size(Nq), who)) != SA_OK) return st;
+  if (Nq == 0) return SA_OK;
+  uint8_t* p = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
+  int64_t* soff = reinterpret_cast<int64_t*>(p);
+  int32_t* slen = reinterpret_cast<int32_t*>(p + round_up(8 * ((size_t)Nq + 1), 256));
+  cudaStream_t s = (cudaStream_t)stream;
+  prefill_rows_kernel<<<(Nq + 256) / 256, 256, 0, s>>>(q_pos, Nq, max_pos, soff, slen, status_of(ws));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("sa_index_score_prefill rows", e);
+  // every query is a row of its own over the one cache: the decode kernel with
+  // seq_off = 0 and seq_len = q_pos + 1
+  return run_index_decode(qI, w, KI, soff, slen, Nq, S, max_pos + 1, H_I, d_I, scores, ld, ws, s);
+}
+
+// ---------------------------------------------------------------- top-k
+size_t sa_topk_workspace_size(int Nq, int n_max, int k) {
+  (void)Nq;
+  (void)n_max;
+  (void)k;
+  return SA_WS_HEADER_BYTES;
+}
+
+sa_status sa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max, int k, int32_t* idx,
+                  float* top_scores, void* ws, size_t ws_bytes, void* stream) {
+  const char* who = "sa_topk";
+  if (Nq < 0) return fail(SA_ERR_INVALID_ARG, "%s: Nq=%d < 0", who, Nq);
+  if (k < 1) return fail(SA_ERR_INVALID_ARG, "%s: k=%d < 1", who, k);
+  if (n_max < 0 || ld < n_max) return fail(SA_ERR_INVALID_ARG, "%s: need 0 <= n_max <= ld", who);
+  if (Nq > 0 && (!scores || !n_valid || !idx)) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  sa_status st = check_ws(ws, ws_bytes, sa_topk_workspace_size(Nq, n_max, k), who);
+  if (st != SA_OK) return st;
+  if (Nq == 0) return SA_OK;
+  cudaError_t e = sa::launch_topk_rows(scores, ld, n_valid, Nq, n_max, k, idx, top_scores, status_of(ws),
+                                       (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail("sa_topk launch", e);
+  return SA_OK;
+}
+
+// ---------------------------------------------------------------- attention
+size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int d, int k) {
+  (void)d;
+  if (L_g < 1 || B < 1 || Hkv < 1 || Hq < Hkv || k < 1) return SA_WS_HEADER_BYTES;
+  return attn_ws_bytes(plan_decode_attn(L_g, B, Hq, Hkv, k));
+}
+
+static sa_status run_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
+                                 const int32_t* seq_len, const int32_t* idx, int L_g, int B, int Hq, int Hkv, int d,
+                                 int k, float scale, void* O, sa_dtype out_dtype, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream) {
+  const char* who = "sa_sparse_decode_attn";
+  if (L_g < 1 || B < 1 || Hq < 1 || Hkv < 1 || k < 1)
+    return fail(SA_ERR_INVALID_ARG, "%s: L_g, B, Hq, Hkv, k must be >= 1", who);
+  if (d != 128) return fail(SA_ERR_UNSUPPORTED, "%s: d=%d (only 128 is built)", who, d);
+  if (Hq % Hkv != 0) return fail(SA_ERR_INVALID_ARG, "%s: Hq=%d not a multiple of Hkv=%d", who, Hq, Hkv);
+  if (out_dtype != SA_BF16 && out_dtype != SA_F32) return fail(SA_ERR_INVALID_ARG, "%s: bad out_dtype", who);
+  if (!Q || !K || !V || !seq_off || !seq_len || !idx || !O) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
+    return fail(SA_ERR_INVALID_ARG, "%s: Q, K, V, O must be 16-byte aligned", who);
+  if (!(scale > 0.f)) return fail(SA_ERR_INVALID_ARG, "%s: scale must be > 0", who);
+  const AttnPlan p = plan_decode_attn(L_g, B, Hq, Hkv, k);
+  sa_status st = check_ws(ws, ws_bytes, attn_ws_bytes(p), who);
+  if (st != SA_OK) return st;
+  sa::AttnArgs a{};
+  a.Q = reinterpret_cast<const uint16_t*>(Q);
+  a.K = reinterpret_cast<const uint16_t*>(K);
+  a.V = reinterpret_cast<const uint16_t*>(V);
+  a.seq_off = seq_off;
+  a.seq_len = seq_len;
+  a.idx = idx;
+  a.k = k;
+  a.prefill = 0;
+  a.L = L_g;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.R = L_g * a.G;
+  a.n_mtiles = p.n_mtiles;
+  a.n_split = p.n_split;
+  a.keys_per_split = p.keys_per_split;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = O;
+  a.out_f32 = out_dtype == SA_F32;
+  a.part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES);
+  a.status = status_of(ws);
+  cudaError_t e = sa::launch_sparse_attn(a, out_dtype == SA_F32, stream);
+  if (e != cudaSuccess) return cuda_fail("sa_sparse_decode_attn launch", e);
+  return SA_OK;
+}
+
+sa_status sa_sparse_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
+                                const int32_t* seq_len, const int32_t* idx, int L_g, int B, int Hq, int Hkv, int d,
+                                int k, float scale, void* O, sa_dtype out_dtype, void* ws, size_t ws_bytes,
+                                void* stream) {
+  return run_decode_attn(Q, K, V, seq_off, seq_len, idx, L_g, B, Hq, Hkv, d, k, scale, O, out_dtype, ws, ws_bytes,
+                         (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------- decode step
+size_t sa_decode_step_workspace_size(int n_layers, int B, int S_max, int Hq, int Hkv, int d, int k) {
+  size_t need = SA_WS_HEADER_BYTES;
+  // the largest fused group is the whole pattern
+  for (int L = 1; L <= n_layers; ++L) {
+    const size_t a = sa_sparse_decode_attn_workspace_size(L, B, Hq, Hkv, d, k);
+    if (a > need) need = a;
+  }
+  const size_t t = sa_topk_workspace_size(B, S_max, k);
+  return t > need ? t : need;
+}
+
+sa_status sa_decode_step(const char* pattern, int n_layers, const void* const* qI, const float* const* w,
+                         const void* const* KI, const void* const* K, const void* const* V, const int64_t* seq_off,
+                         const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I, int k,
+                         const void* Q, int Hq, int Hkv, int d, float scale, void* O, sa_dtype out_dtype, int32_t* idx,
+                         float* scores, int64_t ld, void* ws, size_t ws_bytes, void* stream) {
+  const char* who = "sa_decode_step";
+  if (!pattern || n_layers < 1) return fail(SA_ERR_INVALID_ARG, "%s: empty layer pattern", who);
+  if ((int)strnlen(pattern, (size_t)n_layers + 1) < n_layers)
+    return fail(SA_ERR_INVALID_ARG, "%s: pattern shorter than n_layers", who);
+  if (pattern[0] != 'F')
+    return fail(SA_ERR_INVALID_ARG, "%s: the first layer must be F (an S layer reuses an upstream F index)", who);
+  for (int l = 0; l < n_layers; ++l)
+    if (pattern[l] != 'F' && pattern[l] != 'S') return fail(SA_ERR_INVALID_ARG, "%s: pattern letters are F or S", who);
+  if (!qI || !w || !KI || !K || !V) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer array", who);
+  if (B < 1 || !Q || !O || !idx || !scores) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer or B < 1", who);
+  sa_status st = check_ws(ws, ws_bytes, sa_decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k), who);
+  if (st != SA_OK) return st;
+  const size_t esize = out_dtype == SA_F32 ? 4 : 2;
+  const size_t layer_elems = (size_t)B * Hq * d;
+  int l = 0;
+  while (l < n_layers) {
+    if (pattern[l] == 'F') {
+      st = sa_index_score(qI[l], w[l], KI[l], seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, ws,
+                          ws_bytes, stream);
+      if (st != SA_OK) return st;
+      st = sa_topk(scores, ld, seq_len, B, S_max, k, idx, nullptr, ws, ws_bytes, stream);
+      if (st != SA_OK) return st;
+    }
+    // fuse the following S layers that read the same cache into one group call
+    int m = l;
+    while (m + 1 < n_layers && pattern[m + 1] == 'S' && K[m + 1] == K[l] && V[m + 1] == V[l]) ++m;
+    st = run_decode_attn(reinterpret_cast<const uint8_t*>(Q) + (size_t)l * layer_elems * 2, K[l], V[l], seq_off,
+                         seq_len, idx, m - l + 1, B, Hq, Hkv, d, k, scale,
+                         reinterpret_cast<uint8_t*>(O) + (size_t)l * layer_elems * esize, out_dtype, ws, ws_bytes,
+                         (cudaStream_t)stream);
+    if (st != SA_OK) return st;
+    l = m + 1;
+  }
+  return SA_OK;
+}
+
+// ---------------------------------------------------------------- prefill union
+size_t sa_block_union_prefill_workspace_size(int S, int Nq, int Hq, int Hkv, int d, int k, int block) {
+  (void)Nq;
+  (void)Hq;
+  (void)Hkv;
+  (void)d;
+  (void)k;
+  if (S < 1 || block < 1) return SA_WS_HEADER_BYTES;
+  return SA_WS_HEADER_BYTES + round_up((size_t)(S + block - 1) / block, 256);
+}
+
+sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const void* Q, const void* K, const void* V,
+                                 int S, int Nq, int Hq, int Hkv, int d, int k, int block, float scale,
+                                 int32_t* kv_indptr, int32_t* kv_indices, void* O, sa_dtype out_dtype, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  const char* who = "sa_block_union_prefill";
+  if (S < 1 || Nq < 1 || Hq < 1 || Hkv < 1 || k < 1) return fail(SA_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+  if (d != 128) return fail(SA_ERR_UNSUPPORTED, "%s: d=%d (only 128 is built)", who, d);
+  if (block != 64) return fail(SA_ERR_UNSUPPORTED, "%s: block=%d (only 64 is built)", who, block);
+  if (Hq % Hkv != 0) return fail(SA_ERR_INVALID_ARG, "%s: Hq not a multiple of Hkv", who);
+  if ((int64_t)Nq * (Hq / Hkv) > (1 << 30)) return fail(SA_ERR_INVALID_ARG, "%s: too many query rows", who);
+  if (out_dtype != SA_BF16 && out_dtype != SA_F32) return fail(SA_ERR_INVALID_ARG, "%s: bad out_dtype", who);
+  if (!idx || !q_pos || !Q || !K || !V || !kv_indptr || !kv_indices || !O)
+    return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
+    return fail(SA_ERR_INVALID_ARG, "%s: Q, K, V, O must be 16-byte aligned", who);
+  if (!(scale > 0.f)) return fail(SA_ERR_INVALID_ARG, "%s: scale must be > 0", who);
+  sa_status st = check_ws(ws, ws_bytes, sa_block_union_prefill_workspace_size(S, Nq, Hq, Hkv, d, k, block), who);
+  if (st != SA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* mark = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
+  cudaError_t e = sa::launch_block_union(idx, Nq, k, S, block, Hkv, mark, kv_indptr, kv_indices, status_of(ws), s);
+  if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill union", e);
+  sa::AttnArgs a{};
+  a.Q = reinterpret_cast<const uint16_t*>(Q);
+  a.K = reinterpret_cast<const uint16_t*>(K);
+  a.V = reinterpret_cast<const uint16_t*>(V);
+  a.prefill = 1;
+  a.q_pos = q_pos;
+  a.kv_indptr = kv_indptr;
+  a.kv_indices = kv_indices;
+  a.S = S;
+  a.block = block;
+  a.Nq = Nq;
+  a.L = 1;
+  a.B = 1;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.R = Nq * a.G;
+  a.n_mtiles = (a.R + 127) / 128;
+  a.n_split = 1;
+  a.keys_per_split = (int)round_up((size_t)((S + block - 1) / block) * block, 128);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = O;
+  a.out_f32 = out_dtype == SA_F32;
+  a.part = nullptr;
+  a.status = status_of(ws);
+  e = sa::launch_sparse_attn(a, out_dtype == SA_F32, s);
+  if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill attention", e);
+  return SA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Launch interface of the sparse attention kernels (internal to libsa).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "status.cuh"
+
+namespace sa {
+
+struct AttnArgs {
+  const uint16_t* Q;
+  const uint16_t* K;
+  const uint16_t* V;
+  // decode: keys of (b, g) are idx[b, 0:k]; the cache of sequence b starts at
+  // seq_off[b]*Hkv*d and is laid out [Hkv, seq_len[b], d]
+  const int64_t* seq_off;
+  const int32_t* seq_len;
+  const int32_t* idx;
+  int k;
+  // prefill (prefill != 0): keys of group g are the blocks
+  // kv_indices[kv_indptr[g] : kv_indptr[g+1]] of `block` tokens; cache [Hkv, S, d];
+  // query p sees keys t <= q_pos[p]
+  int prefill;
+  const int32_t* q_pos;
+  const int32_t* kv_indptr;
+  const int32_t* kv_indices;
+  int S;
+  int block;
+  int Nq;
+
+  int L;  // decode: layers in the group
+  int B;
+  int Hq;
+  int Hkv;
+  int G;       // Hq / Hkv
+  int R;       // query rows per (b, g): L*G (decode) or Nq*G (prefill)
+  int n_mtiles;
+  int n_split;
+  int keys_per_split;  // multiple of 128
+  float scale_log2;    // softmax scale * log2(e)
+  void* O;
+  int out_f32;
+  float* part;  // [units][128][d + 2] partial (O, m, l) when n_split > 1
+  DeviceStatus* status;
+};
+
+int attn_num_units(const AttnArgs& a);
+size_t attn_partial_bytes(int units);
+cudaError_t launch_sparse_attn(const AttnArgs& a, bool precise_p, cudaStream_t stream);
+
+}  // namespace sa

@@ -1,0 +1,261 @@
+// Lightning-indexer score on tcgen05 tensor cores.
+//
+// Definition [IndexCache: Accelerating Sparse Attention via Cross-Layer
+// Index Reuse, technical summary section 1: the indexer scores every
+// previous token for the current query; CLSA news article, "Comment CLSA
+// fonctionne": the shared indexer layer computes the scores once]:
+//   score[b,t] = sum_j w[b,j] * max(0, qI[b,j,:] . KI[seq_off[b]+t, :])
+//
+// Decode form.  The step is HBM-bound: every visible key row (d_I bf16) is
+// read once, and each row feeds H_I dot products of length d_I (16 flop per
+// byte at H_I=16), above what the fp32 FMA pipes sustain at HBM rate, so the
+// contraction runs on the tensor cores:
+//   A = 128 key rows x d_I   (TMA, 128-byte swizzle, K-major)
+//   B = H_I (padded to N) query heads x d_I (TMA, same layout)
+//   D = 128 x N fp32 in TMEM; the epilogue warps read one token per thread,
+//       apply ReLU, weight, sum over heads and store one fp32 score.
+// Persistent CTAs (one per SM) walk the ragged list of (sequence, 128-token
+// tile) pairs; warp 0 issues TMA into a STAGES-deep ring, warp 1 issues the
+// MMAs into ACC TMEM accumulators, warps 2-5 run the epilogue.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "indexer.cuh"
+#include "sm100.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kAcc = 4;
+constexpr int kThreads = 192;
+constexpr int kRingBudget = 196608;  // bytes of shared memory for the TMA ring
+
+template <int NHALF, int NPAD>
+struct IdxLayout {
+  static constexpr int kABytes = NHALF * kTile * 128;
+  static constexpr int kBBytes = NHALF * NPAD * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (kRingBudget / kStageBytes) > 5 ? 5 : (kRingBudget / kStageBytes);
+  static constexpr int kTmemCols = (kAcc * NPAD <= 32) ? 32 : (kAcc * NPAD <= 64) ? 64 : (kAcc * NPAD <= 128) ? 128 : 256;
+  // ring | full[kStages] empty[kStages] tfull[kAcc] tempty[kAcc] | tmem slot | prefix[B+1]
+  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kTmemSlotOffset = kBarOffset + 8 * (2 * kStages + 2 * kAcc);
+  static constexpr int kPrefixOffset = kTmemSlotOffset + 16;
+  static size_t smem_bytes(int B) { return 1024 + kPrefixOffset + 4 * (size_t)(B + 1); }
+};
+
+__device__ __forceinline__ int locate_tile(const int* prefix, int B, int g) {
+  // largest b with prefix[b] <= g (prefix[0] = 0, prefix[B] = total)
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int NHALF, int NPAD>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_constant__ CUtensorMap tm_qi,
+                      const float* __restrict__ w, const int64_t* __restrict__ seq_off,
+                      const int32_t* __restrict__ seq_len, int B, int64_t n_tokens, int S_max, int H_I,
+                      float* __restrict__ scores, int64_t ld, DeviceStatus* __restrict__ status) {
+  using Lay = IdxLayout<NHALF, NPAD>;
+  constexpr int kStages = Lay::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kBarOffset);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + kAcc;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kTmemSlotOffset);
+  int* prefix = reinterpret_cast<int*>(smem + Lay::kPrefixOffset);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- set-up: tile prefix over sequences, barriers, TMEM ---------------
+  if (warp == 0) {
+    // prefix[b] = sum of ceil(len/128) over earlier sequences (warp scan in chunks)
+    int carry = 0;
+    for (int base = 0; base < B; base += 32) {
+      const int b = base + lane;
+      int n = 0;
+      if (b < B) {
+        int len = seq_len[b];
+        if (len > S_max || len < 0) {
+          report(status, kErrDevice, kKernIndexer, b, len, S_max);
+          len = len < 0 ? 0 : S_max;
+        }
+        n = (len + kTile - 1) / kTile;
+      }
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (b < B) prefix[b] = carry + incl - n;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) prefix[B] = carry;
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+      for (int a = 0; a < kAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+      fence_mbar_init();
+      tma_prefetch_desc(&tm_ki);
+      tma_prefetch_desc(&tm_qi);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, Lay::kTmemCols);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = prefix[B];
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int i = 0;
+      for (int g = blockIdx.x; g < total; g += gridDim.x, ++i) {
+        const int s = i % kStages;
+        if (!mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, kWaitLimitNs)) {
+          report(status, kErrTimeout, kKernIndexer, blockIdx.x, 0, i);
+          break;
+        }
+        const int b = locate_tile(prefix, B, g);
+        const int tl = g - prefix[b];
+        const int64_t row = seq_off[b] + (int64_t)tl * kTile;
+        uint8_t* st = smem + s * Lay::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], Lay::kStageBytes);
+#pragma unroll
+        for (int h = 0; h < NHALF; ++h) tma_load_2d(st + h * kTile * 128, &tm_ki, &full[s], h * 64, (int)row);
+#pragma unroll
+        for (int h = 0; h < NHALF; ++h)
+          tma_load_3d(st + Lay::kABytes + h * NPAD * 128, &tm_qi, &full[s], h * 64, 0, b);
+      }
+      // drain: every load issued by this thread has landed before the CTA exits
+      const int issued = i;
+      for (int j = issued - kStages; j < issued; ++j)
+        if (j >= 0) mbar_wait(&full[j % kStages], (j / kStages) & 1, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(128, NPAD, false, false);
+      int i = 0;
+      for (int g = blockIdx.x; g < total; g += gridDim.x, ++i) {
+        const int s = i % kStages;
+        const int a = i % kAcc;
+        if (!mbar_wait(&full[s], (i / kStages) & 1, kWaitLimitNs) ||
+            !mbar_wait(&tempty[a], ((i / kAcc) & 1) ^ 1, kWaitLimitNs)) {
+          report(status, kErrTimeout, kKernIndexer, blockIdx.x, 1, i);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + s * Lay::kStageBytes);
+        const uint32_t b_base = a_base + Lay::kABytes;
+        const uint32_t d = tmem_base + a * NPAD;
+#pragma unroll
+        for (int h = 0; h < NHALF; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = umma_desc_sw128(a_base + h * kTile * 128 + kk * 32, 16, 1024);
+            const uint64_t bd = umma_desc_sw128(b_base + h * NPAD * 128 + kk * 32, 16, 1024);
+            umma_bf16(d, ad, bd, idesc, (h | kk) != 0);
+          }
+        }
+        umma_commit(&empty[s]);
+        umma_commit(&tfull[a]);
+      }
+    }
+  } else {
+    // ---------------- epilogue: ReLU, head weights, sum ----------------
+    const int quarter = warp & 3;  // TMEM lanes this warp may read
+    const int r = quarter * 32 + lane;
+    int i = 0;
+    int cur_b = -1;
+    float wr[NPAD];
+#pragma unroll
+    for (int j = 0; j < NPAD; ++j) wr[j] = 0.f;
+    for (int g = blockIdx.x; g < total; g += gridDim.x, ++i) {
+      const int a = i % kAcc;
+      if (!mbar_wait(&tfull[a], (i / kAcc) & 1, kWaitLimitNs)) {
+        report(status, kErrTimeout, kKernIndexer, blockIdx.x, 2, i);
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[NPAD];
+#pragma unroll
+      for (int c = 0; c < NPAD; c += 16)
+        tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + a * NPAD + c, &v[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[a]);
+
+      const int b = locate_tile(prefix, B, g);
+      if (b != cur_b) {
+        cur_b = b;
+#pragma unroll
+        for (int j = 0; j < NPAD; ++j) wr[j] = (j < H_I) ? __ldg(&w[(int64_t)b * H_I + j]) : 0.f;
+      }
+      int len = seq_len[b];
+      len = len < 0 ? 0 : (len > S_max ? S_max : len);
+      const int t = (g - prefix[b]) * kTile + r;
+      if (t < len) {
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < NPAD; ++j)
+          if (j < H_I) acc = fmaf(wr[j], fmaxf(__uint_as_float(v[j]), 0.f), acc);
+        scores[(int64_t)b * ld + t] = __fadd_rn(acc, 0.f);  // canonical +0
+        if (t == 0 && seq_off[b] + len > n_tokens)
+          report(status, kErrDevice, kKernIndexer, b, seq_off[b] + len, n_tokens);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Lay::kTmemCols);
+  }
+}
+
+template <int NHALF, int NPAD>
+cudaError_t launch_decode(const IndexerArgs& a, const CUtensorMap& tm_ki, const CUtensorMap& tm_qi,
+                          int num_sms, cudaStream_t stream) {
+  using Lay = IdxLayout<NHALF, NPAD>;
+  auto kern = indexer_decode_kernel<NHALF, NPAD>;
+  const size_t smem = Lay::smem_bytes(a.B);
+  cudaError_t e = ensure_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles_ub = (int64_t)a.B * ((a.S_max + kTile - 1) / kTile);
+  int grid = (int)(tiles_ub < num_sms ? tiles_ub : num_sms);
+  if (grid < 1) grid = 1;
+  kern<<<grid, kThreads, smem, stream>>>(tm_ki, tm_qi, a.w, a.seq_off, a.seq_len, a.B, a.n_tokens, a.S_max,
+                                        a.H_I, a.scores, a.ld, a.status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_indexer_decode(const IndexerArgs& a, const CUtensorMap& tm_ki, const CUtensorMap& tm_qi,
+                                  int npad, int num_sms, cudaStream_t stream) {
+  const int nh = a.d_I / 64;
+#define SA_IDX_CASE(NH, NP) \
+  if (nh == NH && npad == NP) return launch_decode<NH, NP>(a, tm_ki, tm_qi, num_sms, stream);
+  SA_IDX_CASE(1, 16) SA_IDX_CASE(1, 32) SA_IDX_CASE(1, 48) SA_IDX_CASE(1, 64)
+  SA_IDX_CASE(2, 16) SA_IDX_CASE(2, 32) SA_IDX_CASE(2, 48) SA_IDX_CASE(2, 64)
+  SA_IDX_CASE(3, 16) SA_IDX_CASE(3, 32) SA_IDX_CASE(3, 48) SA_IDX_CASE(3, 64)
+  SA_IDX_CASE(4, 16) SA_IDX_CASE(4, 32) SA_IDX_CASE(4, 48) SA_IDX_CASE(4, 64)
+#undef SA_IDX_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sa

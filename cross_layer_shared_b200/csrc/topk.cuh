@@ -1,0 +1,17 @@
+// Launch interface of the top-k kernels (internal to libsa).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "status.cuh"
+
+namespace sa {
+
+size_t topk_rows_smem_bytes();
+
+// One CTA per row: exact top-k with ties to the lower index, ascending output.
+cudaError_t launch_topk_rows(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max, int k,
+                             int32_t* idx, float* top_scores, DeviceStatus* status, cudaStream_t stream);
+
+}  // namespace sa

@@ -127,6 +127,22 @@ def distinct_positions(seed: int, tid: int, count: int, lo: int, hi: int, align:
     return out
 
 
+def gather_selected_rows(rows_fn, idx_row, Hkv: int, d: int):
+    """Copy the cache rows a selection uses into a compact [Hkv, m, d] cache
+    and remap the index to it (-1 entries stay -1).  rows_fn(head, rows)
+    returns the bf16 rows.  Pure data movement."""
+    idx_row = np.asarray(idx_row)
+    valid = idx_row[idx_row >= 0]
+    m = max(len(valid), 1)
+    K = np.zeros((Hkv, m, d), np.uint16)
+    for h in range(Hkv):
+        if len(valid):
+            K[h] = rows_fn(h, valid)
+    remap = np.full(len(idx_row), -1, np.int32)
+    remap[idx_row >= 0] = np.arange(len(valid), dtype=np.int32)
+    return K, remap, m
+
+
 def _unit(v: np.ndarray) -> np.ndarray:
     v = np.asarray(v, dtype=np.float64)
     return v / np.linalg.norm(v)

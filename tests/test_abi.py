@@ -1,0 +1,98 @@
+"""libsa loads on a machine without a GPU, exports every symbol include/sa.h
+declares, and rejects bad arguments on the host (no device call needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import cross_layer_shared_b200 as sa
+from cross_layer_shared_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return sa.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_path_entry_points():
+    names = declared_symbols()
+    for n in ("sa_index_score", "sa_topk", "sa_sparse_decode_attn", "sa_block_union_prefill", "sa_decode_step"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert name in sa.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.sa_abi_version() == 1
+    assert lib.sa_status_string(0) == b"SA_OK"
+    assert lib.sa_status_string(5) == b"SA_ERR_TIMEOUT"
+
+
+FAKE = ctypes.c_void_p(0x7F0000001000)  # never dereferenced: validation fails first
+FAKE_WS = ctypes.c_void_p(0x7F0000002000)
+
+
+def test_topk_rejects_bad_k_and_missing_workspace(lib):
+    rc = lib.sa_topk(FAKE, 100, FAKE, 2, 100, 0, FAKE, None, FAKE_WS, 4096, None)
+    assert rc == sa.SA_ERR_INVALID_ARG and b"k=0" in lib.sa_last_error()
+    rc = lib.sa_topk(FAKE, 100, FAKE, 2, 100, 8, FAKE, None, None, 0, None)
+    assert rc == sa.SA_ERR_WORKSPACE
+    rc = lib.sa_topk(FAKE, 100, FAKE, 2, 100, 8, FAKE, None, ctypes.c_void_p(0x7F0000002010), 4096, None)
+    assert rc == sa.SA_ERR_WORKSPACE and b"aligned" in lib.sa_last_error()
+    rc = lib.sa_topk(FAKE, 50, FAKE, 2, 100, 8, FAKE, None, FAKE_WS, 4096, None)
+    assert rc == sa.SA_ERR_INVALID_ARG  # ld below n_max
+
+
+def test_index_score_rejects_unsupported_shapes(lib):
+    rc = lib.sa_index_score(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 100, 100, 65, 128, FAKE, 100, FAKE_WS, 4096, None)
+    assert rc == sa.SA_ERR_UNSUPPORTED
+    rc = lib.sa_index_score(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 100, 100, 16, 96, FAKE, 100, FAKE_WS, 4096, None)
+    assert rc == sa.SA_ERR_UNSUPPORTED
+    rc = lib.sa_index_score(ctypes.c_void_p(0x7F0000001002), FAKE, FAKE, FAKE, FAKE, 1, 100, 100, 16, 128, FAKE,
+                            100, FAKE_WS, 4096, None)
+    assert rc == sa.SA_ERR_INVALID_ARG and b"aligned" in lib.sa_last_error()
+
+
+def test_attention_rejects_bad_head_counts(lib):
+    rc = lib.sa_sparse_decode_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1, 30, 4, 128, 256, 0.088, FAKE, 0,
+                                   FAKE_WS, 1 << 20, None)
+    assert rc == sa.SA_ERR_INVALID_ARG and b"multiple" in lib.sa_last_error()
+    rc = lib.sa_sparse_decode_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1, 32, 4, 64, 256, 0.125, FAKE, 0,
+                                   FAKE_WS, 1 << 20, None)
+    assert rc == sa.SA_ERR_UNSUPPORTED
+
+
+def test_decode_step_pattern_must_start_with_full_layer(lib):
+    arr = (ctypes.c_void_p * 4)(*([0x7F0000001000] * 4))
+    pp = ctypes.cast(arr, sa._PP)
+    for pat, want in ((b"SFSS", b"first layer must be F"), (b"FSXS", b"F or S")):
+        rc = lib.sa_decode_step(pat, 4, pp, pp, pp, pp, pp, FAKE, FAKE, 1, 4096, 4096, 4, 64, 256, FAKE, 8, 1, 128,
+                                0.088, FAKE, 0, FAKE, FAKE, 4096, FAKE_WS, 1 << 24, None)
+        assert rc == sa.SA_ERR_INVALID_ARG and want in lib.sa_last_error()
+
+
+def test_block_union_rejects_other_block_sizes(lib):
+    rc = lib.sa_block_union_prefill(FAKE, FAKE, FAKE, FAKE, FAKE, 4096, 16, 8, 2, 128, 64, 32, 0.088, FAKE, FAKE,
+                                    FAKE, 0, FAKE_WS, 1 << 20, None)
+    assert rc == sa.SA_ERR_UNSUPPORTED
+
+
+def test_workspace_sizes_are_host_computable(lib):
+    assert lib.sa_topk_workspace_size(4, 131072, 2048) >= sa.WS_HEADER_BYTES
+    w1 = lib.sa_sparse_decode_attn_workspace_size(24, 4, 32, 8, 128, 2048)
+    assert w1 >= sa.WS_HEADER_BYTES
+    assert lib.sa_decode_step_workspace_size(24, 4, 131072, 32, 8, 128, 2048) >= w1

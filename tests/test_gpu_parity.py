@@ -1,0 +1,311 @@
+"""CUDA path vs the CPU oracle, stage by stage and end to end, on the seeded
+workloads (full size, sampled sequences where the oracle would be slow) and
+on edge cases.  Every call goes through the C ABI (libsa.so)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import cross_layer_shared_b200 as sa
+import oracle
+import synth
+from cross_layer_shared_b200 import build
+from synth import gpu as sgpu
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch.device("cuda")
+
+
+def assert_status_ok(ws):
+    code, det = sa.read_status(ws)
+    assert code == 0, f"device status {code} detail {det}"
+
+
+def bf16_dev(bits, dev):
+    return sgpu.to_dev_bf16(np.asarray(bits, np.uint16), dev)
+
+
+# --------------------------------------------------------------------------
+def test_generator_twin_is_bit_exact(dev):
+    rng = np.random.default_rng(0)
+    for seed, tid, scale, n in ((1237, 2, 0.125, 1 << 20), (1239, 5 + 64 * 3, 1.0, (1 << 20) + 13)):
+        t = sgpu.normal_bf16_gpu(n, seed, tid, scale, dev)
+        pick = np.unique(np.concatenate([rng.integers(0, n, 4096), [0, n - 1, n - 2]]))
+        got = t.view(torch.int16).cpu().numpy().view(np.uint16)[pick]
+        want = synth.normal_bf16_at(seed, tid, pick.astype(np.uint64), scale)
+        assert np.array_equal(got, want)
+    # offset form (the fill of a slice far into a stream)
+    off = 3_000_000_017
+    t = sgpu.normal_bf16_gpu(1000, 5, 9, 1.0, dev, offset=off)
+    want = synth.normal_bf16_at(5, 9, np.arange(off, off + 1000, dtype=np.uint64), 1.0)
+    assert np.array_equal(t.view(torch.int16).cpu().numpy().view(np.uint16), want)
+
+
+# --------------------------------------------------------------------------
+def decode_group_parity(cfg, g, seqs, dev, out_dtypes=(torch.bfloat16, torch.float32)):
+    wl = sgpu.decode_workload(cfg, dev, groups=[g])
+    gr = wl["groups"][g]
+    ws = sa.workspace(1 << 16, dev)
+    scores = sa.index_score(gr["qI"], gr["w"], gr["KI"], wl["seq_off"], wl["seq_len"], cfg.S_max, ws=ws)
+    idx = sa.topk(scores, wl["seq_len"], cfg.S_max, cfg.k, ws=ws)
+    layers = list(cfg.groups[g])
+    Qg = wl["Q"][layers[0]:layers[-1] + 1].contiguous()
+    outs = {}
+    for dt in out_dtypes:
+        aws = sa.workspace(sa.sparse_decode_attn_workspace_size(len(layers), cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.k), dev)
+        outs[dt] = sa.sparse_decode_attn(Qg, gr["K"], gr["V"], wl["seq_off"], wl["seq_len"], idx, cfg.Hkv, cfg.scale,
+                                         out_dtype=dt, ws=aws)
+        assert_status_ok(aws)
+    assert_status_ok(ws)
+    scores_h = scores.cpu().numpy()
+    idx_h = idx.cpu().numpy()
+    outs_h = {dt: o.float().cpu().numpy() for dt, o in outs.items()}
+    qI, w, Q = cfg.qI(g), cfg.w(g), cfg.Q()
+    for b in seqs:
+        S = cfg.seq_lens[b]
+        KI = cfg.KI_rows(g, b, np.arange(S))
+        ora = oracle.index_score(qI[b:b + 1], w[b:b + 1], KI, [0, S], [0], [S - 1])[0]
+        parity.assert_scores_close(scores_h[b, :S], ora, parity.index_error_bound(qI[b], w[b], KI), f"{cfg.name} b={b}")
+        exact = oracle.topk(scores_h[b:b + 1, :S], [S], cfg.k)[0]
+        assert np.array_equal(idx_h[b], exact), f"{cfg.name} b={b}: top-k differs on identical scores"
+        parity.assert_topk_band(idx_h[b], ora, S, cfg.k, f"{cfg.name} b={b}")
+        Kc, remap, m = parity.compact_selected(lambda h, r: cfg.KV_rows(g, b, h, r, "K"), idx_h[b], cfg.Hkv, cfg.d)
+        Vc, _, _ = parity.compact_selected(lambda h, r: cfg.KV_rows(g, b, h, r, "V"), idx_h[b], cfg.Hkv, cfg.d)
+        O_ora = oracle.sparse_decode_attn(Q[layers][:, b:b + 1], Kc.ravel(), Vc.ravel(), [0, m], [m], remap[None],
+                                          cfg.Hkv, cfg.scale)[:, 0]
+        for dt, O in outs_h.items():
+            tol = parity.ATOL_F32 if dt == torch.float32 else parity.ATOL_BF16
+            err = np.abs(O[:, b] - O_ora).max()
+            assert err <= tol, f"{cfg.name} b={b} {dt}: max-abs {err} > {tol}"
+    return idx_h, scores_h
+
+
+def test_c1_decode_group_with_needles(dev):
+    cfg = synth.workload("c1")
+    idx_h, _ = decode_group_parity(cfg, 0, [0], dev)
+    needles = [t for (_, t, _, kr) in cfg.planted(0) if kr is not None]
+    assert set(needles) <= set(idx_h[0].tolist())
+
+
+@pytest.mark.parametrize("name,seqs", [("c2", [0, 5]), ("c3", [0, 3])])
+def test_full_size_decode_group(name, seqs, dev):
+    cfg = synth.workload(name)
+    decode_group_parity(cfg, len(cfg.groups) - 1, seqs, dev)
+
+
+def test_c5_ragged_group_sampled(dev):
+    cfg = synth.workload("c5")
+    lens = np.array(cfg.seq_lens)
+    seqs = [int(np.argmin(lens)), int(np.argmax(lens)), 7]
+    decode_group_parity(cfg, 0, seqs, dev, out_dtypes=(torch.bfloat16,))
+
+
+# --------------------------------------------------------------------------
+def test_topk_edge_cases(dev):
+    rng = np.random.default_rng(3)
+    n = 100_000
+    rows, nval, ks = [], [], []
+    rows.append(np.full(n, 0.75, np.float32)); nval.append(5000)                           # all equal
+    rows.append((rng.integers(0, 20, n) / 4).astype(np.float32)); nval.append(n)           # heavy ties at threshold
+    rows.append(rng.standard_normal(n).astype(np.float32)); nval.append(n)                 # negative scores
+    z = np.zeros(n, np.float32); z[::2] = -0.0; z[5::7] = 1.0; rows.append(z); nval.append(n)  # signed zeros
+    rows.append(rng.random(n).astype(np.float32)); nval.append(1500)                       # n_valid < k
+    rows.append(rng.random(n).astype(np.float32)); nval.append(0)                          # empty row
+    big = (1.0 + np.arange(n, dtype=np.float64) * 2 ** -23).astype(np.float32)            # one huge bucket
+    rows.append(rng.permutation(big)); nval.append(n)
+    rows.append(rng.random(n).astype(np.float32)); nval.append(2048)                       # n_valid == k
+    S = np.stack(rows)
+    nv = np.array(nval, np.int32)
+    for k in (1, 2048, 3000):
+        d_scores = torch.from_numpy(S).to(dev)
+        ws = sa.workspace(sa.lib().sa_topk_workspace_size(len(rows), n, k), dev)
+        idx, ts = sa.topk(d_scores, torch.from_numpy(nv).to(dev), n, k, want_scores=True, ws=ws)
+        assert_status_ok(ws)
+        want, want_s = oracle.topk(S, nv, k, with_scores=True)
+        got = idx.cpu().numpy()
+        for r in range(len(rows)):
+            assert np.array_equal(got[r], want[r]), f"row {r} k={k}"
+        assert np.array_equal(ts.cpu().numpy().view(np.uint32), want_s.view(np.uint32)) or \
+            np.array_equal(ts.cpu().numpy(), want_s)
+
+
+def test_topk_reports_bad_n_valid(dev):
+    s = torch.rand(2, 1000, device=dev)
+    ws = sa.workspace(256, dev)
+    idx = sa.topk(s, torch.tensor([1000, 5000], dtype=torch.int32, device=dev), 1000, 10, ws=ws)
+    code, det = sa.read_status(ws)
+    assert code == sa.SA_ERR_DEVICE and det[0] == 2 and det[2] == 5000
+    parity.assert_valid_index_row(idx[1].cpu().numpy(), 1000, 10)
+
+
+# --------------------------------------------------------------------------
+def _attn_case(dev, L, B, Hq, Hkv, lens, k, idx_fn, seed=0, out_dtype=torch.float32):
+    rng = np.random.default_rng(seed)
+    d = 128
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    T = int(seq_off[-1])
+    Q = synth.f32_to_bf16_bits(rng.standard_normal((L, B, Hq, d)).astype(np.float32))
+    K = synth.f32_to_bf16_bits(rng.standard_normal(T * Hkv * d).astype(np.float32))
+    V = synth.f32_to_bf16_bits(rng.standard_normal(T * Hkv * d).astype(np.float32))
+    idx = np.stack([idx_fn(rng, b, lens[b]) for b in range(B)]).astype(np.int32)
+    ws = sa.workspace(sa.sparse_decode_attn_workspace_size(L, B, Hq, Hkv, d, k), dev)
+    O = sa.sparse_decode_attn(bf16_dev(Q, dev), bf16_dev(K, dev), bf16_dev(V, dev), torch.from_numpy(seq_off).to(dev),
+                              torch.tensor(lens, dtype=torch.int32, device=dev), torch.from_numpy(idx).to(dev), Hkv,
+                              1 / math.sqrt(d), out_dtype=out_dtype, ws=ws)
+    want = oracle.sparse_decode_attn(Q, K, V, seq_off, lens, idx, Hkv, 1 / math.sqrt(d))
+    err = np.abs(O.float().cpu().numpy() - want).max()
+    return err, ws
+
+
+@pytest.mark.parametrize("case", ["full_selection", "padding", "ragged_k", "two_mtiles", "mha", "mqa"])
+def test_attention_edge_cases(case, dev):
+    def pick(k):
+        return lambda rng, b, S: np.sort(rng.choice(S, k, replace=False))
+    if case == "full_selection":  # k = S: dense attention
+        err, ws = _attn_case(dev, 2, 2, 8, 2, [700, 700], 700, lambda rng, b, S: np.arange(S))
+    elif case == "padding":       # -1 entries anywhere, and one row with none valid
+        def f(rng, b, S):
+            r = rng.choice(S, 256, replace=False)
+            r[rng.random(256) < 0.3] = -1
+            return r if b else np.full(256, -1)
+        err, ws = _attn_case(dev, 3, 2, 8, 1, [900, 400], 256, f)
+    elif case == "ragged_k":      # k not a multiple of the 128-key tile
+        err, ws = _attn_case(dev, 4, 3, 16, 4, [500, 333, 1200], 300, pick(300))
+    elif case == "two_mtiles":    # L*G = 200 query rows > one 128-row tile
+        err, ws = _attn_case(dev, 25, 1, 32, 4, [3000], 512, pick(512))
+    elif case == "mha":
+        err, ws = _attn_case(dev, 2, 2, 8, 8, [1000, 800], 384, pick(384))
+    else:
+        err, ws = _attn_case(dev, 6, 1, 16, 1, [5000], 1024, pick(1024), out_dtype=torch.bfloat16)
+    assert_status_ok(ws)
+    assert err <= (parity.ATOL_BF16 if case == "mqa" else parity.ATOL_F32), err
+
+
+def test_attention_reports_out_of_range_index(dev):
+    def f(rng, b, S):
+        r = np.arange(64)
+        r[3] = S + 5
+        return r
+    err, ws = _attn_case(dev, 1, 1, 4, 1, [100], 64, lambda rng, b, S: np.where(np.arange(64) == 3, -1, np.arange(64)))
+    assert err <= parity.ATOL_F32
+    rng = np.random.default_rng(1)
+    d = 128
+    Q = bf16_dev(synth.f32_to_bf16_bits(rng.standard_normal((1, 1, 4, d)).astype(np.float32)), dev)
+    K = bf16_dev(synth.f32_to_bf16_bits(rng.standard_normal(100 * d).astype(np.float32)), dev)
+    idx = torch.from_numpy(f(None, 0, 100).astype(np.int32)[None]).to(dev)
+    ws = sa.workspace(1 << 20, dev)
+    sa.sparse_decode_attn(Q, K, K, torch.tensor([0, 100], device=dev), torch.tensor([100], dtype=torch.int32, device=dev),
+                          idx, 1, 0.0884, ws=ws)
+    code, det = sa.read_status(ws)
+    assert code == sa.SA_ERR_DEVICE and det[0] == 3 and det[2] == 105
+
+
+# --------------------------------------------------------------------------
+def test_decode_step_c1_matches_oracle_walk(dev):
+    cfg = synth.workload("c1")
+    wl = sgpu.decode_workload(cfg, dev)
+    gr = wl["groups"][0]
+    n = cfg.L
+    O, idx = sa.decode_step(cfg.pattern, [gr["qI"]] + [None] * (n - 1), [gr["w"]] + [None] * (n - 1),
+                            [gr["KI"]] + [None] * (n - 1), [gr["K"]] * n, [gr["V"]] * n, wl["seq_off"],
+                            wl["seq_len"], cfg.S_max, cfg.k, wl["Q"], cfg.Hkv, cfg.scale, out_dtype=torch.float32)
+    KI = cfg.KI_full(0)
+    K, V = cfg.KV_full(0, "K"), cfg.KV_full(0, "V")
+    O_ora, used = oracle.decode_step(cfg.pattern, [cfg.qI(0)] * n, [cfg.w(0)] * n, [KI] * n, cfg.seq_off, cfg.seq_lens,
+                                     cfg.k, cfg.Q(), [K] * n, [V] * n, cfg.Hkv, cfg.scale)
+    got_idx = idx.cpu().numpy()
+    parity.assert_topk_band(got_idx[0], oracle.index_score(cfg.qI(0), cfg.w(0), KI, cfg.seq_off, [0],
+                                                           [cfg.S_max - 1])[0], cfg.S_max, cfg.k)
+    if np.array_equal(got_idx, used[0]):
+        assert np.abs(O.cpu().numpy() - O_ora).max() <= parity.ATOL_F32
+
+
+def test_shared_index_equals_per_layer_recompute(dev):
+    """F,F,F,F with identical indexer inputs gives what F,S,S,S gives."""
+    cfg = synth.workload("c1")
+    wl = sgpu.decode_workload(cfg, dev)
+    gr = wl["groups"][0]
+    n = 4
+    common = ([gr["K"]] * n, [gr["V"]] * n, wl["seq_off"], wl["seq_len"], cfg.S_max, cfg.k, wl["Q"], cfg.Hkv, cfg.scale)
+    O1, i1 = sa.decode_step("FFFF", [gr["qI"]] * n, [gr["w"]] * n, [gr["KI"]] * n, *common, out_dtype=torch.float32)
+    O2, i2 = sa.decode_step("FSSS", [gr["qI"]] * n, [gr["w"]] * n, [gr["KI"]] * n, *common, out_dtype=torch.float32)
+    assert torch.equal(i1, i2)
+    assert torch.allclose(O1, O2, rtol=0, atol=1e-6)
+
+
+def test_step_is_deterministic(dev):
+    cfg = synth.workload("c1")
+    wl = sgpu.decode_workload(cfg, dev)
+    gr = wl["groups"][0]
+    n = cfg.L
+    args = ([gr["qI"]] + [None] * (n - 1), [gr["w"]] + [None] * (n - 1), [gr["KI"]] + [None] * (n - 1),
+            [gr["K"]] * n, [gr["V"]] * n, wl["seq_off"], wl["seq_len"], cfg.S_max, cfg.k, wl["Q"], cfg.Hkv, cfg.scale)
+    a = sa.decode_step(cfg.pattern, *args)
+    b = sa.decode_step(cfg.pattern, *args)
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16)) and torch.equal(a[1], b[1])
+
+
+# --------------------------------------------------------------------------
+def prefill_parity(cfg, dev, q_sample=None, heads=None):
+    wl = sgpu.prefill_workload(cfg, dev)
+    ws = sa.workspace(sa.lib().sa_index_score_prefill_workspace_size(cfg.chunk), dev)
+    scores = sa.index_score_prefill(wl["qI"], wl["w"], wl["KI"], wl["q_pos"], cfg.S - 1, ws=ws)
+    n_valid = (wl["q_pos"] + 1).to(torch.int32)
+    idx = sa.topk(scores, n_valid, cfg.S, cfg.k, ws=ws)
+    uws = sa.workspace(sa.lib().sa_block_union_prefill_workspace_size(cfg.S, cfg.chunk, cfg.Hq, cfg.Hkv, cfg.d,
+                                                                       cfg.k, cfg.block), dev)
+    indptr, indices, O = sa.block_union_prefill(idx, wl["q_pos"], wl["Q"], wl["K"], wl["V"], cfg.block, cfg.scale,
+                                                out_dtype=torch.float32, ws=uws)
+    assert_status_ok(ws)
+    assert_status_ok(uws)
+    idx_h = idx.cpu().numpy()
+    q_pos = cfg.q_pos
+    sample = range(cfg.chunk) if q_sample is None else q_sample
+    KI = cfg.KI_full()
+    qI, w = cfg.qI(), cfg.w()
+    scores_h = scores.cpu().numpy() if q_sample is None else scores[torch.tensor(list(sample), device=dev)].cpu().numpy()
+    for i, p in enumerate(sample):
+        n = int(q_pos[p]) + 1
+        ora = oracle.index_score(qI[p:p + 1], w[p:p + 1], KI, [0, cfg.S], [0], [n - 1])[0][:n]
+        parity.assert_scores_close(scores_h[i, :n], ora, parity.index_error_bound(qI[p], w[p], KI[:n]), f"p={p}")
+        assert np.array_equal(idx_h[p], oracle.topk(scores_h[i:i + 1, :n], [n], cfg.k)[0])
+        parity.assert_topk_band(idx_h[p], ora, n, cfg.k, f"p={p}")
+    # the union of the GPU's index, exactly
+    want_ptr, want_ind = oracle.block_union(idx_h, cfg.S, cfg.block, cfg.Hkv)
+    got_ptr = indptr.cpu().numpy()
+    assert np.array_equal(got_ptr, want_ptr)
+    assert np.array_equal(indices.cpu().numpy()[:got_ptr[-1]], want_ind)
+    # paged causal attention over the union, sampled rows of the chosen heads
+    heads = range(cfg.Hq) if heads is None else heads
+    G = cfg.Hq // cfg.Hkv
+    O_h = O.cpu().numpy()
+    Qh = cfg.Q()
+    for h in heads:
+        g = h // G
+        Kg = cfg.KV_rows(g, np.arange(cfg.S), "K")[None]
+        Vg = cfg.KV_rows(g, np.arange(cfg.S), "V")[None]
+        rows = list(sample)
+        Qs = Qh[rows][:, h:h + 1]
+        ptr1 = np.array([0, want_ptr[1]], np.int32)
+        want = oracle.paged_prefill_attn(Qs, q_pos[rows], Kg, Vg, cfg.block, ptr1, want_ind[:want_ptr[1]], cfg.scale)
+        err = np.abs(O_h[rows, h] - want[:, 0]).max()
+        assert err <= parity.ATOL_F32, f"head {h}: {err}"
+
+
+def test_prefill_small_full_oracle(dev):
+    cfg = synth.PrefillConfig("small", S=4096, chunk=256, H_I=16, d_I=128, k=256, block=64, Hq=8, Hkv=2, d=128,
+                              seed=77, hot_regions=4, region_len=128)
+    prefill_parity(cfg, dev)
+
+
+def test_prefill_c4_full_size_sampled(dev):
+    cfg = synth.workload("c4")
+    prefill_parity(cfg, dev, q_sample=[0, 1, 1000, 2047], heads=[0, 13, 31])
