@@ -45,6 +45,8 @@ SIGNATURES = {
     "sa_block_union_prefill_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "sa_block_union_prefill": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
                                _I),
+    "sa_block_union_prefill_noalloc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P],
+                                       _I),
 }
 
 
@@ -242,4 +244,22 @@ def block_union_prefill(idx, q_pos, Q, K, V, block: int, scale: float, out_dtype
     _check(lib().sa_block_union_prefill(_ptr(idx), _ptr(q_pos), _ptr(Q), _ptr(K), _ptr(V), S, Nq, Hq, Hkv, d, k,
                                         block, float(scale), _ptr(kv_indptr), _ptr(kv_indices), _ptr(O), code,
                                         _ptr(ws), ws.numel(), _stream(stream)))
+    return kv_indptr, kv_indices, O
+
+
+def block_union_prefill_noalloc(idx, q_pos, Q, K, V, block: int, scale: float, kv_indptr, kv_indices, O,
+                                stream=None):
+    """sa_block_union_prefill_noalloc: the same result as block_union_prefill
+    without a workspace, for callers that cannot allocate device memory around
+    the call (outputs are passed in).  Its scratch is a fixed array inside
+    libsa; calls that can overlap on the GPU must not be issued together."""
+    Nq, Hq, d = Q.shape
+    Hkv, S, _ = K.shape
+    k = idx.shape[1]
+    _dev(idx, torch.int32, "idx"), _dev(q_pos, torch.int32, "q_pos")
+    _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
+    code = SA_F32 if O.dtype == torch.float32 else SA_BF16
+    _check(lib().sa_block_union_prefill_noalloc(_ptr(idx), _ptr(q_pos), _ptr(Q), _ptr(K), _ptr(V), S, Nq, Hq, Hkv,
+                                                d, k, block, float(scale), _ptr(kv_indptr), _ptr(kv_indices),
+                                                _ptr(O), code, _stream(stream)))
     return kv_indptr, kv_indices, O

@@ -486,3 +486,94 @@ sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc variant
+// Scratch of sa_block_union_prefill_noalloc: a status block followed by one
+// byte per KV block.  It lives in the library's own device memory (every GPU
+// that loads libsa keeps these bytes until the process exits), so the caller
+// needs no workspace.  All calls on a device share it.
+#define SA_NOALLOC_MARK_BYTES SA_NOALLOC_MAX_KV_BLOCKS
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SA_WS_HEADER_BYTES + SA_NOALLOC_MARK_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (host code cannot use the symbol itself as a device pointer).
+sa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc: cudaGetDevice", e);
+  if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "sa_block_union_prefill_noalloc: device %d >= 64", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc: cudaGetSymbolAddress", e);
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return SA_OK;
+}
+}  // namespace
+
+extern "C" sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const int32_t* q_pos, const void* Q,
+                                                    const void* K, const void* V, int S, int Nq, int Hq, int Hkv,
+                                                    int d, int k, int block, float scale, int32_t* kv_indptr,
+                                                    int32_t* kv_indices, void* O, sa_dtype out_dtype, void* stream) {
+  const char* who = "sa_block_union_prefill_noalloc";
+  if (S < 1 || Nq < 1 || Hq < 1 || Hkv < 1 || k < 1) return fail(SA_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+  if (d != 128) return fail(SA_ERR_UNSUPPORTED, "%s: d=%d (only 128 is built)", who, d);
+  if (block != 64) return fail(SA_ERR_UNSUPPORTED, "%s: block=%d (only 64 is built)", who, block);
+  const int64_t nb = ((int64_t)S + block - 1) / block;
+  if (nb > SA_NOALLOC_MARK_BYTES)
+    return fail(SA_ERR_UNSUPPORTED, "%s: S=%d needs %lld KV blocks; the static scratch holds at most %d (S <= %d)",
+                who, S, (long long)nb, SA_NOALLOC_MARK_BYTES, SA_NOALLOC_MARK_BYTES * 64);
+  if (Hq % Hkv != 0) return fail(SA_ERR_INVALID_ARG, "%s: Hq not a multiple of Hkv", who);
+  if ((int64_t)Nq * (Hq / Hkv) > (1 << 30)) return fail(SA_ERR_INVALID_ARG, "%s: too many query rows", who);
+  if (out_dtype != SA_BF16 && out_dtype != SA_F32) return fail(SA_ERR_INVALID_ARG, "%s: bad out_dtype", who);
+  if (!idx || !q_pos || !Q || !K || !V || !kv_indptr || !kv_indices || !O)
+    return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
+    return fail(SA_ERR_INVALID_ARG, "%s: Q, K, V, O must be 16-byte aligned", who);
+  if (!(scale > 0.f)) return fail(SA_ERR_INVALID_ARG, "%s: scale must be > 0", who);
+  void* scratch = nullptr;
+  sa_status st = noalloc_scratch(&scratch);
+  if (st != SA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the previous call's status and marks are still in the array: start clean
+  cudaError_t e = cudaMemsetAsync(scratch, 0, SA_WS_HEADER_BYTES, s);
+  if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc clear", e);
+  uint8_t* mark = reinterpret_cast<uint8_t*>(scratch) + SA_WS_HEADER_BYTES;
+  e = sa::launch_block_union(idx, Nq, k, S, block, Hkv, mark, kv_indptr, kv_indices, status_of(scratch), s);
+  if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc union", e);
+  sa::AttnArgs a{};
+  a.Q = reinterpret_cast<const uint16_t*>(Q);
+  a.K = reinterpret_cast<const uint16_t*>(K);
+  a.V = reinterpret_cast<const uint16_t*>(V);
+  a.prefill = 1;
+  a.q_pos = q_pos;
+  a.kv_indptr = kv_indptr;
+  a.kv_indices = kv_indices;
+  a.S = S;
+  a.block = block;
+  a.Nq = Nq;
+  a.L = 1;
+  a.B = 1;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.R = Nq * a.G;
+  a.n_mtiles = (a.R + 127) / 128;
+  a.n_split = 1;
+  a.keys_per_split = (int)round_up((size_t)nb * block, 128);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = O;
+  a.out_f32 = out_dtype == SA_F32;
+  a.part = nullptr;
+  a.status = status_of(scratch);
+  e = sa::launch_sparse_attn(a, out_dtype == SA_F32, s);
+  if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc attention", e);
+  return SA_OK;
+}

@@ -45,7 +45,9 @@
  *   rest is scratch owned by the call while it runs on `stream`: calls that
  *   overlap on the GPU must not share one workspace.
  * - The library keeps no global state between calls apart from a cached
- *   driver entry point; calls are reentrant and thread-safe.
+ *   driver entry point and the fixed scratch array of
+ *   sa_block_union_prefill_noalloc (see there); the workspace entry points
+ *   are reentrant and thread-safe.
  */
 #ifndef CROSS_LAYER_SHARED_SA_H
 #define CROSS_LAYER_SHARED_SA_H
@@ -232,6 +234,35 @@ sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const
                                  int d, int k, int block, float scale, int32_t* kv_indptr,
                                  int32_t* kv_indices, void* O, sa_dtype out_dtype, void* ws,
                                  size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * sa_block_union_prefill without a workspace.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory around the call - code running inside a CUDA graph capture
+ * (where cudaMalloc is not allowed), runtimes without a device allocator
+ * hook, or a host that has handed all memory to another pool.
+ *
+ * Same arguments, results and device-side skipping as
+ * sa_block_union_prefill, minus ws / ws_bytes.  Its scratch (a status block
+ * and one byte per KV block) is a fixed array inside libsa's own device
+ * memory, SA_NOALLOC_MAX_KV_BLOCKS bytes plus 256, held by every GPU that
+ * loads the library until the process exits.  Limits:
+ *   - ceil(S / block) <= SA_NOALLOC_MAX_KV_BLOCKS (S <= 2,097,152 at block 64),
+ *     larger S returns SA_ERR_UNSUPPORTED before anything is enqueued;
+ *   - the first call on each device looks up the array's device address, so
+ *     make that first call before any stream capture begins;
+ *   - every call shares the one array: calls that may overlap on the GPU
+ *     (different streams, or different host threads on one device) race and
+ *     must be ordered by the caller;
+ *   - device-side range errors are skipped as usual, but their record stays
+ *     in the library's array (cleared at every call) and is not reported.
+ * Allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
+ * ---------------------------------------------------------------------- */
+#define SA_NOALLOC_MAX_KV_BLOCKS 32768
+sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const int32_t* q_pos, const void* Q,
+                                         const void* K, const void* V, int S, int Nq, int Hq, int Hkv,
+                                         int d, int k, int block, float scale, int32_t* kv_indptr,
+                                         int32_t* kv_indices, void* O, sa_dtype out_dtype, void* stream);
 
 #ifdef __cplusplus
 }
