@@ -287,9 +287,9 @@ sa_status sa_index_score_prefill(const void* qI, const float* w, const void* KI,
 
 // ---------------------------------------------------------------- top-k
 size_t sa_topk_workspace_size(int Nq, int n_max, int k) {
-  (void)Nq;
-  (void)n_max;
   (void)k;
+  if (Nq > 0 && n_max > 0 && sa::topk_use_split(Nq, n_max, num_sms()))
+    return SA_WS_HEADER_BYTES + sa::topk_split_ws_bytes(Nq, n_max);
   return SA_WS_HEADER_BYTES;
 }
 
@@ -303,8 +303,13 @@ sa_status sa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int N
   sa_status st = check_ws(ws, ws_bytes, sa_topk_workspace_size(Nq, n_max, k), who);
   if (st != SA_OK) return st;
   if (Nq == 0) return SA_OK;
-  cudaError_t e = sa::launch_topk_rows(scores, ld, n_valid, Nq, n_max, k, idx, top_scores, status_of(ws),
-                                       (cudaStream_t)stream);
+  cudaError_t e;
+  if (sa::topk_use_split(Nq, n_max, num_sms()))
+    e = sa::launch_topk_split(scores, ld, n_valid, Nq, n_max, k, idx, top_scores, status_of(ws),
+                              reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES, num_sms(), (cudaStream_t)stream);
+  else
+    e = sa::launch_topk_rows(scores, ld, n_valid, Nq, n_max, k, idx, top_scores, status_of(ws),
+                             (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail("sa_topk launch", e);
   return SA_OK;
 }

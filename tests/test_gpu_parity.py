@@ -53,7 +53,8 @@ def test_generator_twin_is_bit_exact(dev):
 def decode_group_parity(cfg, g, seqs, dev, out_dtypes=(torch.bfloat16, torch.float32)):
     wl = sgpu.decode_workload(cfg, dev, groups=[g])
     gr = wl["groups"][g]
-    ws = sa.workspace(1 << 16, dev)
+    ws = sa.workspace(max(sa.lib().sa_topk_workspace_size(cfg.B, cfg.S_max, cfg.k),
+                          sa.lib().sa_index_score_workspace_size(cfg.B)), dev)
     scores = sa.index_score(gr["qI"], gr["w"], gr["KI"], wl["seq_off"], wl["seq_len"], cfg.S_max, ws=ws)
     idx = sa.topk(scores, wl["seq_len"], cfg.S_max, cfg.k, ws=ws)
     layers = list(cfg.groups[g])
@@ -109,7 +110,8 @@ def test_c5_ragged_group_sampled(dev):
 
 
 # --------------------------------------------------------------------------
-def test_topk_edge_cases(dev):
+@pytest.mark.parametrize("replicas", [1, 10])  # 8 rows: many CTAs per row; 80 rows: one CTA per row
+def test_topk_edge_cases(dev, replicas):
     rng = np.random.default_rng(3)
     n = 100_000
     rows, nval, ks = [], [], []
@@ -122,8 +124,9 @@ def test_topk_edge_cases(dev):
     big = (1.0 + np.arange(n, dtype=np.float64) * 2 ** -23).astype(np.float32)            # one huge bucket
     rows.append(rng.permutation(big)); nval.append(n)
     rows.append(rng.random(n).astype(np.float32)); nval.append(2048)                       # n_valid == k
-    S = np.stack(rows)
-    nv = np.array(nval, np.int32)
+    S = np.concatenate([np.stack(rows)] * replicas)
+    nv = np.array(nval * replicas, np.int32)
+    rows = rows * replicas
     for k in (1, 2048, 3000):
         d_scores = torch.from_numpy(S).to(dev)
         ws = sa.workspace(sa.lib().sa_topk_workspace_size(len(rows), n, k), dev)
@@ -256,7 +259,8 @@ def test_step_is_deterministic(dev):
 # --------------------------------------------------------------------------
 def prefill_parity(cfg, dev, q_sample=None, heads=None):
     wl = sgpu.prefill_workload(cfg, dev)
-    ws = sa.workspace(sa.lib().sa_index_score_prefill_workspace_size(cfg.chunk), dev)
+    ws = sa.workspace(max(sa.lib().sa_index_score_prefill_workspace_size(cfg.chunk),
+                          sa.lib().sa_topk_workspace_size(cfg.chunk, cfg.S, cfg.k)), dev)
     scores = sa.index_score_prefill(wl["qI"], wl["w"], wl["KI"], wl["q_pos"], cfg.S - 1, ws=ws)
     n_valid = (wl["q_pos"] + 1).to(torch.int32)
     idx = sa.topk(scores, n_valid, cfg.S, cfg.k, ws=ws)
