@@ -342,19 +342,19 @@ def run_ours(args):
             step(st)
         graphs.append(g)
 
-    # kernel launches inside one step (indexer + top-k per F layer, attention
-    # [+ split combine] per fused group)
+    # kernels of ours inside one step: per F layer the indexer and the top-k
+    # (two kernels when rows are few and long, one otherwise), per fused group
+    # one attention launch
+    split_topk = cfg.B * 2 <= torch.cuda.get_device_properties(dev).multi_processor_count and cfg.S_max > 8192
     launches_per_step = 0
-    splits = []
     l = 0
     while l < n:
         if cfg.pattern[l] == "F":
-            launches_per_step += 2
+            launches_per_step += 1 + (2 if split_topk else 1)
         m = l
         while m + 1 < n and cfg.pattern[m + 1] == "S" and sets[0]["K"][m + 1] is sets[0]["K"][l]:
             m += 1
-        ws_sz = sa.sparse_decode_attn_workspace_size(m - l + 1, cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.k)
-        launches_per_step += 1 + (1 if ws_sz > sa.WS_HEADER_BYTES else 0)
+        launches_per_step += 1
         l = m + 1
 
     for i in range(args.warmup):

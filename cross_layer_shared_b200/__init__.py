@@ -38,7 +38,7 @@ SIGNATURES = {
     "sa_topk_workspace_size": ([_I, _I, _I], _SZ),
     "sa_topk": ([_P, _I64, _P, _I, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "sa_sparse_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
-    "sa_sparse_decode_attn": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _SZ, _P], _I),
+    "sa_sparse_decode_attn": ([_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _F, _P, _I, _P, _SZ, _P], _I),
     "sa_decode_step_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "sa_decode_step": ([ctypes.c_char_p, _I, _PP, _PP, _PP, _PP, _PP, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _I,
                         _I, _I, _F, _P, _I, _P, _P, _I64, _P, _SZ, _P], _I),
@@ -167,8 +167,10 @@ def sparse_decode_attn_workspace_size(L_g, B, Hq, Hkv, d, k) -> int:
 
 def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, out_dtype=torch.bfloat16, O=None,
                        ws=None, stream=None) -> torch.Tensor:
+    """K, V: packed caches of n_tokens * Hkv rows of d (n_tokens = sum of seq_len)."""
     L, B, Hq, d = Q.shape
     k = idx.shape[1]
+    n_tokens = K.numel() // (Hkv * d)
     _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
     _dev(idx, torch.int32, "idx")
     if O is None:
@@ -176,8 +178,8 @@ def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, o
     if ws is None:
         ws = workspace(sparse_decode_attn_workspace_size(L, B, Hq, Hkv, d, k), Q.device)
     code = SA_F32 if O.dtype == torch.float32 else SA_BF16
-    _check(lib().sa_sparse_decode_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), _ptr(idx), L, B, Hq,
-                                       Hkv, d, k, float(scale), _ptr(O), code, _ptr(ws), ws.numel(),
+    _check(lib().sa_sparse_decode_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), _ptr(idx), L, B,
+                                       n_tokens, Hq, Hkv, d, k, float(scale), _ptr(O), code, _ptr(ws), ws.numel(),
                                        _stream(stream)))
     return O
 

@@ -104,6 +104,15 @@ sa_status make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* 
   return SA_OK;
 }
 
+// [rows, 128] bf16 as a 2-D tensor map with a 64 x 1 box (rows gathered four at a time)
+sa_status make_rows_tmap(CUtensorMap* m, const void* base, int64_t rows) {
+  if (rows < 1 || rows >= (1ll << 31)) return fail(SA_ERR_INVALID_ARG, "tensor of %lld rows: need 1 <= rows < 2^31", (long long)rows);
+  const uint64_t dims[2] = {128, (uint64_t)rows};
+  const uint64_t str[1] = {256};
+  const uint32_t box[2] = {64, 1};
+  return make_tmap(m, base, 2, dims, str, box);
+}
+
 sa::DeviceStatus* status_of(void* ws) { return reinterpret_cast<sa::DeviceStatus*>(ws); }
 
 sa_status check_ws(void* ws, size_t ws_bytes, size_t need, const char* who) {
@@ -130,18 +139,21 @@ AttnPlan plan_decode_attn(int L_g, int B, int Hq, int Hkv, int k) {
   const int base = B * Hkv * p.n_mtiles;
   const int max_split = (k + 127) / 128;
   int s = num_sms() / (base > 0 ? base : 1);
-  if (s < 1) s = 1;
   if (s > max_split) s = max_split;
+  if (s > 8) s = 8;
+  int p2 = 1;  // splits form a cluster: 1, 2, 4 or 8 CTAs
+  while (p2 * 2 <= s) p2 *= 2;
+  s = p2;
   p.keys_per_split = (int)round_up((size_t)((k + s - 1) / s), 128);
   if (p.keys_per_split < 128) p.keys_per_split = 128;
-  p.n_split = (k + p.keys_per_split - 1) / p.keys_per_split;
-  if (p.n_split < 1) p.n_split = 1;
+  p.n_split = s;  // trailing splits may get no keys; they merge as empty
   p.units = base * p.n_split;
   return p;
 }
 
 size_t attn_ws_bytes(const AttnPlan& p) {
-  return SA_WS_HEADER_BYTES + (p.n_split > 1 ? round_up(sa::attn_partial_bytes(p.units), 256) : 0);
+  (void)p;
+  return SA_WS_HEADER_BYTES;
 }
 
 sa_status validate_index(const void* qI, const float* w, const void* KI, int H_I, int d_I, const char* who) {
@@ -322,9 +334,9 @@ size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int
 }
 
 static sa_status run_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
-                                 const int32_t* seq_len, const int32_t* idx, int L_g, int B, int Hq, int Hkv, int d,
-                                 int k, float scale, void* O, sa_dtype out_dtype, void* ws, size_t ws_bytes,
-                                 cudaStream_t stream) {
+                                 const int32_t* seq_len, const int32_t* idx, int L_g, int B, int64_t n_tokens, int Hq,
+                                 int Hkv, int d, int k, float scale, void* O, sa_dtype out_dtype, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream) {
   const char* who = "sa_sparse_decode_attn";
   if (L_g < 1 || B < 1 || Hq < 1 || Hkv < 1 || k < 1)
     return fail(SA_ERR_INVALID_ARG, "%s: L_g, B, Hq, Hkv, k must be >= 1", who);
@@ -338,6 +350,10 @@ static sa_status run_decode_attn(const void* Q, const void* K, const void* V, co
   const AttnPlan p = plan_decode_attn(L_g, B, Hq, Hkv, k);
   sa_status st = check_ws(ws, ws_bytes, attn_ws_bytes(p), who);
   if (st != SA_OK) return st;
+  CUtensorMap tm_q, tm_k, tm_v;
+  if ((st = make_rows_tmap(&tm_q, Q, (int64_t)L_g * B * Hq)) != SA_OK) return st;
+  if ((st = make_rows_tmap(&tm_k, K, n_tokens * Hkv)) != SA_OK) return st;
+  if ((st = make_rows_tmap(&tm_v, V, n_tokens * Hkv)) != SA_OK) return st;
   sa::AttnArgs a{};
   a.Q = reinterpret_cast<const uint16_t*>(Q);
   a.K = reinterpret_cast<const uint16_t*>(K);
@@ -359,19 +375,18 @@ static sa_status run_decode_attn(const void* Q, const void* K, const void* V, co
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;
   a.out_f32 = out_dtype == SA_F32;
-  a.part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES);
   a.status = status_of(ws);
-  cudaError_t e = sa::launch_sparse_attn(a, out_dtype == SA_F32, stream);
+  cudaError_t e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, stream);
   if (e != cudaSuccess) return cuda_fail("sa_sparse_decode_attn launch", e);
   return SA_OK;
 }
 
 sa_status sa_sparse_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
-                                const int32_t* seq_len, const int32_t* idx, int L_g, int B, int Hq, int Hkv, int d,
-                                int k, float scale, void* O, sa_dtype out_dtype, void* ws, size_t ws_bytes,
-                                void* stream) {
-  return run_decode_attn(Q, K, V, seq_off, seq_len, idx, L_g, B, Hq, Hkv, d, k, scale, O, out_dtype, ws, ws_bytes,
-                         (cudaStream_t)stream);
+                                const int32_t* seq_len, const int32_t* idx, int L_g, int B, int64_t n_tokens, int Hq,
+                                int Hkv, int d, int k, float scale, void* O, sa_dtype out_dtype, void* ws,
+                                size_t ws_bytes, void* stream) {
+  return run_decode_attn(Q, K, V, seq_off, seq_len, idx, L_g, B, n_tokens, Hq, Hkv, d, k, scale, O, out_dtype, ws,
+                         ws_bytes, (cudaStream_t)stream);
 }
 
 // ---------------------------------------------------------------- decode step
@@ -418,7 +433,7 @@ sa_status sa_decode_step(const char* pattern, int n_layers, const void* const* q
     int m = l;
     while (m + 1 < n_layers && pattern[m + 1] == 'S' && K[m + 1] == K[l] && V[m + 1] == V[l]) ++m;
     st = run_decode_attn(reinterpret_cast<const uint8_t*>(Q) + (size_t)l * layer_elems * 2, K[l], V[l], seq_off,
-                         seq_len, idx, m - l + 1, B, Hq, Hkv, d, k, scale,
+                         seq_len, idx, m - l + 1, B, n_tokens, Hq, Hkv, d, k, scale,
                          reinterpret_cast<uint8_t*>(O) + (size_t)l * layer_elems * esize, out_dtype, ws, ws_bytes,
                          (cudaStream_t)stream);
     if (st != SA_OK) return st;
@@ -483,9 +498,15 @@ sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;
   a.out_f32 = out_dtype == SA_F32;
-  a.part = nullptr;
   a.status = status_of(ws);
-  e = sa::launch_sparse_attn(a, out_dtype == SA_F32, s);
+  {
+    CUtensorMap tm_q, tm_k, tm_v;
+    sa_status st2;
+    if ((st2 = make_rows_tmap(&tm_q, Q, (int64_t)Nq * Hq)) != SA_OK) return st2;
+    if ((st2 = make_rows_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
+    if ((st2 = make_rows_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
+    e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, s);
+  }
   if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill attention", e);
   return SA_OK;
 }
@@ -576,9 +597,15 @@ extern "C" sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const in
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;
   a.out_f32 = out_dtype == SA_F32;
-  a.part = nullptr;
   a.status = status_of(scratch);
-  e = sa::launch_sparse_attn(a, out_dtype == SA_F32, s);
+  {
+    CUtensorMap tm_q, tm_k, tm_v;
+    sa_status st2;
+    if ((st2 = make_rows_tmap(&tm_q, Q, (int64_t)Nq * Hq)) != SA_OK) return st2;
+    if ((st2 = make_rows_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
+    if ((st2 = make_rows_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
+    e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, s);
+  }
   if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc attention", e);
   return SA_OK;
 }

@@ -14,20 +14,25 @@
 // with rows = (query, head of the group), keys = the tokens of the group's
 // union blocks, and a causal limit per row.
 //
-// Per CTA (256 threads, warp-specialised):
-//   warps 5-7  gather 128 K rows and 128 V rows per tile with cp.async into
-//              128-byte swizzled shared memory, a 3-deep ring (2 in the
-//              precise-P variant); completion signalled on an mbarrier;
-//   warp 4     owns TMEM (512 columns: S double buffer + O) and issues
-//              S = Q K^T (M=128 rows, N=128 keys, K=d=128) and O += P V
-//              (V read MN-major), so the next tile's QK^T overlaps this
-//              tile's softmax;
-//   warps 0-3  one query row per thread: softmax in registers (exp2
-//              domain, running max with lazy rescale: O is rescaled only
-//              when the max grows by more than 2^8), P in bf16 (or a hi+lo
-//              bf16 pair for fp32 outputs) written over the consumed K
-//              tile; warps whose rows are all padding skip the work.
-//   Key splits write (O, m, l) partials merged by attn_combine_kernel.
+// Per CTA (384 threads, warp-specialised):
+//   warps 9-11  gather 128 K rows and 128 V rows per tile with TMA
+//               (tile::gather4: 4 rows x 128 bytes per instruction) into
+//               128-byte swizzled shared memory, a 3-deep ring (2 in the
+//               precise-P variant); each warp signals its bytes on the
+//               stage's mbarrier; the next tile's indices load early;
+//   warp 8      owns TMEM (512 columns: S double buffer, O0, O1) and issues
+//               S = Q K^T (M=128 rows, N=128 keys, K=d=128) and, per key
+//               half h, O_h += P_h V_h (V read MN-major), so the next
+//               tile's QK^T overlaps this tile's softmax;
+//   warps 0-7   softmax: warp w owns rows 32(w%4).. and key half w/4, one
+//               row per thread, with its own running max / sum / O_h (exp2
+//               domain, lazy rescale: O_h is rescaled only when the max
+//               grows by more than 2^8); P in bf16 (or a hi+lo bf16 pair for
+//               fp32 outputs) written over the consumed K tile.
+//   The two halves are merged at the end; key splits of one row tile run as
+//   a thread-block cluster: each CTA stages its (m, l, O) per output slice
+//   and bulk-copies slice t into CTA t's shared memory, which merges it.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -41,6 +46,11 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kKT = 128;  // keys per tile
+constexpr int kSoftWarps = 8;
+constexpr int kMmaWarp = 8;
+constexpr int kProdWarp0 = 9;  // warps 9, 10, 11
+constexpr int kAttnThreads = 384;
+constexpr int kMlxOff = 188 * 1024;  // half-merge exchange, past every epilogue slot
 
 template <bool PRECISE>
 struct AttnLayout {
@@ -51,19 +61,23 @@ struct AttnLayout {
   static constexpr int kStageOff = kTile;
   static constexpr int kStageBytes = 2 * kTile;  // K then V
   static constexpr int kPloOff = kStageOff + kStages * kStageBytes;
-  static constexpr int kKposOff = kPloOff + (PRECISE ? 2 * kTile : 0);
-  static constexpr int kBarOff = kKposOff + kStages * kKT * 4;
-  // kv_full[ST] kv_empty[ST] s_full[2] s_free[2] p_full[2] o_done
-  static constexpr int kNBar = 2 * kStages + 7;
+  // per stage: 4 validity words (bit c: key 32w+c is real) and the position of
+  // key 32w of each word (positions inside a 32-key word are consecutive in prefill)
+  static constexpr int kMaskOff = kPloOff + (PRECISE ? 2 * kTile : 0);
+  static constexpr int kBarOff = kMaskOff + kStages * 8 * 4;
+  // kv_full[ST] kv_empty[ST] s_full[2] s_free[2] p_full[2] o_done[4] recv
+  static constexpr int kNBar = 2 * kStages + 11;
   static constexpr int kSlotOff = kBarOff + 8 * kNBar;
   static constexpr size_t kSmem = 1024 + kSlotOff + 16;
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
-constexpr int kSoftWarps = 4;       // warps 0-3: one query row per thread
-constexpr int kMmaWarp = 4;         // warp 4: TMEM owner, one thread issues MMAs
-constexpr int kProdWarp0 = 5;       // warps 5-7: cp.async gathers
-constexpr int kProdThreads = 96;
-constexpr int kAttnThreads = 256;
+// 2^x on the special-function unit (ex2.approx.ftz.f32; 2^-inf = +0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
@@ -77,23 +91,42 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// arrive on `bar` when every cp.async issued so far by this thread has landed
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
 }
 
-// OR-reduction + barrier over the producer threads (named barrier 1)
-__device__ __forceinline__ bool producers_sync_or(bool v) {
+__device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 96, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v)
-      : "memory");
-  return r != 0;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Bulk copy of `bytes` from this CTA's shared memory to the same-offset
+// layout in CTA `rank` of the cluster, completion counted on that CTA's
+// mbarrier (both given as this CTA's addresses, mapped with mapa).
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_local, uint32_t src_local, uint32_t bytes,
+                                                  uint64_t* bar_local, int rank) {
+  uint32_t dst, bar;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(dst) : "r"(dst_local), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(bar) : "r"(smem_u32(bar_local)), "r"(rank));
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(src_local), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// A wait whose outcome is the same for every lane of the warp (lane 0 waits,
+// the result is broadcast), so that a wait that gives up never splits a warp
+// that is about to execute warp-collective instructions.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, kWaitLimitNs);
+  return __shfl_sync(0xffffffffu, ok, 0);
 }
 
 struct RowMap {
@@ -118,44 +151,68 @@ __device__ __forceinline__ RowMap map_row(const AttnArgs& a, int b, int g, int r
   return m;
 }
 
+// row of Q (as a 2-D [rows, d] tensor) holding query row r of (b, g)
+__device__ __forceinline__ int q_row(const AttnArgs& a, int b, int g, int r) {
+  const int h = g * a.G + r % a.G;
+  return a.prefill ? (r / a.G) * a.Hq + h : ((r / a.G) * a.B + b) * a.Hq + h;
+}
+
 struct KeySrc {
-  const uint16_t* Kb;
-  const uint16_t* Vb;
-  int len;     // decode: seq_len[b]
-  int base;    // prefill: kv_indptr[g]
+  int len;   // decode: seq_len[b]
+  int base;  // prefill: kv_indptr[g]
   int kbeg, kend;
 };
 
-// position of list entry jj, or -1 when the entry is padding / invalid
-__device__ __forceinline__ int key_at(const AttnArgs& a, const KeySrc& ks, int b, int jj) {
+// Raw list entry jj (a token index in decode, a block id in prefill), loaded
+// without looking at it so that several loads can be in flight; -1 past the
+// split's end.  key_fix turns it into a key position, or -1 when the entry is
+// padding / invalid (an index past the sequence is reported and skipped).
+__device__ __forceinline__ int key_raw(const AttnArgs& a, const KeySrc& ks, int b, int jj) {
   if (jj >= ks.kend) return -1;
+  return a.prefill ? __ldg(&a.kv_indices[ks.base + jj / a.block]) : __ldg(&a.idx[(int64_t)b * a.k + jj]);
+}
+
+__device__ __forceinline__ int key_fix(const AttnArgs& a, const KeySrc& ks, int b, int jj, int raw, bool rep) {
+  if (jj >= ks.kend || raw < 0) return -1;
   if (!a.prefill) {
-    const int t = a.idx[(int64_t)b * a.k + jj];
-    if (t >= ks.len) {
-      report(a.status, kErrDevice, kKernAttn, (int64_t)b * a.k + jj, t, ks.len);
+    if (raw >= ks.len) {
+      if (rep) report(a.status, kErrDevice, kKernAttn, (int64_t)b * a.k + jj, raw, ks.len);
       return -1;
     }
-    return t < 0 ? -1 : t;
+    return raw;
   }
-  const int blk = a.kv_indices[ks.base + jj / a.block];
-  const int t = blk * a.block + jj % a.block;
-  return (blk >= 0 && t < a.S) ? t : -1;
+  const int t = raw * a.block + jj % a.block;
+  return t < a.S ? t : -1;
+}
+
+// n (a multiple of 4) output values of one row, at element offset off of O
+__device__ __forceinline__ void store_out(const AttnArgs& a, int64_t off, const float* f, int n) {
+  if (a.out_f32) {
+    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.O) + off);
+    for (int e = 0; e < n / 4; ++e) o[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+  } else {
+    uint2* o = reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.O) + off);
+    for (int e = 0; e < n / 4; ++e) o[e] = make_uint2(pack_bf16(f[4 * e], f[4 * e + 1]), pack_bf16(f[4 * e + 2], f[4 * e + 3]));
+  }
 }
 
 template <bool PRECISE>
-__global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kAttnThreads, 1)
+sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v) {
   using Lay = AttnLayout<PRECISE>;
   constexpr int ST = Lay::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  int* kpos = reinterpret_cast<int*>(smem + Lay::kKposOff);
+  uint32_t* kmask = reinterpret_cast<uint32_t*>(smem + Lay::kMaskOff);  // [ST][8]
   uint64_t* kv_full = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
   uint64_t* kv_empty = kv_full + ST;
   uint64_t* s_full = kv_empty + ST;
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 2;
+  uint64_t* o_done = p_full + 2;  // [4]: completion of PV_i on o_done[i % 4]
+  uint64_t* recv_bar = o_done + 4;
   uint32_t* slot = reinterpret_cast<uint32_t*>(smem + Lay::kSlotOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -170,26 +227,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const Attn
   int n_keys;
   if (!a.prefill) {
     ks.len = a.seq_len[b];
-    const int64_t base = (a.seq_off[b] * a.Hkv + (int64_t)g * ks.len) * kD;
-    ks.Kb = a.K + base;
-    ks.Vb = a.V + base;
     ks.base = 0;
     n_keys = a.k;
   } else {
     ks.len = a.S;
     ks.base = a.kv_indptr[g];
     n_keys = (a.kv_indptr[g + 1] - ks.base) * a.block;
-    ks.Kb = a.K + (int64_t)g * a.S * kD;
-    ks.Vb = a.V + (int64_t)g * a.S * kD;
   }
   ks.kbeg = split * a.keys_per_split;
   ks.kend = min(n_keys, ks.kbeg + a.keys_per_split);
   const int nt = ks.kend > ks.kbeg ? (ks.kend - ks.kbeg + kKT - 1) / kKT : 0;
 
+  // producer lanes: raw entries of tile rows 4*lane .. 4*lane+3, one tile ahead
+  int raw_next[4];
+  if (warp >= kProdWarp0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) raw_next[i] = key_raw(a, ks, b, ks.kbeg + 4 * lane + i);
+  }
   if (warp == kMmaWarp) tmem_alloc(slot, 512);
   if (tid == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
     for (int s = 0; s < ST; ++s) {
-      mbar_init(&kv_full[s], 2 * kProdThreads);  // cp.async completions + plain arrivals
+      mbar_init(&kv_full[s], 3);  // one arrival (with its byte count) per producer warp
       mbar_init(&kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -197,52 +258,91 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const Attn
       mbar_init(&s_free[i], kSoftWarps);
       mbar_init(&p_full[i], kSoftWarps);
     }
-    mbar_init(o_done, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&o_done[i], 1);
+    mbar_init(recv_bar, 1);
     fence_mbar_init();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
-  const uint32_t tmem_o = tmem + 256;
+
+  // softmax state: thread (row r, key half h)
+  const int half = (warp >> 2) & 1;
+  const int r_loc = (warp & 3) * 32 + lane;
+  const RowMap me = map_row(a, b, g, mt * 128 + r_loc);
+  const bool warp_active = warp < kSoftWarps && mt * 128 + (warp & 3) * 32 < a.R;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t tmem_oh = tmem + 256 + 128 * half;  // this half's O accumulator
+  float m_ref = -INFINITY, l_run = 0.f;
+  bool have_o = false;
 
   if (warp >= kProdWarp0) {
-    // ======================= producers: gather K/V rows =======================
-    const int pt = tid - kProdWarp0 * 32;
-    const int cchunk = pt & 15, crow0 = pt >> 4;  // rows crow0, crow0 + 6, ...
+    // =============== producer warps: TMA gathers of K/V (and Q) rows ===============
+    // warp 9: K columns 0-63 and V columns 64-127 (+ validity words);
+    // warp 10: K columns 64-127 (+ Q columns 0-63 on the first tile);
+    // warp 11: V columns 0-63 (+ Q columns 64-127 on the first tile).
+    const int pw = warp - kProdWarp0;
+    const int64_t row_base = a.prefill ? (int64_t)g * a.S : a.seq_off[b] * a.Hkv + (int64_t)g * ks.len;
     for (int j = 0; j < nt; ++j) {
       const int s = j % ST;
-      bool bad = false;
-      if (j >= ST) bad = !mbar_wait(&kv_empty[s], ((j / ST) & 1) ^ 1, kWaitLimitNs);
-      for (int r = pt; r < kKT; r += kProdThreads) kpos[s * kKT + r] = bad ? -1 : key_at(a, ks, b, ks.kbeg + j * kKT + r);
-      if (producers_sync_or(bad)) {
-        if (pt == 0) report(a.status, kErrTimeout, kKernAttn, u, 0, j);
+      int tc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tc[i] = key_fix(a, ks, b, ks.kbeg + j * kKT + 4 * lane + i, raw_next[i], pw == 0);
+      if (j + 1 < nt) {  // next tile's entries: loads in flight while this tile is issued
+#pragma unroll
+        for (int i = 0; i < 4; ++i) raw_next[i] = key_raw(a, ks, b, ks.kbeg + (j + 1) * kKT + 4 * lane + i);
+      }
+      bool ok = true;
+      if (j >= ST && lane == 0) ok = mbar_wait(&kv_empty[s], ((j / ST) & 1) ^ 1, kWaitLimitNs);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 0, j);
         break;
       }
-      if (j == 0) {
-#pragma unroll 4
-        for (int rr = crow0; rr < 128; rr += 6) {
-          const RowMap rm = map_row(a, b, g, mt * 128 + rr);
-          const uint32_t dst = sbase + Lay::kQOff + (cchunk >> 3) * Lay::kHalf + sw128_offset(rr, cchunk & 7);
-          cp_async_16(dst, rm.valid ? (const void*)(a.Q + rm.qoff + cchunk * 8) : (const void*)a.Q,
-                      rm.valid ? 16u : 0u);
+      if (pw == 0) {
+        // validity words (keys 32w..32w+31 are entries 4l+i of lanes 8w..8w+7)
+        // and the position of each word's first key
+        uint32_t bal[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bal[i] = __ballot_sync(0xffffffffu, tc[i] >= 0);
+        if (lane < 4) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int l8 = 0; l8 < 8; ++l8)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) word |= ((bal[i] >> (8 * lane + l8)) & 1u) << (4 * l8 + i);
+          kmask[s * 8 + lane] = word;
         }
+        if ((lane & 7) == 0) kmask[s * 8 + 4 + (lane >> 3)] = (uint32_t)tc[0];
+        __syncwarp();
       }
-      const uint32_t kdst = sbase + Lay::kStageOff + s * Lay::kStageBytes;
-      const uint32_t vdst = kdst + Lay::kTile;
-#pragma unroll 4
-      for (int rr = crow0; rr < 128; rr += 6) {
-        const int t = kpos[s * kKT + rr];
-        const uint32_t off = (cchunk >> 3) * Lay::kHalf + sw128_offset(rr, cchunk & 7);
-        const int64_t e = (int64_t)(t < 0 ? 0 : t) * kD + cchunk * 8;
-        const uint32_t nb = t < 0 ? 0u : 16u;
-        cp_async_16(kdst + off, ks.Kb + e, nb);
-        cp_async_16(vdst + off, ks.Vb + e, nb);
+      const uint32_t tx = (pw == 0 ? 2 * Lay::kHalf : Lay::kHalf) + (j == 0 && pw > 0 ? Lay::kHalf : 0);
+      if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx);
+      __syncwarp();
+      int rk[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) rk[i] = (int)(row_base + (tc[i] < 0 ? 0 : tc[i]));
+      const uint32_t kst = sbase + Lay::kStageOff + s * Lay::kStageBytes + 4 * lane * 128;
+      const uint32_t vst = kst + Lay::kTile;
+      if (pw == 0) {
+        tma_gather4(kst, &tm_k, &kv_full[s], 0, rk);
+        tma_gather4(vst + Lay::kHalf, &tm_v, &kv_full[s], 64, rk);
+      } else if (pw == 1) {
+        tma_gather4(kst + Lay::kHalf, &tm_k, &kv_full[s], 64, rk);
+      } else {
+        tma_gather4(vst, &tm_v, &kv_full[s], 0, rk);
       }
-      cp_async_mbar_arrive(&kv_full[s]);
-      mbar_arrive(&kv_full[s]);
+      if (j == 0 && pw > 0) {
+        int rq[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = mt * 128 + 4 * lane + i;
+          rq[i] = q_row(a, b, g, r < a.R ? r : mt * 128);
+        }
+        tma_gather4(sbase + Lay::kQOff + (pw - 1) * Lay::kHalf + 4 * lane * 128, &tm_q, &kv_full[0], (pw - 1) * 64,
+                    rq);
+      }
     }
-    cp_async_wait<0>();
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
@@ -251,21 +351,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const Attn
       auto pv = [&](int i) -> bool {
         if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, kWaitLimitNs)) return false;
         tc_fence_after();
-        const uint32_t kst = sbase + Lay::kStageOff + (i % ST) * Lay::kStageBytes;
+        const uint32_t kst = sbase + Lay::kStageOff + (i % ST) * Lay::kStageBytes;  // P lives here now
         const uint32_t vst = kst + Lay::kTile;
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16) {
-          const uint64_t vd = umma_desc_sw128(vst + k16 * 2048, Lay::kHalf, 1024);
-          umma_bf16(tmem_o, umma_desc_sw128(kst + (k16 >> 2) * Lay::kHalf + (k16 & 3) * 32, 16, 1024), vd,
-                    idesc_pv, (i | k16) != 0);
-          if constexpr (PRECISE)
-            umma_bf16(tmem_o,
-                      umma_desc_sw128(sbase + Lay::kPloOff + (i & 1) * Lay::kTile + (k16 >> 2) * Lay::kHalf +
-                                          (k16 & 3) * 32, 16, 1024),
-                      vd, idesc_pv, 1);
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // keys 64h + 16kk .. +15
+            const uint64_t vd = umma_desc_sw128(vst + h * 8192 + kk * 2048, Lay::kHalf, 1024);
+            umma_bf16(tmem + 256 + 128 * h, umma_desc_sw128(kst + h * Lay::kHalf + kk * 32, 16, 1024), vd, idesc_pv,
+                      (i | kk) != 0);
+            if constexpr (PRECISE)
+              umma_bf16(tmem + 256 + 128 * h,
+                        umma_desc_sw128(sbase + Lay::kPloOff + (i & 1) * Lay::kTile + h * Lay::kHalf + kk * 32, 16,
+                                        1024),
+                        vd, idesc_pv, 1);
+          }
         }
         umma_commit(&kv_empty[i % ST]);
-        umma_commit(o_done);
+        umma_commit(&o_done[i & 3]);
         return true;
       };
       bool ok = true;
@@ -289,81 +392,93 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const Attn
       if (!ok) report(a.status, kErrTimeout, kKernAttn, u, 1, 0);
     }
   } else {
-    // ======================= softmax rows (warps 0-3) =======================
-    const RowMap me = map_row(a, b, g, mt * 128 + tid);
-    const bool warp_active = mt * 128 + warp * 32 < a.R;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float m_ref = -INFINITY, l_run = 0.f;
+    // ======================= softmax (warps 0-7) =======================
     bool failed = false;
     for (int j = 0; j < nt; ++j) {
       const int s = j % ST, sb = j & 1;
-      if (!mbar_wait(&s_full[sb], (j >> 1) & 1, kWaitLimitNs)) { failed = true; break; }
+      if (!warp_wait(&s_full[sb], (j >> 1) & 1)) { failed = true; break; }
       tc_fence_after();
-      uint32_t sv[kKT];
       if (warp_active) {
+        if (!warp_wait(&kv_full[s], (j / ST) & 1)) { failed = true; break; }
+        // keys of this half this row may see: the real ones, and in prefill
+        // those at or before the row's position (positions are consecutive
+        // inside a 32-key word)
+        uint32_t vis[2];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + sb * 128 + lane_base + c * 32, &sv[c * 32]);
-        tmem_wait_ld();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      if (warp_active) {
-        if (!mbar_wait(&kv_full[s], (j / ST) & 1, kWaitLimitNs) ||
-            (j >= 1 && !mbar_wait(o_done, (j - 1) & 1, kWaitLimitNs))) { failed = true; break; }
-        const int* kp = kpos + s * kKT;
-        float tmax = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < kKT; ++c) {
-          const int t = kp[c];
-          const bool vis = me.valid && t >= 0 && t <= me.limit;
-          const float x = vis ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
-          sv[c] = __float_as_uint(x);
-          tmax = fmaxf(tmax, x);
+        for (int w2 = 0; w2 < 2; ++w2) {
+          uint32_t v = me.valid ? kmask[s * 8 + 2 * half + w2] : 0u;
+          if (a.prefill && v) {
+            const int first = (int)kmask[s * 8 + 4 + 2 * half + w2];
+            const int room = me.limit - first;  // keys first..first+room are visible
+            v &= room >= 31 ? 0xffffffffu : (room < 0 ? 0u : ((2u << room) - 1u));
+          }
+          vis[w2] = v;
         }
+        const bool all_vis = (vis[0] & vis[1]) == 0xffffffffu;
+        uint32_t sv[64];
+        tmem_ld32(tmem + sb * 128 + 64 * half + lane_base, sv);
+        tmem_ld32(tmem + sb * 128 + 64 * half + 32 + lane_base, sv + 32);
+        tmem_wait_ld();
+        float tmax = -INFINITY;
+        if (all_vis) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) tmax = fmaxf(tmax, __uint_as_float(sv[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if ((vis[e >> 5] >> (e & 31)) & 1u) tmax = fmaxf(tmax, __uint_as_float(sv[e]));
+        }
+        tmax *= a.scale_log2;
         float alpha = 1.f;
         bool rescale = false;
         if (j == 0) {
           m_ref = tmax;
         } else if (tmax > m_ref + 8.f) {
-          alpha = exp2f(m_ref - tmax);
+          alpha = ex2_approx(m_ref - tmax);
           m_ref = tmax;
           rescale = true;
         }
         l_run *= alpha;
         if (__any_sync(0xffffffffu, rescale)) {
+          // O_h is about to be rescaled: the previous tile's PV must have landed.
+          // (Its P_lo buffer is never rewritten before then either: PV_{j-2}
+          // precedes S_j in the in-order tensor pipe.)
+          if (!warp_wait(&o_done[(j - 1) & 3], ((j - 1) >> 2) & 1)) { failed = true; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t ov[32];
-            tmem_ld32(tmem_o + lane_base + c * 32, ov);
+            tmem_ld32(tmem_oh + lane_base + c * 32, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tmem_o + lane_base + c * 32, ov);
+            tmem_st32(tmem_oh + lane_base + c * 32, ov);
           }
           tmem_wait_st();
         }
-        const float mr = (m_ref == -INFINITY) ? 0.f : m_ref;
-        const uint32_t kst = sbase + Lay::kStageOff + s * Lay::kStageBytes;  // P overwrites the used K tile
+        // p = 2^(s*scale*log2e - m_ref), bf16, over this half of the used K tile
+        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        const uint32_t pst = sbase + Lay::kStageOff + s * Lay::kStageBytes + half * Lay::kHalf;
         float lsum = 0.f;
 #pragma unroll
-        for (int c16 = 0; c16 < 16; ++c16) {
+        for (int c16 = 0; c16 < 8; ++c16) {
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            p[e] = exp2f(__uint_as_float(sv[c16 * 8 + e]) - mr);
+            const int col = c16 * 8 + e;
+            p[e] = ex2_approx(fmaf(__uint_as_float(sv[col]), a.scale_log2, neg_m));
+            if (!all_vis && !((vis[col >> 5] >> (col & 31)) & 1u)) p[e] = 0.f;
             lsum += p[e];
           }
-          const uint32_t off = (c16 >> 3) * Lay::kHalf + sw128_offset(tid, c16 & 7);
-          st_shared_v4(kst + off, pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]),
+          const uint32_t off = sw128_offset(r_loc, c16);
+          st_shared_v4(pst + off, pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]),
                        pack_bf16(p[6], p[7]));
           if constexpr (PRECISE) {
             float q[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) q[e] = p[e] - bf16_round(p[e]);
-            st_shared_v4(sbase + Lay::kPloOff + sb * Lay::kTile + off, pack_bf16(q[0], q[1]), pack_bf16(q[2], q[3]),
-                         pack_bf16(q[4], q[5]), pack_bf16(q[6], q[7]));
+            st_shared_v4(sbase + Lay::kPloOff + sb * Lay::kTile + half * Lay::kHalf + off, pack_bf16(q[0], q[1]),
+                         pack_bf16(q[2], q[3]), pack_bf16(q[4], q[5]), pack_bf16(q[6], q[7]));
           }
         }
         l_run += lsum;
@@ -371,56 +486,163 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const Attn
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
+      if (lane == 0) {
+        mbar_arrive(&s_free[sb]);
+        mbar_arrive(&p_full[sb]);
+      }
     }
     if (failed) {
       if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 2, warp);
     } else if (warp_active) {
-      if (nt > 0 && !mbar_wait(o_done, (nt - 1) & 1, kWaitLimitNs)) {
+      if (nt > 0 && !warp_wait(&o_done[(nt - 1) & 3], ((nt - 1) >> 2) & 1)) {
         if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 3, warp);
       } else {
-        tc_fence_after();
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        const int units = gridDim.x;
+        have_o = true;
+      }
+    }
+  }
+
+  // ======================= output: all threads =======================
+  tc_fence_before();
+  __syncthreads();  // every MMA has completed (o_done) and no stage is in use
+  tc_fence_after();
+  // the two key halves of each row: (m, l) of both, merged per row
+  float2* mlx = reinterpret_cast<float2*>(smem + Lay::kStageOff + kMlxOff);  // [2][128]
+  if (warp < kSoftWarps)
+    mlx[half * 128 + r_loc] = (warp_active && have_o && me.valid) ? make_float2(m_ref, l_run)
+                                                                 : make_float2(-INFINITY, 0.f);
+  __syncthreads();
+  float f0 = 0.f, f1 = 0.f, l_row = 0.f, m_row = -INFINITY;
+  if (warp < kSoftWarps) {
+    const float2 h0 = mlx[r_loc], h1 = mlx[128 + r_loc];
+    m_row = fmaxf(h0.x, h1.x);
+    if (m_row != -INFINITY) {
+      f0 = ex2_approx(h0.x - m_row);
+      f1 = ex2_approx(h1.x - m_row);
+      l_row = f0 * h0.y + f1 * h1.y;
+    }
+  }
+  // this thread's 64 output columns of the row: f0 O0 + f1 O1 (unnormalised)
+  auto row_out = [&](int c2, float* f) {  // columns 64*half + 32*c2 .. +31
+    uint32_t o0[32], o1[32];
+    tmem_ld32(tmem + 256 + lane_base + 64 * half + 32 * c2, o0);
+    tmem_ld32(tmem + 384 + lane_base + 64 * half + 32 * c2, o1);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) f[e] = f0 * __uint_as_float(o0[e]) + f1 * __uint_as_float(o1[e]);
+  };
+  if (a.n_split == 1) {
+    if (warp_active && have_o) {
+      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {  // 32 output columns at a time
-          uint32_t ov[32];
-          if (nt > 0) {
-            tmem_ld32(tmem_o + lane_base + c * 32, ov);
-            tmem_wait_ld();
-          } else {
+      for (int c2 = 0; c2 < 2; ++c2) {
+        float f[32];
+        if (nt > 0) {
+          row_out(c2, f);
+        } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = 0u;
-          }
-          if (!me.valid) continue;
-          if (a.n_split == 1) {
-            if (a.out_f32) {
-              float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.O) + me.qoff + c * 32);
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                o[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
-                                   __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
-            } else {
-              uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.O) + me.qoff + c * 32);
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                o[e] = make_uint4(pack_bf16(__uint_as_float(ov[8 * e]) * inv, __uint_as_float(ov[8 * e + 1]) * inv),
-                                  pack_bf16(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv),
-                                  pack_bf16(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv),
-                                  pack_bf16(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv));
-            }
-          } else {
-            uint4* po = reinterpret_cast<uint4*>(a.part + ((int64_t)u * 128 + tid) * kD + c * 32);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) po[e] = make_uint4(ov[4 * e], ov[4 * e + 1], ov[4 * e + 2], ov[4 * e + 3]);
-          }
+          for (int e = 0; e < 32; ++e) f[e] = 0.f;
         }
-        if (me.valid && a.n_split > 1) {
-          float2* pml = reinterpret_cast<float2*>(a.part + (int64_t)units * 128 * kD) + (int64_t)u * 128 + tid;
-          *pml = make_float2(m_ref, l_run);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] *= inv;
+        if (me.valid) store_out(a, me.qoff + 64 * half + 32 * c2, f, 32);
+      }
+    }
+  } else {
+    // Key splits of this row tile form one cluster.  Output slice t (128 /
+    // n_split columns) is merged by CTA t: every CTA stages, per slice, its
+    // unnormalised rows and (m, l) in its own shared memory, then one bulk
+    // copy per peer moves the slice into that peer's receive slot, completion
+    // counted in bytes on the peer's mbarrier.
+    const int ns = a.n_split;
+    const int rank = (int)cluster_rank();
+    const int cw = 32 / ns;                        // 16-byte chunks per slice row
+    // chunk c of row r sits at chunk c ^ swz(r): one row per lane would
+    // otherwise put all 32 lanes' 16-byte accesses in the same banks
+    const int swz = r_loc & (cw >= 8 ? 7 : cw - 1);
+    const uint32_t slot_bytes = 128u * (16u * cw + 8u);  // [128][cw] chunks + [128] (m, l)
+    const uint32_t recv = sbase + Lay::kStageOff;                      // [ns] slots, slot s from CTA s
+    const uint32_t send = recv + ((ns * slot_bytes + 1023u) & ~1023u);  // [ns] slots, slot t for CTA t
+    if (tid == 0) mbar_arrive_expect_tx(recv_bar, (uint32_t)(ns - 1) * slot_bytes);
+    cluster_sync();  // every CTA is done with its stages and has armed its receive barrier
+    if (warp_active) {
+      const bool live = have_o && me.valid;
+      if (half == 0)
+        for (int t = 0; t < ns; ++t)
+          *reinterpret_cast<float2*>(smem + (send - sbase) + t * slot_bytes + 128u * 16u * cw + r_loc * 8u) =
+              make_float2(live ? m_row : -INFINITY, live ? l_row : 0.f);
+#pragma unroll 1
+      for (int c2 = 0; c2 < 2; ++c2) {
+        float f[32];
+        if (have_o && nt > 0) {  // warp-uniform: TMEM loads are warp-collective
+          row_out(c2, f);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) f[e] = 0.f;
+        }
+        if (!live) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) f[e] = 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int chunk = 16 * half + 8 * c2 + q;  // 16-byte chunk of the 512-byte row
+          const int owner = chunk / cw;
+          st_shared_v4(send + owner * slot_bytes + (uint32_t)((r_loc * cw + ((chunk - owner * cw) ^ swz)) * 16),
+                       __float_as_uint(f[4 * q]), __float_as_uint(f[4 * q + 1]), __float_as_uint(f[4 * q + 2]),
+                       __float_as_uint(f[4 * q + 3]));
         }
       }
     }
+    fence_proxy_async_smem();  // the staged slices are read by the bulk copies (async proxy)
+    __syncthreads();
+    if (warp == kMmaWarp && lane < ns && lane != rank)
+      bulk_copy_to_peer(recv + rank * slot_bytes, send + lane * slot_bytes, slot_bytes, recv_bar, lane);
+    bool got = true;
+    if (warp < kSoftWarps) got = warp_wait(recv_bar, 0);
+    if (!got && lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 4, warp);
+    if (warp_active && me.valid && got) {
+      const uint8_t* base = smem + (recv - sbase);
+      const uint8_t* own = smem + (send - sbase) + rank * slot_bytes;
+      float M = -INFINITY;
+      float2 mls[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (t < ns) {
+          const uint8_t* sl = (t == rank ? own : base + t * slot_bytes);
+          mls[t] = *reinterpret_cast<const float2*>(sl + 128u * 16u * cw + r_loc * 8u);
+          M = fmaxf(M, mls[t].x);
+        }
+      }
+      float wt[8], L = 0.f;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        wt[t] = 0.f;
+        if (t < ns && M != -INFINITY) {
+          wt[t] = ex2_approx(mls[t].x - M);
+          L += wt[t] * mls[t].y;
+        }
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      // the slice's chunks, split between the row's two threads
+      const int per = cw / 2 > 0 ? cw / 2 : 1;
+      for (int ci = half * per; ci < (half + 1) * per && ci < cw; ++ci) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (t >= ns) break;
+          const uint32_t sl = (t == rank ? send + rank * slot_bytes : recv + t * slot_bytes);
+          const float4 v = ld_shared_f4(sl + (uint32_t)((r_loc * cw + (ci ^ swz)) * 16));
+          acc.x += wt[t] * v.x;
+          acc.y += wt[t] * v.y;
+          acc.z += wt[t] * v.z;
+          acc.w += wt[t] * v.w;
+        }
+        const float f[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+        store_out(a, me.qoff + (rank * cw + ci) * 4, f, 4);
+      }
+    }
+    cluster_sync();  // every bulk copy out of this CTA has been consumed
   }
 
   tc_fence_before();
@@ -431,48 +653,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const Attn
   }
 }
 
-// Merge the key-split partials of one output row per warp:
-//   o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
-__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnArgs a, int units) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int n_bg = a.prefill ? a.Hkv : a.B * a.Hkv;
-  if (warp >= n_bg * a.R) return;
-  const int bg = warp / a.R, r = warp % a.R;
-  const int b = a.prefill ? 0 : bg / a.Hkv;
-  const int g = a.prefill ? bg : bg % a.Hkv;
-  const int mt = r / 128, lr = r % 128;
-  const float2* ml = reinterpret_cast<const float2*>(a.part + (int64_t)units * 128 * kD);
-  float M = -INFINITY;
-  for (int s = 0; s < a.n_split; ++s) {
-    const int uu = (bg * a.n_mtiles + mt) * a.n_split + s;
-    M = fmaxf(M, ml[(int64_t)uu * 128 + lr].x);
-  }
-  const float Mr = (M == -INFINITY) ? 0.f : M;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lsum = 0.f;
-  for (int s = 0; s < a.n_split; ++s) {
-    const int uu = (bg * a.n_mtiles + mt) * a.n_split + s;
-    const float2 v = ml[(int64_t)uu * 128 + lr];
-    const float wgt = exp2f(v.x - Mr);
-    lsum += wgt * v.y;
-    const float4 o = reinterpret_cast<const float4*>(a.part + ((int64_t)uu * 128 + lr) * kD)[lane];
-    acc.x += wgt * o.x;
-    acc.y += wgt * o.y;
-    acc.z += wgt * o.z;
-    acc.w += wgt * o.w;
-  }
-  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-  const RowMap rm = map_row(a, b, g, r);
-  if (a.out_f32) {
-    reinterpret_cast<float4*>(reinterpret_cast<float*>(a.O) + rm.qoff)[lane] =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  } else {
-    reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.O) + rm.qoff)[lane] =
-        make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
-  }
-}
-
 }  // namespace
 
 int attn_num_units(const AttnArgs& a) {
@@ -480,29 +660,29 @@ int attn_num_units(const AttnArgs& a) {
   return n_bg * a.n_mtiles * a.n_split;
 }
 
-size_t attn_partial_bytes(int units) { return (size_t)units * 128 * (kD + 2) * sizeof(float); }
-
-cudaError_t launch_sparse_attn(const AttnArgs& a, bool precise_p, cudaStream_t stream) {
+cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                               const CUtensorMap& tm_v, bool precise_p, cudaStream_t stream) {
   const int units = attn_num_units(a);
   if (units == 0) return cudaSuccess;
-  cudaError_t e;
-  if (precise_p) {
-    auto kern = sparse_attn_kernel<true>;
-    e = ensure_smem(kern, AttnLayout<true>::kSmem);
-    if (e != cudaSuccess) return e;
-    kern<<<units, kAttnThreads, AttnLayout<true>::kSmem, stream>>>(a);
-  } else {
-    auto kern = sparse_attn_kernel<false>;
-    e = ensure_smem(kern, AttnLayout<false>::kSmem);
-    if (e != cudaSuccess) return e;
-    kern<<<units, kAttnThreads, AttnLayout<false>::kSmem, stream>>>(a);
-  }
-  e = cudaGetLastError();
-  if (e != cudaSuccess || a.n_split == 1) return e;
-  const int n_bg = a.prefill ? a.Hkv : a.B * a.Hkv;
-  const int64_t rows = (int64_t)n_bg * a.R;
-  const int blocks = (int)((rows * 32 + 255) / 256);
-  attn_combine_kernel<<<blocks, 256, 0, stream>>>(a, units);
+  if (a.n_split != 1 && a.n_split != 2 && a.n_split != 4 && a.n_split != 8) return cudaErrorInvalidValue;
+  auto kern = precise_p ? sparse_attn_kernel<true> : sparse_attn_kernel<false>;
+  const size_t smem = precise_p ? AttnLayout<true>::kSmem : AttnLayout<false>::kSmem;
+  cudaError_t e = ensure_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(units);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.n_split;  // the key splits of one row tile share a cluster
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, a, tm_q, tm_k, tm_v);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

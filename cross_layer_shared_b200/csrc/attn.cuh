@@ -1,6 +1,7 @@
 // Launch interface of the sparse attention kernels (internal to libsa).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,17 +37,18 @@ struct AttnArgs {
   int G;       // Hq / Hkv
   int R;       // query rows per (b, g): L*G (decode) or Nq*G (prefill)
   int n_mtiles;
-  int n_split;
+  int n_split;         // 1, 2, 4 or 8: the splits of a row tile form one cluster
   int keys_per_split;  // multiple of 128
   float scale_log2;    // softmax scale * log2(e)
   void* O;
   int out_f32;
-  float* part;  // [units][128][d + 2] partial (O, m, l) when n_split > 1
   DeviceStatus* status;
 };
 
 int attn_num_units(const AttnArgs& a);
-size_t attn_partial_bytes(int units);
-cudaError_t launch_sparse_attn(const AttnArgs& a, bool precise_p, cudaStream_t stream);
+// tm_q / tm_k / tm_v: Q, K, V as 2-D [rows, 128] bf16 tensors, box 64 x 1,
+// 128-byte swizzle (rows gathered four at a time).
+cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                               const CUtensorMap& tm_v, bool precise_p, cudaStream_t stream);
 
 }  // namespace sa

@@ -184,8 +184,10 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
     for (int j = 0; j < NPAD; ++j) wr[j] = 0.f;
     for (int g = blockIdx.x; g < total; g += gridDim.x, ++i) {
       const int a = i % kAcc;
-      if (!mbar_wait(&tfull[a], (i / kAcc) & 1, kWaitLimitNs)) {
-        report(status, kErrTimeout, kKernIndexer, blockIdx.x, 2, i);
+      bool ok = true;  // lane 0 waits for the warp, so a give-up never splits it
+      if (lane == 0) ok = mbar_wait(&tfull[a], (i / kAcc) & 1, kWaitLimitNs);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) report(status, kErrTimeout, kKernIndexer, blockIdx.x, 2, i);
         break;
       }
       tc_fence_after();

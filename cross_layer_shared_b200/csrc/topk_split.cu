@@ -176,14 +176,27 @@ __device__ uint32_t radix_desc(int nc, Val val, Pred pred, uint32_t prefix, uint
   return prefix;
 }
 
+constexpr int kGroups = 8;            // 32-key groups per warp per chunk pass (registers)
+constexpr int kCandSmem = 6144;       // candidates refined in shared memory
+constexpr int kWordsSmem = 4096;      // bitmap words staged in shared memory (rows <= 131072)
+
+struct SelectSmem {
+  uint2 cand[kCandSmem];
+  uint32_t words[kWordsSmem];
+  uint32_t hist[2048];
+  int ws[kWarps + 1];
+  int warp_cnt[kWarps];
+  int cta_base;
+  int last, bin, before;
+};
+
 __global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __restrict__ scores, int64_t ld, int k,
                                                                int chunk, RowState* __restrict__ st,
                                                                uint32_t* __restrict__ bitmap, int wpr,
                                                                uint2* __restrict__ cand, int cap,
                                                                int32_t* __restrict__ idx, float* __restrict__ top_scores) {
-  __shared__ uint32_t sh[2048];
-  __shared__ int ws[kWarps + 1];
-  __shared__ int s_last, s_bin, s_before;
+  extern __shared__ uint8_t smem_raw[];
+  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
   const int q = blockIdx.y, c = blockIdx.x, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int beta = __ldcg(&st[q].beta), above = __ldcg(&st[q].above), n = __ldcg(&st[q].n);
@@ -191,66 +204,101 @@ __global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __re
   uint32_t* bm = bitmap + (int64_t)q * wpr;
   uint2* cq = cand + (int64_t)q * cap;
 
+  // ---- this CTA's chunk: selected-bit words and threshold-bucket candidates ----
   const int beg = c * chunk, end = min(n, beg + chunk);
-  for (int base = beg + warp * 32; base < end; base += kWarps * 32) {
-    const int i = base + lane;
-    const bool in = i < end;
-    const uint32_t key = in ? order_key(row[i]) : 0u;
-    const int d = (int)(key >> 20);
-    const bool sel = in && (beta < 0 || d > beta);
-    const bool eq = in && beta >= 0 && d == beta;
-    const uint32_t word = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) bm[base >> 5] = word;
-    const uint32_t m = __ballot_sync(0xffffffffu, eq);
-    if (m) {
-      int b0 = 0;
-      if (lane == 0) b0 = atomicAdd(&st[q].ncand, __popc(m));
-      b0 = __shfl_sync(0xffffffffu, b0, 0);
-      if (eq) {
-        const int pos = b0 + __popc(m & ((1u << lane) - 1u));
-        if (pos < cap) cq[pos] = make_uint2(key, (uint32_t)i);
-      }
+  for (int base0 = beg; base0 < end; base0 += kThreads * kGroups) {
+    uint32_t key[kGroups];
+    uint32_t eqm[kGroups];
+    int my = 0;  // candidates of this warp in this pass
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int base = base0 + (gi * kWarps + warp) * 32;
+      const int i = base + lane;
+      const bool in = i < end;
+      key[gi] = in ? order_key(row[i]) : 0u;
+      const int d = (int)(key[gi] >> 20);
+      const bool sel = in && (beta < 0 || d > beta);
+      const bool eq = in && beta >= 0 && d == beta;
+      const uint32_t word = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0 && base < end) bm[base >> 5] = word;
+      eqm[gi] = __ballot_sync(0xffffffffu, eq);
+      my += __popc(eqm[gi]);
     }
+    if (lane == 0) sm.warp_cnt[warp] = my;
+    __syncthreads();
+    if (tid == 0) {
+      int tot = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        const int x = sm.warp_cnt[w];
+        sm.warp_cnt[w] = tot;
+        tot += x;
+      }
+      sm.cta_base = tot ? atomicAdd(&st[q].ncand, tot) : 0;  // one reservation per CTA
+    }
+    __syncthreads();
+    int pos = sm.cta_base + sm.warp_cnt[warp];
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int base = base0 + (gi * kWarps + warp) * 32;
+      if ((eqm[gi] >> lane) & 1u) {
+        const int p = pos + __popc(eqm[gi] & ((1u << lane) - 1u));
+        if (p < cap) cq[p] = make_uint2(key[gi], (uint32_t)(base + lane));
+      }
+      pos += __popc(eqm[gi]);
+    }
+    __syncthreads();
   }
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&st[q].ticket2, 1) == (int)gridDim.x - 1;
+  if (tid == 0) sm.last = atomicAdd(&st[q].ticket2, 1) == (int)gridDim.x - 1;
   __syncthreads();
-  if (!s_last) return;
+  if (!sm.last) return;
   __threadfence();
 
-  // ---- the row's last CTA: finish the select among the candidates -------
+  // ---- the row's last CTA ---------------------------------------------------
+  const int nw = (n + 31) >> 5;
+  const bool words_in_smem = nw <= kWordsSmem;
+  if (words_in_smem)
+    for (int w = tid; w < nw; w += kThreads) sm.words[w] = __ldcg(&bm[w]);
   if (beta >= 0) {
     int nc = __ldcg(&st[q].ncand);
     nc = nc < cap ? nc : cap;
+    const bool in_smem = nc <= kCandSmem;
+    if (in_smem)
+      for (int j = tid; j < nc; j += kThreads) sm.cand[j] = __ldcg(&cq[j]);
+    __syncthreads();
+    const uint2* cs = in_smem ? sm.cand : cq;
+    auto ckey = [&](int j) { return in_smem ? sm.cand[j].x : __ldcg(&cq[j].x); };
+    auto cidx = [&](int j) { return in_smem ? sm.cand[j].y : __ldcg(&cq[j].y); };
     int need = k - above;
     int n_eq = 0;
     const int ks[2] = {10, 0}, kw[2] = {10, 10};
-    const uint32_t T = radix_desc(
-        nc, [&](int j) { return __ldcg(&cq[j].x); }, [](int) { return true; }, (uint32_t)beta << 20, 0xFFF00000u,
-        ks, kw, 2, &need, &n_eq, sh, ws, &s_bin, &s_before);
+    const uint32_t T = radix_desc(nc, ckey, [](int) { return true; }, (uint32_t)beta << 20, 0xFFF00000u, ks, kw,
+                                  2, &need, &n_eq, sm.hist, sm.ws, &sm.bin, &sm.before);
     uint32_t cut = 0xFFFFFFFFu;
     if (need < n_eq) {
       // the `need` lowest indices among keys == T: largest values of ~index
       int need2 = need, n2 = 0;
       const int is[3] = {21, 10, 0}, iw[3] = {11, 11, 10};
-      const uint32_t V = radix_desc(
-          nc, [&](int j) { return ~__ldcg(&cq[j].y); }, [&](int j) { return __ldcg(&cq[j].x) == T; }, 0u, 0u, is,
-          iw, 3, &need2, &n2, sh, ws, &s_bin, &s_before);
+      const uint32_t V = radix_desc(nc, [&](int j) { return ~cidx(j); }, [&](int j) { return ckey(j) == T; }, 0u,
+                                    0u, is, iw, 3, &need2, &n2, sm.hist, sm.ws, &sm.bin, &sm.before);
       cut = ~V;
     }
+    (void)cs;
     for (int j = tid; j < nc; j += kThreads) {
-      const uint2 e = __ldcg(&cq[j]);
-      if (e.x > T || (e.x == T && e.y <= cut)) atomicOr(&bm[e.y >> 5], 1u << (e.y & 31));
+      const uint32_t kx = ckey(j), ix = cidx(j);
+      if (kx > T || (kx == T && ix <= cut)) {
+        if (words_in_smem) atomicOr(&sm.words[ix >> 5], 1u << (ix & 31));
+        else atomicOr(&bm[ix >> 5], 1u << (ix & 31));
+      }
     }
-    __threadfence();
-    __syncthreads();
+    if (!words_in_smem) __threadfence();
   }
+  __syncthreads();
 
   // ---- emit set bits in index order ----------------------------------------
   int32_t* out = idx + (int64_t)q * k;
   float* out_s = top_scores ? top_scores + (int64_t)q * k : nullptr;
-  const int nw = (n + 31) >> 5;
   constexpr int kWpt = 8;
   int written = 0;
   for (int w0 = 0; w0 < nw; w0 += kThreads * kWpt) {
@@ -259,12 +307,12 @@ __global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __re
 #pragma unroll
     for (int j = 0; j < kWpt; ++j) {
       const int wi = w0 + tid * kWpt + j;
-      wv[j] = wi < nw ? __ldcg(&bm[wi]) : 0u;
+      wv[j] = wi < nw ? (words_in_smem ? sm.words[wi] : __ldcg(&bm[wi])) : 0u;
       if (wi == nw - 1 && (n & 31)) wv[j] &= (1u << (n & 31)) - 1u;
       cnt += __popc(wv[j]);
     }
     int tot;
-    int pos = written + block_scan_excl(cnt, ws, &tot);
+    int pos = written + block_scan_excl(cnt, sm.ws, &tot);
 #pragma unroll
     for (int j = 0; j < kWpt; ++j) {
       uint32_t x = wv[j];
@@ -289,10 +337,11 @@ __global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __re
 }
 
 int chunk_for(int Nq, int n_max, int num_sms) {
-  // about four CTAs per SM over all rows, chunks a multiple of 32 keys
-  int64_t want = ((int64_t)Nq * n_max) / (4 * (int64_t)num_sms);
-  if (want < 2048) want = 2048;
-  want = (want + 31) / 32 * 32;
+  // about one CTA per SM over all rows; a multiple of one select pass
+  int64_t want = ((int64_t)Nq * n_max + num_sms - 1) / num_sms;
+  const int pass = kThreads * kGroups;
+  want = (want + pass - 1) / pass * pass;
+  if (want < pass) want = pass;
   return (int)want;
 }
 
@@ -324,8 +373,10 @@ cudaError_t launch_topk_split(const float* scores, int64_t ld, const int32_t* n_
   topk_hist_kernel<<<grid, kThreads, 0, stream>>>(scores, ld, n_valid, n_max, k, chunk, hist, st, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  topk_select_kernel<<<grid, kThreads, 0, stream>>>(scores, ld, k, chunk, st, bm, (int)wpr, cand, n_max, idx,
-                                                    top_scores);
+  e = ensure_smem(topk_select_kernel, sizeof(SelectSmem));
+  if (e != cudaSuccess) return e;
+  topk_select_kernel<<<grid, kThreads, sizeof(SelectSmem), stream>>>(scores, ld, k, chunk, st, bm, (int)wpr, cand,
+                                                                     n_max, idx, top_scores);
   return cudaGetLastError();
 }
 

@@ -173,6 +173,8 @@ sa_status sa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int N
  *            seq_off[b]*Hkv*d and is laid out [Hkv, seq_len[b], d]
  *            (KV-head-major); every layer of the group reads this cache
  *   seq_off  int64 [B+1], seq_len int32 [B] (device)
+ *   n_tokens rows of the packed cache per KV head (sum of seq_len); the
+ *            caches hold n_tokens * Hkv rows of d elements
  *   idx      int32 [B, k] (device) shared index of the group
  *   O        [L_g, B, Hq, d], bf16 or fp32 per out_dtype
  * Each selected K/V row is brought from HBM once per (sequence, KV head)
@@ -181,9 +183,9 @@ sa_status sa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int N
  * ---------------------------------------------------------------------- */
 size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int d, int k);
 sa_status sa_sparse_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
-                                const int32_t* seq_len, const int32_t* idx, int L_g, int B, int Hq,
-                                int Hkv, int d, int k, float scale, void* O, sa_dtype out_dtype,
-                                void* ws, size_t ws_bytes, void* stream);
+                                const int32_t* seq_len, const int32_t* idx, int L_g, int B,
+                                int64_t n_tokens, int Hq, int Hkv, int d, int k, float scale, void* O,
+                                sa_dtype out_dtype, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * One decode step over a layer pattern  [IC section 2: a binary pattern

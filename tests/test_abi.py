@@ -68,10 +68,10 @@ def test_index_score_rejects_unsupported_shapes(lib):
 
 
 def test_attention_rejects_bad_head_counts(lib):
-    rc = lib.sa_sparse_decode_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1, 30, 4, 128, 256, 0.088, FAKE, 0,
+    rc = lib.sa_sparse_decode_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1, 4096, 30, 4, 128, 256, 0.088, FAKE, 0,
                                    FAKE_WS, 1 << 20, None)
     assert rc == sa.SA_ERR_INVALID_ARG and b"multiple" in lib.sa_last_error()
-    rc = lib.sa_sparse_decode_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1, 32, 4, 64, 256, 0.125, FAKE, 0,
+    rc = lib.sa_sparse_decode_attn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1, 4096, 32, 4, 64, 256, 0.125, FAKE, 0,
                                    FAKE_WS, 1 << 20, None)
     assert rc == sa.SA_ERR_UNSUPPORTED
 
