@@ -18,6 +18,7 @@ path shards by sequence with no data-path collective, so scaling is weak and
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -55,6 +56,34 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--out-f32", action="store_true", help="fp32 attention output instead of bf16")
     return p.parse_args()
+
+
+# ---------------------------------------------------------------- ranks
+def rank_workload(name: str, rank: int):
+    """The workload one rank decodes: the named configuration, its seed offset
+    by the rank so that every rank serves sequences of its own (weak scaling:
+    the per-GPU work stays fixed as the number of GPUs grows)."""
+    cfg = synth.workload(name)
+    if rank:
+        cfg = dataclasses.replace(cfg, seed=cfg.seed + 7919 * rank)
+    return cfg
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's elapsed time (every rank gets it)."""
+    if world == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time."""
+    return world * units_per_rank / (ms / 1e3)
 
 
 # ---------------------------------------------------------------- accounting
@@ -296,7 +325,7 @@ def run_ours(args):
         dist.barrier()
     sa.lib()
 
-    cfg = synth.workload(args.workload)
+    cfg = rank_workload(args.workload, rank)
     out_dtype = torch.float32 if args.out_f32 else torch.bfloat16
     n = cfg.L
     nb = algorithmic_bytes(cfg, 4 if args.out_f32 else 2)
@@ -372,18 +401,15 @@ def run_ours(args):
             fn(i)
         e1.record()
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1)
+        ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
             dist.barrier()
         return ms
 
     with ClockSampler(local) as clocks:
         ms = timed(lambda i: graphs[i % len(graphs)].replay(), args.steps)
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1e3)
+    value = aggregate_rate(args.steps, world, ms)
 
     # ---- dominant kernel alone: the indexer, in its own graph of launches ----
     # interleave the sets so consecutive launches read different inputs
@@ -440,7 +466,7 @@ def run_ours(args):
         e2e_step(i)
     n_e2e = max(50, min(2000, args.steps))
     ms_e2e = timed(e2e_step, n_e2e)
-    e2e_value = world * n_e2e / (ms_e2e / 1e3)
+    e2e_value = aggregate_rate(n_e2e, world, ms_e2e)
     code, det = sa.read_status(st["ws"])
     if code != 0:
         raise RuntimeError(f"device status {code} {det}")

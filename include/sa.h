@@ -131,7 +131,8 @@ sa_status sa_index_score(const void* qI, const float* w, const void* KI, const i
  *   qI bf16 [Nq, H_I, d_I]; w fp32 [Nq, H_I]; KI bf16 [S, d_I];
  *   q_pos int32 [Nq] (device), each in [0, S); max_pos = host upper bound
  *   of q_pos (< S); scores fp32 [Nq, ld] with ld >= max_pos + 1.
- * Supported: H_I * 16 <= 256 ... see sa_index_score; Nq >= 1.
+ * Supported: 1 <= H_I <= 64, d_I in {64, 128, 192, 256} (as sa_index_score),
+ * 0 <= Nq <= 4096 (Nq = 0 returns SA_OK without a launch).
  * Device errors: q_pos out of [0, max_pos] -> SA_ERR_DEVICE, row skipped.
  * ---------------------------------------------------------------------- */
 size_t sa_index_score_prefill_workspace_size(int Nq);

@@ -1,0 +1,58 @@
+"""Host logic of bench.py for N > 1 ranks, run as a world-size-2 gloo group on
+CPU: every rank gets its own sequences, the elapsed time is the slowest
+rank's, and the aggregate rate counts every rank's units over that time."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank r "took" 10 + 5r ms: everyone must see the slowest, 15 ms
+        ms = bench.max_over_ranks(10.0 + 5.0 * rank, world, "cpu")
+        cfg = bench.rank_workload("c3", rank)
+        results[rank] = (ms, cfg.seed, bench.aggregate_rate(300, world, ms))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_and_workload_split():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_rank_main, args=(world, free_port(), results), nprocs=world, start_method="spawn", join=True)
+    (ms0, seed0, v0), (ms1, seed1, v1) = results[0], results[1]
+    assert ms0 == ms1 == 15.0
+    assert seed0 == synth.workload("c3").seed and seed1 != seed0
+    assert v0 == v1 == pytest.approx(2 * 300 / 0.015)
+
+
+def test_single_rank_is_unchanged():
+    assert bench.max_over_ranks(3.5, 1, "cpu") == 3.5
+    assert bench.rank_workload("c3", 0) == synth.workload("c3")
+    assert bench.aggregate_rate(10, 1, 1000.0) == pytest.approx(10.0)
+
+
+def test_rank_workloads_differ_only_in_seed():
+    a, b = bench.rank_workload("c5", 0), bench.rank_workload("c5", 3)
+    assert a.seed != b.seed
+    assert (a.seq_lens, a.k, a.pattern, a.Hq, a.Hkv, a.d) == (b.seq_lens, b.k, b.pattern, b.Hq, b.Hkv, b.d)
