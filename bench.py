@@ -411,36 +411,39 @@ def run_ours(args):
     ms_per_step = ms / args.steps
     value = aggregate_rate(args.steps, world, ms)
 
-    # ---- dominant kernel alone: the indexer, in its own graph of launches ----
-    # interleave the sets so consecutive launches read different inputs
-    inter = []
-    for st in sets:
+    # ---- per-kernel device time: each graph holds REP back-to-back launches
+    # (alternating input sets, so consecutive launches read different data),
+    # which keeps the host's replay cost out of the figure ----
+    REP = 16
+
+    def rep_graph(fn):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cap):
-            sa.index_score(st["qI"][0], st["w"][0], st["KI"][0], st["wl"]["seq_off"], st["wl"]["seq_len"],
-                           cfg.S_max, scores=st["scores"], ws=st["ws"])
-        inter.append(g)
-    for i in range(8):
-        inter[i % len(inter)].replay()
-    n_idx = max(200, min(4000, args.steps))
-    ms_idx = timed(lambda i: inter[i % len(inter)].replay(), n_idx) / n_idx
-    # top-k and attention alone (breakdown)
-    topk_g, attn_g = [], []
-    for st in sets:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap):
-            sa.topk(st["scores"], st["wl"]["seq_len"], cfg.S_max, cfg.k, idx=st["idx"], ws=st["ws"])
-        topk_g.append(g)
-        g = torch.cuda.CUDAGraph()
-        l0 = cfg.groups[0]
-        with torch.cuda.graph(g, stream=cap):
-            sa.sparse_decode_attn(st["wl"]["Q"][l0[0]:l0[-1] + 1], st["K"][0], st["V"][0], st["wl"]["seq_off"],
-                                  st["wl"]["seq_len"], st["idx"], cfg.Hkv, cfg.scale, O=st["O"][l0[0]:l0[-1] + 1],
-                                  ws=st["ws"])
-        attn_g.append(g)
-    n_k = max(200, min(4000, args.steps))
-    ms_topk = timed(lambda i: topk_g[i % len(topk_g)].replay(), n_k) / n_k
-    ms_attn = timed(lambda i: attn_g[i % len(attn_g)].replay(), n_k) / n_k
+            for r in range(REP):
+                fn(sets[r % len(sets)])
+        return g
+
+    l0 = cfg.groups[0]
+
+    def run_index(st):
+        sa.index_score(st["qI"][0], st["w"][0], st["KI"][0], st["wl"]["seq_off"], st["wl"]["seq_len"], cfg.S_max,
+                       scores=st["scores"], ws=st["ws"])
+
+    def run_topk(st):
+        sa.topk(st["scores"], st["wl"]["seq_len"], cfg.S_max, cfg.k, idx=st["idx"], ws=st["ws"])
+
+    def run_attn(st):
+        sa.sparse_decode_attn(st["wl"]["Q"][l0[0]:l0[-1] + 1], st["K"][0], st["V"][0], st["wl"]["seq_off"],
+                              st["wl"]["seq_len"], st["idx"], cfg.Hkv, cfg.scale, O=st["O"][l0[0]:l0[-1] + 1],
+                              ws=st["ws"])
+
+    g_idx, g_topk, g_attn = rep_graph(run_index), rep_graph(run_topk), rep_graph(run_attn)
+    for g in (g_idx, g_topk, g_attn):
+        g.replay()
+    n_rep = max(20, min(250, args.steps // REP))
+    ms_idx = timed(lambda i: g_idx.replay(), n_rep) / (n_rep * REP)
+    ms_topk = timed(lambda i: g_topk.replay(), n_rep) / (n_rep * REP)
+    ms_attn = timed(lambda i: g_attn.replay(), n_rep) / (n_rep * REP)
 
     # ---- end to end through the public API: pinned host in, host out ---------
     st = sets[0]
@@ -480,7 +483,8 @@ def run_ours(args):
                          f"key, top-{cfg.k}, attention of all {cfg.L} layers); steps/s = sequences/{cfg.B}/s"}
 
     if world > 1:
-        graphs.clear(); inter.clear(); topk_g.clear(); attn_g.clear()
+        graphs.clear()
+        del g_idx, g_topk, g_attn
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:

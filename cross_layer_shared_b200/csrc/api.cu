@@ -301,7 +301,7 @@ sa_status sa_index_score_prefill(const void* qI, const float* w, const void* KI,
 size_t sa_topk_workspace_size(int Nq, int n_max, int k) {
   (void)k;
   if (Nq > 0 && n_max > 0 && sa::topk_use_split(Nq, n_max, num_sms()))
-    return SA_WS_HEADER_BYTES + sa::topk_split_ws_bytes(Nq, n_max);
+    return SA_WS_HEADER_BYTES + sa::topk_split_ws_bytes(Nq, n_max, num_sms());
   return SA_WS_HEADER_BYTES;
 }
 

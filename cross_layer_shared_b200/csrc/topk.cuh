@@ -14,9 +14,9 @@ size_t topk_rows_smem_bytes();
 cudaError_t launch_topk_rows(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max, int k,
                              int32_t* idx, float* top_scores, DeviceStatus* status, cudaStream_t stream);
 
-// Few long rows (Nq <= num_sms / 2, n_max > 8192): many CTAs per row.
+// Few long rows (Nq <= num_sms / 2, n_max > 8192): one cluster of CTAs per row.
 bool topk_use_split(int Nq, int n_max, int num_sms);
-size_t topk_split_ws_bytes(int Nq, int n_max);
+size_t topk_split_ws_bytes(int Nq, int n_max, int num_sms);
 cudaError_t launch_topk_split(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max, int k,
                               int32_t* idx, float* top_scores, DeviceStatus* status, void* scratch, int num_sms,
                               cudaStream_t stream);

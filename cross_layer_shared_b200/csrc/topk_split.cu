@@ -1,20 +1,27 @@
-// Top-k for few long rows (decode: one row per sequence), spread over many
-// CTAs per row.  Same definition as topk.cu [IndexCache technical summary
-// section 1: keep the k most relevant tokens]: the min(k, n) largest scores,
-// ties to the lower index, ascending output, -1 padding.
+// Top-k for few long rows (decode: one row per sequence), each row spread
+// over one thread-block cluster of G CTAs.  Same definition as topk.cu
+// [IndexCache technical summary section 1: keep the k most relevant tokens]:
+// the min(k, n) largest scores, ties to the LOWER index, ascending output,
+// -1 padding.
 //
-// Two kernels, no spin-wait anywhere (the last CTA of a row to finish does
-// the row's serial part; it learns it is last from an atomic ticket):
-//   hist    each CTA histograms key bits [31:20] of its chunk in shared
-//           memory and adds it into the row's global histogram; the row's
-//           last CTA finds the threshold bucket and how many keys lie above.
-//   select  each CTA turns its chunk into bitmap words (warp ballot: key
-//           above the bucket = selected) and appends the keys inside the
-//           bucket to the row's candidate list; the row's last CTA finishes
-//           the radix select on the candidates (key bits [19:10], [9:0], then
-//           the index among keys equal to the k-th, for the lower-index
-//           rule), ORs the winners into the bitmap and emits the set bits in
-//           index order from a block-wide prefix sum of popcounts.
+// The CTAs of a row exchange everything through distributed shared memory
+// and the hardware cluster barrier -- no global atomics, no spin-waits, no
+// scratch to clear between calls:
+//   0  each CTA loads its chunk of keys into shared memory, histograms key
+//      bits [31:20] and lists its non-empty bins;
+//   A  each CTA sums the G lists of its cluster into the row histogram,
+//      finds the threshold bucket (the one holding the k-th largest key) and
+//      the count above it, counts its own keys above the bucket and lists
+//      its keys inside the bucket (the candidates);
+//   B  each CTA gathers the row's candidates, finishes the radix select on
+//      them (key bits [19:10], [9:0], then the index among keys equal to the
+//      k-th, for the lower-index rule) -- the same answer in every CTA of
+//      the row -- and writes its own chunk's selected indices, in index
+//      order, at the offset given by the earlier chunks' counts.
+// A CTA whose candidates overflow its shared list spills them to its slot in
+// the workspace; a row with many candidates refines them in place, from the
+// owners' shared memory or their slots (slow, but exact).
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,21 +29,34 @@
 #include "status.cuh"
 #include "topk.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace sa {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins1 = 4096;
+constexpr int kBins1 = 4096;                // digit [31:20]
+constexpr int kGroups = 8;                  // 32-key groups per warp per pass
+constexpr int kPass = kThreads * kGroups;   // keys per pass (8192)
+constexpr int kChunkUnit = kPass;           // chunks are whole passes
+constexpr int kKeyCache = 16384;            // chunk keys kept in shared memory
+constexpr int kCandLocal = 2048;            // this CTA's candidates, in shared memory
+constexpr int kCandRow = 6144;              // the row's candidates gathered for the refine
+constexpr int kMaxCluster = 16;
 
-struct RowState {
-  int beta;    // threshold bucket of bits [31:20]; -1: the whole row is selected
-  int above;   // keys in buckets above beta
-  int n;       // valid length
-  int ncand;   // keys appended to the candidate list
-  int ticket1;
-  int ticket2;
-  int pad[2];
+struct Smem {
+  uint32_t keys[kKeyCache];
+  uint32_t hist[kBins1];
+  uint2 list[kBins1];         // (bin, count) of the non-empty bins of this chunk
+  uint2 cand[kCandLocal];     // (key, index) of this chunk's keys in the bucket
+  uint2 row_cand[kCandRow];
+  int nlist, cnt_above, ncand, spilled;
+  int cpre[kMaxCluster + 1];  // candidate prefix over the cluster's CTAs
+  int peer_above[kMaxCluster], peer_spill[kMaxCluster];
+  int spill_any, cand_ctr;
+  int ws[kWarps + 1];
+  int bin, before;
 };
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -78,6 +98,10 @@ __device__ int block_scan_excl(int v, int* ws, int* total) {
 // reaches `need`; *before = count strictly above it.
 __device__ void find_bin_desc(const uint32_t* hist, int nb, int need, int* ws, int* s_bin, int* s_before) {
   const int per = (nb + kThreads - 1) / kThreads;
+  if (threadIdx.x == 0) {  // stays in range even if the counts fall short (a timed-out barrier)
+    *s_bin = 0;
+    *s_before = 0;
+  }
   int local = 0;
   for (int j = 0; j < per; ++j) {
     const int bin = nb - 1 - (threadIdx.x * per + j);
@@ -101,256 +125,348 @@ __device__ void find_bin_desc(const uint32_t* hist, int nb, int need, int* ws, i
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads) topk_hist_kernel(const float* __restrict__ scores, int64_t ld,
-                                                             const int32_t* __restrict__ n_valid, int n_max, int k,
-                                                             int chunk, uint32_t* __restrict__ hist,
-                                                             RowState* __restrict__ st, DeviceStatus* status) {
-  __shared__ uint32_t sh[kBins1];
-  __shared__ int ws[kWarps + 1];
-  __shared__ int s_last, s_bin, s_before;
-  const int q = blockIdx.y, c = blockIdx.x, tid = threadIdx.x;
+// radix select, descending, over candidate values v(j) with pred(j): finds
+// the need-th largest value T among those matching (prefix, mask); returns
+// in *need the count of values == T that are taken, in *n_eq how many equal T.
+template <class Val, class Pred>
+__device__ uint32_t radix_desc(int nc, Val val, Pred pred, uint32_t prefix, uint32_t mask, const int* shifts,
+                               const int* widths, int nlev, int* need, int* n_eq, Smem& sm) {
+  for (int lv = 0; lv < nlev; ++lv) {
+    const int shift = shifts[lv], nb = 1 << widths[lv];
+    for (int i = threadIdx.x; i < nb; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < nc; j += kThreads) {
+      if (!pred(j)) continue;
+      const uint32_t v = val(j);
+      if ((v & mask) == prefix) atomicAdd(&sm.hist[(v >> shift) & (uint32_t)(nb - 1)], 1u);
+    }
+    __syncthreads();
+    find_bin_desc(sm.hist, nb, *need, sm.ws, &sm.bin, &sm.before);
+    prefix |= (uint32_t)sm.bin << shift;
+    mask |= (uint32_t)(nb - 1) << shift;
+    *need -= sm.before;
+    *n_eq = (int)sm.hist[sm.bin];
+    __syncthreads();
+  }
+  return prefix;
+}
+
+// Pass layout: warp w covers keys [base0 + 256 w, +256) of a pass, as 8
+// groups of 32 (one key per lane), so group ballots come out in index order
+// and lane gi < 8 can own the word of group gi.
+__device__ __forceinline__ int pass_pos(int base0, int warp, int gi, int lane) {
+  return base0 + (warp * kGroups + gi) * 32 + lane;
+}
+
+__global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                const int32_t* __restrict__ n_valid, int n_max,
+                                                                int k, int chunk, uint2* __restrict__ spill,
+                                                                int32_t* __restrict__ idx,
+                                                                float* __restrict__ top_scores, DeviceStatus* status) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  cg::cluster_group cluster = cg::this_cluster();
+  const int G = (int)cluster.num_blocks();
+  const int c = (int)cluster.block_rank();
+  const int q = blockIdx.x / G, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   int n = n_valid[q];
   if (n < 0 || n > n_max) {
     if (c == 0 && tid == 0) report(status, kErrDevice, kKernTopk, q, n, n_max);
     n = n < 0 ? 0 : n_max;
   }
   const float* row = scores + (int64_t)q * ld;
-  for (int i = tid; i < kBins1; i += kThreads) sh[i] = 0;
-  __syncthreads();
-  const int beg = c * chunk, end = min(n, beg + chunk);
-  if (n > k)
-    for (int i = beg + tid; i < end; i += kThreads) atomicAdd(&sh[order_key(row[i]) >> 20], 1u);
-  __syncthreads();
-  uint32_t* h = hist + (int64_t)q * kBins1;
-  if (n > k)
-    for (int i = tid; i < kBins1; i += kThreads)
-      if (sh[i]) atomicAdd(&h[i], sh[i]);
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&st[q].ticket1, 1) == (int)gridDim.x - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  if (n <= k) {
-    if (tid == 0) {
-      st[q].beta = -1;
-      st[q].above = n;
-      st[q].n = n;
-    }
-    return;
-  }
-  for (int i = tid; i < kBins1; i += kThreads) sh[i] = __ldcg(&h[i]);
-  __syncthreads();
-  find_bin_desc(sh, kBins1, k, ws, &s_bin, &s_before);
-  if (tid == 0) {
-    st[q].beta = s_bin;
-    st[q].above = s_before;
-    st[q].n = n;
-  }
-}
-
-// radix select, descending, over candidate values v(j) with pred(j): finds
-// the need-th largest value T among those matching (prefix, mask); returns
-// in *need the count of values == T that are taken, in *n_eq how many equal T.
-template <class Val, class Pred>
-__device__ uint32_t radix_desc(int nc, Val val, Pred pred, uint32_t prefix, uint32_t mask, const int* shifts,
-                               const int* widths, int nlev, int* need, int* n_eq, uint32_t* sh, int* ws, int* s_bin,
-                               int* s_before) {
-  for (int lv = 0; lv < nlev; ++lv) {
-    const int shift = shifts[lv], nb = 1 << widths[lv];
-    for (int i = threadIdx.x; i < nb; i += kThreads) sh[i] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < nc; j += kThreads) {
-      if (!pred(j)) continue;
-      const uint32_t v = val(j);
-      if ((v & mask) == prefix) atomicAdd(&sh[(v >> shift) & (uint32_t)(nb - 1)], 1u);
-    }
-    __syncthreads();
-    find_bin_desc(sh, nb, *need, ws, s_bin, s_before);
-    prefix |= (uint32_t)*s_bin << shift;
-    mask |= (uint32_t)(nb - 1) << shift;
-    *need -= *s_before;
-    *n_eq = (int)sh[*s_bin];
-    __syncthreads();
-  }
-  return prefix;
-}
-
-constexpr int kGroups = 8;            // 32-key groups per warp per chunk pass (registers)
-constexpr int kCandSmem = 6144;       // candidates refined in shared memory
-constexpr int kWordsSmem = 4096;      // bitmap words staged in shared memory (rows <= 131072)
-
-struct SelectSmem {
-  uint2 cand[kCandSmem];
-  uint32_t words[kWordsSmem];
-  uint32_t hist[2048];
-  int ws[kWarps + 1];
-  int warp_cnt[kWarps];
-  int cta_base;
-  int last, bin, before;
-};
-
-__global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __restrict__ scores, int64_t ld, int k,
-                                                               int chunk, RowState* __restrict__ st,
-                                                               uint32_t* __restrict__ bitmap, int wpr,
-                                                               uint2* __restrict__ cand, int cap,
-                                                               int32_t* __restrict__ idx, float* __restrict__ top_scores) {
-  extern __shared__ uint8_t smem_raw[];
-  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
-  const int q = blockIdx.y, c = blockIdx.x, tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int beta = __ldcg(&st[q].beta), above = __ldcg(&st[q].above), n = __ldcg(&st[q].n);
-  const float* row = scores + (int64_t)q * ld;
-  uint32_t* bm = bitmap + (int64_t)q * wpr;
-  uint2* cq = cand + (int64_t)q * cap;
-
-  // ---- this CTA's chunk: selected-bit words and threshold-bucket candidates ----
-  const int beg = c * chunk, end = min(n, beg + chunk);
-  for (int base0 = beg; base0 < end; base0 += kThreads * kGroups) {
-    uint32_t key[kGroups];
-    uint32_t eqm[kGroups];
-    int my = 0;  // candidates of this warp in this pass
-#pragma unroll
-    for (int gi = 0; gi < kGroups; ++gi) {
-      const int base = base0 + (gi * kWarps + warp) * 32;
-      const int i = base + lane;
-      const bool in = i < end;
-      key[gi] = in ? order_key(row[i]) : 0u;
-      const int d = (int)(key[gi] >> 20);
-      const bool sel = in && (beta < 0 || d > beta);
-      const bool eq = in && beta >= 0 && d == beta;
-      const uint32_t word = __ballot_sync(0xffffffffu, sel);
-      if (lane == 0 && base < end) bm[base >> 5] = word;
-      eqm[gi] = __ballot_sync(0xffffffffu, eq);
-      my += __popc(eqm[gi]);
-    }
-    if (lane == 0) sm.warp_cnt[warp] = my;
-    __syncthreads();
-    if (tid == 0) {
-      int tot = 0;
-      for (int w = 0; w < kWarps; ++w) {
-        const int x = sm.warp_cnt[w];
-        sm.warp_cnt[w] = tot;
-        tot += x;
-      }
-      sm.cta_base = tot ? atomicAdd(&st[q].ncand, tot) : 0;  // one reservation per CTA
-    }
-    __syncthreads();
-    int pos = sm.cta_base + sm.warp_cnt[warp];
-#pragma unroll
-    for (int gi = 0; gi < kGroups; ++gi) {
-      const int base = base0 + (gi * kWarps + warp) * 32;
-      if ((eqm[gi] >> lane) & 1u) {
-        const int p = pos + __popc(eqm[gi] & ((1u << lane) - 1u));
-        if (p < cap) cq[p] = make_uint2(key[gi], (uint32_t)(base + lane));
-      }
-      pos += __popc(eqm[gi]);
-    }
-    __syncthreads();
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) sm.last = atomicAdd(&st[q].ticket2, 1) == (int)gridDim.x - 1;
-  __syncthreads();
-  if (!sm.last) return;
-  __threadfence();
-
-  // ---- the row's last CTA ---------------------------------------------------
-  const int nw = (n + 31) >> 5;
-  const bool words_in_smem = nw <= kWordsSmem;
-  if (words_in_smem)
-    for (int w = tid; w < nw; w += kThreads) sm.words[w] = __ldcg(&bm[w]);
-  if (beta >= 0) {
-    int nc = __ldcg(&st[q].ncand);
-    nc = nc < cap ? nc : cap;
-    const bool in_smem = nc <= kCandSmem;
-    if (in_smem)
-      for (int j = tid; j < nc; j += kThreads) sm.cand[j] = __ldcg(&cq[j]);
-    __syncthreads();
-    const uint2* cs = in_smem ? sm.cand : cq;
-    auto ckey = [&](int j) { return in_smem ? sm.cand[j].x : __ldcg(&cq[j].x); };
-    auto cidx = [&](int j) { return in_smem ? sm.cand[j].y : __ldcg(&cq[j].y); };
-    int need = k - above;
-    int n_eq = 0;
-    const int ks[2] = {10, 0}, kw[2] = {10, 10};
-    const uint32_t T = radix_desc(nc, ckey, [](int) { return true; }, (uint32_t)beta << 20, 0xFFF00000u, ks, kw,
-                                  2, &need, &n_eq, sm.hist, sm.ws, &sm.bin, &sm.before);
-    uint32_t cut = 0xFFFFFFFFu;
-    if (need < n_eq) {
-      // the `need` lowest indices among keys == T: largest values of ~index
-      int need2 = need, n2 = 0;
-      const int is[3] = {21, 10, 0}, iw[3] = {11, 11, 10};
-      const uint32_t V = radix_desc(nc, [&](int j) { return ~cidx(j); }, [&](int j) { return ckey(j) == T; }, 0u,
-                                    0u, is, iw, 3, &need2, &n2, sm.hist, sm.ws, &sm.bin, &sm.before);
-      cut = ~V;
-    }
-    (void)cs;
-    for (int j = tid; j < nc; j += kThreads) {
-      const uint32_t kx = ckey(j), ix = cidx(j);
-      if (kx > T || (kx == T && ix <= cut)) {
-        if (words_in_smem) atomicOr(&sm.words[ix >> 5], 1u << (ix & 31));
-        else atomicOr(&bm[ix >> 5], 1u << (ix & 31));
-      }
-    }
-    if (!words_in_smem) __threadfence();
-  }
-  __syncthreads();
-
-  // ---- emit set bits in index order ----------------------------------------
+  const int beg = c * chunk;
+  const int len = n - beg < 0 ? 0 : (n - beg < chunk ? n - beg : chunk);
+  const bool cached = chunk <= kKeyCache;
   int32_t* out = idx + (int64_t)q * k;
   float* out_s = top_scores ? top_scores + (int64_t)q * k : nullptr;
-  constexpr int kWpt = 8;
-  int written = 0;
-  for (int w0 = 0; w0 < nw; w0 += kThreads * kWpt) {
-    uint32_t wv[kWpt];
+  if (n <= k) {  // every valid key is selected (uniform over the cluster: no barrier is skipped by half of it)
+    for (int i = tid; i < len; i += kThreads) {
+      out[beg + i] = beg + i;
+      if (out_s) out_s[beg + i] = row[beg + i];
+    }
+    if (c == G - 1)
+      for (int p = n + tid; p < k; p += kThreads) {
+        out[p] = -1;
+        if (out_s) out_s[p] = 0.f;
+      }
+    return;
+  }
+  auto key_at = [&](int i) -> uint32_t { return cached ? sm.keys[i] : order_key(__ldg(&row[beg + i])); };
+
+  // ---- phase 0: keys into shared memory, chunk histogram, non-empty bins ----
+  for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
+  if (tid == 0) sm.cand_ctr = 0;
+  __syncthreads();
+  for (int base0 = 0; base0 < len; base0 += kPass) {
+    uint32_t key[kGroups];
+#pragma unroll
+    for (int u = 0; u < kGroups; ++u) {  // all loads of the pass in flight together
+      const int i = base0 + u * kThreads + tid;
+      key[u] = i < len ? order_key(__ldg(&row[beg + i])) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kGroups; ++u) {
+      const int i = base0 + u * kThreads + tid;
+      if (i < len) {
+        if (cached) sm.keys[i] = key[u];
+        atomicAdd(&sm.hist[key[u] >> 20], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  {
+    constexpr int kPer = kBins1 / kThreads;
     int cnt = 0;
 #pragma unroll
-    for (int j = 0; j < kWpt; ++j) {
-      const int wi = w0 + tid * kWpt + j;
-      wv[j] = wi < nw ? (words_in_smem ? sm.words[wi] : __ldcg(&bm[wi])) : 0u;
-      if (wi == nw - 1 && (n & 31)) wv[j] &= (1u << (n & 31)) - 1u;
-      cnt += __popc(wv[j]);
+    for (int j = 0; j < kPer; ++j) cnt += sm.hist[tid * kPer + j] != 0u;
+    int tot;
+    int pos = block_scan_excl(cnt, sm.ws, &tot);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const uint32_t h = sm.hist[tid * kPer + j];
+      if (h) sm.list[pos++] = make_uint2((uint32_t)(tid * kPer + j), h);
+    }
+    if (tid == 0) sm.nlist = tot;
+  }
+  cluster.sync();
+
+  // ---- phase A: row histogram, threshold bucket, this chunk's candidates ----
+  for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
+  __syncthreads();
+  for (int r = warp; r < G; r += kWarps) {
+    const Smem* peer = cluster.map_shared_rank(&sm, r);
+    const int nl = peer->nlist;
+    for (int e0 = 0; e0 < nl; e0 += 128) {
+      uint2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * 32 + lane;
+        v[u] = e < nl ? peer->list[e] : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v[u].y) atomicAdd(&sm.hist[v[u].x & (kBins1 - 1)], v[u].y);
+    }
+  }
+  __syncthreads();
+  find_bin_desc(sm.hist, kBins1, k, sm.ws, &sm.bin, &sm.before);
+  const int beta = sm.bin, above = sm.before;
+  uint2* my_spill = spill + (int64_t)blockIdx.x * chunk;
+  {
+    int my_above = 0;
+    for (int base0 = 0; base0 < len; base0 += kPass) {
+      uint32_t key[kGroups], eqm[kGroups];
+#pragma unroll
+      for (int gi = 0; gi < kGroups; ++gi) {
+        const int i = pass_pos(base0, warp, gi, lane);
+        key[gi] = i < len ? key_at(i) : 0u;
+      }
+      int my = 0;
+#pragma unroll
+      for (int gi = 0; gi < kGroups; ++gi) {
+        const bool in = pass_pos(base0, warp, gi, lane) < len;
+        const int d = (int)(key[gi] >> 20);
+        my_above += (in && d > beta) ? 1 : 0;
+        eqm[gi] = __ballot_sync(0xffffffffu, in && d == beta);
+        my += __popc(eqm[gi]);
+      }
+      if (my) {  // one slot reservation per warp and pass; candidate order is free
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(&sm.cand_ctr, my);
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+#pragma unroll
+        for (int gi = 0; gi < kGroups; ++gi) {
+          if ((eqm[gi] >> lane) & 1u) {
+            const int p = slot + __popc(eqm[gi] & ((1u << lane) - 1u));
+            const uint2 v = make_uint2(key[gi], (uint32_t)(beg + pass_pos(base0, warp, gi, lane)));
+            if (p < kCandLocal) sm.cand[p] = v;
+            else my_spill[p] = v;
+          }
+          slot += __popc(eqm[gi]);
+        }
+      }
+    }
+    int tot_above;
+    block_scan_excl(my_above, sm.ws, &tot_above);
+    if (tid == 0) {
+      const int ncand = sm.cand_ctr;
+      sm.cnt_above = tot_above;
+      sm.ncand = ncand;
+      sm.spilled = ncand > kCandLocal;
+    }
+    __syncthreads();
+    if (sm.spilled)  // the whole list then lives in the workspace
+      for (int p = tid; p < kCandLocal; p += kThreads) my_spill[p] = sm.cand[p];
+  }
+  cluster.sync();
+
+  // ---- phase B: exact k-th key, then this chunk's part of the output ----
+  if (tid < G) {
+    const Smem* peer = cluster.map_shared_rank(&sm, tid);
+    sm.cpre[tid + 1] = peer->ncand;
+    sm.peer_above[tid] = peer->cnt_above;
+    sm.peer_spill[tid] = peer->spilled;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int above_before = 0, spill_any = 0;
+    sm.cpre[0] = 0;
+    for (int r = 0; r < G; ++r) {
+      sm.cpre[r + 1] += sm.cpre[r];
+      if (r < c) above_before += sm.peer_above[r];
+      spill_any |= sm.peer_spill[r];
+    }
+    sm.before = above_before;  // keys above the bucket in chunks < c
+    sm.spill_any = spill_any;
+  }
+  __syncthreads();
+  const int above_before = sm.before;
+  const int nc = sm.cpre[G];
+  const bool fast = !sm.spill_any && nc <= kCandRow;
+  auto cand_at = [&](int j) -> uint2 {  // j-th candidate of the row, from its owner
+    int lo = 0, hi = G;                 // owner r with cpre[r] <= j < cpre[r + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (sm.cpre[mid] <= j) lo = mid; else hi = mid;
+    }
+    const int e = j - sm.cpre[lo];
+    if (sm.peer_spill[lo]) return __ldcg(&spill[((int64_t)q * G + lo) * chunk + e]);
+    return cluster.map_shared_rank(&sm, lo)->cand[e];
+  };
+  if (fast) {
+    for (int j0 = 0; j0 < nc; j0 += 4 * kThreads) {
+      uint2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u * kThreads + tid;
+        v[u] = j < nc ? cand_at(j) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u * kThreads + tid;
+        if (j < nc) sm.row_cand[j] = v[u];
+      }
+    }
+    __syncthreads();
+  }
+  auto ckey = [&](int j) { return fast ? sm.row_cand[j].x : cand_at(j).x; };
+  auto cidx = [&](int j) { return fast ? sm.row_cand[j].y : cand_at(j).y; };
+  int need = k - above, n_eq = 0;
+  const int ks[2] = {10, 0}, kw[2] = {10, 10};
+  const uint32_t T = radix_desc(nc, ckey, [](int) { return true; }, (uint32_t)beta << 20, 0xFFF00000u, ks, kw, 2,
+                                &need, &n_eq, sm);
+  uint32_t cut = 0xFFFFFFFFu;
+  if (need < n_eq) {
+    // the `need` lowest indices among keys == T: largest values of ~index
+    int need2 = need, n2 = 0;
+    const int is[3] = {21, 10, 0}, iw[3] = {11, 11, 10};
+    const uint32_t V = radix_desc(nc, [&](int j) { return ~cidx(j); }, [&](int j) { return ckey(j) == T; }, 0u, 0u,
+                                  is, iw, 3, &need2, &n2, sm);
+    cut = ~V;
+  }
+  // selected candidates of earlier chunks (candidates are grouped by owner,
+  // owners in chunk order)
+  int sel_before = 0;
+  for (int j = tid; j < sm.cpre[c]; j += kThreads) {
+    const uint32_t kx = ckey(j), ix = cidx(j);
+    if (kx > T || (kx == T && ix <= cut)) ++sel_before;
+  }
+  int tot_sel_before;
+  block_scan_excl(sel_before, sm.ws, &tot_sel_before);
+  int written = above_before + tot_sel_before;
+  for (int base0 = 0; base0 < len; base0 += kPass) {
+    uint32_t key[kGroups];
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int i = pass_pos(base0, warp, gi, lane);
+      key[gi] = i < len ? key_at(i) : 0u;
+    }
+    uint32_t x = 0;
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int i = pass_pos(base0, warp, gi, lane);
+      const int d = (int)(key[gi] >> 20);
+      const bool sel = i < len && (d > beta || (d == beta && (key[gi] > T || (key[gi] == T && (uint32_t)(beg + i) <= cut))));
+      const uint32_t w = __ballot_sync(0xffffffffu, sel);
+      if (lane == gi) x = w;
     }
     int tot;
-    int pos = written + block_scan_excl(cnt, sm.ws, &tot);
-#pragma unroll
-    for (int j = 0; j < kWpt; ++j) {
-      uint32_t x = wv[j];
-      const int wi = w0 + tid * kWpt + j;
-      while (x) {
-        const int b = __ffs(x) - 1;
-        x &= x - 1;
-        const int i = (wi << 5) + b;
-        if (pos < k) {
-          out[pos] = i;
-          if (out_s) out_s[pos] = row[i];
-        }
-        ++pos;
+    int pos = written + block_scan_excl(__popc(x), sm.ws, &tot);
+    const int base = beg + pass_pos(base0, warp, lane, 0);  // lane < 8: its group's first key
+    while (x) {
+      const int b = __ffs(x) - 1;
+      x &= x - 1;
+      if (pos < k) {
+        out[pos] = base + b;
+        if (out_s) out_s[pos] = row[base + b];
       }
+      ++pos;
     }
     written += tot;
   }
-  for (int p = written + tid; p < k; p += kThreads) {
-    out[p] = -1;
-    if (out_s) out_s[p] = 0.f;
-  }
+  cluster.sync();  // peers may still be reading this CTA's lists
 }
 
-int chunk_for(int Nq, int n_max, int num_sms) {
-  // about one CTA per SM over all rows; a multiple of one select pass
-  int64_t want = ((int64_t)Nq * n_max + num_sms - 1) / num_sms;
-  const int pass = kThreads * kGroups;
-  want = (want + pass - 1) / pass * pass;
-  if (want < pass) want = pass;
-  return (int)want;
+struct Plan {
+  int G, chunk;
+};
+
+// G: CTAs per row (a cluster), a power of two up to max_g with Nq * G <= SMs
+Plan plan_for(int Nq, int n_max, int num_sms, int max_g) {
+  Plan p;
+  int G = 1;
+  while (G * 2 <= max_g && (int64_t)Nq * G * 2 <= num_sms && (int64_t)G * kChunkUnit < n_max) G *= 2;
+  int64_t chunk = ((int64_t)n_max + G - 1) / G;
+  chunk = (chunk + kChunkUnit - 1) / kChunkUnit * kChunkUnit;
+  p.G = G;
+  p.chunk = (int)chunk;
+  return p;
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Largest cluster the device schedules for this kernel (16 needs the
+// non-portable size; some parts only give 8).  Looked up once per device.
+int max_cluster() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  if (cached[dev]) return cached[dev];
+  int g = 8;
+  if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+      ensure_smem(topk_cluster_kernel, sizeof(Smem)) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kMaxCluster);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sizeof(Smem);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kMaxCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &cfg) == cudaSuccess && n >= 1) g = kMaxCluster;
+  }
+  cudaGetLastError();
+  cached[dev] = g;
+  return g;
 }
 
 }  // namespace
 
-size_t topk_split_ws_bytes(int Nq, int n_max) {
-  const size_t wpr = ((size_t)n_max + 31) / 32;
-  auto r = [](size_t x) { return (x + 255) / 256 * 256; };
-  return r(sizeof(RowState) * Nq) + r(4ull * kBins1 * Nq) + r(4 * wpr * Nq) + r(8ull * (size_t)n_max * Nq);
+size_t topk_split_ws_bytes(int Nq, int n_max, int num_sms) {
+  // candidate spill slots: one chunk per CTA, for either cluster size
+  size_t most = 0;
+  for (int g = 8; g <= kMaxCluster; g *= 2) {
+    const Plan p = plan_for(Nq, n_max, num_sms, g);
+    const size_t b = 8ull * p.chunk * (size_t)Nq * p.G;
+    if (b > most) most = b;
+  }
+  return round256(most);
 }
 
 bool topk_use_split(int Nq, int n_max, int num_sms) { return Nq > 0 && Nq * 2 <= num_sms && n_max > 8192; }
@@ -358,25 +474,24 @@ bool topk_use_split(int Nq, int n_max, int num_sms) { return Nq > 0 && Nq * 2 <=
 cudaError_t launch_topk_split(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max, int k,
                               int32_t* idx, float* top_scores, DeviceStatus* status, void* scratch, int num_sms,
                               cudaStream_t stream) {
-  const size_t wpr = ((size_t)n_max + 31) / 32;
-  auto r = [](size_t x) { return (x + 255) / 256 * 256; };
-  uint8_t* p = reinterpret_cast<uint8_t*>(scratch);
-  RowState* st = reinterpret_cast<RowState*>(p);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(p + r(sizeof(RowState) * Nq));
-  uint32_t* bm = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(hist) + r(4ull * kBins1 * Nq));
-  uint2* cand = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(bm) + r(4 * wpr * Nq));
-  // row states and histograms start at zero every call
-  cudaError_t e = cudaMemsetAsync(p, 0, r(sizeof(RowState) * Nq) + r(4ull * kBins1 * Nq), stream);
+  const Plan p = plan_for(Nq, n_max, num_sms, max_cluster());
+  cudaError_t e = ensure_smem(topk_cluster_kernel, sizeof(Smem));
   if (e != cudaSuccess) return e;
-  const int chunk = chunk_for(Nq, n_max, num_sms);
-  const dim3 grid((n_max + chunk - 1) / chunk, Nq);
-  topk_hist_kernel<<<grid, kThreads, 0, stream>>>(scores, ld, n_valid, n_max, k, chunk, hist, st, status);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(Nq * p.G));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = sizeof(Smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;  // the CTAs of one row form one cluster
+  attr[0].val.clusterDim.x = p.G;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, ld, n_valid, n_max, k, p.chunk,
+                         reinterpret_cast<uint2*>(scratch), idx, top_scores, status);
   if (e != cudaSuccess) return e;
-  e = ensure_smem(topk_select_kernel, sizeof(SelectSmem));
-  if (e != cudaSuccess) return e;
-  topk_select_kernel<<<grid, kThreads, sizeof(SelectSmem), stream>>>(scores, ld, k, chunk, st, bm, (int)wpr, cand,
-                                                                     n_max, idx, top_scores);
   return cudaGetLastError();
 }
 
