@@ -223,27 +223,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   const int b = a.prefill ? 0 : bg / a.Hkv;
   const int g = a.prefill ? bg : bg % a.Hkv;
 
-  KeySrc ks;
-  int n_keys;
-  if (!a.prefill) {
-    ks.len = a.seq_len[b];
-    ks.base = 0;
-    n_keys = a.k;
-  } else {
-    ks.len = a.S;
-    ks.base = a.kv_indptr[g];
-    n_keys = (a.kv_indptr[g + 1] - ks.base) * a.block;
-  }
-  ks.kbeg = split * a.keys_per_split;
-  ks.kend = min(n_keys, ks.kbeg + a.keys_per_split);
-  const int nt = ks.kend > ks.kbeg ? (ks.kend - ks.kbeg + kKT - 1) / kKT : 0;
-
-  // producer lanes: raw entries of tile rows 4*lane .. 4*lane+3, one tile ahead
-  int raw_next[4];
-  if (warp >= kProdWarp0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) raw_next[i] = key_raw(a, ks, b, ks.kbeg + 4 * lane + i);
-  }
+  pdl_trigger();
   if (warp == kMmaWarp) tmem_alloc(slot, 512);
   if (tid == 0) {
     tma_prefetch_desc(&tm_q);
@@ -266,6 +246,30 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
+
+  // everything below reads what earlier kernels of the stream wrote
+  pdl_wait();
+  KeySrc ks;
+  int n_keys;
+  if (!a.prefill) {
+    ks.len = a.seq_len[b];
+    ks.base = 0;
+    n_keys = a.k;
+  } else {
+    ks.len = a.S;
+    ks.base = a.kv_indptr[g];
+    n_keys = (a.kv_indptr[g + 1] - ks.base) * a.block;
+  }
+  ks.kbeg = split * a.keys_per_split;
+  ks.kend = min(n_keys, ks.kbeg + a.keys_per_split);
+  const int nt = ks.kend > ks.kbeg ? (ks.kend - ks.kbeg + kKT - 1) / kKT : 0;
+
+  // producer lanes: raw entries of tile rows 4*lane .. 4*lane+3, one tile ahead
+  int raw_next[4];
+  if (warp >= kProdWarp0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) raw_next[i] = key_raw(a, ks, b, ks.kbeg + 4 * lane + i);
+  }
 
   // softmax state: thread (row r, key half h)
   const int half = (warp >> 2) & 1;
@@ -674,13 +678,14 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& tm_q, const
   cfg.blockDim = dim3(kAttnThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = a.n_split;  // the key splits of one row tile share a cluster
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, a, tm_q, tm_k, tm_v);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

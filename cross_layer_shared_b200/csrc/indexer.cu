@@ -76,7 +76,19 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- set-up: tile prefix over sequences, barriers, TMEM ---------------
+  // ---- set-up: barriers and TMEM (overlaps the previous kernel's tail) ----
+  pdl_trigger();
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < kAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_ki);
+    tma_prefetch_desc(&tm_qi);
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, Lay::kTmemCols);
+  }
+  // everything below reads what earlier kernels of the stream wrote
+  pdl_wait();
   if (warp == 0) {
     // prefix[b] = sum of ceil(len/128) over earlier sequences (warp scan in chunks)
     int carry = 0;
@@ -101,15 +113,6 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) prefix[B] = carry;
-    if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-      for (int a = 0; a < kAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
-      fence_mbar_init();
-      tma_prefetch_desc(&tm_ki);
-      tma_prefetch_desc(&tm_qi);
-    }
-  } else if (warp == 1) {
-    tmem_alloc(tmem_slot, Lay::kTmemCols);
   }
   tc_fence_before();
   __syncthreads();
@@ -240,8 +243,17 @@ cudaError_t launch_decode(const IndexerArgs& a, const CUtensorMap& tm_ki, const 
   const int64_t tiles_ub = (int64_t)a.B * ((a.S_max + kTile - 1) / kTile);
   int grid = (int)(tiles_ub < num_sms ? tiles_ub : num_sms);
   if (grid < 1) grid = 1;
-  kern<<<grid, kThreads, smem, stream>>>(tm_ki, tm_qi, a.w, a.seq_off, a.seq_len, a.B, a.n_tokens, a.S_max,
-                                        a.H_I, a.scores, a.ld, a.status);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tm_ki, tm_qi, a.w, a.seq_off, a.seq_len, a.B, a.n_tokens, a.S_max, a.H_I,
+                         a.scores, a.ld, a.status);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -24,6 +24,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel of the stream is still running: it must not touch
+// global memory that kernel writes (or reads) before pdl_wait() returns,
+// which happens once the previous kernel has completed and its writes are
+// visible.  pdl_trigger() lets the next kernel of the stream start its own
+// set-up.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -250,6 +260,16 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
 // never reach the attribute API.
 bool smem_attr_done(int dev, const void* fn);
 void smem_attr_mark(int dev, const void* fn);
+
+// Launch attribute that lets a kernel overlap its set-up with the tail of the
+// previous kernel of the stream (the kernel calls pdl_wait() first thing
+// after its set-up).
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = 1;
+  return at;
+}
 
 template <typename Kernel>
 inline cudaError_t ensure_smem(Kernel kern, size_t bytes) {

@@ -170,6 +170,10 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
   const int c = (int)cluster.block_rank();
   const int q = blockIdx.x / G, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
+  pdl_trigger();
+  for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
+  if (tid == 0) sm.cand_ctr = 0;
+  pdl_wait();  // the scores come from the previous kernel of the stream
   int n = n_valid[q];
   if (n < 0 || n > n_max) {
     if (c == 0 && tid == 0) report(status, kErrDevice, kKernTopk, q, n, n_max);
@@ -196,8 +200,6 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
   auto key_at = [&](int i) -> uint32_t { return cached ? sm.keys[i] : order_key(__ldg(&row[beg + i])); };
 
   // ---- phase 0: keys into shared memory, chunk histogram, non-empty bins ----
-  for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
-  if (tid == 0) sm.cand_ctr = 0;
   __syncthreads();
   for (int base0 = 0; base0 < len; base0 += kPass) {
     uint32_t key[kGroups];
@@ -482,13 +484,14 @@ cudaError_t launch_topk_split(const float* scores, int64_t ld, const int32_t* n_
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = sizeof(Smem);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;  // the CTAs of one row form one cluster
   attr[0].val.clusterDim.x = p.G;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, ld, n_valid, n_max, k, p.chunk,
                          reinterpret_cast<uint2*>(scratch), idx, top_scores, status);
   if (e != cudaSuccess) return e;
