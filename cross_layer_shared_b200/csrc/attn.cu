@@ -605,6 +605,9 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     bool got = true;
     if (warp < kSoftWarps) got = warp_wait(recv_bar, 0);
     if (!got && lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 4, warp);
+    // all that was sent to this CTA has landed; its own send slots are still
+    // read by its peers' copies until every CTA of the cluster arrives here
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     if (warp_active && me.valid && got) {
       const uint8_t* base = smem + (recv - sbase);
       const uint8_t* own = smem + (send - sbase) + rank * slot_bytes;
@@ -646,7 +649,8 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         store_out(a, me.qoff + (rank * cw + ci) * 4, f, 4);
       }
     }
-    cluster_sync();  // every bulk copy out of this CTA has been consumed
+    // every bulk copy out of this CTA has been consumed before it exits
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   }
 
   tc_fence_before();
