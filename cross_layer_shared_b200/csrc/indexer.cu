@@ -30,20 +30,27 @@ namespace {
 constexpr int kTile = 128;
 constexpr int kAcc = 4;
 constexpr int kThreads = 192;
-constexpr int kRingBudget = 196608;  // bytes of shared memory for the TMA ring
+constexpr int kMaxStages = 4;  // measured: 4 beats 3, 5 and 6 on B200 (more in flight is slower)
+constexpr int kSmemMax = 232448;  // dynamic shared memory per CTA on sm_100
+
+// full[kMaxStages] empty[kMaxStages] tfull[kAcc] tempty[kAcc] | tmem slot |
+// prefix[B+1] | ring of n_st stages (1024-aligned; as many as fit, up to 6)
+constexpr int kBarOffset = 0;
+constexpr int kTmemSlotOffset = 8 * (2 * kMaxStages + 2 * kAcc);
+constexpr int kPrefixOffset = kTmemSlotOffset + 16;
 
 template <int NHALF, int NPAD>
 struct IdxLayout {
   static constexpr int kABytes = NHALF * kTile * 128;
   static constexpr int kBBytes = NHALF * NPAD * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (kRingBudget / kStageBytes) > 5 ? 5 : (kRingBudget / kStageBytes);
   static constexpr int kTmemCols = (kAcc * NPAD <= 32) ? 32 : (kAcc * NPAD <= 64) ? 64 : (kAcc * NPAD <= 128) ? 128 : 256;
-  // ring | full[kStages] empty[kStages] tfull[kAcc] tempty[kAcc] | tmem slot | prefix[B+1]
-  static constexpr int kBarOffset = kStages * kStageBytes;
-  static constexpr int kTmemSlotOffset = kBarOffset + 8 * (2 * kStages + 2 * kAcc);
-  static constexpr int kPrefixOffset = kTmemSlotOffset + 16;
-  static size_t smem_bytes(int B) { return 1024 + kPrefixOffset + 4 * (size_t)(B + 1); }
+  static int ring_offset(int B) { return (kPrefixOffset + 4 * (B + 1) + 1023) / 1024 * 1024; }
+  static int stages(int B) {
+    const int n = (kSmemMax - 1024 - ring_offset(B)) / kStageBytes;
+    return n > kMaxStages ? kMaxStages : n;
+  }
+  static size_t smem_bytes(int B) { return 1024 + (size_t)ring_offset(B) + (size_t)stages(B) * kStageBytes; }
 };
 
 __device__ __forceinline__ int locate_tile(const int* prefix, int B, int g) {
@@ -61,17 +68,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_constant__ CUtensorMap tm_qi,
                       const float* __restrict__ w, const int64_t* __restrict__ seq_off,
                       const int32_t* __restrict__ seq_len, int B, int64_t n_tokens, int S_max, int H_I,
-                      float* __restrict__ scores, int64_t ld, DeviceStatus* __restrict__ status) {
+                      float* __restrict__ scores, int64_t ld, DeviceStatus* __restrict__ status, int n_st,
+                      int ring_off) {
   using Lay = IdxLayout<NHALF, NPAD>;
-  constexpr int kStages = Lay::kStages;
+  const int kStages = n_st;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kBarOffset);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + kAcc;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kTmemSlotOffset);
-  int* prefix = reinterpret_cast<int*>(smem + Lay::kPrefixOffset);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlotOffset);
+  int* prefix = reinterpret_cast<int*>(smem + kPrefixOffset);
+  uint8_t* ring = smem + ring_off;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -133,7 +142,7 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
         const int b = locate_tile(prefix, B, g);
         const int tl = g - prefix[b];
         const int64_t row = seq_off[b] + (int64_t)tl * kTile;
-        uint8_t* st = smem + s * Lay::kStageBytes;
+        uint8_t* st = ring + s * Lay::kStageBytes;
         mbar_arrive_expect_tx(&full[s], Lay::kStageBytes);
 #pragma unroll
         for (int h = 0; h < NHALF; ++h) tma_load_2d(st + h * kTile * 128, &tm_ki, &full[s], h * 64, (int)row);
@@ -160,7 +169,7 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
           break;
         }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + s * Lay::kStageBytes);
+        const uint32_t a_base = smem_u32(ring + s * Lay::kStageBytes);
         const uint32_t b_base = a_base + Lay::kABytes;
         const uint32_t d = tmem_base + a * NPAD;
 #pragma unroll
@@ -251,8 +260,9 @@ cudaError_t launch_decode(const IndexerArgs& a, const CUtensorMap& tm_ki, const 
   cudaLaunchAttribute attr[1] = {pdl_attribute()};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (Lay::stages(a.B) < 2) return cudaErrorInvalidValue;  // the prefix table would crowd out the ring
   e = cudaLaunchKernelEx(&cfg, kern, tm_ki, tm_qi, a.w, a.seq_off, a.seq_len, a.B, a.n_tokens, a.S_max, a.H_I,
-                         a.scores, a.ld, a.status);
+                         a.scores, a.ld, a.status, Lay::stages(a.B), Lay::ring_offset(a.B));
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
