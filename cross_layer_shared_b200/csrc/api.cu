@@ -285,10 +285,26 @@ sa_status sa_index_score_prefill(const void* qI, const float* w, const void* KI,
   if (!q_pos || !scores) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
   if ((st = check_ws(ws, ws_bytes, sa_index_score_prefill_workspace_size(Nq), who)) != SA_OK) return st;
   if (Nq == 0) return SA_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (sa::indexer_prefill_supported(H_I, d_I)) {
+    // blocks of 256 / H_I queries share every key tile on the tensor cores
+    CUtensorMap tm_ki, tm_qi;
+    const uint64_t kd[2] = {(uint64_t)d_I, (uint64_t)S};
+    const uint64_t ks[1] = {(uint64_t)d_I * 2};
+    const uint32_t kb[2] = {64, 128};
+    if ((st = make_tmap(&tm_ki, KI, 2, kd, ks, kb)) != SA_OK) return st;
+    const uint64_t qd[2] = {(uint64_t)d_I, (uint64_t)Nq * H_I};
+    const uint64_t qs[1] = {(uint64_t)d_I * 2};
+    const uint32_t qb[2] = {64, 256};
+    if ((st = make_tmap(&tm_qi, qI, 2, qd, qs, qb)) != SA_OK) return st;
+    sa::PrefillIndexerArgs a{w, q_pos, Nq, S, max_pos, H_I, d_I, scores, ld, status_of(ws)};
+    cudaError_t e = sa::launch_indexer_prefill(a, tm_ki, tm_qi, num_sms(), s);
+    if (e != cudaSuccess) return cuda_fail("sa_index_score_prefill launch", e);
+    return SA_OK;
+  }
   uint8_t* p = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
   int64_t* soff = reinterpret_cast<int64_t*>(p);
   int32_t* slen = reinterpret_cast<int32_t*>(p + round_up(8 * ((size_t)Nq + 1), 256));
-  cudaStream_t s = (cudaStream_t)stream;
   prefill_rows_kernel<<<(Nq + 256) / 256, 256, 0, s>>>(q_pos, Nq, max_pos, soff, slen, status_of(ws));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail("sa_index_score_prefill rows", e);

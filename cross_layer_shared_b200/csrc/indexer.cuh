@@ -41,6 +41,8 @@ struct PrefillIndexerArgs {
   DeviceStatus* status;
 };
 
+// Block-of-queries kernel: H_I a power of two in [2, 64], d_I 64 or 128.
+bool indexer_prefill_supported(int H_I, int d_I);
 // tm_ki: KI [S, d_I], box (64, 128); tm_qi: qI as 2-D [Nq*H_I, d_I], box (64, 256), 128B swizzle.
 cudaError_t launch_indexer_prefill(const PrefillIndexerArgs& a, const CUtensorMap& tm_ki,
                                    const CUtensorMap& tm_qi, int num_sms, cudaStream_t stream);

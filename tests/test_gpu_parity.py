@@ -304,6 +304,33 @@ def prefill_parity(cfg, dev, q_sample=None, heads=None):
         assert err <= parity.ATOL_F32, f"head {h}: {err}"
 
 
+@pytest.mark.parametrize("H_I,d_I,Nq,S", [
+    (16, 128, 300, 5000),   # blocks of 16 queries, ragged last block
+    (4, 64, 100, 3000),     # blocks of 64 queries
+    (64, 128, 37, 2500),    # blocks of 4 queries
+    (2, 128, 257, 1500),    # blocks of 128 queries
+    (12, 64, 50, 2000),     # not a power of two: the one-query-per-row path
+])
+def test_prefill_indexer_shapes(dev, H_I, d_I, Nq, S):
+    """Every query's scores over its causal prefix, against the oracle, for
+    the block-of-queries kernel (several block sizes) and the general path."""
+    rng = np.random.default_rng(H_I * 1000 + Nq)
+    qI = synth.f32_to_bf16_bits((rng.standard_normal((Nq, H_I, d_I)) / 8).astype(np.float32))
+    KI = synth.f32_to_bf16_bits((rng.standard_normal((S, d_I)) / 8).astype(np.float32))
+    w = rng.uniform(0.1, 1.0, (Nq, H_I)).astype(np.float32)
+    q_pos = (S - Nq + np.arange(Nq)).astype(np.int32)
+    q_pos[::7] = rng.integers(0, S - Nq, len(q_pos[::7]))  # some queries see a short prefix
+    ws = sa.workspace(sa.lib().sa_index_score_prefill_workspace_size(Nq), dev)
+    scores = sa.index_score_prefill(bf16_dev(qI, dev), torch.from_numpy(w).to(dev), bf16_dev(KI, dev),
+                                    torch.from_numpy(q_pos).to(dev), S - 1, ws=ws)
+    assert_status_ok(ws)
+    got = scores.cpu().numpy()
+    for p in range(Nq):
+        n = int(q_pos[p]) + 1
+        ora = oracle.index_score(qI[p:p + 1], w[p:p + 1], KI, [0, S], [0], [n - 1])[0][:n]
+        parity.assert_scores_close(got[p, :n], ora, parity.index_error_bound(qI[p], w[p], KI[:n]), f"p={p}")
+
+
 def test_prefill_small_full_oracle(dev):
     cfg = synth.PrefillConfig("small", S=4096, chunk=256, H_I=16, d_I=128, k=256, block=64, Hq=8, Hkv=2, d=128,
                               seed=77, hot_regions=4, region_len=128)
