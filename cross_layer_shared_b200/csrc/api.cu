@@ -113,6 +113,16 @@ sa_status make_rows_tmap(CUtensorMap* m, const void* base, int64_t rows) {
   return make_tmap(m, base, 2, dims, str, box);
 }
 
+// [rows, 128] bf16 as a 2-D tensor map with a 64 x 64 box (one 64-token KV
+// block, half of its columns, per load)
+sa_status make_block_tmap(CUtensorMap* m, const void* base, int64_t rows) {
+  if (rows < 1 || rows >= (1ll << 31)) return fail(SA_ERR_INVALID_ARG, "tensor of %lld rows: need 1 <= rows < 2^31", (long long)rows);
+  const uint64_t dims[2] = {128, (uint64_t)rows};
+  const uint64_t str[1] = {256};
+  const uint32_t box[2] = {64, 64};
+  return make_tmap(m, base, 2, dims, str, box);
+}
+
 sa::DeviceStatus* status_of(void* ws) { return reinterpret_cast<sa::DeviceStatus*>(ws); }
 
 sa_status check_ws(void* ws, size_t ws_bytes, size_t need, const char* who) {
@@ -519,8 +529,8 @@ sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const
     CUtensorMap tm_q, tm_k, tm_v;
     sa_status st2;
     if ((st2 = make_rows_tmap(&tm_q, Q, (int64_t)Nq * Hq)) != SA_OK) return st2;
-    if ((st2 = make_rows_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
-    if ((st2 = make_rows_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
+    if ((st2 = make_block_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
+    if ((st2 = make_block_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
     e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, s);
   }
   if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill attention", e);
@@ -618,8 +628,8 @@ extern "C" sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const in
     CUtensorMap tm_q, tm_k, tm_v;
     sa_status st2;
     if ((st2 = make_rows_tmap(&tm_q, Q, (int64_t)Nq * Hq)) != SA_OK) return st2;
-    if ((st2 = make_rows_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
-    if ((st2 = make_rows_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
+    if ((st2 = make_block_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
+    if ((st2 = make_block_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
     e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, s);
   }
   if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc attention", e);

@@ -320,21 +320,43 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         if ((lane & 7) == 0) kmask[s * 8 + 4 + (lane >> 3)] = (uint32_t)tc[0];
         __syncwarp();
       }
-      const uint32_t tx = (pw == 0 ? 2 * Lay::kHalf : Lay::kHalf) + (j == 0 && pw > 0 ? Lay::kHalf : 0);
+      // decode: the three warps gather (K lo, V hi), (K hi), (V lo) rows;
+      // prefill: the tile is two whole KV blocks, eight 64 x 64 tile loads
+      // issued by warp 9 (a block past the list reads rows past the tensor:
+      // zeros, so the masked rows of the MMA stay finite)
+      const uint32_t tx = (a.prefill ? (pw == 0 ? 2 * Lay::kTile : 0) : (pw == 0 ? 2 * Lay::kHalf : Lay::kHalf)) +
+                          (j == 0 && pw > 0 ? Lay::kHalf : 0);
       if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx);
       __syncwarp();
-      int rk[4];
+      const uint32_t kst0 = sbase + Lay::kStageOff + s * Lay::kStageBytes;
+      if (a.prefill) {
+        if (pw == 0 && lane == 0) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) rk[i] = (int)(row_base + (tc[i] < 0 ? 0 : tc[i]));
-      const uint32_t kst = sbase + Lay::kStageOff + s * Lay::kStageBytes + 4 * lane * 128;
-      const uint32_t vst = kst + Lay::kTile;
-      if (pw == 0) {
-        tma_gather4(kst, &tm_k, &kv_full[s], 0, rk);
-        tma_gather4(vst + Lay::kHalf, &tm_v, &kv_full[s], 64, rk);
-      } else if (pw == 1) {
-        tma_gather4(kst + Lay::kHalf, &tm_k, &kv_full[s], 64, rk);
+          for (int b2 = 0; b2 < 2; ++b2) {
+            const int jj = ks.kbeg + j * kKT + b2 * 64;  // first entry of the block
+            const int row = jj < ks.kend ? (int)(row_base + (int64_t)a.kv_indices[ks.base + jj / 64] * 64)
+                                         : a.Hkv * a.S;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              tma_load_2d_u32(kst0 + h * Lay::kHalf + b2 * 8192, &tm_k, &kv_full[s], h * 64, row);
+              tma_load_2d_u32(kst0 + Lay::kTile + h * Lay::kHalf + b2 * 8192, &tm_v, &kv_full[s], h * 64, row);
+            }
+          }
+        }
       } else {
-        tma_gather4(vst, &tm_v, &kv_full[s], 0, rk);
+        int rk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rk[i] = (int)(row_base + (tc[i] < 0 ? 0 : tc[i]));
+        const uint32_t kst = kst0 + 4 * lane * 128;
+        const uint32_t vst = kst + Lay::kTile;
+        if (pw == 0) {
+          tma_gather4(kst, &tm_k, &kv_full[s], 0, rk);
+          tma_gather4(vst + Lay::kHalf, &tm_v, &kv_full[s], 64, rk);
+        } else if (pw == 1) {
+          tma_gather4(kst + Lay::kHalf, &tm_k, &kv_full[s], 64, rk);
+        } else {
+          tma_gather4(vst, &tm_v, &kv_full[s], 0, rk);
+        }
       }
       if (j == 0 && pw > 0) {
         int rq[4];

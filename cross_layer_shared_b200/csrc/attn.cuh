@@ -46,8 +46,9 @@ struct AttnArgs {
 };
 
 int attn_num_units(const AttnArgs& a);
-// tm_q / tm_k / tm_v: Q, K, V as 2-D [rows, 128] bf16 tensors, box 64 x 1,
-// 128-byte swizzle (rows gathered four at a time).
+// tm_q / tm_k / tm_v: Q, K, V as 2-D [rows, 128] bf16 tensors, 128-byte
+// swizzle.  tm_q, and tm_k / tm_v in decode: box 64 x 1 (rows gathered four at
+// a time).  tm_k / tm_v in prefill: box 64 x 64 (one KV block per load).
 cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                const CUtensorMap& tm_v, bool precise_p, cudaStream_t stream);
 
