@@ -54,7 +54,7 @@ struct Smem {
   int nlist, cnt_above, ncand, spilled;
   int cpre[kMaxCluster + 1];  // candidate prefix over the cluster's CTAs
   int peer_above[kMaxCluster], peer_spill[kMaxCluster];
-  int spill_any, cand_ctr;
+  int spill_any, cand_ctr, above_ctr;
   int ws[kWarps + 1];
   int bin, before;
 };
@@ -172,7 +172,10 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
   const int lane = tid & 31, warp = tid >> 5;
   pdl_trigger();
   for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
-  if (tid == 0) sm.cand_ctr = 0;
+  if (tid == 0) {
+    sm.cand_ctr = 0;
+    sm.above_ctr = 0;
+  }
   pdl_wait();  // the scores come from the previous kernel of the stream
   int n = n_valid[q];
   if (n < 0 || n > n_max) {
@@ -290,38 +293,42 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
         }
       }
     }
-    int tot_above;
-    block_scan_excl(my_above, sm.ws, &tot_above);
-    if (tid == 0) {
-      const int ncand = sm.cand_ctr;
-      sm.cnt_above = tot_above;
-      sm.ncand = ncand;
-      sm.spilled = ncand > kCandLocal;
-    }
+    // this chunk's count above the bucket: warp sums, one shared atomic each
+    const int wsum = __reduce_add_sync(0xffffffffu, my_above);
+    if (lane == 0 && wsum) atomicAdd(&sm.above_ctr, wsum);
     __syncthreads();
-    if (sm.spilled)  // the whole list then lives in the workspace
+    const int ncand = sm.cand_ctr;
+    const int spilled = ncand > kCandLocal;
+    if (spilled)  // the whole list then lives in the workspace
       for (int p = tid; p < kCandLocal; p += kThreads) my_spill[p] = sm.cand[p];
+    // push this chunk's counts into every CTA of the row (read after the barrier)
+    if (tid < G) {
+      Smem* peer = cluster.map_shared_rank(&sm, tid);
+      peer->cpre[c + 1] = ncand;
+      peer->peer_above[c] = sm.above_ctr;
+      peer->peer_spill[c] = spilled;
+    }
   }
   cluster.sync();
 
   // ---- phase B: exact k-th key, then this chunk's part of the output ----
-  if (tid < G) {
-    const Smem* peer = cluster.map_shared_rank(&sm, tid);
-    sm.cpre[tid + 1] = peer->ncand;
-    sm.peer_above[tid] = peer->cnt_above;
-    sm.peer_spill[tid] = peer->spilled;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int above_before = 0, spill_any = 0;
-    sm.cpre[0] = 0;
-    for (int r = 0; r < G; ++r) {
-      sm.cpre[r + 1] += sm.cpre[r];
-      if (r < c) above_before += sm.peer_above[r];
-      spill_any |= sm.peer_spill[r];
+  if (warp == 0) {  // candidate prefix over the chunks, keys above the bucket before this chunk
+    const int n_r = lane < G ? sm.cpre[lane + 1] : 0;
+    int incl = n_r;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
     }
-    sm.before = above_before;  // keys above the bucket in chunks < c
-    sm.spill_any = spill_any;
+    const int ab = __reduce_add_sync(0xffffffffu, lane < c ? sm.peer_above[lane] : 0);
+    const int sp = __reduce_or_sync(0xffffffffu, lane < G ? sm.peer_spill[lane] : 0);
+    __syncwarp();
+    if (lane < G) sm.cpre[lane + 1] = incl;
+    if (lane == 0) {
+      sm.cpre[0] = 0;
+      sm.before = ab;
+      sm.spill_any = sp;
+    }
   }
   __syncthreads();
   const int above_before = sm.before;
@@ -378,6 +385,9 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
   int tot_sel_before;
   block_scan_excl(sel_before, sm.ws, &tot_sel_before);
   int written = above_before + tot_sel_before;
+  // this CTA reads nothing of its peers from here on; the matching wait
+  // before exit keeps its own lists alive until every peer is past this point
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   for (int base0 = 0; base0 < len; base0 += kPass) {
     uint32_t key[kGroups];
 #pragma unroll
@@ -408,7 +418,7 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
     }
     written += tot;
   }
-  cluster.sync();  // peers may still be reading this CTA's lists
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 struct Plan {
