@@ -42,6 +42,8 @@ SIGNATURES = {
     "sa_decode_step_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "sa_decode_step": ([ctypes.c_char_p, _I, _PP, _PP, _PP, _PP, _PP, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _I,
                         _I, _I, _F, _P, _I, _P, _P, _I64, _P, _SZ, _P], _I),
+    "sa_decode_step_ex": ([ctypes.c_char_p, _I, _PP, _PP, _PP, _PP, _PP, _PP, _PP, _PP, _P, _P, _I, _I64, _I, _I,
+                           _I, _I, _P, _I, _I, _I, _F, _P, _I, _P, _P, _I64, _I, _P, _SZ, _P], _I),
     "sa_block_union_prefill_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "sa_block_union_prefill": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
                                _I),
@@ -193,11 +195,18 @@ def _ptr_array(ts: Sequence[Optional[torch.Tensor]]):
     return ctypes.cast(arr, _PP), arr
 
 
+STEP_PER_LAYER = 1
+
+
 def decode_step(pattern: str, qI: Sequence, w: Sequence, KI: Sequence, K: Sequence, V: Sequence, seq_off, seq_len,
                 S_max: int, k: int, Q, Hkv: int, scale: float, out_dtype=torch.bfloat16, O=None, idx=None,
-                scores=None, ws=None, stream=None):
+                scores=None, ws=None, stream=None, new_KI: Optional[Sequence] = None,
+                new_K: Optional[Sequence] = None, new_V: Optional[Sequence] = None, per_layer: bool = False):
     """One decode step over `pattern` (per-layer lists; entries of S layers'
-    indexer inputs may be None).  Returns (O, idx of the last F layer)."""
+    indexer inputs may be None).  With new_KI (and new_K / new_V) per layer,
+    the new token's rows are written into the caches first (sa_decode_step_ex);
+    per_layer runs one attention launch per layer.  Returns (O, idx of the
+    last F layer)."""
     L, B, Hq, d = Q.shape
     n = len(pattern)
     assert L == n and len(K) == n and len(V) == n
@@ -219,9 +228,23 @@ def decode_step(pattern: str, qI: Sequence, w: Sequence, KI: Sequence, K: Sequen
         arrays.append(p)
         keep.append(a)
     code = SA_F32 if O.dtype == torch.float32 else SA_BF16
-    _check(lib().sa_decode_step(pattern.encode(), n, *arrays, _ptr(seq_off), _ptr(seq_len), B, n_tokens, S_max, H_I,
-                                d_I, k, _ptr(Q), Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(idx), _ptr(scores),
-                                scores.shape[1], _ptr(ws), ws.numel(), _stream(stream)))
+    if new_KI is None and new_K is None and not per_layer:
+        _check(lib().sa_decode_step(pattern.encode(), n, *arrays, _ptr(seq_off), _ptr(seq_len), B, n_tokens, S_max,
+                                    H_I, d_I, k, _ptr(Q), Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(idx),
+                                    _ptr(scores), scores.shape[1], _ptr(ws), ws.numel(), _stream(stream)))
+        return O, idx
+    extra = []
+    for lst in (new_KI, new_K, new_V):
+        if lst is None:
+            extra.append(None)
+        else:
+            p, a = _ptr_array(lst)
+            extra.append(p)
+            keep.append(a)
+    _check(lib().sa_decode_step_ex(pattern.encode(), n, *arrays, *extra, _ptr(seq_off), _ptr(seq_len), B, n_tokens,
+                                   S_max, H_I, d_I, k, _ptr(Q), Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(idx),
+                                   _ptr(scores), scores.shape[1], STEP_PER_LAYER if per_layer else 0, _ptr(ws),
+                                   ws.numel(), _stream(stream)))
     return O, idx
 
 

@@ -178,7 +178,8 @@ sa_status validate_index(const void* qI, const float* w, const void* KI, int H_I
 
 sa_status run_index_decode(const void* qI, const float* w, const void* KI, const int64_t* seq_off,
                            const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I,
-                           float* scores, int64_t ld, void* ws, cudaStream_t stream) {
+                           float* scores, int64_t ld, void* ws, cudaStream_t stream,
+                           const sa::AppendArgs& ap = sa::AppendArgs{}) {
   CUtensorMap tm_ki, tm_qi;
   {
     const uint64_t dims[2] = {(uint64_t)d_I, (uint64_t)n_tokens};
@@ -195,7 +196,7 @@ sa_status run_index_decode(const void* qI, const float* w, const void* KI, const
     sa_status st = make_tmap(&tm_qi, qI, 3, dims, str, box);
     if (st != SA_OK) return st;
   }
-  sa::IndexerArgs a{w, seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, status_of(ws)};
+  sa::IndexerArgs a{w, seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, status_of(ws), ap};
   cudaError_t e = sa::launch_indexer_decode(a, tm_ki, tm_qi, npad, num_sms(), stream);
   if (e != cudaSuccess) return cuda_fail("sa_index_score launch", e);
   return SA_OK;
@@ -262,10 +263,22 @@ size_t sa_index_score_workspace_size(int B) {
   return SA_WS_HEADER_BYTES;
 }
 
+static sa_status index_score_impl(const void* qI, const float* w, const void* KI, const int64_t* seq_off,
+                                  const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I,
+                                  float* scores, int64_t ld, void* ws, size_t ws_bytes, void* stream,
+                                  const sa::AppendArgs& ap, const char* who);
+
 sa_status sa_index_score(const void* qI, const float* w, const void* KI, const int64_t* seq_off,
                          const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I, float* scores,
                          int64_t ld, void* ws, size_t ws_bytes, void* stream) {
-  const char* who = "sa_index_score";
+  return index_score_impl(qI, w, KI, seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, ws, ws_bytes,
+                          stream, sa::AppendArgs{}, "sa_index_score");
+}
+
+static sa_status index_score_impl(const void* qI, const float* w, const void* KI, const int64_t* seq_off,
+                                  const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I,
+                                  float* scores, int64_t ld, void* ws, size_t ws_bytes, void* stream,
+                                  const sa::AppendArgs& ap, const char* who) {
   if (B < 0 || B > 4096) return fail(SA_ERR_INVALID_ARG, "%s: B=%d outside [0, 4096]", who, B);
   if (S_max < 0) return fail(SA_ERR_INVALID_ARG, "%s: S_max=%d < 0", who, S_max);
   if (n_tokens < 1 || n_tokens >= (1ll << 31)) return fail(SA_ERR_INVALID_ARG, "%s: n_tokens=%lld outside [1, 2^31)", who, (long long)n_tokens);
@@ -276,7 +289,7 @@ sa_status sa_index_score(const void* qI, const float* w, const void* KI, const i
   if ((st = check_ws(ws, ws_bytes, sa_index_score_workspace_size(B), who)) != SA_OK) return st;
   if (B == 0 || S_max == 0) return SA_OK;
   return run_index_decode(qI, w, KI, seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, ws,
-                          (cudaStream_t)stream);
+                          (cudaStream_t)stream, ap);
 }
 
 size_t sa_index_score_prefill_workspace_size(int Nq) {
@@ -432,6 +445,19 @@ sa_status sa_decode_step(const char* pattern, int n_layers, const void* const* q
                          const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I, int k,
                          const void* Q, int Hq, int Hkv, int d, float scale, void* O, sa_dtype out_dtype, int32_t* idx,
                          float* scores, int64_t ld, void* ws, size_t ws_bytes, void* stream) {
+  return sa_decode_step_ex(pattern, n_layers, qI, w, const_cast<void* const*>(KI), const_cast<void* const*>(K),
+                           const_cast<void* const*>(V), nullptr, nullptr, nullptr, seq_off, seq_len, B, n_tokens,
+                           S_max, H_I, d_I, k, Q, Hq, Hkv, d, scale, O, out_dtype, idx, scores, ld, 0, ws, ws_bytes,
+                           stream);
+}
+
+sa_status sa_decode_step_ex(const char* pattern, int n_layers, const void* const* qI, const float* const* w,
+                            void* const* KI, void* const* K, void* const* V, const void* const* new_KI,
+                            const void* const* new_K, const void* const* new_V, const int64_t* seq_off,
+                            const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I, int d_I, int k,
+                            const void* Q, int Hq, int Hkv, int d, float scale, void* O, sa_dtype out_dtype,
+                            int32_t* idx, float* scores, int64_t ld, int flags, void* ws, size_t ws_bytes,
+                            void* stream) {
   const char* who = "sa_decode_step";
   if (!pattern || n_layers < 1) return fail(SA_ERR_INVALID_ARG, "%s: empty layer pattern", who);
   if ((int)strnlen(pattern, (size_t)n_layers + 1) < n_layers)
@@ -442,6 +468,24 @@ sa_status sa_decode_step(const char* pattern, int n_layers, const void* const* q
     if (pattern[l] != 'F' && pattern[l] != 'S') return fail(SA_ERR_INVALID_ARG, "%s: pattern letters are F or S", who);
   if (!qI || !w || !KI || !K || !V) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer array", who);
   if (B < 1 || !Q || !O || !idx || !scores) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer or B < 1", who);
+  if (flags & ~SA_STEP_PER_LAYER) return fail(SA_ERR_INVALID_ARG, "%s: unknown flags 0x%x", who, flags);
+  if ((new_K == nullptr) != (new_V == nullptr))
+    return fail(SA_ERR_INVALID_ARG, "%s: new_K and new_V come together", who);
+  if (new_K && !new_KI) return fail(SA_ERR_INVALID_ARG, "%s: a K/V append needs new_KI too", who);
+  if (new_KI) {
+    int f = 0;
+    for (int l = 0; l < n_layers; ++l) {
+      if (pattern[l] == 'F') {
+        f = l;
+        if (!new_KI[l] || !aligned(new_KI[l], 16) || (new_K && (!new_K[l] || !new_V[l] || !aligned(new_K[l], 16) ||
+                                                                !aligned(new_V[l], 16))))
+          return fail(SA_ERR_INVALID_ARG, "%s: layer %d: new rows must be non-NULL and 16-byte aligned", who, l);
+      } else if (new_K && (K[l] != K[f] || V[l] != V[f])) {
+        return fail(SA_ERR_UNSUPPORTED, "%s: appending needs every layer to read its F layer's KV cache (layer %d)",
+                    who, l);
+      }
+    }
+  }
   sa_status st = check_ws(ws, ws_bytes, sa_decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k), who);
   if (st != SA_OK) return st;
   const size_t esize = out_dtype == SA_F32 ? 4 : 2;
@@ -449,15 +493,31 @@ sa_status sa_decode_step(const char* pattern, int n_layers, const void* const* q
   int l = 0;
   while (l < n_layers) {
     if (pattern[l] == 'F') {
-      st = sa_index_score(qI[l], w[l], KI[l], seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, ws,
-                          ws_bytes, stream);
+      sa::AppendArgs ap{};
+      if (new_KI) {
+        ap.qI = static_cast<const uint16_t*>(qI[l]);
+        ap.new_KI = static_cast<const uint16_t*>(new_KI[l]);
+        ap.KI = static_cast<uint16_t*>(KI[l]);
+        if (new_K) {
+          ap.new_K = static_cast<const uint16_t*>(new_K[l]);
+          ap.new_V = static_cast<const uint16_t*>(new_V[l]);
+          ap.K = static_cast<uint16_t*>(K[l]);
+          ap.V = static_cast<uint16_t*>(V[l]);
+        }
+        ap.Hkv = Hkv;
+        ap.d = d;
+      }
+      st = index_score_impl(qI[l], w[l], KI[l], seq_off, seq_len, B, n_tokens, S_max, H_I, d_I, scores, ld, ws,
+                            ws_bytes, stream, ap, who);
       if (st != SA_OK) return st;
       st = sa_topk(scores, ld, seq_len, B, S_max, k, idx, nullptr, ws, ws_bytes, stream);
       if (st != SA_OK) return st;
     }
-    // fuse the following S layers that read the same cache into one group call
+    // fuse the following S layers that read the same cache into one group
+    // call, unless each layer is to run on its own
     int m = l;
-    while (m + 1 < n_layers && pattern[m + 1] == 'S' && K[m + 1] == K[l] && V[m + 1] == V[l]) ++m;
+    if (!(flags & SA_STEP_PER_LAYER))
+      while (m + 1 < n_layers && pattern[m + 1] == 'S' && K[m + 1] == K[l] && V[m + 1] == V[l]) ++m;
     st = run_decode_attn(reinterpret_cast<const uint8_t*>(Q) + (size_t)l * layer_elems * 2, K[l], V[l], seq_off,
                          seq_len, idx, m - l + 1, B, n_tokens, Hq, Hkv, d, k, scale,
                          reinterpret_cast<uint8_t*>(O) + (size_t)l * layer_elems * esize, out_dtype, ws, ws_bytes,

@@ -63,13 +63,49 @@ __device__ __forceinline__ int locate_tile(const int* prefix, int B, int g) {
   return lo;
 }
 
+// One warp, for the new token of sequence b (row len-1 of its caches): copies
+// its indexer key and its K / V rows of every KV head into the caches, then
+// stores its score computed from the fresh key (lane l takes key components
+// l, l+32, ..; the per-head sums are butterfly reductions, identical in
+// every lane).  Tiles that loaded this row from the cache are not used for it.
+__device__ __noinline__ void append_new_token(const AppendArgs& ap, const float* __restrict__ w,
+                                              const int64_t* __restrict__ seq_off, int b, int len, int H_I,
+                                              int d_I, float* score_out, int lane) {
+  const int64_t off = seq_off[b];
+  const uint16_t* nk = ap.new_KI + (int64_t)b * d_I;
+  uint16_t* kdst = ap.KI + (off + len - 1) * d_I;
+  for (int c = lane * 8; c < d_I; c += 256)
+    *reinterpret_cast<uint4*>(kdst + c) = *reinterpret_cast<const uint4*>(nk + c);
+  if (ap.new_K != nullptr) {
+    const int per_row = ap.d / 8;  // 16-byte pieces of a row
+    for (int i = lane; i < ap.Hkv * per_row; i += 32) {
+      const int h = i / per_row, pc = i % per_row;
+      const int64_t row = off * ap.Hkv + (int64_t)h * len + (len - 1);
+      const int64_t src = ((int64_t)b * ap.Hkv + h) * ap.d;
+      reinterpret_cast<uint4*>(ap.K + row * ap.d)[pc] = reinterpret_cast<const uint4*>(ap.new_K + src)[pc];
+      reinterpret_cast<uint4*>(ap.V + row * ap.d)[pc] = reinterpret_cast<const uint4*>(ap.new_V + src)[pc];
+    }
+  }
+  float acc = 0.f;
+  for (int j = 0; j < H_I; ++j) {
+    const uint16_t* q = ap.qI + ((int64_t)b * H_I + j) * d_I;
+    float part = 0.f;
+    for (int c = lane; c < d_I; c += 32)
+      part = fmaf(__uint_as_float((uint32_t)q[c] << 16), __uint_as_float((uint32_t)nk[c] << 16), part);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    acc = fmaf(__ldg(&w[(int64_t)b * H_I + j]), fmaxf(part, 0.f), acc);
+  }
+  if (lane == 0) *score_out = __fadd_rn(acc, 0.f);  // canonical +0
+}
+
 template <int NHALF, int NPAD>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_constant__ CUtensorMap tm_qi,
                       const float* __restrict__ w, const int64_t* __restrict__ seq_off,
                       const int32_t* __restrict__ seq_len, int B, int64_t n_tokens, int S_max, int H_I,
                       float* __restrict__ scores, int64_t ld, DeviceStatus* __restrict__ status, int n_st,
-                      int ring_off) {
+                      int ring_off, const AppendArgs ap) {
   using Lay = IdxLayout<NHALF, NPAD>;
   const int kStages = n_st;
   extern __shared__ uint8_t smem_raw[];
@@ -221,7 +257,10 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
       int len = seq_len[b];
       len = len < 0 ? 0 : (len > S_max ? S_max : len);
       const int t = (g - prefix[b]) * kTile + r;
-      if (t < len) {
+      // the new token's row, when this call appends it, is scored below from
+      // its fresh key (the tile may hold the stale cache row)
+      const int t_new = (ap.new_KI != nullptr) ? len - 1 : -1;
+      if (t < len && t != t_new) {
         float acc = 0.f;
 #pragma unroll
         for (int j = 0; j < NPAD; ++j)
@@ -230,6 +269,8 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
         if (t == 0 && seq_off[b] + len > n_tokens)
           report(status, kErrDevice, kKernIndexer, b, seq_off[b] + len, n_tokens);
       }
+      if (t_new >= 0 && t_new / kTile == g - prefix[b] && (t_new % kTile) / 32 == quarter)
+        append_new_token(ap, w, seq_off, b, len, H_I, 64 * NHALF, scores + (int64_t)b * ld + t_new, lane);
     }
   }
 
@@ -262,7 +303,7 @@ cudaError_t launch_decode(const IndexerArgs& a, const CUtensorMap& tm_ki, const 
   cfg.numAttrs = 1;
   if (Lay::stages(a.B) < 2) return cudaErrorInvalidValue;  // the prefix table would crowd out the ring
   e = cudaLaunchKernelEx(&cfg, kern, tm_ki, tm_qi, a.w, a.seq_off, a.seq_len, a.B, a.n_tokens, a.S_max, a.H_I,
-                         a.scores, a.ld, a.status, Lay::stages(a.B), Lay::ring_offset(a.B));
+                         a.scores, a.ld, a.status, Lay::stages(a.B), Lay::ring_offset(a.B), a.ap);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -9,6 +9,21 @@
 
 namespace sa {
 
+// The new token of every sequence (position seq_len[b] - 1), written into
+// the caches by the decode indexer and scored from its fresh indexer key.
+// All pointers null: no append.
+struct AppendArgs {
+  const uint16_t* qI;      // [B, H_I, d_I]: the queries, for the new token's score
+  const uint16_t* new_KI;  // [B, d_I]
+  uint16_t* KI;            // the indexer-key cache (rows packed by seq_off)
+  const uint16_t* new_K;   // [B, Hkv, d] (may be null: no K/V append)
+  const uint16_t* new_V;
+  uint16_t* K;             // the KV cache: sequence b at seq_off[b]*Hkv*d, [Hkv, seq_len[b], d]
+  uint16_t* V;
+  int Hkv;
+  int d;
+};
+
 struct IndexerArgs {
   const float* w;
   const int64_t* seq_off;
@@ -21,6 +36,7 @@ struct IndexerArgs {
   float* scores;
   int64_t ld;
   DeviceStatus* status;
+  AppendArgs ap;
 };
 
 // tm_ki: KI [n_tokens, d_I] bf16, box (64, 128), 128B swizzle.

@@ -212,6 +212,40 @@ sa_status sa_decode_step(const char* pattern, int n_layers, const void* const* q
                          void* stream);
 
 /* ------------------------------------------------------------------------
+ * The decode step with the new token appended to the caches, and/or one
+ * attention launch per layer.  The pages define neither; they are the steps
+ * either side of the shared-index path in a real decoder: the new token's
+ * indexer key and K/V rows enter the caches before they are searched, and
+ * layer l+1's queries only exist after layer l has run.
+ *
+ * Same arguments as sa_decode_step, plus:
+ *   new_KI  host array (n_layers entries, read at F layers; or NULL: no
+ *           append): device pointer to [B, d_I] bf16, the new token's
+ *           indexer key of every sequence.  It is written to row
+ *           seq_off[b] + seq_len[b] - 1 of KI[l] (seq_len counts the new
+ *           token) and its score is computed from this fresh row.
+ *   new_K, new_V  host arrays (or both NULL): device pointers to [B, Hkv, d]
+ *           bf16, the new token's K / V rows, written to position
+ *           seq_len[b] - 1 of every head of the cache K[l], V[l] of each F
+ *           layer.  Every S layer must then read its F layer's cache
+ *           (SA_ERR_UNSUPPORTED otherwise).  Needs new_KI.
+ *   flags   0, or SA_STEP_PER_LAYER: one attention launch per layer, no
+ *           fusion of a group's layers (each layer's queries are ready only
+ *           after the previous layer in a real model).  Results are the same
+ *           either way.
+ * KI, K and V are written, hence non-const.  All new rows 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+#define SA_STEP_PER_LAYER 1
+sa_status sa_decode_step_ex(const char* pattern, int n_layers, const void* const* qI,
+                            const float* const* w, void* const* KI, void* const* K, void* const* V,
+                            const void* const* new_KI, const void* const* new_K,
+                            const void* const* new_V, const int64_t* seq_off,
+                            const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int H_I,
+                            int d_I, int k, const void* Q, int Hq, int Hkv, int d, float scale,
+                            void* O, sa_dtype out_dtype, int32_t* idx, float* scores, int64_t ld,
+                            int flags, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Block union + zero-copy paged causal attention for one prefill chunk
  * [CA selection step: map each selected token to its KV block, union over
  * the query blocks of the chunk (Q-block union) and over the query heads

@@ -139,6 +139,28 @@ def paged_prefill_attn(Q, q_pos, K, V, block: int, kv_indptr, kv_indices, scale:
     return out
 
 
+def kv_append(KI, K, V, seq_off, seq_len, new_KI, new_K, new_V, Hkv: int, d: int):
+    """The caches after the new token of every sequence is written at
+    position seq_len[b] - 1 (the length counts the new token): row
+    seq_off[b] + seq_len[b] - 1 of KI gets new_KI[b]; in sequence b's KV
+    region ([Hkv, seq_len[b], d] from element seq_off[b]*Hkv*d) the row of
+    every head at that position gets new_K[b, h] / new_V[b, h].  Plain
+    copies; returns (KI, K, V) as new arrays."""
+    KI = np.array(KI, copy=True)
+    K = np.array(K, copy=True).reshape(-1)
+    V = np.array(V, copy=True).reshape(-1)
+    new_K = np.asarray(new_K).reshape(len(seq_len), Hkv, d)
+    new_V = np.asarray(new_V).reshape(len(seq_len), Hkv, d)
+    for b, n in enumerate(seq_len):
+        t = int(n) - 1
+        KI[int(seq_off[b]) + t] = new_KI[b]
+        for h in range(Hkv):
+            row = (int(seq_off[b]) * Hkv + h * int(n) + t) * d
+            K[row:row + d] = new_K[b, h]
+            V[row:row + d] = new_V[b, h]
+    return KI, K, V
+
+
 def decode_step(pattern: str, qI: Sequence, w: Sequence, KI: Sequence, seq_off, seq_len, k: int,
                 Q, K: Sequence, V: Sequence, Hkv: int, scale: float):
     """One decode step over the layers of `pattern` [IndexCache, technical

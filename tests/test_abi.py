@@ -96,3 +96,19 @@ def test_workspace_sizes_are_host_computable(lib):
     w1 = lib.sa_sparse_decode_attn_workspace_size(24, 4, 32, 8, 128, 2048)
     assert w1 >= sa.WS_HEADER_BYTES
     assert lib.sa_decode_step_workspace_size(24, 4, 131072, 32, 8, 128, 2048) >= w1
+
+
+def test_decode_step_ex_rejects_bad_append_requests(lib):
+    arr = (ctypes.c_void_p * 4)(*([0x7F0000001000] * 4))
+    pp = ctypes.cast(arr, sa._PP)
+    other = (ctypes.c_void_p * 4)(0x7F0000001000, 0x7F0000003000, 0x7F0000001000, 0x7F0000001000)
+    po = ctypes.cast(other, sa._PP)
+
+    def call(K, new_KI, new_K, new_V, flags=0):
+        return lib.sa_decode_step_ex(b"FSSS", 4, pp, pp, pp, K, pp, new_KI, new_K, new_V, FAKE, FAKE, 1, 4096, 4096, 4,
+                                     64, 256, FAKE, 8, 1, 128, 0.088, FAKE, 0, FAKE, FAKE, 4096, flags, FAKE_WS,
+                                     1 << 24, None)
+    assert call(pp, pp, pp, None) == sa.SA_ERR_INVALID_ARG and b"together" in lib.sa_last_error()
+    assert call(pp, None, pp, pp) == sa.SA_ERR_INVALID_ARG and b"new_KI" in lib.sa_last_error()
+    assert call(po, pp, pp, pp) == sa.SA_ERR_UNSUPPORTED and b"F layer" in lib.sa_last_error()
+    assert call(pp, None, None, None, flags=4) == sa.SA_ERR_INVALID_ARG and b"flags" in lib.sa_last_error()

@@ -231,6 +231,53 @@ def test_decode_step_c1_matches_oracle_walk(dev):
         assert np.abs(O.cpu().numpy() - O_ora).max() <= parity.ATOL_F32
 
 
+def test_decode_step_append_and_per_layer(dev):
+    """The new token's rows land in the caches bit-exactly (nothing else
+    changes), the step over the appended caches matches the oracle on them,
+    and one attention launch per layer gives the fused group's output bit for
+    bit."""
+    rng = np.random.default_rng(5)
+    lens, H_I, d_I, Hq, Hkv, d, k, pattern = [3000, 1500], 4, 64, 8, 2, 128, 128, "FSSS"
+    B, L = len(lens), len(pattern)
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    T = int(seq_off[-1])
+    scale = 1.0 / math.sqrt(d)
+
+    def bf(shape, sd=1.0):
+        return synth.f32_to_bf16_bits((rng.standard_normal(shape) * sd).astype(np.float32))
+
+    qI, KI, K, V, Q = bf((B, H_I, d_I), 1 / 8), bf((T, d_I), 1 / 8), bf(T * Hkv * d), bf(T * Hkv * d), bf((L, B, Hq, d))
+    w = rng.uniform(0.1, 1.0, (B, H_I)).astype(np.float32)
+    nKI, nK, nV = bf((B, d_I), 1 / 8), bf((B, Hkv, d)), bf((B, Hkv, d))
+    KIa, Ka, Va = oracle.kv_append(KI, K, V, seq_off, lens, nKI, nK, nV, Hkv, d)
+    dKI, dK, dV = bf16_dev(KI, dev), bf16_dev(K, dev), bf16_dev(V, dev)
+    dqI, dw, dQ = bf16_dev(qI, dev), torch.from_numpy(w).to(dev), bf16_dev(Q, dev)
+    d_off = torch.from_numpy(seq_off).to(dev)
+    d_len = torch.tensor(lens, dtype=torch.int32, device=dev)
+    none = [None] * (L - 1)
+    common = ([dK] * L, [dV] * L, d_off, d_len, max(lens), k, dQ, Hkv, scale)
+    O, idx = sa.decode_step(pattern, [dqI] + none, [dw] + none, [dKI] + none, *common, out_dtype=torch.float32,
+                            new_KI=[bf16_dev(nKI, dev)] + none, new_K=[bf16_dev(nK, dev)] + none,
+                            new_V=[bf16_dev(nV, dev)] + none)
+    assert np.array_equal(dKI.cpu().view(torch.int16).numpy().view(np.uint16), KIa)
+    assert np.array_equal(dK.cpu().view(torch.int16).numpy().view(np.uint16), Ka)
+    assert np.array_equal(dV.cpu().view(torch.int16).numpy().view(np.uint16), Va)
+    O_ora, used = oracle.decode_step(pattern, [qI] * L, [w] * L, [KIa] * L, seq_off, lens, k, Q, [Ka] * L, [Va] * L,
+                                     Hkv, scale)
+    got_idx = idx.cpu().numpy()
+    for b in range(B):
+        ora = oracle.index_score(qI[b:b + 1], w[b:b + 1], KIa, seq_off, [b], [lens[b] - 1])[0][:lens[b]]
+        parity.assert_topk_band(got_idx[b], ora, lens[b], k, f"b={b}")
+    if np.array_equal(got_idx, used[0]):
+        assert np.abs(O.cpu().numpy() - O_ora).max() <= parity.ATOL_F32
+    # the caches now hold the new token: per-layer launches against the fused group
+    args = (pattern, [dqI] + none, [dw] + none, [dKI] + none, *common)
+    O_fused, i_fused = sa.decode_step(*args, out_dtype=torch.float32)
+    O_layer, i_layer = sa.decode_step(*args, out_dtype=torch.float32, per_layer=True)
+    assert torch.equal(i_fused, i_layer)
+    assert torch.equal(O_fused, O_layer)
+
+
 def test_shared_index_equals_per_layer_recompute(dev):
     """F,F,F,F with identical indexer inputs gives what F,S,S,S gives."""
     cfg = synth.workload("c1")

@@ -416,3 +416,27 @@ def test_c1_needles_are_selected():
     kth = np.sort(s[0])[::-1][cfg.k - 1]
     for t in needles:
         assert s[0, t] > kth and t in set(idx.tolist())
+
+
+def test_kv_append_writes_only_the_new_token_rows():
+    """The appended caches differ from the old ones exactly at each
+    sequence's last position (every KV head), where they hold the new rows."""
+    rng = np.random.default_rng(3)
+    lens, Hkv, d, d_I = [5, 3], 2, 4, 3
+    seq_off = np.array([0, 5, 8])
+    KI = rng.integers(0, 1000, (8, d_I)).astype(np.uint16)
+    K = rng.integers(0, 1000, 8 * Hkv * d).astype(np.uint16)
+    V = rng.integers(0, 1000, 8 * Hkv * d).astype(np.uint16)
+    nKI = np.full((2, d_I), 7, np.uint16)
+    nK = np.arange(2 * Hkv * d, dtype=np.uint16).reshape(2, Hkv, d) + 2000
+    nV = nK + 1000
+    KIa, Ka, Va = oracle.kv_append(KI, K, V, seq_off, lens, nKI, nK, nV, Hkv, d)
+    assert np.array_equal(KIa[[4, 7]], nKI) and np.array_equal(np.delete(KIa, [4, 7], 0), np.delete(KI, [4, 7], 0))
+    # sequence 0: heads at element rows 0*2+h*5+4; sequence 1: 5*2 + h*3 + 2
+    rows = [4, 9, 12, 15]
+    want = [nK[0, 0], nK[0, 1], nK[1, 0], nK[1, 1]]
+    K3, Ka3 = K.reshape(-1, d), Ka.reshape(-1, d)
+    for r, wv in zip(rows, want):
+        assert np.array_equal(Ka3[r], wv)
+    assert np.array_equal(np.delete(Ka3, rows, 0), np.delete(K3, rows, 0))
+    assert np.array_equal(Va.reshape(-1, d)[rows], np.stack([nV[0, 0], nV[0, 1], nV[1, 0], nV[1, 1]]))
