@@ -610,6 +610,36 @@ def run_ours(args):
     ms_per_step = ms / args.steps
     value = aggregate_rate(args.steps, world, ms)
 
+    # ---- the same step as a real decoder runs it: the new token appended to
+    # the caches first, then one attention launch per layer ----
+    gen = torch.Generator(device="cpu").manual_seed(cfg.seed)
+    rows = {"KI": (torch.randn((cfg.B, cfg.d_I), generator=gen) / 8).to(torch.bfloat16).to(dev),
+            "K": torch.randn((cfg.B, cfg.Hkv, cfg.d), generator=gen).to(torch.bfloat16).to(dev),
+            "V": torch.randn((cfg.B, cfg.Hkv, cfg.d), generator=gen).to(torch.bfloat16).to(dev)}
+
+    def step_seq(st):
+        new_KI = [rows["KI"] if t is not None else None for t in st["qI"]]
+        new_K = [rows["K"] if t is not None else None for t in st["qI"]]
+        new_V = [rows["V"] if t is not None else None for t in st["qI"]]
+        sa.decode_step(cfg.pattern, st["qI"], st["w"], st["KI"], st["K"], st["V"], st["wl"]["seq_off"],
+                       st["wl"]["seq_len"], cfg.S_max, cfg.k, st["wl"]["Q"], cfg.Hkv, cfg.scale, O=st["O"],
+                       idx=st["idx"], scores=st["scores"], ws=st["ws"], new_KI=new_KI, new_K=new_K, new_V=new_V,
+                       per_layer=True)
+
+    for st in sets:
+        step_seq(st)
+    torch.cuda.synchronize()
+    g_seq = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_seq, stream=cap):
+        for j in range(STEPS_PER_GRAPH):
+            step_seq(sets[j % len(sets)])
+    g_seq.replay()
+    n_seq = max(2, min(250, args.steps // STEPS_PER_GRAPH))
+    ms_seq = timed(lambda i: g_seq.replay(), n_seq) / (n_seq * STEPS_PER_GRAPH)
+    seq_launches = 0
+    for l in range(cfg.L):
+        seq_launches += (2 if cfg.pattern[l] == "F" else 0) + 1
+
     # ---- per-kernel device time: each graph holds REP back-to-back launches
     # (alternating input sets, so consecutive launches read different data),
     # which keeps the host's replay cost out of the figure ----
@@ -730,7 +760,7 @@ def run_ours(args):
 
     if world > 1:
         graphs.clear()
-        del multi, g_idx, g_topk, g_attn
+        del multi, g_idx, g_topk, g_attn, g_seq
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
@@ -754,6 +784,11 @@ def run_ours(args):
                      "algorithmic_bytes_per_launch": idx_bytes, "launch_ms": ms_idx,
                      "peak_kind": f"{peak_kind} (burst copy, kernel timed alone)"},
         "kernels_ms": {"indexer": ms_idx, "topk": ms_topk, "attention_group": ms_attn},
+        "per_layer_with_append": {"value": aggregate_rate(1, world, ms_seq), "unit": "steps/s", "ms_per_step": ms_seq,
+                                  "launches_per_step": seq_launches,
+                                  "note": "the new token's rows appended to the caches by the indexer, then one "
+                                          "attention launch per layer (no fusion of the group's layers), as a "
+                                          "decoder that computes layer l+1's queries from layer l runs it"},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "per step: pinned host -> device copy of that step's queries, indexer queries and head "
