@@ -283,9 +283,9 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
 
   if (warp >= kProdWarp0) {
     // =============== producer warps: TMA gathers of K/V (and Q) rows ===============
-    // warp 9: K columns 0-63 and V columns 64-127 (+ validity words);
-    // warp 10: K columns 64-127 (+ Q columns 0-63 on the first tile);
-    // warp 11: V columns 0-63 (+ Q columns 64-127 on the first tile).
+    // warp 9: K columns 0-63 (+ validity words); warp 10: K columns 64-127
+    // (+ Q columns 0-63 on the first tile); warp 11: V columns 0-63 (+ Q
+    // columns 64-127 on the first tile); V columns 64-127 split between them.
     const int pw = warp - kProdWarp0;
     const int64_t row_base = a.prefill ? (int64_t)g * a.S : a.seq_off[b] * a.Hkv + (int64_t)g * ks.len;
     for (int j = 0; j < nt; ++j) {
@@ -324,7 +324,10 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
       // prefill: the tile is two whole KV blocks, eight 64 x 64 tile loads
       // issued by warp 9 (a block past the list reads rows past the tensor:
       // zeros, so the masked rows of the MMA stay finite)
-      const uint32_t tx = (a.prefill ? (pw == 0 ? 2 * Lay::kTile : 0) : (pw == 0 ? 2 * Lay::kHalf : Lay::kHalf)) +
+      // decode: V columns 64-127 are split over the three warps by row group
+      // (lanes [vlo, vhi)), so each issues about 43 gathers per tile
+      const int vlo = pw == 0 ? 0 : (pw == 1 ? 10 : 21), vhi = pw == 0 ? 10 : (pw == 1 ? 21 : 32);
+      const uint32_t tx = (a.prefill ? (pw == 0 ? 2 * Lay::kTile : 0) : Lay::kHalf + (uint32_t)(vhi - vlo) * 512u) +
                           (j == 0 && pw > 0 ? Lay::kHalf : 0);
       if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx);
       __syncwarp();
@@ -349,14 +352,13 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         for (int i = 0; i < 4; ++i) rk[i] = (int)(row_base + (tc[i] < 0 ? 0 : tc[i]));
         const uint32_t kst = kst0 + 4 * lane * 128;
         const uint32_t vst = kst + Lay::kTile;
-        if (pw == 0) {
+        if (pw == 0)
           tma_gather4(kst, &tm_k, &kv_full[s], 0, rk);
-          tma_gather4(vst + Lay::kHalf, &tm_v, &kv_full[s], 64, rk);
-        } else if (pw == 1) {
+        else if (pw == 1)
           tma_gather4(kst + Lay::kHalf, &tm_k, &kv_full[s], 64, rk);
-        } else {
+        else
           tma_gather4(vst, &tm_v, &kv_full[s], 0, rk);
-        }
+        if (lane >= vlo && lane < vhi) tma_gather4(vst + Lay::kHalf, &tm_v, &kv_full[s], 64, rk);
       }
       if (j == 0 && pw > 0) {
         int rq[4];
