@@ -99,7 +99,7 @@ __device__ __noinline__ void append_new_token(const AppendArgs& ap, const float*
   if (lane == 0) *score_out = __fadd_rn(acc, 0.f);  // canonical +0
 }
 
-template <int NHALF, int NPAD>
+template <int NHALF, int NPAD, bool APPEND>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_constant__ CUtensorMap tm_qi,
                       const float* __restrict__ w, const int64_t* __restrict__ seq_off,
@@ -259,7 +259,7 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
       const int t = (g - prefix[b]) * kTile + r;
       // the new token's row, when this call appends it, is scored below from
       // its fresh key (the tile may hold the stale cache row)
-      const int t_new = (ap.new_KI != nullptr) ? len - 1 : -1;
+      const int t_new = APPEND ? len - 1 : -1;
       if (t < len && t != t_new) {
         float acc = 0.f;
 #pragma unroll
@@ -269,7 +269,7 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
         if (t == 0 && seq_off[b] + len > n_tokens)
           report(status, kErrDevice, kKernIndexer, b, seq_off[b] + len, n_tokens);
       }
-      if (t_new >= 0 && t_new / kTile == g - prefix[b] && (t_new % kTile) / 32 == quarter)
+      if (APPEND && t_new >= 0 && t_new / kTile == g - prefix[b] && (t_new % kTile) / 32 == quarter)
         append_new_token(ap, w, seq_off, b, len, H_I, 64 * NHALF, scores + (int64_t)b * ld + t_new, lane);
     }
   }
@@ -286,7 +286,9 @@ template <int NHALF, int NPAD>
 cudaError_t launch_decode(const IndexerArgs& a, const CUtensorMap& tm_ki, const CUtensorMap& tm_qi,
                           int num_sms, cudaStream_t stream) {
   using Lay = IdxLayout<NHALF, NPAD>;
-  auto kern = indexer_decode_kernel<NHALF, NPAD>;
+  // the new-token append is compiled only into the kernel that does it
+  auto kern = a.ap.new_KI != nullptr ? indexer_decode_kernel<NHALF, NPAD, true>
+                                     : indexer_decode_kernel<NHALF, NPAD, false>;
   const size_t smem = Lay::smem_bytes(a.B);
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
