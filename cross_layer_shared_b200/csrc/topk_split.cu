@@ -44,6 +44,7 @@ constexpr int kKeyCache = 16384;            // chunk keys kept in shared memory
 constexpr int kCandLocal = 2048;            // this CTA's candidates, in shared memory
 constexpr int kCandRow = 6144;              // the row's candidates gathered for the refine
 constexpr int kMaxCluster = 16;
+constexpr int kBitWords = 4096;             // chunks up to 131072 keys emit from a bitmap
 
 struct Smem {
   uint32_t keys[kKeyCache];
@@ -51,6 +52,7 @@ struct Smem {
   uint2 list[kBins1];         // (bin, count) of the non-empty bins of this chunk
   uint2 cand[kCandLocal];     // (key, index) of this chunk's keys in the bucket
   uint2 row_cand[kCandRow];
+  uint32_t bits[kBitWords];   // this chunk's selected keys, one bit per key
   int nlist, cnt_above, ncand, spilled;
   int cpre[kMaxCluster + 1];  // candidate prefix over the cluster's CTAs
   int peer_above[kMaxCluster], peer_spill[kMaxCluster];
@@ -259,6 +261,7 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
   find_bin_desc(sm.hist, kBins1, k, sm.ws, &sm.bin, &sm.before);
   const int beta = sm.bin, above = sm.before;
   uint2* my_spill = spill + (int64_t)blockIdx.x * chunk;
+  const bool use_bits = chunk <= kBitWords * 32;
   {
     int my_above = 0;
     for (int base0 = 0; base0 < len; base0 += kPass) {
@@ -276,6 +279,8 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
         my_above += (in && d > beta) ? 1 : 0;
         eqm[gi] = __ballot_sync(0xffffffffu, in && d == beta);
         my += __popc(eqm[gi]);
+        const uint32_t up = __ballot_sync(0xffffffffu, in && d > beta);
+        if (use_bits && lane == 0) sm.bits[pass_pos(base0, warp, gi, 0) >> 5] = up;  // the group's 32 keys, one word
       }
       if (my) {  // one slot reservation per warp and pass; candidate order is free
         int slot = 0;
@@ -388,6 +393,46 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
   // this CTA reads nothing of its peers from here on; the matching wait
   // before exit keeps its own lists alive until every peer is past this point
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  if (use_bits) {
+    // the keys above the bucket are already set; add this chunk's kept bucket
+    // keys, then emit the set bits in index order
+    const int my_nc = sm.cand_ctr;
+    const bool mine_spilled = my_nc > kCandLocal;
+    for (int j = tid; j < my_nc; j += kThreads) {
+      const uint2 v = mine_spilled ? __ldcg(&my_spill[j]) : sm.cand[j];
+      if (v.x > T || (v.x == T && v.y <= cut)) {
+        const uint32_t li = v.y - (uint32_t)beg;
+        atomicOr(&sm.bits[li >> 5], 1u << (li & 31));
+      }
+    }
+    __syncthreads();
+    const int nwl = (len + 31) >> 5;
+    const int per = (nwl + kThreads - 1) / kThreads;
+    int cnt = 0;
+    for (int q2 = 0; q2 < per; ++q2) {
+      const int wi = tid * per + q2;
+      if (wi < nwl) cnt += __popc(sm.bits[wi]);
+    }
+    int tot;
+    int pos = written + block_scan_excl(cnt, sm.ws, &tot);
+    for (int q2 = 0; q2 < per; ++q2) {
+      const int wi = tid * per + q2;
+      if (wi >= nwl) break;
+      uint32_t x = sm.bits[wi];
+      while (x) {
+        const int b = __ffs(x) - 1;
+        x &= x - 1;
+        const int i = beg + (wi << 5) + b;
+        if (pos < k) {
+          out[pos] = i;
+          if (out_s) out_s[pos] = row[i];
+        }
+        ++pos;
+      }
+    }
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    return;
+  }
   for (int base0 = 0; base0 < len; base0 += kPass) {
     uint32_t key[kGroups];
 #pragma unroll
