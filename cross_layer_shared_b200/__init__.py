@@ -9,6 +9,7 @@ Build:  python -m cross_layer_shared_b200.build
 """
 from __future__ import annotations
 
+import array
 import ctypes
 import os
 from typing import List, Optional, Sequence
@@ -191,8 +192,13 @@ def decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k) -> int:
 
 
 def _ptr_array(ts: Sequence[Optional[torch.Tensor]]):
-    arr = (ctypes.c_void_p * len(ts))(*[None if t is None else t.data_ptr() for t in ts])
-    return ctypes.cast(arr, _PP), arr
+    """Host array of device pointers (NULL for None); a tensor listed for many
+    layers is asked for its address once."""
+    memo = {}
+    vals = [0 if t is None else (memo.get(id(t)) or memo.setdefault(id(t), t.data_ptr())) for t in ts]
+    buf = array.array("Q", vals)
+    arr = (ctypes.c_void_p * len(vals)).from_buffer(buf)
+    return ctypes.cast(arr, _PP), (buf, arr)
 
 
 STEP_PER_LAYER = 1
