@@ -22,6 +22,8 @@
 // the workspace; a row with many candidates refines them in place, from the
 // owners' shared memory or their slots (slow, but exact).
 #include <cooperative_groups.h>
+
+#include <atomic>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -487,10 +489,10 @@ size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 // Largest cluster the device schedules for this kernel (16 needs the
 // non-portable size; some parts only give 8).  Looked up once per device.
 int max_cluster() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64];  // per device; every writer stores the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  if (cached[dev]) return cached[dev];
+  if (const int c = cached[dev].load(std::memory_order_relaxed)) return c;
   int g = 8;
   if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
       ensure_smem(topk_cluster_kernel, sizeof(Smem)) == cudaSuccess) {
@@ -509,7 +511,7 @@ int max_cluster() {
     if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &cfg) == cudaSuccess && n >= 1) g = kMaxCluster;
   }
   cudaGetLastError();
-  cached[dev] = g;
+  cached[dev].store(g, std::memory_order_relaxed);
   return g;
 }
 

@@ -44,8 +44,10 @@
  *   there, so the status is sticky until sa_clear_device_status()).  The
  *   rest is scratch owned by the call while it runs on `stream`: calls that
  *   overlap on the GPU must not share one workspace.
- * - The library keeps no global state between calls apart from a cached
- *   driver entry point and the fixed scratch array of
+ * - Between calls the library keeps only per-device facts it looks up once
+ *   (the driver's tensor-map entry point, the SM count, the largest cluster
+ *   the top-k kernel can be scheduled with, which kernels have had their
+ *   shared-memory limit raised) and the fixed scratch array of
  *   sa_block_union_prefill_noalloc (see there); the workspace entry points
  *   are reentrant and thread-safe.
  */
