@@ -534,6 +534,13 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   tc_fence_before();
   __syncthreads();  // every MMA has completed (o_done) and no stage is in use
   tc_fence_after();
+  if (a.n_split > 1) {
+    // this CTA's stages are free for its peers' slices: arm the receive
+    // barrier and arrive; the wait comes after the half merge below
+    if (tid == 0)
+      mbar_arrive_expect_tx(recv_bar, (uint32_t)(a.n_split - 1) * (128u * (16u * (32 / a.n_split) + 8u)));
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  }
   // the two key halves of each row: (m, l) of both, merged per row
   float2* mlx = reinterpret_cast<float2*>(smem + Lay::kStageOff + kMlxOff);  // [2][128]
   if (warp < kSoftWarps)
@@ -591,8 +598,8 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     const uint32_t slot_bytes = 128u * (16u * cw + 8u);  // [128][cw] chunks + [128] (m, l)
     const uint32_t recv = sbase + Lay::kStageOff;                      // [ns] slots, slot s from CTA s
     const uint32_t send = recv + ((ns * slot_bytes + 1023u) & ~1023u);  // [ns] slots, slot t for CTA t
-    if (tid == 0) mbar_arrive_expect_tx(recv_bar, (uint32_t)(ns - 1) * slot_bytes);
-    cluster_sync();  // every CTA is done with its stages and has armed its receive barrier
+    // every CTA is done with its stages and has armed its receive barrier
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
     if (warp_active) {
       const bool live = have_o && me.valid;
       if (half == 0)
