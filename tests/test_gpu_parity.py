@@ -378,6 +378,15 @@ def test_prefill_indexer_shapes(dev, H_I, d_I, Nq, S):
         parity.assert_scores_close(got[p, :n], ora, parity.index_error_bound(qI[p], w[p], KI[:n]), f"p={p}")
 
 
+def test_prefill_ragged_last_block(dev):
+    """A context that is not a whole number of 64-token blocks: the last
+    block is partial (its tile load reaches past the head's keys), every
+    query of the chunk sees it, and G = 2 query heads per KV head."""
+    cfg = synth.PrefillConfig("ragged", S=4000, chunk=160, H_I=16, d_I=128, k=512, block=64, Hq=4, Hkv=2, d=128,
+                              seed=78, hot_regions=3, region_len=128)
+    prefill_parity(cfg, dev)
+
+
 def test_prefill_small_full_oracle(dev):
     cfg = synth.PrefillConfig("small", S=4096, chunk=256, H_I=16, d_I=128, k=256, block=64, Hq=8, Hkv=2, d=128,
                               seed=77, hot_regions=4, region_len=128)
