@@ -49,6 +49,75 @@ def test_generator_twin_is_bit_exact(dev):
     assert np.array_equal(t.view(torch.int16).cpu().numpy().view(np.uint16), want)
 
 
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c5"])
+def test_decode_workload_tensors_match_host_rows(dev, name):
+    """Every device tensor of the decode workloads (first group; planted rows
+    included) equals the host generator's rows bit for bit, on sampled rows
+    of every sequence and KV head."""
+    cfg = synth.workload(name)
+    wl = sgpu.decode_workload(cfg, dev, groups=[0])
+    gr = wl["groups"][0]
+    rng = np.random.default_rng(11)
+
+    def bits(t):
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+    planted = {(b, t) for (b, t, _, _) in cfg.planted(0)}
+    for b in range(0, cfg.B, max(1, cfg.B // 4)):
+        S = cfg.seq_lens[b]
+        rows = np.unique(np.concatenate([rng.integers(0, S, 64), [0, S - 1],
+                                         [t for (bb, t) in planted if bb == b][:8]])).astype(np.int64)
+        got = bits(gr["KI"][torch.from_numpy(cfg.seq_off[b] + rows).to(dev)])
+        assert np.array_equal(got, cfg.KI_rows(0, b, rows)), f"KI b={b}"
+        K3 = gr["K"].view(-1, cfg.d)
+        V3 = gr["V"].view(-1, cfg.d)
+        for h in (0, cfg.Hkv - 1):
+            flat = torch.from_numpy(cfg.seq_off[b] * cfg.Hkv + h * S + rows).to(dev)
+            assert np.array_equal(bits(K3[flat]), cfg.KV_rows(0, b, h, rows, "K")), f"K b={b} h={h}"
+            assert np.array_equal(bits(V3[flat]), cfg.KV_rows(0, b, h, rows, "V")), f"V b={b} h={h}"
+    assert np.array_equal(bits(wl["Q"]), cfg.Q())
+    assert np.array_equal(bits(gr["qI"]), cfg.qI(0))
+
+
+def test_prefill_workload_tensors_match_host_rows(dev):
+    cfg = synth.workload("c4")
+    wl = sgpu.prefill_workload(cfg, dev)
+    rng = np.random.default_rng(12)
+    rows = np.unique(np.concatenate([rng.integers(0, cfg.S, 256), cfg.hot_ki_rows()[0][:16], [cfg.S - 1]]))
+    KI = cfg.KI_full()
+    got = wl["KI"][torch.from_numpy(rows).to(dev)].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, KI[rows])
+    for h in (0, cfg.Hkv - 1):
+        for which in ("K", "V"):
+            got = wl[which][h][torch.from_numpy(rows).to(dev)].view(torch.int16).cpu().numpy().view(np.uint16)
+            assert np.array_equal(got, cfg.KV_rows(h, rows, which)), f"{which} h={h}"
+
+
+def test_key_split_count_does_not_change_the_output(dev):
+    """One (sequence, KV head) alone is split over 8 CTAs of a cluster; the
+    same data inside a batch of 148 units runs unsplit: same output within
+    the fp32 tolerance (only the merge order differs)."""
+    rng = np.random.default_rng(21)
+    d, k, S, Hq, L = 128, 1024, 5000, 4, 6
+    K = synth.f32_to_bf16_bits(rng.standard_normal(S * d).astype(np.float32))
+    V = synth.f32_to_bf16_bits(rng.standard_normal(S * d).astype(np.float32))
+    Q = synth.f32_to_bf16_bits(rng.standard_normal((L, 1, Hq, d)).astype(np.float32))
+    sel = np.sort(rng.choice(S, k, replace=False)).astype(np.int32)
+    one = sa.sparse_decode_attn(bf16_dev(Q, dev), bf16_dev(K, dev), bf16_dev(V, dev),
+                                torch.tensor([0, S], device=dev), torch.tensor([S], dtype=torch.int32, device=dev),
+                                torch.from_numpy(sel[None]).to(dev), 1, 1 / math.sqrt(d), out_dtype=torch.float32)
+    B = 148  # as many units as SMs: no room to split
+    Kb = bf16_dev(np.tile(K, B), dev)
+    Vb = bf16_dev(np.tile(V, B), dev)
+    Qb = bf16_dev(np.repeat(Q, B, axis=1), dev)
+    offs = torch.arange(0, (B + 1) * S, S, device=dev)
+    many = sa.sparse_decode_attn(Qb, Kb, Vb, offs, torch.full((B,), S, dtype=torch.int32, device=dev),
+                                 torch.from_numpy(np.tile(sel, (B, 1))).to(dev), 1, 1 / math.sqrt(d),
+                                 out_dtype=torch.float32)
+    err = (many - one.expand(-1, B, -1, -1)).abs().max().item()
+    assert err <= parity.ATOL_F32, err
+
+
 # --------------------------------------------------------------------------
 def decode_group_parity(cfg, g, seqs, dev, out_dtypes=(torch.bfloat16, torch.float32)):
     wl = sgpu.decode_workload(cfg, dev, groups=[g])

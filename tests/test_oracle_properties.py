@@ -1,0 +1,84 @@
+"""Property-based checks of the oracle on tiny random shapes (CPU): each
+property follows from the definitions, independent of how the oracle
+computes them."""
+import math
+
+import numpy as np
+from hypothesis import given, settings, strategies as st
+
+import oracle
+import synth
+
+
+def bf16(x):
+    return synth.f32_to_bf16_bits(np.asarray(x, np.float32))
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.integers(1, 48), st.integers(1, 20), st.integers(0, 2**31 - 1), st.integers(0, 48))
+def test_topk_is_the_stable_sort_prefix(n, k, seed, n_valid):
+    """Top-k = the first min(k, n_valid) entries of the sort by (score
+    descending, index ascending), emitted in ascending index order, padded
+    with -1.  Scores drawn from a few values so that ties are common."""
+    n_valid = min(n_valid, n)
+    rng = np.random.default_rng(seed)
+    s = rng.integers(-3, 4, n).astype(np.float32) / 2
+    got = oracle.topk(s[None], [n_valid], k)[0]
+    order = sorted(range(n_valid), key=lambda i: (-float(s[i]), i))[:k]
+    want = np.full(k, -1, np.int32)
+    want[: len(order)] = sorted(order)
+    assert np.array_equal(got, want)
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.integers(1, 40), st.integers(1, 6), st.integers(0, 2**31 - 1))
+def test_attention_is_invariant_to_selection_order_and_duplicate_padding(S, k, seed):
+    """Softmax attention over a set of keys: permuting the selected entries
+    or appending -1 padding changes nothing."""
+    rng = np.random.default_rng(seed)
+    d, Hq, Hkv = 8, 2, 1
+    k = min(k, S)
+    Q = bf16(rng.standard_normal((1, 1, Hq, d)))
+    K = bf16(rng.standard_normal(S * Hkv * d))
+    V = bf16(rng.standard_normal(S * Hkv * d))
+    sel = rng.choice(S, k, replace=False).astype(np.int32)
+    a = oracle.sparse_decode_attn(Q, K, V, [0, S], [S], np.sort(sel)[None], Hkv, 1 / math.sqrt(d))
+    perm = rng.permutation(sel)
+    padded = np.concatenate([perm, np.full(3, -1, np.int32)])[None]
+    b = oracle.sparse_decode_attn(Q, K, V, [0, S], [S], padded, Hkv, 1 / math.sqrt(d))
+    assert np.allclose(a, b, rtol=0, atol=1e-12)
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.integers(1, 12), st.integers(64, 700), st.integers(1, 40), st.integers(0, 2**31 - 1))
+def test_block_union_covers_exactly_the_selected_blocks(Nq, S, k, seed):
+    """The table of every group is the sorted set of blocks holding a
+    selected token: every selected token's block is listed (coverage) and
+    every listed block holds one (minimality)."""
+    rng = np.random.default_rng(seed)
+    k = min(k, S)
+    idx = np.stack([rng.choice(S, k, replace=False) for _ in range(Nq)]).astype(np.int32)
+    idx[rng.random(idx.shape) < 0.1] = -1
+    ptr, ind = oracle.block_union(idx, S, 64, 2)
+    want = sorted({int(t) // 64 for t in idx.ravel() if t >= 0})
+    assert ptr[0] == 0 and ptr[1] - ptr[0] == len(want) and ptr[2] - ptr[1] == len(want)
+    assert list(ind[: len(want)]) == want and list(ind[len(want): 2 * len(want)]) == want
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.integers(1, 30), st.integers(1, 4), st.integers(0, 2**31 - 1))
+def test_index_score_is_monotone_in_each_head_weight(S, H_I, seed):
+    """Raising one head's weight never lowers a score (ReLU terms are >= 0),
+    and scaling every weight by 2 doubles every score exactly."""
+    rng = np.random.default_rng(seed)
+    d_I = 8
+    qI = bf16(rng.standard_normal((1, H_I, d_I)) / 4)
+    KI = bf16(rng.standard_normal((S, d_I)) / 4)
+    w = rng.uniform(0.1, 1.0, (1, H_I)).astype(np.float32)
+    base = oracle.index_score(qI, w, KI, [0, S], [0], [S - 1])[0][:S]
+    w2 = w.copy()
+    w2[0, rng.integers(H_I)] *= 1.5
+    up = oracle.index_score(qI, w2, KI, [0, S], [0], [S - 1])[0][:S]
+    assert np.all(up >= base)
+    dbl = oracle.index_score(qI, 2 * w, KI, [0, S], [0], [S - 1])[0][:S]
+    assert np.array_equal(dbl, 2 * base)
