@@ -50,6 +50,7 @@ def load(path: str):
     lb.oracle_block_union.argtypes = [P, I, I, I, I, I, P, P]
     lb.oracle_block_union.restype = I
     lb.oracle_paged_prefill_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, D, P]
+    lb.oracle_indexer_layer_attn.argtypes = [P, P, P, P, P, I, I, I, I, I, D, P, P, I64, P]
     lb.oracle_num_threads.restype = I
     return lb
 
@@ -111,6 +112,39 @@ def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float) -
                                     _p(_c(seq_len, np.int32)), _p(idx), L, B, Hq, Hkv, d, k,
                                     float(scale), _p(out))
     return out
+
+
+def indexer_layer_attn(Q, K, V, seq_off, seq_len, Hkv: int, scale: float, ld: Optional[int] = None):
+    """The CLSA indexer layer as a full attention layer whose weights route
+    the shared index: (O [B,Hq,d] fp64 dense output, route [B, ld] fp32 with
+    route[b,t] = sum over heads of the attention weight of token t; entries
+    past seq_len[b] are NaN)."""
+    Q = _c(Q, np.uint16)
+    B, Hq, d = Q.shape
+    seq_len = _c(seq_len, np.int32)
+    S_max = int(seq_len.max()) if B else 0
+    ld = int(ld if ld is not None else max(S_max, 1))
+    O = np.empty((B, Hq, d), dtype=np.float64)
+    route = np.full((B, ld), np.nan, dtype=np.float32)
+    P = np.empty((B, Hq, max(S_max, 1)), dtype=np.float64)
+    lib().oracle_indexer_layer_attn(_p(Q), _p(_c(K, np.uint16)), _p(_c(V, np.uint16)), _p(_c(seq_off, np.int64)),
+                                    _p(seq_len), B, Hq, Hkv, d, max(S_max, 1), float(scale), _p(O), _p(route), ld,
+                                    _p(P))
+    return O, route
+
+
+def decode_step_attn_route(Q, K, V, seq_off, seq_len, k: int, Hkv: int, scale: float):
+    """One decode step of a cross-decoder group under the CLSA reading in
+    which layer 0 is the indexer layer: it attends densely, the top-k of its
+    summed attention weights is the index, and layers 1..L-1 reuse that index
+    over the same cache.  Returns (O [L,B,Hq,d] fp64, idx [B,k], route)."""
+    Q = np.asarray(Q)
+    O0, route = indexer_layer_attn(Q[0], K, V, seq_off, seq_len, Hkv, scale)
+    idx = topk(route, seq_len, k)
+    out = [O0]
+    if Q.shape[0] > 1:
+        out.extend(sparse_decode_attn(Q[1:], K, V, seq_off, seq_len, idx, Hkv, scale))
+    return np.stack(out), idx, route
 
 
 def block_union(idx, S: int, block: int, Hkv: int):

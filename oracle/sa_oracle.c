@@ -263,6 +263,62 @@ void oracle_paged_prefill_attn(const uint16_t* Q, const int32_t* q_pos, const ui
   }
 }
 
+/*
+ * The CLSA indexer layer read as a full attention layer whose attention
+ * weights give the routing index [CLSA, section "La precision reste
+ * stable": the index is computed once from the attention scores of the
+ * indexer layer, which sees the same query state and cache as every other
+ * layer].  For sequence b and query head h (KV head g = h / (Hq/Hkv)), over
+ * every cached token t < seq_len[b]:
+ *   z_t     = scale * (Q[b,h] . K[g,t])
+ *   p_{h,t} = exp(z_t - max z) / sum_u exp(z_u - max z)     (the attention weights)
+ *   O[b,h]  = sum_t p_{h,t} V[g,t]                           (the layer's dense output)
+ *   route[b,t] = sum_h p_{h,t}, heads in ascending order, rounded once to fp32
+ * Q [B,Hq,d]; K, V as in oracle_sparse_decode_attn; O [B,Hq,d] fp64;
+ * route [B, ld] fp32, entries t >= seq_len[b] untouched.  P is scratch of
+ * B*Hq*S_max doubles (the weights of every head, summed in head order).
+ */
+void oracle_indexer_layer_attn(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                               const int64_t* seq_off, const int32_t* seq_len, int B, int Hq, int Hkv,
+                               int d, int S_max, double scale, double* O, float* route, int64_t ld,
+                               double* P) {
+  const int G = Hq / Hkv;
+  const int64_t rows = (int64_t)B * Hq;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < rows; ++r) {
+    const int b = (int)(r / Hq);
+    const int h = (int)(r % Hq);
+    const int g = h / G;
+    const int64_t S = seq_len[b];
+    const uint16_t* Kb = K + seq_off[b] * Hkv * d + (int64_t)g * S * d;
+    const uint16_t* Vb = V + seq_off[b] * Hkv * d + (int64_t)g * S * d;
+    const uint16_t* q = Q + r * d;
+    double* o = O + r * d;
+    double* p = P + r * (int64_t)S_max;
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    double m = -INFINITY;
+    for (int64_t t = 0; t < S; ++t) {
+      double dot = 0.0;
+      for (int c = 0; c < d; ++c) dot += bf(q[c]) * bf(Kb[t * d + c]);
+      p[t] = scale * dot;
+      if (p[t] > m) m = p[t];
+    }
+    double den = 0.0;
+    for (int64_t t = 0; t < S; ++t) den += exp(p[t] - m);
+    for (int64_t t = 0; t < S; ++t) {
+      p[t] = exp(p[t] - m) / den;
+      for (int c = 0; c < d; ++c) o[c] += p[t] * bf(Vb[t * d + c]);
+    }
+  }
+#pragma omp parallel for schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int64_t t = 0; t < seq_len[b]; ++t) {
+      double acc = 0.0;
+      for (int h = 0; h < Hq; ++h) acc += P[((int64_t)b * Hq + h) * S_max + t];
+      route[(int64_t)b * ld + t] = (float)acc;
+    }
+}
+
 /* threads OpenMP will use (reported next to CPU timings) */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

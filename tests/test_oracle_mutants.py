@@ -26,6 +26,14 @@ MUTANTS = {
     "ceil block map": ("if (t >= 0) mark[t / block] = 1;", "if (t >= 0) mark[(t + block - 1) / block] = 1;"),
     "causal strict": ("if (t <= q_pos[p] && t < S) keys[n++] = t;", "if (t < q_pos[p] && t < S) keys[n++] = t;"),
     "value row of the wrong token": ("const uint16_t* vr = Vb + keys[j] * d;", "const uint16_t* vr = Vb + keys[0] * d;"),
+    "routing weights not normalised": ("p[t] = exp(p[t] - m) / den;", "p[t] = exp(p[t] - m);"),
+    "routing GQA map modulo": ("const int g = h / G;\n    const int64_t S = seq_len[b];",
+                               "const int g = h % Hkv;\n    const int64_t S = seq_len[b];"),
+    "routing from the last head only": ("for (int h = 0; h < Hq; ++h) acc += P[",
+                                        "for (int h = Hq - 1; h < Hq; ++h) acc += P["),
+    "routing logits unscaled": ("p[t] = scale * dot;", "p[t] = dot;"),
+    "routing drops the last token": ("for (int64_t t = 0; t < seq_len[b]; ++t) {\n      double acc",
+                                     "for (int64_t t = 0; t + 1 < seq_len[b]; ++t) {\n      double acc"),
 }
 
 PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

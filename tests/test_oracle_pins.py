@@ -440,3 +440,104 @@ def test_kv_append_writes_only_the_new_token_rows():
         assert np.array_equal(Ka3[r], wv)
     assert np.array_equal(np.delete(Ka3, rows, 0), np.delete(K3, rows, 0))
     assert np.array_equal(Va.reshape(-1, d)[rows], np.stack([nV[0, 0], nV[0, 1], nV[1, 0], nV[1, 1]]))
+
+
+# ----------------------------------------------------------------------------
+# CLSA indexer layer read as full attention whose weights route the index
+# ----------------------------------------------------------------------------
+def _torch_weights(q, Kb, scale):
+    """Library routine: the softmax attention weights of one query row (fp64)."""
+    qq = torch.from_numpy(bf16_bits_to_f32(q).astype(np.float64))
+    kk = torch.from_numpy(bf16_bits_to_f32(Kb).astype(np.float64))
+    return torch.softmax(scale * kk @ qq, dim=0).numpy()
+
+
+def test_indexer_layer_output_is_dense_attention():
+    rng = np.random.default_rng(11)
+    seq_off, S, Q, K, V = _tiny_decode(rng)
+    _, B, Hq, d = Q.shape
+    Hkv, scale = 2, 1 / math.sqrt(d)
+    O, _ = oracle.indexer_layer_attn(Q[0], K, V, seq_off, S, Hkv, scale)
+    for b, h in itertools.product(range(B), range(Hq)):
+        g = h // (Hq // Hkv)
+        want = _dense_attention_torch(Q[0, b, h][None], _kv(K, seq_off, S, Hkv, d, b, g),
+                                      _kv(V, seq_off, S, Hkv, d, b, g), scale)[0]
+        np.testing.assert_allclose(O[b, h], want, rtol=0, atol=1e-12)
+
+
+def test_indexer_layer_route_is_the_head_sum_of_attention_weights():
+    rng = np.random.default_rng(12)
+    seq_off, S, Q, K, V = _tiny_decode(rng, Hq=8, Hkv=2)
+    _, B, Hq, d = Q.shape
+    Hkv, scale = 2, 1 / math.sqrt(d)
+    _, route = oracle.indexer_layer_attn(Q[0], K, V, seq_off, S, Hkv, scale, ld=16)
+    for b in range(B):
+        want = sum(_torch_weights(Q[0, b, h], _kv(K, seq_off, S, Hkv, d, b, h // (Hq // Hkv)), scale)
+                   for h in range(Hq))
+        np.testing.assert_allclose(route[b, :S[b]], want, rtol=2e-7, atol=0)
+        assert np.all(np.isnan(route[b, S[b]:]))  # nothing written past the sequence
+        # each head's weights sum to one, so the routing scores sum to Hq
+        assert abs(float(route[b, :S[b]].astype(np.float64).sum()) - Hq) < 1e-5
+
+
+def test_indexer_layer_single_head_routes_by_logit():
+    # one head, integer-valued q and k: the logits are exact integers, and the
+    # softmax is monotone, so the top-k of the routing scores is the top-k of
+    # the logits under the tie rule (brute force), ties included
+    rng = np.random.default_rng(13)
+    S, d, k = 40, 8, 9
+    q = rng.integers(-2, 3, (1, 1, d)).astype(np.float32)
+    Kt = rng.integers(-2, 3, (S, d)).astype(np.float32)
+    V = rng.standard_normal(S * d).astype(np.float32)
+    _, route = oracle.indexer_layer_attn(bf(q), bf(Kt.ravel()), bf(V), [0, S], [S], 1, 0.5)
+    logits = Kt @ q[0, 0]
+    order = sorted(range(S), key=lambda t: (-logits[t], t))[:k]
+    assert list(oracle.topk(route, [S], k)[0]) == sorted(order)
+    for a, b2 in itertools.combinations(range(S), 2):
+        if logits[a] == logits[b2]:
+            assert route[0, a] == route[0, b2]
+
+
+def test_indexer_layer_identical_keys_route_uniformly():
+    S, d, Hq = 24, 8, 4
+    Q = bf(np.random.default_rng(14).standard_normal((1, Hq, d)))
+    K = bf(np.tile(np.linspace(-1, 1, d), S))
+    V = bf(np.arange(S * d, dtype=np.float32) / 64)
+    O, route = oracle.indexer_layer_attn(Q, K, V, [0, S], [S], 1, 0.3)
+    np.testing.assert_allclose(route[0], np.float32(Hq / S), rtol=1e-7, atol=0)
+    assert list(oracle.topk(route, [S], 5)[0]) == [0, 1, 2, 3, 4]  # all tied: lowest indices
+    # uniform weights: the output is the mean value row
+    np.testing.assert_allclose(O[0, 0], bf16_bits_to_f32(V).reshape(S, d).mean(0), rtol=0, atol=1e-12)
+
+
+def test_indexer_layer_reads_each_head_group_cache():
+    # heads 0,1 (KV head 0) and heads 2,3 (KV head 1): a key aligned with the
+    # group's queries sits at token 3 in KV head 0 and at token 7 in KV head
+    # 1, so the routing score peaks at both with about 2 (two heads each)
+    S, d, Hq, Hkv = 12, 8, 4, 2
+    Q = np.zeros((1, Hq, d), np.float32)
+    Q[0, :2, 0] = 4.0
+    Q[0, 2:, 1] = 4.0
+    K = np.zeros((Hkv, S, d), np.float32)
+    K[0, 3, 0] = 4.0
+    K[1, 7, 1] = 4.0
+    V = np.zeros(Hkv * S * d, np.float32)
+    _, route = oracle.indexer_layer_attn(bf(Q), bf(K.ravel()), bf(V), [0, S], [S], Hkv, 1.0)
+    assert set(oracle.topk(route, [S], 2)[0]) == {3, 7}
+    assert route[0, 3] > 1.99 and route[0, 7] > 1.99
+
+
+def test_attn_route_step_with_every_token_selected_is_dense():
+    # k = S: every later layer attends to every token, i.e. dense attention
+    rng = np.random.default_rng(15)
+    seq_off, S, Q, K, V = _tiny_decode(rng, L=3)
+    L, B, Hq, d = Q.shape
+    Hkv, scale = 2, 1 / math.sqrt(d)
+    O, idx, _ = oracle.decode_step_attn_route(Q, K, V, seq_off, S, int(S.max()), Hkv, scale)
+    for b in range(B):
+        assert list(idx[b, :S[b]]) == list(range(S[b]))
+    for l, b, h in itertools.product(range(L), range(B), range(Hq)):
+        g = h // (Hq // Hkv)
+        want = _dense_attention_torch(Q[l, b, h][None], _kv(K, seq_off, S, Hkv, d, b, g),
+                                      _kv(V, seq_off, S, Hkv, d, b, g), scale)[0]
+        np.testing.assert_allclose(O[l, b, h], want, rtol=0, atol=1e-12)
