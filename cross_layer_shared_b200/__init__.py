@@ -40,6 +40,8 @@ SIGNATURES = {
     "sa_topk": ([_P, _I64, _P, _I, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "sa_sparse_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "sa_sparse_decode_attn": ([_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _F, _P, _I, _P, _SZ, _P], _I),
+    "sa_indexer_layer_attn_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
+    "sa_indexer_layer_attn": ([_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _F, _P, _I, _P, _I64, _P, _SZ, _P], _I),
     "sa_decode_step_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "sa_decode_step": ([ctypes.c_char_p, _I, _PP, _PP, _PP, _PP, _PP, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _I,
                         _I, _I, _F, _P, _I, _P, _P, _I64, _P, _SZ, _P], _I),
@@ -185,6 +187,56 @@ def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, o
                                        n_tokens, Hq, Hkv, d, k, float(scale), _ptr(O), code, _ptr(ws), ws.numel(),
                                        _stream(stream)))
     return O
+
+
+def indexer_layer_attn_workspace_size(B, S_max, Hq, Hkv, d) -> int:
+    return int(lib().sa_indexer_layer_attn_workspace_size(B, S_max, Hq, Hkv, d))
+
+
+def indexer_layer_attn(Q, K, V, seq_off, seq_len, S_max: int, Hkv: int, scale: float, out_dtype=torch.bfloat16,
+                       O=None, scores=None, ws=None, stream=None):
+    """The CLSA indexer layer as full attention whose weights route the index
+    (sa_indexer_layer_attn): Q [B, Hq, d] -> (O [B, Hq, d] dense output,
+    scores [B, ld] fp32 routing scores, the sum over heads of each token's
+    attention weight)."""
+    B, Hq, d = Q.shape
+    n_tokens = K.numel() // (Hkv * d)
+    _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
+    if O is None:
+        O = torch.empty((B, Hq, d), dtype=out_dtype, device=Q.device)
+    if scores is None:
+        scores = torch.empty((B, max(S_max, 1)), dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws = workspace(indexer_layer_attn_workspace_size(B, S_max, Hq, Hkv, d), Q.device)
+    code = SA_F32 if O.dtype == torch.float32 else SA_BF16
+    _check(lib().sa_indexer_layer_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), B, n_tokens, S_max,
+                                       Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(scores), scores.stride(0),
+                                       _ptr(ws), ws.numel(), _stream(stream)))
+    return O, scores
+
+
+def decode_step_attn_route_workspace_size(B, S_max, Hq, Hkv, d, k, L) -> int:
+    return max(indexer_layer_attn_workspace_size(B, S_max, Hq, Hkv, d), int(lib().sa_topk_workspace_size(B, S_max, k)),
+               sparse_decode_attn_workspace_size(max(L - 1, 1), B, Hq, Hkv, d, k))
+
+
+def decode_step_attn_route(Q, K, V, seq_off, seq_len, S_max: int, k: int, Hkv: int, scale: float,
+                           out_dtype=torch.bfloat16, O=None, idx=None, scores=None, ws=None, stream=None):
+    """One decode step of a cross-decoder group under the CLSA reading in
+    which layer 0 is the indexer layer: it attends densely and its summed
+    attention weights give the routing scores; their top-k is the index that
+    layers 1..L-1 share over the same cache.  Q [L, B, Hq, d] -> (O, idx)."""
+    L, B, Hq, d = Q.shape
+    if O is None:
+        O = torch.empty((L, B, Hq, d), dtype=out_dtype, device=Q.device)
+    if ws is None:
+        ws = workspace(decode_step_attn_route_workspace_size(B, S_max, Hq, Hkv, d, k, L), Q.device)
+    _, scores = indexer_layer_attn(Q[0], K, V, seq_off, seq_len, S_max, Hkv, scale, O=O[0], scores=scores, ws=ws,
+                                   stream=stream)
+    idx = topk(scores, seq_len, S_max, k, idx=idx, ws=ws, stream=stream)
+    if L > 1:
+        sparse_decode_attn(Q[1:], K, V, seq_off, seq_len, idx, Hkv, scale, O=O[1:], ws=ws, stream=stream)
+    return O, idx
 
 
 def decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k) -> int:

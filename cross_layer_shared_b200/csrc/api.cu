@@ -17,6 +17,7 @@
 #include "attn.cuh"
 #include "sm100.cuh"
 #include "indexer.cuh"
+#include "route_attn.cuh"
 #include "status.cuh"
 #include "topk.cuh"
 #include "union.cuh"
@@ -430,6 +431,66 @@ sa_status sa_sparse_decode_attn(const void* Q, const void* K, const void* V, con
                                 size_t ws_bytes, void* stream) {
   return run_decode_attn(Q, K, V, seq_off, seq_len, idx, L_g, B, n_tokens, Hq, Hkv, d, k, scale, O, out_dtype, ws,
                          ws_bytes, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------- indexer layer (CLSA routing)
+size_t sa_indexer_layer_attn_workspace_size(int B, int S_max, int Hq, int Hkv, int d) {
+  (void)Hkv;
+  (void)d;
+  if (B < 1 || S_max < 1 || Hq < 1) return SA_WS_HEADER_BYTES;
+  return SA_WS_HEADER_BYTES + sa::route_ws_bytes(B, S_max, Hq);
+}
+
+sa_status sa_indexer_layer_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
+                                const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int Hq, int Hkv, int d,
+                                float scale, void* O, sa_dtype out_dtype, float* scores, int64_t ld, void* ws,
+                                size_t ws_bytes, void* stream) {
+  const char* who = "sa_indexer_layer_attn";
+  if (B < 0 || S_max < 0 || n_tokens < 0) return fail(SA_ERR_INVALID_ARG, "%s: negative size", who);
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+    return fail(SA_ERR_INVALID_ARG, "%s: Hq=%d must be a positive multiple of Hkv=%d", who, Hq, Hkv);
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(SA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d not in {1, 2, 4, 8}", who, G);
+  if (Hq > 256) return fail(SA_ERR_UNSUPPORTED, "%s: Hq=%d above 256", who, Hq);
+  if (d != 128) return fail(SA_ERR_UNSUPPORTED, "%s: d=%d (only 128 is built)", who, d);
+  if (out_dtype != SA_BF16 && out_dtype != SA_F32) return fail(SA_ERR_INVALID_ARG, "%s: bad out_dtype", who);
+  if (ld < S_max) return fail(SA_ERR_INVALID_ARG, "%s: ld=%lld below S_max=%d", who, (long long)ld, S_max);
+  sa_status st = check_ws(ws, ws_bytes, sa_indexer_layer_attn_workspace_size(B, S_max, Hq, Hkv, d), who);
+  if (st != SA_OK) return st;
+  if (B == 0 || S_max == 0) return SA_OK;
+  if (!Q || !K || !V || !seq_off || !seq_len || !O || !scores)
+    return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(scores, 4))
+    return fail(SA_ERR_INVALID_ARG, "%s: Q, K, V, O must be 16-byte aligned and scores 4-byte aligned", who);
+  sa::RouteArgs a{};
+  a.Q = reinterpret_cast<const uint16_t*>(Q);
+  a.K = reinterpret_cast<const uint16_t*>(K);
+  a.V = reinterpret_cast<const uint16_t*>(V);
+  a.seq_off = seq_off;
+  a.seq_len = seq_len;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.S_max = S_max;
+  a.n_tokens = n_tokens;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.n_split = (S_max + sa::kRouteChunk - 1) / sa::kRouteChunk;
+  a.zld = (int64_t)round_up((size_t)S_max, 64);
+  uint8_t* p = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
+  a.z = reinterpret_cast<float*>(p);
+  p += round_up((size_t)B * Hq * a.zld * 4, 256);
+  a.part_ml = reinterpret_cast<float2*>(p);
+  p += round_up((size_t)B * Hq * a.n_split * 8, 256);
+  a.part_o = reinterpret_cast<float*>(p);
+  a.scores = scores;
+  a.ld = ld;
+  a.O = O;
+  a.out_f32 = out_dtype == SA_F32;
+  a.status = status_of(ws);
+  const cudaError_t e = sa::launch_indexer_layer_attn(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail("sa_indexer_layer_attn launch", e);
+  return SA_OK;
 }
 
 // ---------------------------------------------------------------- decode step

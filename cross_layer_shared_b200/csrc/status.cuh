@@ -29,6 +29,7 @@ enum : int {
   kKernCombine = 4,
   kKernUnion = 5,
   kKernIndexerPrefill = 6,
+  kKernRoute = 7,
 };
 
 struct DeviceStatus {

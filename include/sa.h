@@ -191,6 +191,37 @@ sa_status sa_sparse_decode_attn(const void* Q, const void* K, const void* V, con
                                 sa_dtype out_dtype, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * The CLSA indexer layer read as a full attention layer whose attention
+ * weights route the shared index  [CLSA news article, section "La
+ * precision reste stable": the routing index is computed once from the
+ * attention scores of the indexer layer, which sees the same query state
+ * and cache as every other layer].  The pages give no formula for the
+ * aggregation over heads; this reads it as the sum of the attention weights.
+ *
+ * For sequence b, query head h (KV head g = h / (Hq/Hkv)), every cached
+ * token t < seq_len[b]:
+ *   z[h,t] = scale * Q[b,h,:] . K_b[g,t,:],   p[h,t] = softmax_t z[h,t]
+ *   O[b,h,:]     = sum_t p[h,t] * V_b[g,t,:]        (the layer's dense output)
+ *   scores[b,t]  = sum_h p[h,t]                     (fp32 routing score)
+ * sa_topk(scores, seq_len, ...) then gives the index the later layers share.
+ *
+ *   Q        bf16 [B, Hq, d]: the indexer layer's queries
+ *   K, V     packed cache as in sa_sparse_decode_attn
+ *   seq_off  int64 [B+1], seq_len int32 [B] (device); S_max >= every seq_len
+ *   O        [B, Hq, d], bf16 or fp32 per out_dtype
+ *   scores   fp32 [B, ld], ld >= S_max; entries t >= seq_len[b] untouched
+ * Supported: d = 128, Hq/Hkv in {1, 2, 4, 8}, Hq <= 256.  The workspace
+ * holds the logits (B*Hq*S_max fp32) and per-2048-key partial results.
+ * Device errors: seq_len[b] outside [0, S_max] or past n_tokens ->
+ * SA_ERR_DEVICE, the sequence is treated as empty.
+ * ---------------------------------------------------------------------- */
+size_t sa_indexer_layer_attn_workspace_size(int B, int S_max, int Hq, int Hkv, int d);
+sa_status sa_indexer_layer_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
+                                const int32_t* seq_len, int B, int64_t n_tokens, int S_max, int Hq,
+                                int Hkv, int d, float scale, void* O, sa_dtype out_dtype,
+                                float* scores, int64_t ld, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * One decode step over a layer pattern  [IC section 2: a binary pattern
  * marks F layers, which run their indexer and overwrite the cached top-k
  * index, and S layers, which reuse the index of the nearest upstream F

@@ -10,6 +10,12 @@
   scores, exact outside the ambiguous band A = {t: |s_t - s_(k)| <= 1e-3 |s_(k)|}.
 * Attention: max-abs 1e-2 for bf16 outputs, 1e-4 for fp32 outputs, computed
   by the oracle on the GPU's (validated) index.
+* Routing scores of the indexer layer (sum over heads of attention weights):
+  each GPU logit is an fp32 sum of 16-term chains and a 3-level butterfly,
+  so |dz| <= gamma_20 * scale * sum_c |q_c k_c| (natural units).  A weight
+  2^(z - M) / L then carries at most |dz| from z, |dz| from M, 2|dz| +
+  gamma_n from L, and a few ulp from exp2; the head sum adds gamma_Hq.  The
+  relative bound is 4 |dz|_max + gamma_64 + gamma_Hq + 8 ulp.
 """
 from __future__ import annotations
 
@@ -32,6 +38,24 @@ def index_error_bound(qI_bits, w, KI_bits) -> np.ndarray:
     u = 2.0 ** -23
     gamma = n * u / (1 - n * u)
     return gamma * mag
+
+
+def route_rtol(Q_bits, K_bits, scale) -> float:
+    """Relative bound on GPU vs oracle routing scores (see module doc).
+    Q_bits [Hq, d]; K_bits [Hkv, S, d] of one sequence."""
+    Hq, d = Q_bits.shape
+    Hkv = K_bits.shape[0]
+    G = Hq // Hkv
+    q = np.abs(bf16_bits_to_f32(Q_bits).astype(np.float64))
+    mag = 0.0
+    for g in range(Hkv):
+        k = np.abs(bf16_bits_to_f32(K_bits[g]).astype(np.float64))
+        mag = max(mag, float((k @ q[g * G:(g + 1) * G].T).max()))
+    u = 2.0 ** -23
+
+    def gamma(n):
+        return n * u / (1 - n * u)
+    return 4 * gamma(20) * scale * mag + gamma(64) + gamma(Hq) + 8 * u
 
 
 def assert_scores_close(gpu, ora, bound, what=""):

@@ -112,3 +112,20 @@ def test_decode_step_ex_rejects_bad_append_requests(lib):
     assert call(pp, None, pp, pp) == sa.SA_ERR_INVALID_ARG and b"new_KI" in lib.sa_last_error()
     assert call(po, pp, pp, pp) == sa.SA_ERR_UNSUPPORTED and b"F layer" in lib.sa_last_error()
     assert call(pp, None, None, None, flags=4) == sa.SA_ERR_INVALID_ARG and b"flags" in lib.sa_last_error()
+
+
+def test_indexer_layer_attn_rejects_bad_requests(lib):
+    need = lib.sa_indexer_layer_attn_workspace_size(4, 131072, 32, 8, 128)
+    # logits of every head and token, plus the partial results
+    assert need >= sa.WS_HEADER_BYTES + 4 * 32 * 131072 * 4
+
+    def call(Hq=32, Hkv=8, d=128, ld=4096, ws_bytes=1 << 30, S_max=4096, Q=FAKE):
+        return lib.sa_indexer_layer_attn(Q, FAKE, FAKE, FAKE, FAKE, 2, 8192, S_max, Hq, Hkv, d, 0.088, FAKE, 0,
+                                         FAKE, ld, FAKE_WS, ws_bytes, None)
+
+    assert call(Hq=24, Hkv=8) == sa.SA_ERR_UNSUPPORTED and b"{1, 2, 4, 8}" in lib.sa_last_error()
+    assert call(Hq=30, Hkv=8) == sa.SA_ERR_INVALID_ARG
+    assert call(d=64) == sa.SA_ERR_UNSUPPORTED
+    assert call(ld=100) == sa.SA_ERR_INVALID_ARG and b"ld" in lib.sa_last_error()
+    assert call(ws_bytes=1024) == sa.SA_ERR_WORKSPACE
+    assert call(Q=ctypes.c_void_p(0x7F0000001008)) == sa.SA_ERR_INVALID_ARG

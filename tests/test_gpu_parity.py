@@ -465,3 +465,83 @@ def test_prefill_small_full_oracle(dev):
 def test_prefill_c4_full_size_sampled(dev):
     cfg = synth.workload("c4")
     prefill_parity(cfg, dev, q_sample=[0, 1, 1000, 2047], heads=[0, 13, 31])
+
+
+# --------------------------------------------------------------------------
+# CLSA indexer layer read as full attention whose weights route the index
+def _route_case(dev, B, Hq, Hkv, lens, k, seed, out_dtype=torch.float32):
+    rng = np.random.default_rng(seed)
+    d = 128
+    lens = list(lens)
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    T = int(seq_off[-1])
+    S_max = max(max(lens), 1)
+    Q = synth.f32_to_bf16_bits(rng.standard_normal((2, B, Hq, d)).astype(np.float32))
+    K = synth.f32_to_bf16_bits(rng.standard_normal(max(T, 1) * Hkv * d).astype(np.float32))
+    V = synth.f32_to_bf16_bits(rng.standard_normal(max(T, 1) * Hkv * d).astype(np.float32))
+    scale = 1 / math.sqrt(d)
+    ws = sa.workspace(sa.decode_step_attn_route_workspace_size(B, S_max, Hq, Hkv, d, k, 2), dev)
+    scores = torch.full((B, S_max + 5), float("nan"), dtype=torch.float32, device=dev)
+    O, idx = sa.decode_step_attn_route(bf16_dev(Q, dev), bf16_dev(K, dev), bf16_dev(V, dev),
+                                       torch.from_numpy(seq_off).to(dev), torch.tensor(lens, dtype=torch.int32, device=dev),
+                                       S_max, k, Hkv, scale, out_dtype=out_dtype, scores=scores, ws=ws)
+    assert_status_ok(ws)
+    O_ora, route = oracle.indexer_layer_attn(Q[0], K, V, seq_off, lens, Hkv, scale)
+    sc, idx_h, O_h = scores.cpu().numpy(), idx.cpu().numpy(), O.float().cpu().numpy()
+    tol = parity.ATOL_F32 if out_dtype == torch.float32 else parity.ATOL_BF16
+    assert np.abs(O_h[0] - O_ora).max() <= tol
+    for b in range(B):
+        S = lens[b]
+        assert np.all(np.isnan(sc[b, S:])), "nothing is written past the sequence"
+        if S:
+            Kb = K[seq_off[b] * Hkv * d:(seq_off[b] + S) * Hkv * d].reshape(Hkv, S, d)
+            rtol = parity.route_rtol(Q[0, b], Kb, scale)
+            err = np.abs(sc[b, :S].astype(np.float64) - route[b, :S]) / np.maximum(route[b, :S], 1e-30)
+            assert err.max() <= rtol, (b, float(err.max()), rtol)
+        assert np.array_equal(idx_h[b], oracle.topk(sc[b:b + 1, :S], [S], k)[0]) if S else np.all(idx_h[b] == -1)
+        if S:
+            parity.assert_topk_band(idx_h[b], route[b], S, k, f"route b={b}")
+    # layer 1 reads the GPU's index: dense-routed sparse attention
+    O1 = oracle.sparse_decode_attn(Q[1:], K, V, seq_off, lens, idx_h, Hkv, scale)
+    assert np.abs(O_h[1:] - O1).max() <= tol
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,lens,k", [
+    (2, 32, 8, [5000, 2048], 256),          # G = 4, several 2048-key chunks, exact chunk edge
+    (3, 16, 2, [77, 4099, 31], 64),          # G = 8, ragged tiles, a sequence shorter than k
+    (2, 4, 4, [1000, 0], 128),               # G = 1 and an empty sequence
+    (1, 8, 4, [300], 300),                   # G = 2, k = S: every token routed
+])
+def test_indexer_layer_routing_small(dev, B, Hq, Hkv, lens, k):
+    _route_case(dev, B, Hq, Hkv, lens, k, seed=B * 100 + Hq)
+
+
+def test_indexer_layer_routing_bf16_output(dev):
+    _route_case(dev, 2, 32, 8, [3000, 1500], 512, seed=7, out_dtype=torch.bfloat16)
+
+
+def test_attn_route_step_c3_full_size_sampled(dev):
+    """The c3 group (4 x 131072 tokens, 32 / 8 heads, 24 layers) under the
+    attention-routing reading: layer 0 dense with its routing scores, top-2048,
+    23 sparse layers; sequences 0 and 3 against the oracle."""
+    cfg = synth.workload("c3")
+    wl = sgpu.decode_workload(cfg, dev, groups=[0])
+    gr = wl["groups"][0]
+    ws = sa.workspace(sa.decode_step_attn_route_workspace_size(cfg.B, cfg.S_max, cfg.Hq, cfg.Hkv, cfg.d, cfg.k,
+                                                               cfg.L), dev)
+    O, idx = sa.decode_step_attn_route(wl["Q"], gr["K"], gr["V"], wl["seq_off"], wl["seq_len"], cfg.S_max, cfg.k,
+                                       cfg.Hkv, cfg.scale, out_dtype=torch.float32, ws=ws)
+    assert_status_ok(ws)
+    O_h, idx_h = O.cpu().numpy(), idx.cpu().numpy()
+    Q = cfg.Q()
+    for b in (0, 3):
+        S = cfg.seq_lens[b]
+        rows = np.arange(S)
+        K = np.stack([cfg.KV_rows(0, b, h, rows, "K") for h in range(cfg.Hkv)])
+        V = np.stack([cfg.KV_rows(0, b, h, rows, "V") for h in range(cfg.Hkv)])
+        O0, route = oracle.indexer_layer_attn(Q[0, b:b + 1], K.ravel(), V.ravel(), [0, S], [S], cfg.Hkv, cfg.scale)
+        assert np.abs(O_h[0, b] - O0[0]).max() <= parity.ATOL_F32
+        parity.assert_topk_band(idx_h[b], route[0], S, cfg.k, f"c3 route b={b}")
+        O_rest = oracle.sparse_decode_attn(Q[1:, b:b + 1], K.ravel(), V.ravel(), [0, S], [S], idx_h[b:b + 1],
+                                           cfg.Hkv, cfg.scale)[:, 0]
+        assert np.abs(O_h[1:, b] - O_rest).max() <= parity.ATOL_F32
