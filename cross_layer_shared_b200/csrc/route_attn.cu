@@ -22,7 +22,8 @@
 //   memory (thread = one key x 16 of its 128 dims, then an 8-lane sum).
 //   Then per head (warp h): the chunk max m, p = 2^(z - m) in place,
 //   l = sum p, and z out to global memory for the routing scores.
-//   Phase 2: o[h] = sum_t p[h,t] V[t] (thread = 2 dims x its heads).
+//   Phase 2: o[h] = sum_t p[h,t] V[t] (thread = 4 dims x 2 heads x one
+//   residue class of rows; the row classes are summed at the end).
 //   Writes (m, l) and o per (head, chunk).
 // Combine kernel: per sequence, CTAs 0..n_tc-1 write the routing scores of
 //   1024 tokens each, r_t = sum_h 2^(z[h,t] - M_h) / L_h, with (M_h, L_h) the
@@ -51,8 +52,8 @@ template <int G>
 struct PartLayout {
   static constexpr int kRingOff = 0;                             // [kStages][kRows][128] bf16
   static constexpr int kZOff = kRingOff + kStages * kTileBytes;  // [G][kRouteChunk] fp32: z, then p
-  static constexpr int kQOff = kZOff + G * kRouteChunk * 4;      // [G][128] bf16
-  static constexpr int kBarOff = kQOff + G * kD * 2;             // full[kStages] empty[kStages]
+  static constexpr int kQOff = kZOff + G * kRouteChunk * 4;      // [G][4][8][4] fp32 (see q_slot)
+  static constexpr int kBarOff = kQOff + G * kD * 4;             // full[kStages] empty[kStages]
   static constexpr int kFlagOff = kBarOff + 16 * kStages;
   static constexpr size_t kSmem = kFlagOff + 16;
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -86,6 +87,25 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Slot of query dim c of head h in shared memory: the 16 dims a phase-1
+// thread dq uses (8dq..8dq+7, 64+8dq..64+8dq+7) are four float4 whose j-th
+// ones sit side by side for dq = 0..7, so eight lanes read 128 contiguous bytes.
+__device__ __forceinline__ int q_slot(int h, int c) {
+  const int dq = (c & 63) >> 3;
+  const int e = ((c >> 6) << 3) | (c & 7);  // 0..15 within the thread's dims
+  return ((h * 4 + (e >> 2)) * 8 + dq) * 4 + (e & 3);
+}
+
+// a shared-memory load the compiler keeps in the loop (hoisting the query
+// slices out of it would hold 16*G registers and cost a resident CTA)
+__device__ __forceinline__ float4 lds_f4(const float* p) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
+
 __device__ __forceinline__ void unpack8(const uint4 u, float* f) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -108,12 +128,12 @@ __device__ __forceinline__ int checked_len(const RouteArgs& a, int b, bool repor
 }
 
 template <int G>
-__global__ void __launch_bounds__(kPartThreads, 1) indexer_layer_partial_kernel(const RouteArgs a) {
+__global__ void __launch_bounds__(kPartThreads, 3) indexer_layer_partial_kernel(const RouteArgs a) {
   using Lay = PartLayout<G>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* ring = reinterpret_cast<uint16_t*>(smem + Lay::kRingOff);
   float* zs = reinterpret_cast<float*>(smem + Lay::kZOff);
-  uint16_t* qs = reinterpret_cast<uint16_t*>(smem + Lay::kQOff);
+  float* qs = reinterpret_cast<float*>(smem + Lay::kQOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
   uint64_t* empty = full + kStages;
   int* abort_flag = reinterpret_cast<int*>(smem + Lay::kFlagOff);
@@ -137,8 +157,10 @@ __global__ void __launch_bounds__(kPartThreads, 1) indexer_layer_partial_kernel(
   const int nt = (n + kRows - 1) / kRows;             // K tiles, then as many V tiles
   const int64_t row0 = a.seq_off[b] * a.Hkv + (int64_t)g * len + t0;
   const int h0 = g * G;
-  if (tid < G * kD / 8)
-    reinterpret_cast<uint4*>(qs)[tid] = reinterpret_cast<const uint4*>(a.Q + ((int64_t)b * a.Hq + h0) * kD)[tid];
+  for (int e = tid; e < G * kD; e += kPartThreads) {
+    const uint32_t q16 = a.Q[((int64_t)b * a.Hq + h0) * kD + e];
+    qs[q_slot(e / kD, e % kD)] = __uint_as_float(q16 << 16);
+  }
   __syncthreads();
 
   if (warp == kCompWarps) {
@@ -186,12 +208,15 @@ __global__ void __launch_bounds__(kPartThreads, 1) indexer_layer_partial_kernel(
     float acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      float qf[16];
-      unpack8(*reinterpret_cast<const uint4*>(qs + h * kD + 8 * dq), qf);
-      unpack8(*reinterpret_cast<const uint4*>(qs + h * kD + 64 + 8 * dq), qf + 8);
       float x = 0.f;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) x = fmaf(qf[e], kf[e], x);
+      for (int j4 = 0; j4 < 4; ++j4) {
+        const float4 q4 = lds_f4(qs + ((h * 4 + j4) * 8 + dq) * 4);
+        x = fmaf(q4.x, kf[4 * j4], x);
+        x = fmaf(q4.y, kf[4 * j4 + 1], x);
+        x = fmaf(q4.z, kf[4 * j4 + 2], x);
+        x = fmaf(q4.w, kf[4 * j4 + 3], x);
+      }
       acc[h] = x;
     }
 #pragma unroll
@@ -230,12 +255,19 @@ __global__ void __launch_bounds__(kPartThreads, 1) indexer_layer_partial_kernel(
   comp_bar();
 
   // ---------------- phase 2: o[h] = sum_t p[h,t] V[t] ----------------
-  constexpr int HPT = (G + 3) / 4;  // heads of this thread: hq, hq + 4, ...
-  const int dp = tid & 63;          // dims 2dp, 2dp + 1
-  const int hq = tid >> 6;
-  float o0[HPT], o1[HPT];
+  // thread: dims [4 dq4, 4 dq4 + 4) of HP heads, rows r = rg (mod NRG) of
+  // each tile; the NRG row groups are summed through shared memory at the end
+  constexpr int HP = G < 2 ? G : 2;         // heads per thread
+  constexpr int NHS = G / HP;               // head slots
+  constexpr int NRG = kCompWarps / NHS;     // row groups (8, 8, 4, 2 for G = 1, 2, 4, 8)
+  const int dq4 = tid & 31;
+  const int hs = (tid >> 5) % NHS;
+  const int rg = (tid >> 5) / NHS;
+  float o[HP][4];
 #pragma unroll
-  for (int x = 0; x < HPT; ++x) o0[x] = o1[x] = 0.f;
+  for (int x = 0; x < HP; ++x)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[x][e] = 0.f;
   bool ok = true;
   for (int j = 0; j < nt; ++j) {
     const int i = nt + j, s = i % kStages;
@@ -245,32 +277,39 @@ __global__ void __launch_bounds__(kPartThreads, 1) indexer_layer_partial_kernel(
       break;
     }
     const int rows = min(kRows, n - j * kRows);
-    const uint32_t* vt = reinterpret_cast<const uint32_t*>(ring + s * kRows * kD) + dp;
-    const float* pr = zs + j * kRows;
+    const uint2* vt = reinterpret_cast<const uint2*>(ring + s * kRows * kD) + dq4;
+    const float* pr = zs + (hs * HP) * kRouteChunk + j * kRows;
 #pragma unroll 4
-    for (int r = 0; r < rows; ++r) {
-      const uint32_t v2 = vt[r * (kD / 2)];
-      const float v0 = __uint_as_float(v2 << 16), v1 = __uint_as_float(v2 & 0xffff0000u);
+    for (int r = rg; r < rows; r += NRG) {
+      const uint2 v4 = vt[r * (kD / 4)];
+      const float v[4] = {__uint_as_float(v4.x << 16), __uint_as_float(v4.x & 0xffff0000u),
+                          __uint_as_float(v4.y << 16), __uint_as_float(v4.y & 0xffff0000u)};
 #pragma unroll
-      for (int x = 0; x < HPT; ++x) {
-        const int h = hq + 4 * x;
-        if (h < G) {
-          const float p = pr[h * kRouteChunk + r];
-          o0[x] = fmaf(p, v0, o0[x]);
-          o1[x] = fmaf(p, v1, o1[x]);
-        }
+      for (int x = 0; x < HP; ++x) {
+        const float p = pr[x * kRouteChunk + r];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[x][e] = fmaf(p, v[e], o[x][e]);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
-  if (!ok) return;
+  if (!ok && lane == 0) atomicExch(abort_flag, 1);
+  // sum the row groups (the weights are no longer needed: reuse their space);
+  // every compute warp reaches each barrier, a warp that gave up included
+  comp_bar();
+  if (*reinterpret_cast<volatile int*>(abort_flag) != 0) return;
+  float* red = zs;  // [NRG][G][128]
 #pragma unroll
-  for (int x = 0; x < HPT; ++x) {
-    const int h = hq + 4 * x;
-    if (h < G)
-      *reinterpret_cast<float2*>(a.part_o + (((int64_t)b * a.Hq + h0 + h) * a.n_split + split) * kD + 2 * dp) =
-          make_float2(o0[x], o1[x]);
+  for (int x = 0; x < HP; ++x)
+    *reinterpret_cast<float4*>(red + ((rg * G) + hs * HP + x) * kD + 4 * dq4) =
+        make_float4(o[x][0], o[x][1], o[x][2], o[x][3]);
+  comp_bar();
+  for (int e = tid; e < G * kD; e += 32 * kCompWarps) {
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < NRG; ++q) sum += red[q * G * kD + e];
+    a.part_o[(((int64_t)b * a.Hq + h0 + e / kD) * a.n_split + split) * kD + e % kD] = sum;
   }
 }
 
