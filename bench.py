@@ -101,6 +101,18 @@ def algorithmic_bytes(cfg: synth.DecodeConfig, out_bytes: int = 2) -> dict:
     return {"KI": ki, "KV": kv, "Q": q, "O": o, "small": small, "total": ki + kv + q + o + small}
 
 
+def attn_route_bytes(cfg: synth.DecodeConfig, out_bytes: int = 2) -> dict:
+    """Strict HBM bytes of one step under the attention-routing reading
+    (layer 0 attends densely; its summed attention weights route the index
+    of layers 1..L-1): every K and V row of the cache once, each selected
+    row once more for the sparse layers, Q and O of every layer."""
+    dense = cfg.T * cfg.Hkv * cfg.d * 2 * 2
+    sel = sum(min(cfg.k, s) for s in cfg.seq_lens) * cfg.Hkv * cfg.d * 2 * 2
+    q = cfg.L * cfg.B * cfg.Hq * cfg.d * 2
+    o = cfg.L * cfg.B * cfg.Hq * cfg.d * out_bytes
+    return {"dense_KV": dense, "selected_KV": sel, "Q": q, "O": o, "total": dense + sel + q + o}
+
+
 def indexer_launch_bytes(cfg: synth.DecodeConfig) -> int:
     """Bytes one indexer launch must move: each visible key row (d_I bf16) read
     once, the query/weights read, one fp32 score per key written."""
@@ -640,6 +652,43 @@ def run_ours(args):
     for l in range(cfg.L):
         seq_launches += (2 if cfg.pattern[l] == "F" else 0) + 1
 
+    # ---- the attention-routing reading of the indexer layer (one group only):
+    # layer 0 attends densely and its summed attention weights are the
+    # routing scores; their top-k serves layers 1..L-1 ----
+    route = None
+    if len(cfg.groups) == 1 and cfg.L > 1:
+        rws = [sa.workspace(sa.decode_step_attn_route_workspace_size(cfg.B, cfg.S_max, cfg.Hq, cfg.Hkv, cfg.d, cfg.k,
+                                                                     cfg.L), dev) for _ in sets]
+
+        def step_route(j):
+            st = sets[j % len(sets)]
+            sa.decode_step_attn_route(st["wl"]["Q"], st["K"][0], st["V"][0], st["wl"]["seq_off"], st["wl"]["seq_len"],
+                                      cfg.S_max, cfg.k, cfg.Hkv, cfg.scale, O=st["O"], idx=st["idx"],
+                                      scores=st["scores"], ws=rws[j % len(sets)])
+
+        for j in range(len(sets)):
+            step_route(j)
+        torch.cuda.synchronize()
+        for w in rws:
+            code, det = sa.read_status(w)
+            if code != 0:
+                raise RuntimeError(f"device status {code} {det}")
+        g_route = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_route, stream=cap):
+            for j in range(STEPS_PER_GRAPH):
+                step_route(j)
+        g_route.replay()
+        n_route = max(3, min(50, args.steps // (4 * STEPS_PER_GRAPH)))
+        ms_route = timed(lambda i: g_route.replay(), n_route) / (n_route * STEPS_PER_GRAPH)
+        rb = attn_route_bytes(cfg, 4 if args.out_f32 else 2)
+        route = {"value": aggregate_rate(1, world, ms_route), "unit": "steps/s", "ms_per_step": ms_route,
+                 "hbm_gbs": rb["total"] / (ms_route / 1e3) / 1e9 * world, "algorithmic_bytes_per_step": rb,
+                 "launches_per_step": 4,
+                 "note": "CLSA read as routing from the indexer layer's own attention weights: layer 0 attends "
+                         "densely over every cached token, the sum over its query heads of each token's weight "
+                         "is the routing score, its top-k is the index of layers 1..L-1"}
+        del g_route
+
     # ---- per-kernel device time: each graph holds REP back-to-back launches
     # (alternating input sets, so consecutive launches read different data),
     # which keeps the host's replay cost out of the figure ----
@@ -767,6 +816,8 @@ def run_ours(args):
         return 0
 
     peak, peak_kind = measured_peaks()
+    if route is not None:
+        route["hbm_frac"] = route["hbm_gbs"] / world / peak
     step_gbs = nb["total"] / (ms_per_step / 1e3) / 1e9
     idx_bytes = indexer_launch_bytes(cfg)
     idx_gbs = idx_bytes / (ms_idx / 1e3) / 1e9
@@ -789,6 +840,7 @@ def run_ours(args):
                                   "note": "the new token's rows appended to the caches by the indexer, then one "
                                           "attention launch per layer (no fusion of the group's layers), as a "
                                           "decoder that computes layer l+1's queries from layer l runs it"},
+        "attn_route": route,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "per step: pinned host -> device copy of that step's queries, indexer queries and head "
