@@ -41,6 +41,7 @@ METRIC = "decode steps/s and achieved HBM GB/s (% of roofline) at 128K ctx, 1×B
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 PROFILE = os.path.join(ROOT, "profiles", "indexer_decode_c3.md")
+L2_BYTES = 126 * 1024 * 1024  # B200 L2
 INDEXER_SRC = os.path.join(ROOT, "cross_layer_shared_b200", "csrc", "indexer.cu")
 
 
@@ -52,7 +53,8 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5"],
                    help="c4 times one chunked-prefill chunk instead of a decode step")
-    p.add_argument("--sets", type=int, default=2, help="rotating input sets (cold L2 between steps)")
+    p.add_argument("--sets", type=int, default=0,
+                   help="rotating input sets (cold L2 between steps); 0 = two if they fit in device memory, else one")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--out-f32", action="store_true", help="fp32 attention output instead of bf16")
@@ -128,11 +130,14 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profile_traffic():
+def profile_traffic(workload: str):
     """ncu DRAM bytes per indexer launch recorded in profiles/, if the kernel
-    source still matches the one profiled."""
+    source still matches the one profiled and the workload is the one it
+    was taken on."""
     try:
         text = open(PROFILE).read()
+        if re.search(r"workload:\s*(\w+)", text).group(1) != workload:
+            return None
         sha = re.search(r"indexer_source_sha256:\s*([0-9a-f]+)", text).group(1)
         traffic = float(re.search(r"traffic_bytes_per_launch_full:\s*([0-9.eE+]+)", text).group(1))
         cur = hashlib.sha256(open(INDEXER_SRC, "rb").read()).hexdigest()
@@ -495,11 +500,19 @@ def run_reference(args):
     return 0
 
 
+def set_bytes(cfg) -> int:
+    """Device bytes of one input set: the indexer keys and K/V caches of every group."""
+    per_group = cfg.T * (cfg.d_I * 2 + 2 * cfg.Hkv * cfg.d * 2)
+    return len(cfg.groups) * per_group
+
+
 def workload_config(cfg, args):
     return {"workload": f"{cfg.name}: {synth.DESCRIPTIONS[cfg.name]}", "batch": cfg.B, "context": cfg.S_max,
             "layers": cfg.L, "pattern": cfg.pattern if len(cfg.pattern) <= 8 else f"{cfg.pattern[:4]}... ({cfg.L})",
             "top_k": cfg.k, "indexer": f"{cfg.H_I}x{cfg.d_I}", "heads": f"{cfg.Hq}q/{cfg.Hkv}kv", "head_dim": cfg.d,
-            "l2": f"{args.sets} rotating input sets, each larger than L2",
+            "l2": (f"{args.sets} rotating input set(s) of {set_bytes(cfg) / 1e9:.1f} GB each, larger than L2"
+                   if set_bytes(cfg) > L2_BYTES else
+                   f"{args.sets} input set(s) of {set_bytes(cfg) / 1e6:.1f} MB: resident in L2 (warm-cache figure)"),
             "parallelism": "replicas" if args.gpus > 1 else "single"}
 
 
@@ -530,6 +543,9 @@ def run_ours(args):
     n = cfg.L
     nb = algorithmic_bytes(cfg, 4 if args.out_f32 else 2)
 
+    if args.sets <= 0:  # two rotating sets when they fit (with room to spare), else one
+        free, _ = torch.cuda.mem_get_info(dev)
+        args.sets = 2 if 2 * set_bytes(cfg) < 0.8 * free else 1
     sets = []
     for si in range(args.sets):
         wl = sgpu.decode_workload(cfg, dev)
@@ -821,7 +837,7 @@ def run_ours(args):
     step_gbs = nb["total"] / (ms_per_step / 1e3) / 1e9
     idx_bytes = indexer_launch_bytes(cfg)
     idx_gbs = idx_bytes / (ms_idx / 1e3) / 1e9
-    traffic = profile_traffic()
+    traffic = profile_traffic(cfg.name)
     cs = clocks.summary()
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
