@@ -65,9 +65,10 @@ __device__ __forceinline__ int locate_tile(const int* prefix, int B, int g) {
 
 // One warp, for the new token of sequence b (row len-1 of its caches): copies
 // its indexer key and its K / V rows of every KV head into the caches, then
-// stores its score computed from the fresh key (lane l takes key components
-// l, l+32, ..; the per-head sums are butterfly reductions, identical in
-// every lane).  Tiles that loaded this row from the cache are not used for it.
+// stores its score computed from the fresh key.  Lane j takes indexer head j
+// (and j + 32): its whole dot product, with every load issued before the
+// arithmetic, then one butterfly sum of the weighted ReLU terms.  Tiles that
+// loaded this row from the cache are not used for it.
 __device__ __noinline__ void append_new_token(const AppendArgs& ap, const float* __restrict__ w,
                                               const int64_t* __restrict__ seq_off, int b, int len, int H_I,
                                               int d_I, float* score_out, int lane) {
@@ -87,15 +88,33 @@ __device__ __noinline__ void append_new_token(const AppendArgs& ap, const float*
     }
   }
   float acc = 0.f;
-  for (int j = 0; j < H_I; ++j) {
-    const uint16_t* q = ap.qI + ((int64_t)b * H_I + j) * d_I;
-    float part = 0.f;
-    for (int c = lane; c < d_I; c += 32)
-      part = fmaf(__uint_as_float((uint32_t)q[c] << 16), __uint_as_float((uint32_t)nk[c] << 16), part);
+  for (int j = lane; j < H_I; j += 32) {
+    const uint4* q = reinterpret_cast<const uint4*>(ap.qI + ((int64_t)b * H_I + j) * d_I);
+    const uint4* k = reinterpret_cast<const uint4*>(nk);
+    const float wj = __ldg(&w[(int64_t)b * H_I + j]);
+    float dot = 0.f;
+    for (int c8 = 0; c8 < d_I / 8; c8 += 4) {  // d_I is a multiple of 64: four 16-byte pieces at a time
+      uint4 qv[4], kv[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    acc = fmaf(__ldg(&w[(int64_t)b * H_I + j]), fmaxf(part, 0.f), acc);
+      for (int u = 0; u < 4; ++u) {
+        qv[u] = q[c8 + u];
+        kv[u] = k[c8 + u];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t qa[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+        const uint32_t ka[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          dot = fmaf(__uint_as_float(qa[e] << 16), __uint_as_float(ka[e] << 16), dot);
+          dot = fmaf(__uint_as_float(qa[e] & 0xffff0000u), __uint_as_float(ka[e] & 0xffff0000u), dot);
+        }
+      }
+    }
+    acc = fmaf(wj, fmaxf(dot, 0.f), acc);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) *score_out = __fadd_rn(acc, 0.f);  // canonical +0
 }
 
