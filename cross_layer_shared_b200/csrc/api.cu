@@ -118,6 +118,16 @@ sa_status make_rows_tmap(CUtensorMap* m, const void* base, int64_t rows) {
   return make_tmap(m, base, 2, dims, str, box);
 }
 
+// [rows, 128] bf16 as a 2-D tensor map with a 64 x 128 box (half the columns
+// of a 128-row tile per load)
+sa_status make_tile128_tmap(CUtensorMap* m, const void* base, int64_t rows) {
+  if (rows < 1 || rows >= (1ll << 31)) return fail(SA_ERR_INVALID_ARG, "tensor of %lld rows: need 1 <= rows < 2^31", (long long)rows);
+  const uint64_t dims[2] = {128, (uint64_t)rows};
+  const uint64_t str[1] = {256};
+  const uint32_t box[2] = {64, 128};
+  return make_tmap(m, base, 2, dims, str, box);
+}
+
 // [rows, 128] bf16 as a 2-D tensor map with a 64 x 64 box (one 64-token KV
 // block, half of its columns, per load)
 sa_status make_block_tmap(CUtensorMap* m, const void* base, int64_t rows) {
@@ -488,7 +498,16 @@ sa_status sa_indexer_layer_attn(const void* Q, const void* K, const void* V, con
   a.O = O;
   a.out_f32 = out_dtype == SA_F32;
   a.status = status_of(ws);
-  const cudaError_t e = sa::launch_indexer_layer_attn(a, (cudaStream_t)stream);
+  CUtensorMap tm_k, tm_v, tm_q;
+  if ((st = make_tile128_tmap(&tm_k, K, n_tokens * Hkv)) != SA_OK) return st;
+  if ((st = make_tile128_tmap(&tm_v, V, n_tokens * Hkv)) != SA_OK) return st;
+  {
+    const uint64_t dims[3] = {128, (uint64_t)Hq, (uint64_t)B};
+    const uint64_t str[2] = {256, (uint64_t)Hq * 256};
+    const uint32_t box[3] = {64, 16, 1};
+    if ((st = make_tmap(&tm_q, Q, 3, dims, str, box)) != SA_OK) return st;
+  }
+  const cudaError_t e = sa::launch_indexer_layer_attn(a, tm_k, tm_v, tm_q, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail("sa_indexer_layer_attn launch", e);
   return SA_OK;
 }

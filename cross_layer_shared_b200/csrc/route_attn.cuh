@@ -1,6 +1,7 @@
 // Launch interface of the indexer-layer attention kernels (internal to libsa).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -32,6 +33,9 @@ struct RouteArgs {
 };
 
 size_t route_ws_bytes(int B, int S_max, int Hq);  // scratch after the workspace header
-cudaError_t launch_indexer_layer_attn(const RouteArgs& a, cudaStream_t stream);
+// tm_k / tm_v: the packed K / V caches as 2-D [n_tokens*Hkv, 128] bf16, box 64
+// x 128 rows, 128-byte swizzle; tm_q: Q as 3-D (128, Hq, B), box (64, 16, 1).
+cudaError_t launch_indexer_layer_attn(const RouteArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                      const CUtensorMap& tm_q, cudaStream_t stream);
 
 }  // namespace sa

@@ -545,3 +545,28 @@ def test_attn_route_step_c3_full_size_sampled(dev):
         O_rest = oracle.sparse_decode_attn(Q[1:, b:b + 1], K.ravel(), V.ravel(), [0, S], [S], idx_h[b:b + 1],
                                            cfg.Hkv, cfg.scale)[:, 0]
         assert np.abs(O_h[1:, b] - O_rest).max() <= parity.ATOL_F32
+
+
+def test_indexer_layer_reports_bad_length(dev):
+    """A sequence length above S_max is reported (kernel id 7) and the
+    sequence is treated as empty: zero output, nothing routed; the other
+    sequence is unaffected."""
+    rng = np.random.default_rng(5)
+    d, Hq, Hkv, S_max = 128, 8, 2, 300
+    lens_real = [300, 200]
+    seq_off = np.array([0, 300, 500], np.int64)
+    Q = synth.f32_to_bf16_bits(rng.standard_normal((2, Hq, d)).astype(np.float32))
+    K = synth.f32_to_bf16_bits(rng.standard_normal(500 * Hkv * d).astype(np.float32))
+    V = synth.f32_to_bf16_bits(rng.standard_normal(500 * Hkv * d).astype(np.float32))
+    ws = sa.workspace(sa.indexer_layer_attn_workspace_size(2, S_max, Hq, Hkv, d), dev)
+    bad = torch.tensor([300, S_max + 5], dtype=torch.int32, device=dev)
+    O, sc = sa.indexer_layer_attn(bf16_dev(Q, dev), bf16_dev(K, dev), bf16_dev(V, dev),
+                                  torch.from_numpy(seq_off).to(dev), bad, S_max, Hkv, 1 / math.sqrt(d),
+                                  out_dtype=torch.float32, ws=ws)
+    code, det = sa.read_status(ws)
+    assert code == sa.SA_ERR_DEVICE and det[0] == 7 and det[1] == 1 and det[2] == S_max + 5
+    O_h = O.cpu().numpy()
+    assert np.all(O_h[1] == 0)
+    O_ora, _ = oracle.indexer_layer_attn(Q[:1], K[:300 * Hkv * d], V[:300 * Hkv * d], seq_off[:2], lens_real[:1],
+                                         Hkv, 1 / math.sqrt(d))
+    assert np.abs(O_h[0] - O_ora[0]).max() <= parity.ATOL_F32
