@@ -56,3 +56,19 @@ def test_rank_workloads_differ_only_in_seed():
     a, b = bench.rank_workload("c5", 0), bench.rank_workload("c5", 3)
     assert a.seed != b.seed
     assert (a.seq_lens, a.k, a.pattern, a.Hq, a.Hkv, a.d) == (b.seq_lens, b.k, b.pattern, b.Hq, b.Hkv, b.d)
+
+
+def test_byte_counts_and_profile_lookup():
+    cfg = synth.workload("c3")
+    rb = bench.attn_route_bytes(cfg)
+    # the routing step reads every K and V row once (4 x 131072 tokens x 8 heads x 256 B x 2)
+    assert rb["dense_KV"] == 4 * 131072 * 8 * 256 * 2
+    assert rb["selected_KV"] == 4 * 2048 * 8 * 256 * 2
+    assert rb["total"] == sum(v for k, v in rb.items() if k != "total")
+    nb = bench.algorithmic_bytes(cfg)
+    assert nb["KI"] == 4 * 131072 * 256 and nb["KV"] == rb["selected_KV"]
+    # one input set: the indexer keys and both caches of each group
+    assert bench.set_bytes(cfg) == 4 * 131072 * (256 + 2 * 8 * 256)
+    assert bench.set_bytes(synth.workload("c1")) < bench.L2_BYTES < bench.set_bytes(cfg)
+    # ncu traffic is reported only for the workload it was captured on
+    assert bench.profile_traffic("c1") is None
