@@ -103,6 +103,35 @@ def _dev(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
     return t
 
 
+def _out(t: torch.Tensor, shape, dtypes, name: str) -> torch.Tensor:
+    """A caller-supplied output: contiguous, on the GPU, of an accepted dtype
+    and exactly the shape the call writes (a kernel would write past a smaller
+    one)."""
+    if not (t.is_cuda and t.is_contiguous() and t.dtype in dtypes):
+        raise ValueError(f"{name} must be a contiguous CUDA tensor of {' or '.join(str(x) for x in dtypes)}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    return t
+
+
+def _rows_out(t: torch.Tensor, rows: int, min_cols: int, name: str) -> int:
+    """A caller-supplied fp32 score table [rows, ld] with ld >= min_cols; returns ld."""
+    if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.float32 and t.dim() == 2):
+        raise ValueError(f"{name} must be a contiguous 2-D CUDA tensor of torch.float32")
+    if t.shape[0] != rows or t.shape[1] < max(min_cols, 1):
+        raise ValueError(f"{name} must be [{rows}, >= {max(min_cols, 1)}], not {tuple(t.shape)}")
+    return int(t.shape[1])
+
+
+def _seqs(seq_off: torch.Tensor, seq_len: torch.Tensor, B: int) -> None:
+    _out(seq_off, (B + 1,), (torch.int64,), "seq_off")
+    _out(seq_len, (B,), (torch.int32,), "seq_len")
+
+
+def _ws(ws: torch.Tensor) -> torch.Tensor:
+    return _dev(ws, torch.uint8, "ws")
+
+
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     """A zeroed workspace (status block included) of at least nbytes."""
     n = max(int(nbytes), WS_HEADER_BYTES)
@@ -126,12 +155,18 @@ def index_score(qI, w, KI, seq_off, seq_len, S_max: int, scores=None, ld: Option
                 stream=None) -> torch.Tensor:
     B, H_I, d_I = qI.shape
     _dev(qI, torch.bfloat16, "qI"), _dev(w, torch.float32, "w"), _dev(KI, torch.bfloat16, "KI")
-    _dev(seq_off, torch.int64, "seq_off"), _dev(seq_len, torch.int32, "seq_len")
-    ld = int(ld if ld is not None else max(S_max, 1))
+    _seqs(seq_off, seq_len, B)
     if scores is None:
+        ld = int(ld if ld is not None else max(S_max, 1))
         scores = torch.empty((B, ld), dtype=torch.float32, device=qI.device)
+    else:
+        have = _rows_out(scores, B, S_max, "scores")
+        if ld is not None and int(ld) != have:
+            raise ValueError(f"ld={ld} does not match scores of {have} columns")
+        ld = have
     if ws is None:
         ws = workspace(lib().sa_index_score_workspace_size(B), qI.device)
+    _ws(ws)
     _check(lib().sa_index_score(_ptr(qI), _ptr(w), _ptr(KI), _ptr(seq_off), _ptr(seq_len), B, KI.shape[0], S_max,
                                 H_I, d_I, _ptr(scores), ld, _ptr(ws), ws.numel(), _stream(stream)))
     return scores
@@ -141,12 +176,18 @@ def index_score_prefill(qI, w, KI, q_pos, max_pos: int, scores=None, ld: Optiona
                         stream=None) -> torch.Tensor:
     Nq, H_I, d_I = qI.shape
     _dev(qI, torch.bfloat16, "qI"), _dev(w, torch.float32, "w"), _dev(KI, torch.bfloat16, "KI")
-    _dev(q_pos, torch.int32, "q_pos")
-    ld = int(ld if ld is not None else max_pos + 1)
+    _out(q_pos, (Nq,), (torch.int32,), "q_pos")
     if scores is None:
+        ld = int(ld if ld is not None else max_pos + 1)
         scores = torch.empty((Nq, ld), dtype=torch.float32, device=qI.device)
+    else:
+        have = _rows_out(scores, Nq, max_pos + 1, "scores")
+        if ld is not None and int(ld) != have:
+            raise ValueError(f"ld={ld} does not match scores of {have} columns")
+        ld = have
     if ws is None:
         ws = workspace(lib().sa_index_score_prefill_workspace_size(Nq), qI.device)
+    _ws(ws)
     _check(lib().sa_index_score_prefill(_ptr(qI), _ptr(w), _ptr(KI), _ptr(q_pos), Nq, KI.shape[0], max_pos, H_I,
                                         d_I, _ptr(scores), ld, _ptr(ws), ws.numel(), _stream(stream)))
     return scores
@@ -154,13 +195,18 @@ def index_score_prefill(qI, w, KI, q_pos, max_pos: int, scores=None, ld: Optiona
 
 def topk(scores, n_valid, n_max: int, k: int, idx=None, top_scores=None, want_scores=False, ws=None, stream=None):
     Nq, ld = scores.shape
-    _dev(scores, torch.float32, "scores"), _dev(n_valid, torch.int32, "n_valid")
+    _rows_out(scores, Nq, n_max, "scores")
+    _out(n_valid, (Nq,), (torch.int32,), "n_valid")
     if idx is None:
         idx = torch.empty((Nq, k), dtype=torch.int32, device=scores.device)
+    _out(idx, (Nq, k), (torch.int32,), "idx")
     if want_scores and top_scores is None:
         top_scores = torch.empty((Nq, k), dtype=torch.float32, device=scores.device)
+    if top_scores is not None:
+        _out(top_scores, (Nq, k), (torch.float32,), "top_scores")
     if ws is None:
         ws = workspace(lib().sa_topk_workspace_size(Nq, n_max, k), scores.device)
+    _ws(ws)
     _check(lib().sa_topk(_ptr(scores), ld, _ptr(n_valid), Nq, n_max, k, _ptr(idx), _ptr(top_scores), _ptr(ws),
                          ws.numel(), _stream(stream)))
     return (idx, top_scores) if want_scores else idx
@@ -177,11 +223,14 @@ def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, o
     k = idx.shape[1]
     n_tokens = K.numel() // (Hkv * d)
     _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
-    _dev(idx, torch.int32, "idx")
+    _out(idx, (B, k), (torch.int32,), "idx")
+    _seqs(seq_off, seq_len, B)
     if O is None:
         O = torch.empty((L, B, Hq, d), dtype=out_dtype, device=Q.device)
+    _out(O, (L, B, Hq, d), (torch.bfloat16, torch.float32), "O")
     if ws is None:
         ws = workspace(sparse_decode_attn_workspace_size(L, B, Hq, Hkv, d, k), Q.device)
+    _ws(ws)
     code = SA_F32 if O.dtype == torch.float32 else SA_BF16
     _check(lib().sa_sparse_decode_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), _ptr(idx), L, B,
                                        n_tokens, Hq, Hkv, d, k, float(scale), _ptr(O), code, _ptr(ws), ws.numel(),
@@ -202,15 +251,19 @@ def indexer_layer_attn(Q, K, V, seq_off, seq_len, S_max: int, Hkv: int, scale: f
     B, Hq, d = Q.shape
     n_tokens = K.numel() // (Hkv * d)
     _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
+    _seqs(seq_off, seq_len, B)
     if O is None:
         O = torch.empty((B, Hq, d), dtype=out_dtype, device=Q.device)
+    _out(O, (B, Hq, d), (torch.bfloat16, torch.float32), "O")
     if scores is None:
         scores = torch.empty((B, max(S_max, 1)), dtype=torch.float32, device=Q.device)
+    ld = _rows_out(scores, B, S_max, "scores")
     if ws is None:
         ws = workspace(indexer_layer_attn_workspace_size(B, S_max, Hq, Hkv, d), Q.device)
+    _ws(ws)
     code = SA_F32 if O.dtype == torch.float32 else SA_BF16
     _check(lib().sa_indexer_layer_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), B, n_tokens, S_max,
-                                       Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(scores), scores.stride(0),
+                                       Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(scores), ld,
                                        _ptr(ws), ws.numel(), _stream(stream)))
     return O, scores
 
@@ -271,14 +324,20 @@ def decode_step(pattern: str, qI: Sequence, w: Sequence, KI: Sequence, K: Sequen
     f0 = next(t for t in qI if t is not None)
     H_I, d_I = f0.shape[1], f0.shape[2]
     n_tokens = next(t for t in KI if t is not None).shape[0]
+    _dev(Q, torch.bfloat16, "Q")
+    _seqs(seq_off, seq_len, B)
     if O is None:
         O = torch.empty((L, B, Hq, d), dtype=out_dtype, device=Q.device)
+    _out(O, (L, B, Hq, d), (torch.bfloat16, torch.float32), "O")
     if idx is None:
         idx = torch.empty((B, k), dtype=torch.int32, device=Q.device)
+    _out(idx, (B, k), (torch.int32,), "idx")
     if scores is None:
         scores = torch.empty((B, max(S_max, 1)), dtype=torch.float32, device=Q.device)
+    _rows_out(scores, B, S_max, "scores")
     if ws is None:
         ws = workspace(decode_step_workspace_size(n, B, S_max, Hq, Hkv, d, k), Q.device)
+    _ws(ws)
     keep = []
     arrays = []
     for lst in (qI, w, KI, K, V):
@@ -312,17 +371,21 @@ def block_union_prefill(idx, q_pos, Q, K, V, block: int, scale: float, out_dtype
     Nq, Hq, d = Q.shape
     Hkv, S, _ = K.shape
     k = idx.shape[1]
-    _dev(idx, torch.int32, "idx"), _dev(q_pos, torch.int32, "q_pos")
+    _out(idx, (Nq, k), (torch.int32,), "idx"), _out(q_pos, (Nq,), (torch.int32,), "q_pos")
     _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
     nb = (S + block - 1) // block
     if kv_indptr is None:
         kv_indptr = torch.empty(Hkv + 1, dtype=torch.int32, device=Q.device)
+    _out(kv_indptr, (Hkv + 1,), (torch.int32,), "kv_indptr")
     if kv_indices is None:
         kv_indices = torch.empty(Hkv * nb, dtype=torch.int32, device=Q.device)
+    _out(kv_indices, (Hkv * nb,), (torch.int32,), "kv_indices")
     if O is None:
         O = torch.empty((Nq, Hq, d), dtype=out_dtype, device=Q.device)
+    _out(O, (Nq, Hq, d), (torch.bfloat16, torch.float32), "O")
     if ws is None:
         ws = workspace(lib().sa_block_union_prefill_workspace_size(S, Nq, Hq, Hkv, d, k, block), Q.device)
+    _ws(ws)
     code = SA_F32 if O.dtype == torch.float32 else SA_BF16
     _check(lib().sa_block_union_prefill(_ptr(idx), _ptr(q_pos), _ptr(Q), _ptr(K), _ptr(V), S, Nq, Hq, Hkv, d, k,
                                         block, float(scale), _ptr(kv_indptr), _ptr(kv_indices), _ptr(O), code,
@@ -339,8 +402,12 @@ def block_union_prefill_noalloc(idx, q_pos, Q, K, V, block: int, scale: float, k
     Nq, Hq, d = Q.shape
     Hkv, S, _ = K.shape
     k = idx.shape[1]
-    _dev(idx, torch.int32, "idx"), _dev(q_pos, torch.int32, "q_pos")
+    _out(idx, (Nq, k), (torch.int32,), "idx"), _out(q_pos, (Nq,), (torch.int32,), "q_pos")
     _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
+    nb = (S + block - 1) // block
+    _out(kv_indptr, (Hkv + 1,), (torch.int32,), "kv_indptr")
+    _out(kv_indices, (Hkv * nb,), (torch.int32,), "kv_indices")
+    _out(O, (Nq, Hq, d), (torch.bfloat16, torch.float32), "O")
     code = SA_F32 if O.dtype == torch.float32 else SA_BF16
     _check(lib().sa_block_union_prefill_noalloc(_ptr(idx), _ptr(q_pos), _ptr(Q), _ptr(K), _ptr(V), S, Nq, Hq, Hkv,
                                                 d, k, block, float(scale), _ptr(kv_indptr), _ptr(kv_indices),

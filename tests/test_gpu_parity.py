@@ -570,3 +570,25 @@ def test_indexer_layer_reports_bad_length(dev):
     O_ora, _ = oracle.indexer_layer_attn(Q[:1], K[:300 * Hkv * d], V[:300 * Hkv * d], seq_off[:2], lens_real[:1],
                                          Hkv, 1 / math.sqrt(d))
     assert np.abs(O_h[0] - O_ora[0]).max() <= parity.ATOL_F32
+
+
+def test_binding_rejects_outputs_of_the_wrong_shape(dev):
+    """Caller-supplied outputs and sequence tables are checked before any
+    launch: a kernel would otherwise write past a smaller tensor."""
+    d, B, Hq, Hkv, L, k, S = 128, 2, 8, 2, 2, 64, 300
+    Q = torch.zeros((L, B, Hq, d), dtype=torch.bfloat16, device=dev)
+    K = torch.zeros((B * S * Hkv * d,), dtype=torch.bfloat16, device=dev)
+    seq_off = torch.tensor([0, S, 2 * S], device=dev)
+    seq_len = torch.tensor([S, S], dtype=torch.int32, device=dev)
+    idx = torch.zeros((B, k), dtype=torch.int32, device=dev)
+    with pytest.raises(ValueError, match="O must have shape"):
+        sa.sparse_decode_attn(Q, K, K, seq_off, seq_len, idx, Hkv, 0.088,
+                              O=torch.empty((L, B, Hq, d - 1), dtype=torch.bfloat16, device=dev))
+    with pytest.raises(ValueError, match="seq_off"):
+        sa.sparse_decode_attn(Q, K, K, seq_off.to(torch.int32), seq_len, idx, Hkv, 0.088)
+    with pytest.raises(ValueError, match="scores must be"):
+        sa.indexer_layer_attn(Q[0], K, K, seq_off, seq_len, S, Hkv, 0.088,
+                              scores=torch.empty((B, S - 1), dtype=torch.float32, device=dev))
+    with pytest.raises(ValueError, match="idx must have shape"):
+        sa.topk(torch.zeros((B, S), device=dev), seq_len, S, k, idx=torch.empty((B, k - 1), dtype=torch.int32,
+                                                                                 device=dev))
