@@ -740,21 +740,35 @@ def run_ours(args):
     ms_attn = timed(lambda i: g_attn.replay(), n_rep) / (n_rep * REP)
 
     # ---- end to end through the public API: pinned host in, host out ---------
-    # Every step copies its queries, indexer queries and head weights in from
-    # pinned host memory and its outputs back out.  Copies run on their own
-    # streams with two device buffer sets, so step i+1's inputs travel while
-    # step i computes; the steps themselves stay in order on one stream.
+    # Every step copies its inputs in from pinned host memory (the queries of
+    # every layer and the indexer queries and head weights of every F layer,
+    # packed in one buffer: one copy), runs through a DecodeStepPlan (the
+    # call prepared once for these buffers), and copies its outputs back out.
+    # Copies run on their own streams with two device buffer sets, so step
+    # i+1's inputs travel while step i computes; the steps themselves stay in
+    # order on one stream.
     nbuf = len(sets)
-    host_in = []
+    e2e = []
     for st in sets:
-        host_in.append({"qI": [t.cpu().pin_memory() if t is not None else None for t in st["qI"]],
-                        "w": [t.cpu().pin_memory() if t is not None else None for t in st["w"]],
-                        "Q": st["wl"]["Q"].cpu().pin_memory(),
-                        "O": torch.empty(st["O"].shape, dtype=st["O"].dtype).pin_memory()})
-    hi0 = host_in[0]
-    h2d = hi0["Q"].numel() * hi0["Q"].element_size() + sum(
-        t.numel() * t.element_size() for t in hi0["qI"] + hi0["w"] if t is not None)
-    d2h = hi0["O"].numel() * hi0["O"].element_size()
+        parts = [st["wl"]["Q"]] + [t for t in st["qI"] if t is not None] + [t for t in st["w"] if t is not None]
+        offs, total = [], 0
+        for t in parts:
+            offs.append(total)
+            total += (t.numel() * t.element_size() + 255) // 256 * 256
+        dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+        views = [dbuf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for t, o in zip(parts, offs)]
+        for v, t in zip(views, parts):
+            v.copy_(t)
+        rest = iter(views[1:])
+        qIv = [next(rest) if t is not None else None for t in st["qI"]]
+        wv = [next(rest) if t is not None else None for t in st["w"]]
+        plan = sa.DecodeStepPlan(cfg.pattern, qIv, wv, st["KI"], st["K"], st["V"], st["wl"]["seq_off"],
+                                 st["wl"]["seq_len"], cfg.S_max, cfg.k, views[0], cfg.Hkv, cfg.scale, O=st["O"],
+                                 idx=st["idx"], scores=st["scores"], ws=st["ws"])
+        e2e.append({"dbuf": dbuf, "hbuf": dbuf.cpu().pin_memory(), "plan": plan, "O": st["O"],
+                    "O_host": torch.empty(st["O"].shape, dtype=st["O"].dtype).pin_memory()})
+    h2d = e2e[0]["hbuf"].numel()
+    d2h = e2e[0]["O_host"].numel() * e2e[0]["O_host"].element_size()
     cs, hs, ds = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     h2d_ev = [torch.cuda.Event() for _ in range(nbuf)]
     comp_ev = [torch.cuda.Event() for _ in range(nbuf)]
@@ -762,31 +776,25 @@ def run_ours(args):
 
     def e2e_h2d(i):
         b = i % nbuf
-        st, hi = sets[b], host_in[b]
+        e = e2e[b]
+        if i >= nbuf:
+            hs.wait_event(comp_ev[b])  # the step that last read this buffer set is done
         with torch.cuda.stream(hs):
-            if i >= nbuf:
-                hs.wait_event(comp_ev[b])  # the step that last read this buffer set is done
-            for dsrc, hsrc in zip(st["qI"], hi["qI"]):
-                if hsrc is not None:
-                    dsrc.copy_(hsrc, non_blocking=True)
-            for dsrc, hsrc in zip(st["w"], hi["w"]):
-                if hsrc is not None:
-                    dsrc.copy_(hsrc, non_blocking=True)
-            st["wl"]["Q"].copy_(hi["Q"], non_blocking=True)
-            h2d_ev[b].record(hs)
+            e["dbuf"].copy_(e["hbuf"], non_blocking=True)
+        h2d_ev[b].record(hs)
 
     def e2e_step_out(i):
         b = i % nbuf
-        st, hi = sets[b], host_in[b]
+        e = e2e[b]
         cs.wait_event(h2d_ev[b])
         if i >= nbuf:
             cs.wait_event(d2h_ev[b])  # O of this buffer set has been copied out
-        step(st, stream=cs)
+        e["plan"].run(cs)
         comp_ev[b].record(cs)
+        ds.wait_event(comp_ev[b])
         with torch.cuda.stream(ds):
-            ds.wait_event(comp_ev[b])
-            hi["O"].copy_(st["O"], non_blocking=True)
-            d2h_ev[b].record(ds)
+            e["O_host"].copy_(e["O"], non_blocking=True)
+        d2h_ev[b].record(ds)
 
     def e2e_run(n):
         e2e_h2d(0)
@@ -859,10 +867,11 @@ def run_ours(args):
         "attn_route": route,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "note": "per step: pinned host -> device copy of that step's queries, indexer queries and head "
-                        "weights; the step through the public API; device -> pinned host copy of the outputs; "
-                        "copies on their own streams with two buffer sets (step i+1's inputs travel while step i "
-                        "computes; steps run in order on one stream); the KV and indexer-key caches stay resident"},
+                "note": "per step: one pinned host -> device copy of that step's queries, indexer queries and "
+                        "head weights (packed); the step through the public API (a DecodeStepPlan prepared once "
+                        "for these buffers); device -> pinned host copy of the outputs; copies on their own "
+                        "streams with two buffer sets (step i+1's inputs travel while step i computes; steps run "
+                        "in order on one stream); the KV and indexer-key caches stay resident"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": cs,
     }

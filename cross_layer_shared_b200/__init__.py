@@ -43,9 +43,9 @@ SIGNATURES = {
     "sa_indexer_layer_attn_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
     "sa_indexer_layer_attn": ([_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _F, _P, _I, _P, _I64, _P, _SZ, _P], _I),
     "sa_decode_step_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
-    "sa_decode_step": ([ctypes.c_char_p, _I, _PP, _PP, _PP, _PP, _PP, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _I,
+    "sa_decode_step": ([ctypes.c_char_p, _I, _P, _P, _P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _P, _I,
                         _I, _I, _F, _P, _I, _P, _P, _I64, _P, _SZ, _P], _I),
-    "sa_decode_step_ex": ([ctypes.c_char_p, _I, _PP, _PP, _PP, _PP, _PP, _PP, _PP, _PP, _P, _P, _I, _I64, _I, _I,
+    "sa_decode_step_ex": ([ctypes.c_char_p, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I64, _I, _I,
                            _I, _I, _P, _I, _I, _I, _F, _P, _I, _P, _P, _I64, _I, _P, _SZ, _P], _I),
     "sa_block_union_prefill_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "sa_block_union_prefill": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P, _SZ, _P],
@@ -92,9 +92,17 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream) -> int:
+    """The cudaStream_t of `stream`, or of the current stream (the raw query
+    skips building a Stream object on every call)."""
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None:
+        return _raw_stream(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _dev(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
@@ -296,14 +304,30 @@ def decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k) -> int:
     return int(lib().sa_decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k))
 
 
-def _ptr_array(ts: Sequence[Optional[torch.Tensor]]):
-    """Host array of device pointers (NULL for None); a tensor listed for many
-    layers is asked for its address once."""
+def _ptr_arrays(lists: Sequence[Sequence[Optional[torch.Tensor]]]):
+    """Host arrays of device pointers (NULL for None), one per list, in one
+    buffer: returns the buffer (keep it alive across the call) and the
+    address of each array.  A tensor listed many times is asked for its
+    address once."""
     memo = {}
-    vals = [0 if t is None else (memo.get(id(t)) or memo.setdefault(id(t), t.data_ptr())) for t in ts]
+    vals = []
+    for lst in lists:
+        for t in lst:
+            if t is None:
+                vals.append(0)
+            else:
+                p = memo.get(id(t))
+                if p is None:
+                    p = memo[id(t)] = t.data_ptr()
+                vals.append(p)
     buf = array.array("Q", vals)
-    arr = (ctypes.c_void_p * len(vals)).from_buffer(buf)
-    return ctypes.cast(arr, _PP), (buf, arr)
+    base = buf.buffer_info()[0]
+    addrs = []
+    off = 0
+    for lst in lists:
+        addrs.append(base + 8 * off)
+        off += len(lst)
+    return buf, addrs
 
 
 STEP_PER_LAYER = 1
@@ -338,31 +362,70 @@ def decode_step(pattern: str, qI: Sequence, w: Sequence, KI: Sequence, K: Sequen
     if ws is None:
         ws = workspace(decode_step_workspace_size(n, B, S_max, Hq, Hkv, d, k), Q.device)
     _ws(ws)
-    keep = []
-    arrays = []
-    for lst in (qI, w, KI, K, V):
-        p, a = _ptr_array(lst)
-        arrays.append(p)
-        keep.append(a)
     code = SA_F32 if O.dtype == torch.float32 else SA_BF16
     if new_KI is None and new_K is None and not per_layer:
-        _check(lib().sa_decode_step(pattern.encode(), n, *arrays, _ptr(seq_off), _ptr(seq_len), B, n_tokens, S_max,
-                                    H_I, d_I, k, _ptr(Q), Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(idx),
-                                    _ptr(scores), scores.shape[1], _ptr(ws), ws.numel(), _stream(stream)))
+        buf, arrays = _ptr_arrays((qI, w, KI, K, V))
+        _check(lib().sa_decode_step(pattern.encode(), n, *arrays, seq_off.data_ptr(), seq_len.data_ptr(), B,
+                                    n_tokens, S_max, H_I, d_I, k, Q.data_ptr(), Hq, Hkv, d, float(scale),
+                                    O.data_ptr(), code, idx.data_ptr(), scores.data_ptr(), scores.shape[1],
+                                    ws.data_ptr(), ws.numel(), _stream(stream)))
         return O, idx
-    extra = []
-    for lst in (new_KI, new_K, new_V):
-        if lst is None:
-            extra.append(None)
-        else:
-            p, a = _ptr_array(lst)
-            extra.append(p)
-            keep.append(a)
-    _check(lib().sa_decode_step_ex(pattern.encode(), n, *arrays, *extra, _ptr(seq_off), _ptr(seq_len), B, n_tokens,
-                                   S_max, H_I, d_I, k, _ptr(Q), Hq, Hkv, d, float(scale), _ptr(O), code, _ptr(idx),
-                                   _ptr(scores), scores.shape[1], STEP_PER_LAYER if per_layer else 0, _ptr(ws),
-                                   ws.numel(), _stream(stream)))
+    extra_lists = [lst for lst in (new_KI, new_K, new_V) if lst is not None]
+    buf, arrays = _ptr_arrays([qI, w, KI, K, V] + extra_lists)
+    it = iter(arrays[5:])
+    extra = [None if lst is None else next(it) for lst in (new_KI, new_K, new_V)]
+    _check(lib().sa_decode_step_ex(pattern.encode(), n, *arrays[:5], *extra, seq_off.data_ptr(), seq_len.data_ptr(),
+                                   B, n_tokens, S_max, H_I, d_I, k, Q.data_ptr(), Hq, Hkv, d, float(scale),
+                                   O.data_ptr(), code, idx.data_ptr(), scores.data_ptr(), scores.shape[1],
+                                   STEP_PER_LAYER if per_layer else 0, ws.data_ptr(), ws.numel(),
+                                   _stream(stream)))
     return O, idx
+
+
+class DecodeStepPlan:
+    """sa_decode_step prepared once for tensors a decode loop reuses every
+    step (caches, query buffers, outputs, workspace): the arguments are
+    checked and marshalled here, and run() makes only the C call.  The plan
+    holds the tensors it points to; build a new plan if any of them is
+    replaced by another allocation."""
+
+    def __init__(self, pattern: str, qI: Sequence, w: Sequence, KI: Sequence, K: Sequence, V: Sequence, seq_off,
+                 seq_len, S_max: int, k: int, Q, Hkv: int, scale: float, out_dtype=torch.bfloat16, O=None, idx=None,
+                 scores=None, ws=None):
+        L, B, Hq, d = Q.shape
+        n = len(pattern)
+        if not (L == n and len(qI) == n and len(w) == n and len(KI) == n and len(K) == n and len(V) == n):
+            raise ValueError("every per-layer list and Q must have one entry per pattern letter")
+        f0 = next(t for t in qI if t is not None)
+        H_I, d_I = f0.shape[1], f0.shape[2]
+        n_tokens = next(t for t in KI if t is not None).shape[0]
+        _dev(Q, torch.bfloat16, "Q")
+        _seqs(seq_off, seq_len, B)
+        if O is None:
+            O = torch.empty((L, B, Hq, d), dtype=out_dtype, device=Q.device)
+        _out(O, (L, B, Hq, d), (torch.bfloat16, torch.float32), "O")
+        if idx is None:
+            idx = torch.empty((B, k), dtype=torch.int32, device=Q.device)
+        _out(idx, (B, k), (torch.int32,), "idx")
+        if scores is None:
+            scores = torch.empty((B, max(S_max, 1)), dtype=torch.float32, device=Q.device)
+        _rows_out(scores, B, S_max, "scores")
+        if ws is None:
+            ws = workspace(decode_step_workspace_size(n, B, S_max, Hq, Hkv, d, k), Q.device)
+        _ws(ws)
+        self.O, self.idx, self.scores, self.ws = O, idx, scores, ws
+        self._hold = (qI, w, KI, K, V, seq_off, seq_len, Q)
+        self._buf, arrays = _ptr_arrays((qI, w, KI, K, V))
+        code = SA_F32 if O.dtype == torch.float32 else SA_BF16
+        self._args = (pattern.encode(), n, *arrays, seq_off.data_ptr(), seq_len.data_ptr(), B, n_tokens, S_max, H_I,
+                      d_I, k, Q.data_ptr(), Hq, Hkv, d, float(scale), O.data_ptr(), code, idx.data_ptr(),
+                      scores.data_ptr(), scores.shape[1], ws.data_ptr(), ws.numel())
+        self._fn = lib().sa_decode_step
+
+    def run(self, stream=None):
+        """Enqueue the step on `stream` (default: the current stream); returns (O, idx)."""
+        _check(self._fn(*self._args, _stream(stream)))
+        return self.O, self.idx
 
 
 def block_union_prefill(idx, q_pos, Q, K, V, block: int, scale: float, out_dtype=torch.bfloat16, O=None,

@@ -95,10 +95,43 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// A tensor map is a pure function of the address and the geometry, so the
+// last few encoded per host thread are kept and reused (a decode step encodes
+// the same five every call).
+struct TmapKey {
+  const void* base;
+  int rank;
+  uint64_t dims[3], strides[2];
+  uint32_t box[3];
+  bool operator==(const TmapKey& o) const { return memcmp(this, &o, sizeof *this) == 0; }
+};
+struct TmapEntry {
+  TmapKey key;
+  CUtensorMap map;
+  bool used;
+};
+constexpr int kTmapCache = 16;
+thread_local TmapEntry g_tmap_cache[kTmapCache];
+thread_local int g_tmap_next = 0;
+
 // bf16 tensor map with 128-byte swizzle; dims innermost first (elements),
 // strides in bytes for dims 1.. ; box in elements.
 sa_status make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
                     const uint32_t* box) {
+  TmapKey key;
+  memset(&key, 0, sizeof key);  // padding included: the key compares as bytes
+  key.base = base;
+  key.rank = rank;
+  for (int i = 0; i < rank && i < 3; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+    if (i + 1 < rank) key.strides[i] = strides[i];
+  }
+  for (int i = 0; i < kTmapCache; ++i)
+    if (g_tmap_cache[i].used && g_tmap_cache[i].key == key) {
+      *m = g_tmap_cache[i].map;
+      return SA_OK;
+    }
   auto fn = encode_fn();
   if (!fn) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   uint32_t estr[3] = {1, 1, 1};
@@ -106,6 +139,11 @@ sa_status make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* 
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SA_ERR_INVALID_ARG, "tensor map encoding failed (CUresult %d)", (int)r);
+  TmapEntry& e = g_tmap_cache[g_tmap_next];
+  g_tmap_next = (g_tmap_next + 1) % kTmapCache;
+  e.key = key;
+  e.map = *m;
+  e.used = true;
   return SA_OK;
 }
 

@@ -47,7 +47,9 @@
  * - Between calls the library keeps only per-device facts it looks up once
  *   (the driver's tensor-map entry point, the SM count, the largest cluster
  *   the top-k kernel can be scheduled with, which kernels have had their
- *   shared-memory limit raised) and the fixed scratch array of
+ *   shared-memory limit raised), per host thread the last 16 tensor maps it
+ *   encoded (each a function of an address and a shape only), and the fixed
+ *   scratch array of
  *   sa_block_union_prefill_noalloc (see there); the workspace entry points
  *   are reentrant and thread-safe.
  */

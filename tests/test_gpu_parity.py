@@ -592,3 +592,33 @@ def test_binding_rejects_outputs_of_the_wrong_shape(dev):
     with pytest.raises(ValueError, match="idx must have shape"):
         sa.topk(torch.zeros((B, S), device=dev), seq_len, S, k, idx=torch.empty((B, k - 1), dtype=torch.int32,
                                                                                  device=dev))
+
+
+def test_decode_step_plan_matches_decode_step(dev):
+    """A DecodeStepPlan (arguments checked and marshalled once) runs the same
+    step as decode_step, bit for bit, also after its input buffers are
+    refilled in place (c2: three F layers)."""
+    cfg = synth.workload("c2")
+    wl = sgpu.decode_workload(cfg, dev)
+    n = cfg.L
+    gi = [max(i for i, g in enumerate(cfg.groups) if g[0] <= l) for l in range(n)]  # each layer's group
+    grs = wl["groups"]
+    qI = [grs[gi[l]]["qI"] if cfg.pattern[l] == "F" else None for l in range(n)]
+    w = [grs[gi[l]]["w"] if cfg.pattern[l] == "F" else None for l in range(n)]
+    KI = [grs[gi[l]]["KI"] if cfg.pattern[l] == "F" else None for l in range(n)]
+    K = [grs[gi[l]]["K"] for l in range(n)]
+    V = [grs[gi[l]]["V"] for l in range(n)]
+    O0, idx0 = sa.decode_step(cfg.pattern, qI, w, KI, K, V, wl["seq_off"], wl["seq_len"], cfg.S_max, cfg.k, wl["Q"],
+                              cfg.Hkv, cfg.scale)
+    Q = wl["Q"].clone()
+    plan = sa.DecodeStepPlan(cfg.pattern, qI, w, KI, K, V, wl["seq_off"], wl["seq_len"], cfg.S_max, cfg.k, Q, cfg.Hkv,
+                             cfg.scale)
+    O1, idx1 = plan.run()
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O0) and torch.equal(idx1, idx0)
+    Q.copy_(torch.flip(wl["Q"], dims=[1]))  # new queries in the same buffer
+    O2, _ = plan.run()
+    O3, _ = sa.decode_step(cfg.pattern, qI, w, KI, K, V, wl["seq_off"], wl["seq_len"], cfg.S_max, cfg.k, Q, cfg.Hkv,
+                           cfg.scale)
+    assert torch.equal(O2, O3)
+    assert_status_ok(plan.ws)
