@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <cmath>
 #include <mutex>
 #include <string>
 
@@ -212,6 +213,27 @@ AttnPlan plan_decode_attn(int L_g, int B, int Hq, int Hkv, int k) {
   p.n_split = s;  // trailing splits may get no keys; they merge as empty
   p.units = base * p.n_split;
   return p;
+}
+
+// Key splits per prefill row tile (a cluster of 1, 2 or 4 CTAs, merged at the
+// end): the fewest whose launch fills its last wave of one-CTA-per-SM units to
+// within 5 %.  Every unit of a prefill chunk has about the same work (the
+// union of blocks is shared), so a part-empty last wave idles SMs for a
+// whole unit's time: c4's 512 units on 148 SMs are 3.46 waves (86 % busy),
+// split in two 6.92 waves (99 %).
+int prefill_split(int units) {
+  const int sms = num_sms();
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 4; s *= 2) {
+    const double waves = (double)units * s / sms;
+    const double eff = waves / std::ceil(waves);
+    if (eff > best_eff + 0.05) {
+      best = s;
+      best_eff = eff;
+    }
+  }
+  return best;
 }
 
 size_t attn_ws_bytes(const AttnPlan& p) {
@@ -701,7 +723,7 @@ sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const
   a.G = Hq / Hkv;
   a.R = Nq * a.G;
   a.n_mtiles = (a.R + 127) / 128;
-  a.n_split = 1;
+  a.n_split = prefill_split(Hkv * a.n_mtiles);
   a.keys_per_split = (int)round_up((size_t)((S + block - 1) / block) * block, 128);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;
@@ -800,7 +822,7 @@ extern "C" sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const in
   a.G = Hq / Hkv;
   a.R = Nq * a.G;
   a.n_mtiles = (a.R + 127) / 128;
-  a.n_split = 1;
+  a.n_split = prefill_split(Hkv * a.n_mtiles);
   a.keys_per_split = (int)round_up((size_t)nb * block, 128);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;

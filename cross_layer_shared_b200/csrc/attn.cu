@@ -260,8 +260,11 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     ks.base = a.kv_indptr[g];
     n_keys = (a.kv_indptr[g + 1] - ks.base) * a.block;
   }
-  ks.kbeg = split * a.keys_per_split;
-  ks.kend = min(n_keys, ks.kbeg + a.keys_per_split);
+  // decode: the host's even split of k; prefill: the union's size is known
+  // only here, so its split is even over that size (whole 128-key tiles)
+  const int per = a.prefill ? ((n_keys + a.n_split - 1) / a.n_split + kKT - 1) / kKT * kKT : a.keys_per_split;
+  ks.kbeg = split * per;
+  ks.kend = min(n_keys, ks.kbeg + per);
   const int nt = ks.kend > ks.kbeg ? (ks.kend - ks.kbeg + kKT - 1) / kKT : 0;
 
   // producer lanes: raw entries of tile rows 4*lane .. 4*lane+3, one tile ahead
