@@ -506,13 +506,29 @@ def set_bytes(cfg) -> int:
     return len(cfg.groups) * per_group
 
 
+def input_sets(cfg, args) -> int:
+    """Rotating input sets: as asked, else two when they fit in 80 % of the
+    device's free memory (the full 180 GB when no device is visible), else one."""
+    if args.sets > 0:
+        return args.sets
+    free = 180e9
+    try:
+        import torch
+        if torch.cuda.is_available():
+            free, _ = torch.cuda.mem_get_info()
+    except Exception:
+        pass
+    return 2 if 2 * set_bytes(cfg) < 0.8 * free else 1
+
+
 def workload_config(cfg, args):
     return {"workload": f"{cfg.name}: {synth.DESCRIPTIONS[cfg.name]}", "batch": cfg.B, "context": cfg.S_max,
             "layers": cfg.L, "pattern": cfg.pattern if len(cfg.pattern) <= 8 else f"{cfg.pattern[:4]}... ({cfg.L})",
             "top_k": cfg.k, "indexer": f"{cfg.H_I}x{cfg.d_I}", "heads": f"{cfg.Hq}q/{cfg.Hkv}kv", "head_dim": cfg.d,
-            "l2": (f"{args.sets} rotating input set(s) of {set_bytes(cfg) / 1e9:.1f} GB each, larger than L2"
+            "l2": (f"{input_sets(cfg, args)} rotating input set(s) of {set_bytes(cfg) / 1e9:.1f} GB each, larger than L2"
                    if set_bytes(cfg) > L2_BYTES else
-                   f"{args.sets} input set(s) of {set_bytes(cfg) / 1e6:.1f} MB: resident in L2 (warm-cache figure)"),
+                   f"{input_sets(cfg, args)} input set(s) of {set_bytes(cfg) / 1e6:.1f} MB: resident in L2 "
+                   f"(warm-cache figure)"),
             "parallelism": "replicas" if args.gpus > 1 else "single"}
 
 
@@ -543,9 +559,7 @@ def run_ours(args):
     n = cfg.L
     nb = algorithmic_bytes(cfg, 4 if args.out_f32 else 2)
 
-    if args.sets <= 0:  # two rotating sets when they fit (with room to spare), else one
-        free, _ = torch.cuda.mem_get_info(dev)
-        args.sets = 2 if 2 * set_bytes(cfg) < 0.8 * free else 1
+    args.sets = input_sets(cfg, args)
     sets = []
     for si in range(args.sets):
         wl = sgpu.decode_workload(cfg, dev)
