@@ -6,7 +6,10 @@ leg may import this package.  It shares no code with the CUDA path in
 ``oracle/sa_oracle.c`` (fp64, naive loops, OpenMP over independent
 outputs), loaded here through ctypes; the only Python logic is the layer
 pattern walk of ``decode_step`` (IndexCache's F/S rule) and argument
-marshalling.
+marshalling.  The context-parallel pieces (``sparse_decode_attn_partial``,
+``combine_partials``, ``cp_select``) have no oracle of a whole sharded step:
+a sharded step must equal the one-device ``decode_step``, which is the
+oracle for it.
 
 Parity pins: tests/test_oracle_pins.py.
 """
@@ -51,6 +54,9 @@ def load(path: str):
     lb.oracle_block_union.restype = I
     lb.oracle_paged_prefill_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P, D, P]
     lb.oracle_indexer_layer_attn.argtypes = [P, P, P, P, P, I, I, I, I, I, D, P, P, I64, P]
+    lb.oracle_sparse_decode_attn_partial.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, D, P, P]
+    lb.oracle_combine_partials.argtypes = [P, P, I, I64, I, P]
+    lb.oracle_cp_select.argtypes = [P, P, I, I, I, I, P]
     lb.oracle_num_threads.restype = I
     return lb
 
@@ -111,6 +117,42 @@ def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float) -
     lib().oracle_sparse_decode_attn(_p(Q), _p(K), _p(V), _p(_c(seq_off, np.int64)),
                                     _p(_c(seq_len, np.int32)), _p(idx), L, B, Hq, Hkv, d, k,
                                     float(scale), _p(out))
+    return out
+
+
+def sparse_decode_attn_partial(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float):
+    """One rank's share of a context-parallel step: (O_part [L,B,Hq,d],
+    ml [L,B,Hq,2]) fp64, the attention rows before the division, with the
+    row max in log2 units and the sum of weights."""
+    Q = _c(Q, np.uint16)
+    L, B, Hq, d = Q.shape
+    idx = _c(idx, np.int32)
+    k = idx.shape[1]
+    O = np.empty((L, B, Hq, d), dtype=np.float64)
+    ml = np.empty((L, B, Hq, 2), dtype=np.float64)
+    lib().oracle_sparse_decode_attn_partial(_p(Q), _p(_c(K, np.uint16)), _p(_c(V, np.uint16)),
+                                            _p(_c(seq_off, np.int64)), _p(_c(seq_len, np.int32)), _p(idx), L,
+                                            B, Hq, Hkv, d, k, float(scale), _p(O), _p(ml))
+    return O, ml
+
+
+def combine_partials(O_part, ml) -> np.ndarray:
+    """Log-sum-exp merge of P partials: O_part [P, rows, d], ml [P, rows, 2]."""
+    O_part = _c(O_part, np.float64)
+    ml = _c(ml, np.float64)
+    P, rows, d = O_part.shape
+    out = np.empty((rows, d), dtype=np.float64)
+    lib().oracle_combine_partials(_p(O_part), _p(ml), P, rows, d, _p(out))
+    return out
+
+
+def cp_select(cand_scores, cand_idx, rank: int) -> np.ndarray:
+    """Global top-k of N ranks' candidates [N, B, k]; rank's local indices [B, k]."""
+    cand_scores = _c(cand_scores, np.float32)
+    cand_idx = _c(cand_idx, np.int32)
+    N, B, k = cand_idx.shape
+    out = np.empty((B, k), dtype=np.int32)
+    lib().oracle_cp_select(_p(cand_scores), _p(cand_idx), N, B, k, int(rank), _p(out))
     return out
 
 

@@ -319,6 +319,124 @@ void oracle_indexer_layer_attn(const uint16_t* Q, const uint16_t* K, const uint1
     }
 }
 
+/*
+ * Context-parallel decode, one rank's attention share [CLSA, "Ce que cela
+ * signifie pour l'inference sur longs contextes": contexts past one GPU's
+ * reach are left open; sharding each sequence over ranks is this build's
+ * reading].  The rows of oracle_sparse_decode_attn, before the division:
+ *   m = max_t z_t / ln 2                 (the row's max logit in log2 units)
+ *   l = sum_t exp(z_t - max z)           (= sum_t 2^(z_t / ln 2 - m))
+ *   o = sum_t exp(z_t - max z) V_t
+ * ml holds (m, l) per row; a row with no valid index gets m = -inf, l = 0,
+ * o = 0.
+ */
+void oracle_sparse_decode_attn_partial(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                       const int64_t* seq_off, const int32_t* seq_len, const int32_t* idx,
+                                       int L, int B, int Hq, int Hkv, int d, int k, double scale,
+                                       double* O_part, double* ml) {
+  const int G = Hq / Hkv;
+  const int64_t rows = (int64_t)L * B * Hq;
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t r = 0; r < rows; ++r) {
+    const int h = (int)(r % Hq);
+    const int b = (int)((r / Hq) % B);
+    /* query head h reads KV head h / G of sequence b */
+    const int64_t base = (seq_off[b] * Hkv + (int64_t)(h / G) * seq_len[b]) * d;
+    const uint16_t* Kb = K + base;
+    const uint16_t* Vb = V + base;
+    double* o = O_part + r * d;
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    double* z = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+    double mz = -INFINITY;
+    for (int j = 0; j < k; ++j) {
+      const int32_t t = idx[(int64_t)b * k + j];
+      if (t < 0) continue;
+      double dot = 0.0;
+      for (int c = 0; c < d; ++c) dot += bf(Q[r * d + c]) * bf(Kb[(int64_t)t * d + c]);
+      z[j] = dot * scale;
+      if (z[j] > mz) mz = z[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j < k; ++j) {
+      const int32_t t = idx[(int64_t)b * k + j];
+      if (t < 0) continue;
+      const double p = exp(z[j] - mz);
+      l += p;
+      for (int c = 0; c < d; ++c) o[c] += p * bf(Vb[(int64_t)t * d + c]);
+    }
+    ml[2 * r] = l > 0.0 ? mz / log(2.0) : -INFINITY;
+    ml[2 * r + 1] = l;
+    free(z);
+  }
+}
+
+/*
+ * The log-sum-exp merge of P partial results of the same rows: with M the
+ * largest m_p over parts whose l_p > 0,
+ *   O[row] = sum_p 2^(m_p - M) o_p[row] / sum_p 2^(m_p - M) l_p,
+ * and O = 0 where every l_p = 0.  O_part [P, rows, d], ml [P, rows, 2].
+ */
+void oracle_combine_partials(const double* O_part, const double* ml, int P, int64_t rows, int d, double* O) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    double M = -INFINITY;
+    for (int p = 0; p < P; ++p)
+      if (ml[2 * ((int64_t)p * rows + r) + 1] > 0.0 && ml[2 * ((int64_t)p * rows + r)] > M)
+        M = ml[2 * ((int64_t)p * rows + r)];
+    double* o = O + r * d;
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    if (M == -INFINITY) continue;
+    double den = 0.0;
+    for (int p = 0; p < P; ++p) {
+      const double m = ml[2 * ((int64_t)p * rows + r)], l = ml[2 * ((int64_t)p * rows + r) + 1];
+      if (!(l > 0.0)) continue;
+      const double wgt = pow(2.0, m - M);
+      den += wgt * l;
+      for (int c = 0; c < d; ++c) o[c] += wgt * O_part[((int64_t)p * rows + r) * d + c];
+    }
+    for (int c = 0; c < d; ++c) o[c] /= den;
+  }
+}
+
+/*
+ * Context-parallel selection: the global top-k of the ranks' candidates.
+ * cand_scores / cand_idx [N, B, k] hold every rank's top-k over its own
+ * slice (idx < 0 = padding).  Per sequence b: the N*k candidates in order
+ * (rank-major, then the rank's order), padding scoring -inf, go through
+ * oracle_topk; the positions kept that belong to `rank` become its local
+ * indices, in ascending order, then -1.
+ */
+void oracle_cp_select(const float* cand_scores, const int32_t* cand_idx, int N, int B, int k, int rank,
+                      int32_t* local_idx) {
+  const int64_t n = (int64_t)N * k;
+  float* rows = (float*)malloc(sizeof(float) * (size_t)(B * n > 0 ? B * n : 1));
+  int32_t* n_valid = (int32_t*)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
+  int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)(B * k > 0 ? B * k : 1));
+  for (int b = 0; b < B; ++b) {
+    n_valid[b] = (int32_t)n;
+    for (int r = 0; r < N; ++r)
+      for (int j = 0; j < k; ++j) {
+        const int64_t c = ((int64_t)r * B + b) * k + j;
+        rows[(int64_t)b * n + (int64_t)r * k + j] = cand_idx[c] >= 0 ? cand_scores[c] : -INFINITY;
+      }
+  }
+  oracle_topk(rows, n, n_valid, B, k, sel, NULL);
+  for (int b = 0; b < B; ++b) {
+    int m = 0;
+    for (int j = 0; j < k; ++j) {
+      const int32_t pos = sel[(int64_t)b * k + j];
+      if (pos >= 0 && pos / k == rank) {
+        const int32_t t = cand_idx[((int64_t)rank * B + b) * k + pos % k];
+        if (t >= 0) local_idx[(int64_t)b * k + m++] = t;
+      }
+    }
+    for (int j = m; j < k; ++j) local_idx[(int64_t)b * k + j] = -1;
+  }
+  free(rows);
+  free(n_valid);
+  free(sel);
+}
+
 /* threads OpenMP will use (reported next to CPU timings) */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

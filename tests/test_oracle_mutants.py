@@ -32,6 +32,14 @@ MUTANTS = {
     "routing from the last head only": ("for (int h = 0; h < Hq; ++h) acc += P[",
                                         "for (int h = Hq - 1; h < Hq; ++h) acc += P["),
     "routing logits unscaled": ("p[t] = scale * dot;", "p[t] = dot;"),
+    "partial GQA map modulo": ("(int64_t)(h / G) * seq_len[b]) * d;", "(int64_t)(h % Hkv) * seq_len[b]) * d;"),
+    "partial max in natural units": ("ml[2 * r] = l > 0.0 ? mz / log(2.0) : -INFINITY;",
+                                     "ml[2 * r] = l > 0.0 ? mz : -INFINITY;"),
+    "partial scale dropped": ("z[j] = dot * scale;", "z[j] = dot;"),
+    "combine weight in natural units": ("const double wgt = pow(2.0, m - M);", "const double wgt = exp(m - M);"),
+    "candidates gathered rank-minor": ("rows[(int64_t)b * n + (int64_t)r * k + j] =",
+                                       "rows[(int64_t)b * n + (int64_t)j * N + r] ="),
+    "selection keeps every rank's share": ("if (pos >= 0 && pos / k == rank) {", "if (pos >= 0) {"),
     "routing drops the last token": ("for (int64_t t = 0; t < seq_len[b]; ++t) {\n      double acc",
                                      "for (int64_t t = 0; t + 1 < seq_len[b]; ++t) {\n      double acc"),
 }

@@ -541,3 +541,113 @@ def test_attn_route_step_with_every_token_selected_is_dense():
         want = _dense_attention_torch(Q[l, b, h][None], _kv(K, seq_off, S, Hkv, d, b, g),
                                       _kv(V, seq_off, S, Hkv, d, b, g), scale)[0]
         np.testing.assert_allclose(O[l, b, h], want, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# context-parallel decode: partial attention, log-sum-exp combine, selection
+# ----------------------------------------------------------------------------
+def test_cp_partial_is_the_unnormalised_softmax():
+    # library routine: torch fp64 logsumexp / softmax over the selected keys
+    rng = np.random.default_rng(40)
+    seq_off, S, Q, K, V = _tiny_decode(rng)
+    L, B, Hq, d = Q.shape
+    Hkv, k = 2, 6
+    idx = np.stack([np.sort(rng.choice(S[b], 5, replace=False)) for b in range(B)]).astype(np.int32)
+    idx = np.concatenate([idx, np.full((B, 1), -1, np.int32)], axis=1)
+    scale = 0.3
+    o, ml = oracle.sparse_decode_attn_partial(Q, K, V, seq_off, S, idx, Hkv, scale)
+    for l, b, h in itertools.product(range(L), range(B), range(Hq)):
+        g = h // (Hq // Hkv)
+        sel = torch.from_numpy(idx[b][idx[b] >= 0].astype(np.int64))
+        Kb = torch.from_numpy(bf16_bits_to_f32(_kv(K, seq_off, S, Hkv, d, b, g)).astype(np.float64))[sel]
+        Vb = torch.from_numpy(bf16_bits_to_f32(_kv(V, seq_off, S, Hkv, d, b, g)).astype(np.float64))[sel]
+        q = torch.from_numpy(bf16_bits_to_f32(Q[l, b, h]).astype(np.float64))
+        z = scale * (Kb @ q)
+        m = float(z.max())
+        assert ml[l, b, h, 0] == pytest.approx(m / math.log(2), rel=0, abs=1e-12)
+        assert ml[l, b, h, 1] == pytest.approx(math.exp(float(torch.logsumexp(z, 0)) - m), rel=1e-12)
+        np.testing.assert_allclose(o[l, b, h] / ml[l, b, h, 1], (torch.softmax(z, 0) @ Vb).numpy(), rtol=0,
+                                   atol=1e-12)
+
+
+def test_cp_partial_of_an_empty_selection():
+    rng = np.random.default_rng(41)
+    seq_off, S, Q, K, V = _tiny_decode(rng)
+    idx = np.full((2, 4), -1, np.int32)
+    o, ml = oracle.sparse_decode_attn_partial(Q, K, V, seq_off, S, idx, 2, 0.3)
+    assert np.all(o == 0) and np.all(ml[..., 1] == 0) and np.all(np.isneginf(ml[..., 0]))
+
+
+def test_cp_combine_closed_form():
+    # part 0: m = 0, l = 1, o = u; part 1: m = 1, l = 3, o = v  ->  (u + 2 v) / (1 + 6)
+    u = np.arange(4, dtype=np.float64)[None]
+    v = np.full((1, 4), 7.0)
+    ml = np.array([[[0.0, 1.0]], [[1.0, 3.0]]])
+    got = oracle.combine_partials(np.stack([u, v]), ml)
+    np.testing.assert_allclose(got[0], (u[0] + 2 * v[0]) / 7.0, rtol=0, atol=1e-15)
+    # a part with l = 0 is ignored, whatever its m; all-empty rows give 0
+    ml2 = np.array([[[0.0, 1.0], [5.0, 0.0]], [[50.0, 0.0], [-np.inf, 0.0]]])
+    parts = np.stack([np.stack([u[0], v[0]]), np.stack([v[0], u[0]])])
+    got = oracle.combine_partials(parts, ml2)
+    np.testing.assert_allclose(got[0], u[0], rtol=0, atol=0)
+    assert np.all(got[1] == 0)
+
+
+def test_cp_combine_of_a_key_split_equals_attention_over_the_union():
+    # the selected keys of each sequence split into 3 disjoint parts (one of
+    # them empty for sequence 0): the merge equals the one-part attention
+    rng = np.random.default_rng(42)
+    seq_off, S, Q, K, V = _tiny_decode(rng)
+    L, B, Hq, d = Q.shape
+    k, Hkv, scale = 8, 2, 0.4
+    idx = np.stack([np.sort(rng.choice(S[b], k, replace=False)) for b in range(B)]).astype(np.int32)
+    owner = rng.integers(0, 3, (B, k))
+    owner[0][owner[0] == 2] = 1
+    parts, mls = [], []
+    for p in range(3):
+        ip = np.where(owner == p, idx, -1).astype(np.int32)
+        o, ml = oracle.sparse_decode_attn_partial(Q, K, V, seq_off, S, ip, Hkv, scale)
+        parts.append(o.reshape(-1, d))
+        mls.append(ml.reshape(-1, 2))
+    got = oracle.combine_partials(np.stack(parts), np.stack(mls)).reshape(L, B, Hq, d)
+    want = oracle.sparse_decode_attn(Q, K, V, seq_off, S, idx, Hkv, scale)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def _python_topk(row, k):
+    order = sorted(range(len(row)), key=lambda t: (-float(row[t]), t))
+    return sorted(order[:k])
+
+
+def test_cp_select_over_slices_is_the_global_topk():
+    for N in (1, 2, 3, 5):
+        _cp_select_case(N)
+
+
+def _cp_select_case(N):
+    # scores drawn from a few values (many ties), one sequence shorter than
+    # k, one shorter than N (empty slices); brute force on the whole context
+    rng = np.random.default_rng(43 + N)
+    lens = [40, 7, 3, 64]
+    k = 9
+    B = len(lens)
+    full = [rng.integers(0, 6, n).astype(np.float32) * np.float32(0.5) for n in lens]
+    bounds = [[(r * n // N, (r + 1) * n // N) for n in lens] for r in range(N)]
+    cand_s = np.zeros((N, B, k), np.float32)
+    cand_i = np.zeros((N, B, k), np.int32)
+    for r in range(N):
+        lo_hi = bounds[r]
+        width = max(1, max(hi - lo for lo, hi in lo_hi))
+        sc = np.zeros((B, width), np.float32)
+        for b, (lo, hi) in enumerate(lo_hi):
+            sc[b, : hi - lo] = full[b][lo:hi]
+        cand_i[r], cand_s[r] = oracle.topk(sc, [hi - lo for lo, hi in lo_hi], k, with_scores=True)
+    got = [set() for _ in range(B)]
+    for r in range(N):
+        loc = oracle.cp_select(cand_s, cand_i, r)
+        for b in range(B):
+            row = [int(t) for t in loc[b] if t >= 0]
+            assert row == sorted(row) and all(t < 0 for t in loc[b][len(row):])
+            got[b] |= {bounds[r][b][0] + t for t in row}
+    for b in range(B):
+        assert sorted(got[b]) == _python_topk(full[b], k), b
