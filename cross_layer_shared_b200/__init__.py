@@ -52,6 +52,11 @@ SIGNATURES = {
                                _I),
     "sa_block_union_prefill_noalloc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P],
                                        _I),
+    "sa_sparse_decode_attn_partial": ([_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _F, _P, _P, _P, _SZ,
+                                       _P], _I),
+    "sa_cp_select_workspace_size": ([_I, _I, _I], _SZ),
+    "sa_cp_select": ([_P, _P, _I64, _I, _I, _I, _I, _P, _P, _SZ, _P], _I),
+    "sa_combine_partials": ([_P, _I64, _P, _I64, _I, _I64, _I, _P, _I, _P], _I),
 }
 
 
@@ -243,6 +248,80 @@ def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, o
     _check(lib().sa_sparse_decode_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), _ptr(idx), L, B,
                                        n_tokens, Hq, Hkv, d, k, float(scale), _ptr(O), code, _ptr(ws), ws.numel(),
                                        _stream(stream)))
+    return O
+
+
+def sparse_decode_attn_partial(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, O_part=None, ml=None,
+                                ws=None, stream=None):
+    """sparse_decode_attn left unnormalised: O_part fp32 [L, B, Hq, d] and ml
+    fp32 [L, B, Hq, 2], (m, l) with m a reference logit in log2 units (within
+    8 of the row's max) and l the sum of 2^(logit - m); O_part / l is the
+    output."""
+    L, B, Hq, d = Q.shape
+    k = idx.shape[1]
+    n_tokens = K.numel() // (Hkv * d)
+    _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
+    _out(idx, (B, k), (torch.int32,), "idx")
+    _seqs(seq_off, seq_len, B)
+    if O_part is None:
+        O_part = torch.empty((L, B, Hq, d), dtype=torch.float32, device=Q.device)
+    if ml is None:
+        ml = torch.empty((L, B, Hq, 2), dtype=torch.float32, device=Q.device)
+    _out(O_part, (L, B, Hq, d), (torch.float32,), "O_part")
+    _out(ml, (L, B, Hq, 2), (torch.float32,), "ml")
+    if ws is None:
+        ws = workspace(sparse_decode_attn_workspace_size(L, B, Hq, Hkv, d, k), Q.device)
+    _ws(ws)
+    _check(lib().sa_sparse_decode_attn_partial(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), _ptr(idx),
+                                               L, B, n_tokens, Hq, Hkv, d, k, float(scale), _ptr(O_part), _ptr(ml),
+                                               _ptr(ws), ws.numel(), _stream(stream)))
+    return O_part, ml
+
+
+def cp_select_workspace_size(N, B, k) -> int:
+    return int(lib().sa_cp_select_workspace_size(N, B, k))
+
+
+def cp_select(cand_scores, cand_idx, rank: int, local_idx=None, ws=None, stream=None) -> torch.Tensor:
+    """Global top-k of N ranks' candidates, as `rank`'s local indices [B, k].
+
+    cand_scores fp32 / cand_idx int32, each [N, B, k] or a view of one
+    all-gathered int32 buffer [N, 2, B, k] (scores bit-cast in [:, 0])."""
+    N, B, k = cand_idx.shape
+    if not (cand_scores.is_cuda and cand_idx.is_cuda and cand_scores.dtype == torch.float32
+            and cand_idx.dtype == torch.int32 and tuple(cand_scores.shape) == (N, B, k)):
+        raise ValueError("cand_scores fp32 and cand_idx int32 must be CUDA tensors of one shape [N, B, k]")
+    stride = cand_idx.stride(0) if N > 1 else B * k
+    if (cand_scores.stride(0) != stride and N > 1) or cand_idx.stride()[1:] != (k, 1) \
+            or cand_scores.stride()[1:] != (k, 1):
+        raise ValueError("cand_scores and cand_idx must be [B, k] blocks of one rank stride")
+    if local_idx is None:
+        local_idx = torch.empty((B, k), dtype=torch.int32, device=cand_idx.device)
+    _out(local_idx, (B, k), (torch.int32,), "local_idx")
+    if ws is None:
+        ws = workspace(cp_select_workspace_size(N, B, k), cand_idx.device)
+    _ws(ws)
+    _check(lib().sa_cp_select(_ptr(cand_scores), _ptr(cand_idx), stride, N, B, k, int(rank), _ptr(local_idx),
+                              _ptr(ws), ws.numel(), _stream(stream)))
+    return local_idx
+
+
+def combine_partials(O_part, ml, O=None, out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    """Log-sum-exp merge of P partials: O_part fp32 [P, rows, d], ml fp32
+    [P, rows, 2] (each part contiguous; the parts may sit at any common
+    stride, e.g. views of one all-gathered buffer).  Returns O [rows, d]."""
+    P, rows, d = O_part.shape
+    if not (O_part.is_cuda and ml.is_cuda and O_part.dtype == torch.float32 and ml.dtype == torch.float32
+            and tuple(ml.shape) == (P, rows, 2)):
+        raise ValueError("O_part [P, rows, d] and ml [P, rows, 2] must be fp32 CUDA tensors")
+    if O_part.stride()[1:] != (d, 1) or ml.stride()[1:] != (2, 1):
+        raise ValueError("each part of O_part and ml must be contiguous")
+    if O is None:
+        O = torch.empty((rows, d), dtype=out_dtype, device=O_part.device)
+    _out(O, (rows, d), (torch.bfloat16, torch.float32), "O")
+    code = SA_F32 if O.dtype == torch.float32 else SA_BF16
+    _check(lib().sa_combine_partials(_ptr(O_part), O_part.stride(0), _ptr(ml), ml.stride(0), P, rows, d, _ptr(O),
+                                     code, _stream(stream)))
     return O
 
 

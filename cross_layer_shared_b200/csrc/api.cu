@@ -19,6 +19,7 @@
 #include "sm100.cuh"
 #include "indexer.cuh"
 #include "route_attn.cuh"
+#include "cp.cuh"
 #include "status.cuh"
 #include "topk.cuh"
 #include "union.cuh"
@@ -450,8 +451,10 @@ size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int
 static sa_status run_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
                                  const int32_t* seq_len, const int32_t* idx, int L_g, int B, int64_t n_tokens, int Hq,
                                  int Hkv, int d, int k, float scale, void* O, sa_dtype out_dtype, void* ws,
-                                 size_t ws_bytes, cudaStream_t stream) {
-  const char* who = "sa_sparse_decode_attn";
+                                 size_t ws_bytes, cudaStream_t stream, float* ml = nullptr) {
+  const char* who = ml ? "sa_sparse_decode_attn_partial" : "sa_sparse_decode_attn";
+  if (ml && (out_dtype != SA_F32 || !aligned(ml, 8)))
+    return fail(SA_ERR_INVALID_ARG, "%s: partial outputs are fp32 and ml 8-byte aligned", who);
   if (L_g < 1 || B < 1 || Hq < 1 || Hkv < 1 || k < 1)
     return fail(SA_ERR_INVALID_ARG, "%s: L_g, B, Hq, Hkv, k must be >= 1", who);
   if (d != 128) return fail(SA_ERR_UNSUPPORTED, "%s: d=%d (only 128 is built)", who, d);
@@ -489,6 +492,7 @@ static sa_status run_decode_attn(const void* Q, const void* K, const void* V, co
   a.scale_log2 = scale * 1.4426950408889634f;
   a.O = O;
   a.out_f32 = out_dtype == SA_F32;
+  a.ml = reinterpret_cast<float2*>(ml);
   a.status = status_of(ws);
   cudaError_t e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, stream);
   if (e != cudaSuccess) return cuda_fail("sa_sparse_decode_attn launch", e);
@@ -569,6 +573,87 @@ sa_status sa_indexer_layer_attn(const void* Q, const void* K, const void* V, con
   }
   const cudaError_t e = sa::launch_indexer_layer_attn(a, tm_k, tm_v, tm_q, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail("sa_indexer_layer_attn launch", e);
+  return SA_OK;
+}
+
+sa_status sa_sparse_decode_attn_partial(const void* Q, const void* K, const void* V, const int64_t* seq_off,
+                                        const int32_t* seq_len, const int32_t* idx, int L_g, int B, int64_t n_tokens,
+                                        int Hq, int Hkv, int d, int k, float scale, float* O_part, float* ml,
+                                        void* ws, size_t ws_bytes, void* stream) {
+  if (!ml) return fail(SA_ERR_INVALID_ARG, "sa_sparse_decode_attn_partial: NULL ml");
+  return run_decode_attn(Q, K, V, seq_off, seq_len, idx, L_g, B, n_tokens, Hq, Hkv, d, k, scale, O_part, SA_F32, ws,
+                         ws_bytes, (cudaStream_t)stream, ml);
+}
+
+// ---------------------------------------------------------------- context-parallel decode
+namespace {
+struct CpSelectLayout {
+  size_t rows, n_valid, sel, topk, total;  // byte offsets after the header, then the total
+};
+CpSelectLayout cp_select_layout(int N, int B, int k) {
+  CpSelectLayout l{};
+  const size_t n = (size_t)N * k;
+  l.rows = 0;
+  l.n_valid = l.rows + round_up(4 * (size_t)B * n, 256);
+  l.sel = l.n_valid + round_up(4 * (size_t)B, 256);
+  l.topk = l.sel + round_up(4 * (size_t)B * k, 256);
+  const size_t t = sa::topk_use_split(B, (int)n, num_sms()) ? sa::topk_split_ws_bytes(B, (int)n, num_sms()) : 0;
+  l.total = SA_WS_HEADER_BYTES + l.topk + round_up(t, 256);
+  return l;
+}
+}  // namespace
+
+size_t sa_cp_select_workspace_size(int N, int B, int k) {
+  if (N < 1 || B < 1 || k < 1 || (int64_t)N * k > INT32_MAX) return SA_WS_HEADER_BYTES;
+  return cp_select_layout(N, B, k).total;
+}
+
+sa_status sa_cp_select(const float* cand_scores, const int32_t* cand_idx, int64_t cand_stride, int N, int B, int k,
+                       int rank, int32_t* local_idx, void* ws, size_t ws_bytes, void* stream) {
+  const char* who = "sa_cp_select";
+  if (N < 1 || B < 1 || k < 1) return fail(SA_ERR_INVALID_ARG, "%s: N, B, k must be >= 1", who);
+  if ((int64_t)N * k > INT32_MAX) return fail(SA_ERR_INVALID_ARG, "%s: N*k above 2^31 - 1", who);
+  if (rank < 0 || rank >= N) return fail(SA_ERR_INVALID_ARG, "%s: rank=%d outside [0, %d)", who, rank, N);
+  if (!cand_scores || !cand_idx || !local_idx) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (N > 1 && cand_stride < (int64_t)B * k)
+    return fail(SA_ERR_INVALID_ARG, "%s: cand_stride=%lld below B*k", who, (long long)cand_stride);
+  sa_status st = check_ws(ws, ws_bytes, sa_cp_select_workspace_size(N, B, k), who);
+  if (st != SA_OK) return st;
+  const CpSelectLayout l = cp_select_layout(N, B, k);
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
+  float* rows = reinterpret_cast<float*>(base + l.rows);
+  int32_t* n_valid = reinterpret_cast<int32_t*>(base + l.n_valid);
+  int32_t* sel = reinterpret_cast<int32_t*>(base + l.sel);
+  const cudaStream_t s = (cudaStream_t)stream;
+  const int n = N * k;
+  cudaError_t e = sa::launch_cp_gather(cand_scores, cand_idx, cand_stride, N, B, k, rows, n_valid, s);
+  if (e != cudaSuccess) return cuda_fail("sa_cp_select gather launch", e);
+  if (sa::topk_use_split(B, n, num_sms()))
+    e = sa::launch_topk_split(rows, n, n_valid, B, n, k, sel, nullptr, status_of(ws), base + l.topk, num_sms(), s);
+  else
+    e = sa::launch_topk_rows(rows, n, n_valid, B, n, k, sel, nullptr, status_of(ws), s);
+  if (e != cudaSuccess) return cuda_fail("sa_cp_select top-k launch", e);
+  e = sa::launch_cp_local(sel, cand_idx, cand_stride, B, k, rank, local_idx, s);
+  if (e != cudaSuccess) return cuda_fail("sa_cp_select local launch", e);
+  return SA_OK;
+}
+
+sa_status sa_combine_partials(const float* O_part, int64_t o_stride, const float* ml, int64_t ml_stride, int P,
+                              int64_t rows, int d, void* O, sa_dtype out_dtype, void* stream) {
+  const char* who = "sa_combine_partials";
+  if (P < 1 || rows < 0) return fail(SA_ERR_INVALID_ARG, "%s: need P >= 1, rows >= 0", who);
+  if (d != 128) return fail(SA_ERR_UNSUPPORTED, "%s: d=%d (only 128 is built)", who, d);
+  if (out_dtype != SA_BF16 && out_dtype != SA_F32) return fail(SA_ERR_INVALID_ARG, "%s: bad out_dtype", who);
+  if (rows == 0) return SA_OK;
+  if (!O_part || !ml || !O) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned(O_part, 16) || !aligned(ml, 8) || !aligned(O, 16))
+    return fail(SA_ERR_INVALID_ARG, "%s: O_part and O must be 16-byte aligned, ml 8-byte aligned", who);
+  if (P > 1 && (o_stride < rows * d || o_stride % 4 != 0 || ml_stride < 2 * rows || ml_stride % 2 != 0))
+    return fail(SA_ERR_INVALID_ARG, "%s: need o_stride >= rows*d, a multiple of 4, and ml_stride >= 2*rows, even",
+                who);
+  cudaError_t e = sa::launch_combine_partials(O_part, o_stride, reinterpret_cast<const float2*>(ml), ml_stride / 2, P,
+                                              rows, O, out_dtype == SA_F32, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail("sa_combine_partials launch", e);
   return SA_OK;
 }
 

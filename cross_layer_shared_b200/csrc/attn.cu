@@ -571,7 +571,9 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   };
   if (a.n_split == 1) {
     if (warp_active && have_o) {
-      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+      // partial output: the rows as they are, with (m, l) beside them
+      const float inv = a.ml != nullptr ? 1.f : (l_row > 0.f ? 1.f / l_row : 0.f);
+      if (a.ml != nullptr && half == 0 && me.valid) a.ml[me.qoff / kD] = make_float2(m_row, l_row);
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
         float f[32];
@@ -664,7 +666,8 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
           L += wt[t] * mls[t].y;
         }
       }
-      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float inv = a.ml != nullptr ? 1.f : (L > 0.f ? 1.f / L : 0.f);
+      if (a.ml != nullptr && rank == 0 && half == 0) a.ml[me.qoff / kD] = make_float2(M, L);
       // the slice's chunks, split between the row's two threads
       const int per = cw / 2 > 0 ? cw / 2 : 1;
       for (int ci = half * per; ci < (half + 1) * per && ci < cw; ++ci) {

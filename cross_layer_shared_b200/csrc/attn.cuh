@@ -42,6 +42,10 @@ struct AttnArgs {
   float scale_log2;    // softmax scale * log2(e)
   void* O;
   int out_f32;
+  // partial output (context-parallel decode): when set, O (fp32) receives each
+  // row's output before normalisation, relative to the row's reference logit
+  // m (log2 units, within 8 of the max), and ml the row's (m, sum of weights)
+  float2* ml = nullptr;
   DeviceStatus* status;
 };
 

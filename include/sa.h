@@ -336,6 +336,74 @@ sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const int32_t* q_po
                                          int d, int k, int block, float scale, int32_t* kv_indptr,
                                          int32_t* kv_indices, void* O, sa_dtype out_dtype, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Context-parallel decode: one sequence's context sharded over N ranks
+ * [CLSA news article, section "Ce que cela signifie pour l'inference sur
+ * longs contextes": how the method behaves past 128K tokens is left open.
+ * The pages have no sharding scheme.  This one is the plainest that gives
+ * the same result as one GPU.]
+ *
+ * Rank r holds a contiguous slice of every sequence (tokens [lo_r, hi_r),
+ * slices in rank order, possibly empty) as its own packed caches.  A step:
+ *   1. sa_index_score + sa_topk (with top_scores) over the local slice;
+ *   2. all ranks' (top_scores, idx) gathered, rank-major, on every rank;
+ *   3. sa_cp_select: the global top-k of those candidates, mapped back to
+ *      this rank's local indices;
+ *   4. sa_sparse_decode_attn_partial over the local selected rows;
+ *   5. all ranks' (O_part, ml) gathered; sa_combine_partials.
+ * A token of the global top-k is in its slice's top-k.  Candidate position
+ * order (rank-major, then ascending local index) is ascending global
+ * index, so the tie rule (lower index first) carries over.  Softmax over a
+ * union of disjoint key sets is the log-sum-exp merge of the parts.  The
+ * step therefore selects the same index as sa_decode_step on one GPU, and
+ * attends over it.
+ * ---------------------------------------------------------------------- */
+
+/* The sparse decode attention of one rank, left unnormalised.  Arguments as
+ * sa_sparse_decode_attn.  For each row (l, b, h), with a reference m (log2
+ * units) at most 8 below max_t z_t * log2(e) over its valid selected keys:
+ *   O_part[row, :] = sum_t 2^(z_t*log2(e) - m) V_t    fp32 [L_g, B, Hq, d]
+ *   ml[row]        = (m, sum_t 2^(z_t*log2(e) - m))   fp32 pairs [L_g, B, Hq]
+ * so O_part / l is the row's output and m + log2(l) its log-sum-exp in log2
+ * units; m itself is whatever reference the kernel kept.  A row with no
+ * valid index gets l = 0 and O_part = 0.  ml must be 8-byte aligned.
+ * Workspace: sa_sparse_decode_attn_workspace_size. */
+sa_status sa_sparse_decode_attn_partial(const void* Q, const void* K, const void* V,
+                                        const int64_t* seq_off, const int32_t* seq_len,
+                                        const int32_t* idx, int L_g, int B, int64_t n_tokens, int Hq,
+                                        int Hkv, int d, int k, float scale, float* O_part, float* ml,
+                                        void* ws, size_t ws_bytes, void* stream);
+
+/* Global top-k over the gathered candidates.
+ *   cand_scores, cand_idx  rank r's top_scores (fp32 [B, k]) and idx (int32
+ *               [B, k], < 0 = padding) from sa_topk over its slice, at
+ *               element offset r * cand_stride of each (so one all-gathered
+ *               buffer of [N][scores | idx] blocks serves both, with
+ *               cand_idx = cand_scores + B*k and cand_stride = 2*B*k)
+ *   local_idx   int32 [B, k] out: the global top-k entries in rank `rank`'s
+ *               slice, as its local indices, ascending, then -1
+ * The selection is sa_topk's (min(k, candidates) largest, ties to the lower
+ * position) over the N*k candidates of each sequence, padding scoring -inf.
+ * 0 <= rank < N; N*k <= 2^31 - 1; cand_stride >= B*k when N > 1. */
+size_t sa_cp_select_workspace_size(int N, int B, int k);
+sa_status sa_cp_select(const float* cand_scores, const int32_t* cand_idx, int64_t cand_stride, int N,
+                       int B, int k, int rank, int32_t* local_idx, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* The log-sum-exp merge of P partial results of the same rows:
+ *   O[row, :] = sum_p 2^(m_p - M) O_part_p[row, :] / sum_p 2^(m_p - M) l_p,
+ * with M the largest m_p among parts with l_p > 0; O = 0 where every l_p = 0.
+ *   O_part_p  fp32 [rows, d] at O_part + p * o_stride (floats)
+ *   (m_p, l_p) fp32 pairs [rows] at ml + p * ml_stride (floats)
+ *   O         [rows, d] in out_dtype (bf16 or fp32)
+ * With P > 1: o_stride >= rows*d and a multiple of 4, ml_stride >= 2*rows
+ * and even (one all-gathered buffer of [P][O_part | ml] blocks: ml = O_part
+ * + rows*d, both strides rows*(d+2) rounded up to a multiple of 4).
+ * Supported: d = 128, 1 <= P.  rows = 0
+ * returns SA_OK without a launch.  No workspace. */
+sa_status sa_combine_partials(const float* O_part, int64_t o_stride, const float* ml, int64_t ml_stride,
+                              int P, int64_t rows, int d, void* O, sa_dtype out_dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -129,3 +129,41 @@ def test_indexer_layer_attn_rejects_bad_requests(lib):
     assert call(ld=100) == sa.SA_ERR_INVALID_ARG and b"ld" in lib.sa_last_error()
     assert call(ws_bytes=1024) == sa.SA_ERR_WORKSPACE
     assert call(Q=ctypes.c_void_p(0x7F0000001008)) == sa.SA_ERR_INVALID_ARG
+
+
+def test_context_parallel_entry_points_reject_bad_requests(lib):
+    B, k = 4, 2048
+    need = lib.sa_cp_select_workspace_size(8, B, k)
+    # the gathered rows of scores, their counts and the selected positions
+    assert need >= sa.WS_HEADER_BYTES + 4 * B * 8 * k + 4 * B + 4 * B * k
+
+    def select(N=2, rank=0, stride=B * k, ws_bytes=1 << 30):
+        return lib.sa_cp_select(FAKE, FAKE, stride, N, B, k, rank, FAKE, FAKE_WS, ws_bytes, None)
+
+    assert select(rank=2) == sa.SA_ERR_INVALID_ARG and b"rank" in lib.sa_last_error()
+    assert select(rank=-1) == sa.SA_ERR_INVALID_ARG
+    assert select(N=0) == sa.SA_ERR_INVALID_ARG
+    assert select(stride=B * k - 1) == sa.SA_ERR_INVALID_ARG and b"cand_stride" in lib.sa_last_error()
+    assert select(ws_bytes=1024) == sa.SA_ERR_WORKSPACE
+
+    rows = 96
+
+    def combine(P=2, d=128, o_stride=rows * 130, ml_stride=rows * 130, ml=FAKE, dtype=sa.SA_BF16, n=rows):
+        return lib.sa_combine_partials(FAKE, o_stride, ml, ml_stride, P, n, d, FAKE, dtype, None)
+
+    assert combine(d=64) == sa.SA_ERR_UNSUPPORTED
+    assert combine(P=0) == sa.SA_ERR_INVALID_ARG
+    assert combine(dtype=7) == sa.SA_ERR_INVALID_ARG
+    assert combine(o_stride=rows * 128 - 4) == sa.SA_ERR_INVALID_ARG
+    assert combine(o_stride=rows * 130 + 2) == sa.SA_ERR_INVALID_ARG
+    assert combine(ml_stride=rows * 130 + 1) == sa.SA_ERR_INVALID_ARG
+    assert combine(ml=ctypes.c_void_p(0x7F0000001004)) == sa.SA_ERR_INVALID_ARG
+    assert combine(n=0) == sa.SA_OK  # nothing to merge: no launch
+
+    def partial(ml=FAKE, d=128):
+        return lib.sa_sparse_decode_attn_partial(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 8192, 32, 8, d, 64, 0.088,
+                                                 FAKE, ml, FAKE_WS, 1 << 30, None)
+
+    assert partial(ml=None) == sa.SA_ERR_INVALID_ARG and b"ml" in lib.sa_last_error()
+    assert partial(ml=ctypes.c_void_p(0x7F0000001004)) == sa.SA_ERR_INVALID_ARG
+    assert partial(d=64) == sa.SA_ERR_UNSUPPORTED
