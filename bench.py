@@ -58,6 +58,8 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--out-f32", action="store_true", help="fp32 attention output instead of bf16")
+    p.add_argument("--cp-ranks", type=int, default=8,
+                   help="ranks of the emulated context-parallel step (single-group workloads, N=1; 0 = skip)")
     return p.parse_args()
 
 
@@ -533,6 +535,85 @@ def workload_config(cfg, args):
 
 
 # ---------------------------------------------------------------- our arm
+def context_parallel_section(cfg, st, N, cap, dev, reps: int = 16, iters: int = 20) -> dict:
+    """Per-rank device time of a context-parallel step of `cfg`'s one layer
+    group with N ranks, all emulated on this GPU (phases of every rank run in
+    turn; each rank's chain then replayed from a CUDA graph on the gathered
+    buffers of that step)."""
+    import torch
+
+    import cross_layer_shared_b200 as sa
+    from cross_layer_shared_b200 import cp
+
+    lens = [int(x) for x in cfg.seq_lens]
+    bnd = cp.shard_bounds(lens, N)
+    KI, K, V = st["KI"][0].view(-1, cfg.d_I), st["K"][0], st["V"][0]
+    qI, w, Q = st["qI"][0], st["w"][0], st["wl"]["Q"]
+    ranks = []
+    for r in range(N):
+        lo, hi = bnd[r, :, 0], bnd[r, :, 1]
+        ranks.append(cp.CPRank(N, r, cp.shard_cache(KI, lens, 1, cfg.d_I, lo, hi),
+                               cp.shard_cache(K, lens, cfg.Hkv, cfg.d, lo, hi).view(-1),
+                               cp.shard_cache(V, lens, cfg.Hkv, cfg.d, lo, hi).view(-1), hi - lo, cfg.k, cfg.H_I,
+                               cfg.d_I, cfg.Hq, cfg.Hkv, cfg.d, cfg.L, cfg.scale))
+    O_cp, local = cp.emulate_step(ranks, qI, w, Q)
+    # the one-device step on the same inputs, for the record
+    scores = sa.index_score(qI, w, KI, st["wl"]["seq_off"], st["wl"]["seq_len"], cfg.S_max)
+    idx = sa.topk(scores, st["wl"]["seq_len"], cfg.S_max, cfg.k)
+    O1 = sa.sparse_decode_attn(Q, K, V, st["wl"]["seq_off"], st["wl"]["seq_len"], idx, cfg.Hkv, cfg.scale)
+    same_idx = True
+    idx_h = idx.cpu().numpy()
+    for b in range(len(lens)):
+        got = sorted(int(bnd[r, b, 0] + t) for r in range(N) for t in local[r][b].cpu().numpy() if t >= 0)
+        same_idx &= got == [int(t) for t in idx_h[b] if t >= 0]
+    max_abs = (O_cp.float() - O1.float()).abs().max().item()
+    for r in ranks:
+        for ws in (r.ws_index, r.ws_topk, r.ws_sel, r.ws_attn):
+            code, det = sa.read_status(ws)
+            if code != 0:
+                raise RuntimeError(f"context-parallel device status {code} {det}")
+    cand = torch.stack([r.cand for r in ranks])
+    parts = torch.stack([r.part for r in ranks])
+    O = torch.empty_like(O1)
+
+    def graph_ms(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (iters * reps)
+
+    def chain(r):
+        r.candidates(qI, w)
+        r.select(cand)
+        r.partial(Q)
+        r.combine(parts, O)
+
+    per_rank = [graph_ms(lambda r=r: chain(r)) for r in ranks]
+    slow = ranks[max(range(N), key=lambda i: per_rank[i])]
+    phases = {"candidates": graph_ms(lambda: slow.candidates(qI, w)), "select": graph_ms(lambda: slow.select(cand)),
+              "partial_attention": graph_ms(lambda: slow.partial(Q)),
+              "combine": graph_ms(lambda: slow.combine(parts, O))}
+    cand_b, part_b = ranks[0].cand.numel() * 4, ranks[0].part.numel() * 4
+    return {"ranks": N, "context_per_rank": [int(x) for x in (bnd[:, :, 1] - bnd[:, :, 0]).max(1)],
+            "ms_per_rank_step_max": max(per_rank), "ms_per_rank_step": per_rank, "phases_ms_slowest_rank": phases,
+            "selected_per_rank": [int((x >= 0).sum().item()) for x in local],
+            "allgather_bytes_per_rank": {"candidates": cand_b, "partials": part_b},
+            "allgather_bytes_received_per_rank": (N - 1) * (cand_b + part_b),
+            "launches_per_rank_step": 7, "same_index_as_one_device": bool(same_idx),
+            "max_abs_vs_one_device": max_abs,
+            "note": "every rank emulated on one GPU; the two all-gathers are not timed (one GPU): add their "
+                    "NVLink time for the received bytes; one group of all layers shares the index"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -719,6 +800,16 @@ def run_ours(args):
                          "is the routing score, its top-k is the index of layers 1..L-1"}
         del g_route
 
+    # ---- context-parallel decode, every rank emulated on this GPU: each
+    # sequence's context sharded over cp_ranks ranks; a rank's step is its
+    # indexer + top-k over its slice, the global selection over all ranks'
+    # candidates, attention over its share, and the merge of all partials.
+    # The two all-gathers between the phases are not run (one GPU): their
+    # bytes per rank are reported instead ----
+    cpar = None
+    if world == 1 and len(cfg.groups) == 1 and args.cp_ranks > 1:
+        cpar = context_parallel_section(cfg, sets[0], args.cp_ranks, cap, dev)
+
     # ---- per-kernel device time: each graph holds REP back-to-back launches
     # (alternating input sets, so consecutive launches read different data),
     # which keeps the host's replay cost out of the figure ----
@@ -879,6 +970,7 @@ def run_ours(args):
                                           "attention launch per layer (no fusion of the group's layers), as a "
                                           "decoder that computes layer l+1's queries from layer l runs it"},
         "attn_route": route,
+        "context_parallel": cpar,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "per step: one pinned host -> device copy of that step's queries, indexer queries and "

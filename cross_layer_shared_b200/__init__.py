@@ -52,10 +52,10 @@ SIGNATURES = {
                                _I),
     "sa_block_union_prefill_noalloc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P],
                                        _I),
-    "sa_sparse_decode_attn_partial": ([_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _F, _P, _P, _P, _SZ,
-                                       _P], _I),
+    "sa_sparse_decode_attn_partial": ([_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _P, _F, _P, _P, _P,
+                                       _SZ, _P], _I),
     "sa_cp_select_workspace_size": ([_I, _I, _I], _SZ),
-    "sa_cp_select": ([_P, _P, _I64, _I, _I, _I, _I, _P, _P, _SZ, _P], _I),
+    "sa_cp_select": ([_P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "sa_combine_partials": ([_P, _I64, _P, _I64, _I, _I64, _I, _P, _I, _P], _I),
 }
 
@@ -252,16 +252,19 @@ def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, o
 
 
 def sparse_decode_attn_partial(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float, O_part=None, ml=None,
-                                ws=None, stream=None):
+                                idx_count=None, ws=None, stream=None):
     """sparse_decode_attn left unnormalised: O_part fp32 [L, B, Hq, d] and ml
     fp32 [L, B, Hq, 2], (m, l) with m a reference logit in log2 units (within
     8 of the row's max) and l the sum of 2^(logit - m); O_part / l is the
-    output."""
+    output.  idx_count int32 [B] (optional): only the first idx_count[b]
+    entries of idx row b are real."""
     L, B, Hq, d = Q.shape
     k = idx.shape[1]
     n_tokens = K.numel() // (Hkv * d)
     _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
     _out(idx, (B, k), (torch.int32,), "idx")
+    if idx_count is not None:
+        _out(idx_count, (B,), (torch.int32,), "idx_count")
     _seqs(seq_off, seq_len, B)
     if O_part is None:
         O_part = torch.empty((L, B, Hq, d), dtype=torch.float32, device=Q.device)
@@ -273,8 +276,8 @@ def sparse_decode_attn_partial(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: 
         ws = workspace(sparse_decode_attn_workspace_size(L, B, Hq, Hkv, d, k), Q.device)
     _ws(ws)
     _check(lib().sa_sparse_decode_attn_partial(_ptr(Q), _ptr(K), _ptr(V), _ptr(seq_off), _ptr(seq_len), _ptr(idx),
-                                               L, B, n_tokens, Hq, Hkv, d, k, float(scale), _ptr(O_part), _ptr(ml),
-                                               _ptr(ws), ws.numel(), _stream(stream)))
+                                               L, B, n_tokens, Hq, Hkv, d, k, _ptr(idx_count), float(scale),
+                                               _ptr(O_part), _ptr(ml), _ptr(ws), ws.numel(), _stream(stream)))
     return O_part, ml
 
 
@@ -282,8 +285,10 @@ def cp_select_workspace_size(N, B, k) -> int:
     return int(lib().sa_cp_select_workspace_size(N, B, k))
 
 
-def cp_select(cand_scores, cand_idx, rank: int, local_idx=None, ws=None, stream=None) -> torch.Tensor:
-    """Global top-k of N ranks' candidates, as `rank`'s local indices [B, k].
+def cp_select(cand_scores, cand_idx, rank: int, local_idx=None, local_count=None, ws=None,
+              stream=None) -> torch.Tensor:
+    """Global top-k of N ranks' candidates, as `rank`'s local indices [B, k]
+    (and, into local_count int32 [B] if given, how many there are).
 
     cand_scores fp32 / cand_idx int32, each [N, B, k] or a view of one
     all-gathered int32 buffer [N, 2, B, k] (scores bit-cast in [:, 0])."""
@@ -298,11 +303,13 @@ def cp_select(cand_scores, cand_idx, rank: int, local_idx=None, ws=None, stream=
     if local_idx is None:
         local_idx = torch.empty((B, k), dtype=torch.int32, device=cand_idx.device)
     _out(local_idx, (B, k), (torch.int32,), "local_idx")
+    if local_count is not None:
+        _out(local_count, (B,), (torch.int32,), "local_count")
     if ws is None:
         ws = workspace(cp_select_workspace_size(N, B, k), cand_idx.device)
     _ws(ws)
     _check(lib().sa_cp_select(_ptr(cand_scores), _ptr(cand_idx), stride, N, B, k, int(rank), _ptr(local_idx),
-                              _ptr(ws), ws.numel(), _stream(stream)))
+                              _ptr(local_count), _ptr(ws), ws.numel(), _stream(stream)))
     return local_idx
 
 

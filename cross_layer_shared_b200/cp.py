@@ -109,6 +109,7 @@ class CPRank:
         self.part_floats = part_floats(self.rows, d)
         self.part = torch.empty(self.part_floats, dtype=torch.float32, device=dev)
         self.local_idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+        self.local_count = torch.empty(B, dtype=torch.int32, device=dev)
         self.ws_index = workspace(int(lib().sa_index_score_workspace_size(B)), dev)
         self.ws_topk = workspace(int(lib().sa_topk_workspace_size(B, self.S_max, k)), dev)
         self.ws_sel = workspace(cp_select_workspace_size(N, B, k), dev)
@@ -127,14 +128,16 @@ class CPRank:
     def select(self, gathered: torch.Tensor, stream=None) -> torch.Tensor:
         """gathered int32 [N, 2, B, k] -> this rank's share of the global top-k."""
         scores, idx = cand_views(gathered)
-        return cp_select(scores, idx, self.rank, local_idx=self.local_idx, ws=self.ws_sel, stream=stream)
+        return cp_select(scores, idx, self.rank, local_idx=self.local_idx, local_count=self.local_count,
+                         ws=self.ws_sel, stream=stream)
 
     def partial(self, Q: torch.Tensor, stream=None) -> torch.Tensor:
         """Unnormalised attention over the local selected rows, into self.part."""
         o, ml = part_views(self.part, self.rows, self.d)
         sparse_decode_attn_partial(Q, self.K, self.V, self.seq_off, self.seq_len, self.local_idx, self.Hkv,
                                    self.scale, O_part=o.view(self.L_g, self.B, self.Hq, self.d),
-                                   ml=ml.view(self.L_g, self.B, self.Hq, 2), ws=self.ws_attn, stream=stream)
+                                   ml=ml.view(self.L_g, self.B, self.Hq, 2), idx_count=self.local_count,
+                                   ws=self.ws_attn, stream=stream)
         return self.part
 
     def combine(self, gathered: torch.Tensor, O: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16,
@@ -182,3 +185,47 @@ def emulate_step(ranks: Sequence[CPRank], qI: torch.Tensor, w: torch.Tensor, Q: 
         r.select(cand, stream)
     parts = torch.stack([r.partial(Q, stream) for r in ranks])
     return ranks[0].combine(parts, None, out_dtype, stream), [r.local_idx for r in ranks]
+
+
+def main(argv=None) -> int:
+    """Run emulated context-parallel decode steps on one GPU (seeded random
+    inputs of the given shape; defaults: 4 sequences of 128K tokens, a 16x128
+    indexer, k = 2048, one group of 24 layers with 32q/8kv heads of 128)."""
+    import argparse
+    import math
+
+    p = argparse.ArgumentParser(prog="python -m cross_layer_shared_b200.cp")
+    p.add_argument("--ranks", type=int, default=8)
+    p.add_argument("--steps", type=int, default=2)
+    p.add_argument("--batch", type=int, default=4)
+    p.add_argument("--context", type=int, default=131072)
+    p.add_argument("--k", type=int, default=2048)
+    p.add_argument("--layers", type=int, default=24)
+    p.add_argument("--seed", type=int, default=1)
+    a = p.parse_args(argv)
+    H_I, d_I, Hq, Hkv, d = 16, 128, 32, 8, 128
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(a.seed)
+
+    def rnd(*shape, s=1.0):
+        return (torch.randn(*shape, device=dev, generator=g) * s).to(torch.bfloat16)
+
+    qI, w = rnd(a.batch, H_I, d_I, s=0.25), torch.rand(a.batch, H_I, device=dev, generator=g)
+    Q = rnd(a.layers, a.batch, Hq, d)
+    bnd = shard_bounds([a.context] * a.batch, a.ranks)
+    ranks = []
+    for r in range(a.ranks):
+        n = [int(x) for x in bnd[r, :, 1] - bnd[r, :, 0]]
+        T = sum(n)
+        ranks.append(CPRank(a.ranks, r, rnd(T, d_I, s=0.25), rnd(T * Hkv * d), rnd(T * Hkv * d), n, a.k, H_I, d_I, Hq,
+                            Hkv, d, a.layers, 1 / math.sqrt(d)))
+    for _ in range(a.steps):
+        O, local = emulate_step(ranks, qI, w, Q)
+    torch.cuda.synchronize()
+    print(f"{a.steps} emulated steps over {a.ranks} ranks; selected per rank "
+          f"{[int((x >= 0).sum().item()) for x in local]}; |O| max {O.float().abs().max().item():.4f}")
+    return 0
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())

@@ -451,7 +451,8 @@ size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int
 static sa_status run_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,
                                  const int32_t* seq_len, const int32_t* idx, int L_g, int B, int64_t n_tokens, int Hq,
                                  int Hkv, int d, int k, float scale, void* O, sa_dtype out_dtype, void* ws,
-                                 size_t ws_bytes, cudaStream_t stream, float* ml = nullptr) {
+                                 size_t ws_bytes, cudaStream_t stream, float* ml = nullptr,
+                                 const int32_t* idx_count = nullptr) {
   const char* who = ml ? "sa_sparse_decode_attn_partial" : "sa_sparse_decode_attn";
   if (ml && (out_dtype != SA_F32 || !aligned(ml, 8)))
     return fail(SA_ERR_INVALID_ARG, "%s: partial outputs are fp32 and ml 8-byte aligned", who);
@@ -493,6 +494,7 @@ static sa_status run_decode_attn(const void* Q, const void* K, const void* V, co
   a.O = O;
   a.out_f32 = out_dtype == SA_F32;
   a.ml = reinterpret_cast<float2*>(ml);
+  a.idx_count = idx_count;
   a.status = status_of(ws);
   cudaError_t e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, stream);
   if (e != cudaSuccess) return cuda_fail("sa_sparse_decode_attn launch", e);
@@ -578,11 +580,11 @@ sa_status sa_indexer_layer_attn(const void* Q, const void* K, const void* V, con
 
 sa_status sa_sparse_decode_attn_partial(const void* Q, const void* K, const void* V, const int64_t* seq_off,
                                         const int32_t* seq_len, const int32_t* idx, int L_g, int B, int64_t n_tokens,
-                                        int Hq, int Hkv, int d, int k, float scale, float* O_part, float* ml,
-                                        void* ws, size_t ws_bytes, void* stream) {
+                                        int Hq, int Hkv, int d, int k, const int32_t* idx_count, float scale,
+                                        float* O_part, float* ml, void* ws, size_t ws_bytes, void* stream) {
   if (!ml) return fail(SA_ERR_INVALID_ARG, "sa_sparse_decode_attn_partial: NULL ml");
   return run_decode_attn(Q, K, V, seq_off, seq_len, idx, L_g, B, n_tokens, Hq, Hkv, d, k, scale, O_part, SA_F32, ws,
-                         ws_bytes, (cudaStream_t)stream, ml);
+                         ws_bytes, (cudaStream_t)stream, ml, idx_count);
 }
 
 // ---------------------------------------------------------------- context-parallel decode
@@ -609,7 +611,7 @@ size_t sa_cp_select_workspace_size(int N, int B, int k) {
 }
 
 sa_status sa_cp_select(const float* cand_scores, const int32_t* cand_idx, int64_t cand_stride, int N, int B, int k,
-                       int rank, int32_t* local_idx, void* ws, size_t ws_bytes, void* stream) {
+                       int rank, int32_t* local_idx, int32_t* local_count, void* ws, size_t ws_bytes, void* stream) {
   const char* who = "sa_cp_select";
   if (N < 1 || B < 1 || k < 1) return fail(SA_ERR_INVALID_ARG, "%s: N, B, k must be >= 1", who);
   if ((int64_t)N * k > INT32_MAX) return fail(SA_ERR_INVALID_ARG, "%s: N*k above 2^31 - 1", who);
@@ -633,7 +635,7 @@ sa_status sa_cp_select(const float* cand_scores, const int32_t* cand_idx, int64_
   else
     e = sa::launch_topk_rows(rows, n, n_valid, B, n, k, sel, nullptr, status_of(ws), s);
   if (e != cudaSuccess) return cuda_fail("sa_cp_select top-k launch", e);
-  e = sa::launch_cp_local(sel, cand_idx, cand_stride, B, k, rank, local_idx, s);
+  e = sa::launch_cp_local(sel, cand_idx, cand_stride, B, k, rank, local_idx, local_count, s);
   if (e != cudaSuccess) return cuda_fail("sa_cp_select local launch", e);
   return SA_OK;
 }

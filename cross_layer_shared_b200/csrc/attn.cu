@@ -255,14 +255,21 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     ks.len = a.seq_len[b];
     ks.base = 0;
     n_keys = a.k;
+    if (a.idx_count != nullptr) {
+      const int c = a.idx_count[b];
+      n_keys = c < 0 ? 0 : (c < a.k ? c : a.k);
+    }
   } else {
     ks.len = a.S;
     ks.base = a.kv_indptr[g];
     n_keys = (a.kv_indptr[g + 1] - ks.base) * a.block;
   }
-  // decode: the host's even split of k; prefill: the union's size is known
-  // only here, so its split is even over that size (whole 128-key tiles)
-  const int per = a.prefill ? ((n_keys + a.n_split - 1) / a.n_split + kKT - 1) / kKT * kKT : a.keys_per_split;
+  // decode: the host's even split of k; prefill, and decode with a count of
+  // real entries: the size is known only here, so the split is even over it
+  // (whole 128-key tiles)
+  const int per = (a.prefill || a.idx_count != nullptr)
+                      ? ((n_keys + a.n_split - 1) / a.n_split + kKT - 1) / kKT * kKT
+                      : a.keys_per_split;
   ks.kbeg = split * per;
   ks.kend = min(n_keys, ks.kbeg + per);
   const int nt = ks.kend > ks.kbeg ? (ks.kend - ks.kbeg + kKT - 1) / kKT : 0;

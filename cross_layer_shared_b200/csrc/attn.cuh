@@ -46,6 +46,9 @@ struct AttnArgs {
   // row's output before normalisation, relative to the row's reference logit
   // m (log2 units, within 8 of the max), and ml the row's (m, sum of weights)
   float2* ml = nullptr;
+  // decode, optional: idx_count[b] entries of idx row b are real, the rest
+  // padding; the key splits then cover only those entries
+  const int32_t* idx_count = nullptr;
   DeviceStatus* status;
 };
 

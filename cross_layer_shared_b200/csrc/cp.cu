@@ -38,26 +38,53 @@ __global__ void cp_gather_kernel(const float* __restrict__ cand_scores, const in
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) n_valid[b] = N * k;
 }
 
-// One warp per sequence: the selected candidate positions (ascending, -1
-// padded) that fall in this rank's block become its local indices, in order.
-__global__ void cp_local_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ cand_idx, int64_t stride,
-                                int B, int k, int rank, int32_t* __restrict__ local_idx) {
-  const int b = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (b >= B) return;
-  int n = 0;
-  for (int j0 = 0; j0 < k; j0 += 32) {
-    const int j = j0 + lane;
-    int v = -1;
-    if (j < k) {
-      const int p = sel[(int64_t)b * k + j];
-      if (p >= 0 && p / k == rank) v = cand_idx[rank * stride + (int64_t)b * k + p % k];
-    }
-    const uint32_t m = __ballot_sync(0xffffffffu, v >= 0);
-    if (v >= 0) local_idx[(int64_t)b * k + n + __popc(m & ((1u << lane) - 1u))] = v;
-    n += __popc(m);
+// One CTA per sequence: the selected candidate positions (ascending, -1
+// padded) that fall in this rank's block [rank*k, rank*k + k) form one run
+// of the selection; entry j of the run becomes local entry j - lo, where lo
+// counts the selected positions before the block.  The rank's padding
+// candidates (-1) sort last in its block, so its real entries lead the run:
+// local_idx gets them in order, then -1, and count[b] their number.
+__global__ void __launch_bounds__(256) cp_local_kernel(const int32_t* __restrict__ sel,
+                                                       const int32_t* __restrict__ cand_idx, int64_t stride, int k,
+                                                       int rank, int32_t* __restrict__ local_idx,
+                                                       int32_t* __restrict__ count) {
+  __shared__ int red[2][8];
+  const int b = blockIdx.x;
+  const int64_t blo = (int64_t)rank * k, bhi = blo + k;
+  const int32_t* srow = sel + (int64_t)b * k;
+  const int32_t* crow = cand_idx + rank * stride + (int64_t)b * k;
+  int before = 0, valid = 0;
+  for (int j = threadIdx.x; j < k; j += blockDim.x) {
+    const int p = __ldg(srow + j);
+    if (p >= 0 && p < blo) ++before;
+    if (p >= blo && p < bhi && __ldg(crow + (p - blo)) >= 0) ++valid;
   }
-  for (int j = n + lane; j < k; j += 32) local_idx[(int64_t)b * k + j] = -1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    valid += __shfl_xor_sync(0xffffffffu, valid, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = before;
+    red[1][threadIdx.x >> 5] = valid;
+  }
+  __syncthreads();
+  int lo = 0, n = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    lo += red[0][w];
+    n += red[1][w];
+  }
+  int32_t* out = local_idx + (int64_t)b * k;
+  for (int j = threadIdx.x; j < k; j += blockDim.x) {
+    const int p = __ldg(srow + j);
+    if (p >= blo && p < bhi) {
+      const int v = __ldg(crow + (p - blo));
+      if (v >= 0) out[j - lo] = v;
+    }
+    if (j >= n) out[j] = -1;
+  }
+  if (count != nullptr && threadIdx.x == 0) count[b] = n;
 }
 
 // One warp per row: o = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p; part p
@@ -113,8 +140,8 @@ cudaError_t launch_cp_gather(const float* cand_scores, const int32_t* cand_idx, 
 }
 
 cudaError_t launch_cp_local(const int32_t* sel, const int32_t* cand_idx, int64_t stride, int B, int k, int rank,
-                            int32_t* local_idx, cudaStream_t stream) {
-  cp_local_kernel<<<(B + 7) / 8, 256, 0, stream>>>(sel, cand_idx, stride, B, k, rank, local_idx);
+                            int32_t* local_idx, int32_t* count, cudaStream_t stream) {
+  cp_local_kernel<<<B, 256, 0, stream>>>(sel, cand_idx, stride, k, rank, local_idx, count);
   return cudaGetLastError();
 }
 

@@ -360,7 +360,11 @@ sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const int32_t* q_po
  * ---------------------------------------------------------------------- */
 
 /* The sparse decode attention of one rank, left unnormalised.  Arguments as
- * sa_sparse_decode_attn.  For each row (l, b, h), with a reference m (log2
+ * sa_sparse_decode_attn, plus idx_count (nullable, device int32 [B]): when
+ * set, only the first idx_count[b] entries of idx row b are read (the rest
+ * count as padding) and the keys are split over that many, so a rank whose
+ * share of the index is small runs on only that share.  For each row
+ * (l, b, h), with a reference m (log2
  * units) at most 8 below max_t z_t * log2(e) over its valid selected keys:
  *   O_part[row, :] = sum_t 2^(z_t*log2(e) - m) V_t    fp32 [L_g, B, Hq, d]
  *   ml[row]        = (m, sum_t 2^(z_t*log2(e) - m))   fp32 pairs [L_g, B, Hq]
@@ -371,8 +375,9 @@ sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const int32_t* q_po
 sa_status sa_sparse_decode_attn_partial(const void* Q, const void* K, const void* V,
                                         const int64_t* seq_off, const int32_t* seq_len,
                                         const int32_t* idx, int L_g, int B, int64_t n_tokens, int Hq,
-                                        int Hkv, int d, int k, float scale, float* O_part, float* ml,
-                                        void* ws, size_t ws_bytes, void* stream);
+                                        int Hkv, int d, int k, const int32_t* idx_count, float scale,
+                                        float* O_part, float* ml, void* ws, size_t ws_bytes,
+                                        void* stream);
 
 /* Global top-k over the gathered candidates.
  *   cand_scores, cand_idx  rank r's top_scores (fp32 [B, k]) and idx (int32
@@ -382,13 +387,15 @@ sa_status sa_sparse_decode_attn_partial(const void* Q, const void* K, const void
  *               cand_idx = cand_scores + B*k and cand_stride = 2*B*k)
  *   local_idx   int32 [B, k] out: the global top-k entries in rank `rank`'s
  *               slice, as its local indices, ascending, then -1
+ *   local_count int32 [B] out (nullable): the number of those entries, the
+ *               idx_count of sa_sparse_decode_attn_partial
  * The selection is sa_topk's (min(k, candidates) largest, ties to the lower
  * position) over the N*k candidates of each sequence, padding scoring -inf.
  * 0 <= rank < N; N*k <= 2^31 - 1; cand_stride >= B*k when N > 1. */
 size_t sa_cp_select_workspace_size(int N, int B, int k);
 sa_status sa_cp_select(const float* cand_scores, const int32_t* cand_idx, int64_t cand_stride, int N,
-                       int B, int k, int rank, int32_t* local_idx, void* ws, size_t ws_bytes,
-                       void* stream);
+                       int B, int k, int rank, int32_t* local_idx, int32_t* local_count, void* ws,
+                       size_t ws_bytes, void* stream);
 
 /* The log-sum-exp merge of P partial results of the same rows:
  *   O[row, :] = sum_p 2^(m_p - M) O_part_p[row, :] / sum_p 2^(m_p - M) l_p,

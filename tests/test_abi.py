@@ -138,7 +138,7 @@ def test_context_parallel_entry_points_reject_bad_requests(lib):
     assert need >= sa.WS_HEADER_BYTES + 4 * B * 8 * k + 4 * B + 4 * B * k
 
     def select(N=2, rank=0, stride=B * k, ws_bytes=1 << 30):
-        return lib.sa_cp_select(FAKE, FAKE, stride, N, B, k, rank, FAKE, FAKE_WS, ws_bytes, None)
+        return lib.sa_cp_select(FAKE, FAKE, stride, N, B, k, rank, FAKE, None, FAKE_WS, ws_bytes, None)
 
     assert select(rank=2) == sa.SA_ERR_INVALID_ARG and b"rank" in lib.sa_last_error()
     assert select(rank=-1) == sa.SA_ERR_INVALID_ARG
@@ -161,8 +161,8 @@ def test_context_parallel_entry_points_reject_bad_requests(lib):
     assert combine(n=0) == sa.SA_OK  # nothing to merge: no launch
 
     def partial(ml=FAKE, d=128):
-        return lib.sa_sparse_decode_attn_partial(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 8192, 32, 8, d, 64, 0.088,
-                                                 FAKE, ml, FAKE_WS, 1 << 30, None)
+        return lib.sa_sparse_decode_attn_partial(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 8192, 32, 8, d, 64, None,
+                                                 0.088, FAKE, ml, FAKE_WS, 1 << 30, None)
 
     assert partial(ml=None) == sa.SA_ERR_INVALID_ARG and b"ml" in lib.sa_last_error()
     assert partial(ml=ctypes.c_void_p(0x7F0000001004)) == sa.SA_ERR_INVALID_ARG

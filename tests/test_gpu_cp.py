@@ -81,6 +81,39 @@ def test_partial_attention_matches_the_oracle(dev, L, B, Hq, Hkv, lens, k, empty
     assert (one.view_as(full) - full).abs().max().item() <= 1e-6
 
 
+@pytest.mark.parametrize("B,lens,k,counts", [
+    (3, [900, 333, 1500], 1024, [0, 100, 1024]),   # many units
+    (1, [5000], 2048, [300]),                      # one unit over a cluster: splits of the 300 real entries
+    (2, [4000, 64], 2048, [2048, 64]),
+])
+def test_partial_attention_reads_only_the_counted_entries(dev, B, lens, k, counts):
+    """Entries past idx_count[b] are ignored even when they hold valid
+    indices: the result is the oracle's over the counted prefix."""
+    rng = np.random.default_rng(k + B)
+    L, Hq, Hkv, d = 3, 16, 4, 128
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    T = int(seq_off[-1])
+    Q, K, V = bits(rng, (L, B, Hq, d)), bits(rng, T * Hkv * d), bits(rng, T * Hkv * d)
+    idx = np.full((B, k), -1, np.int32)
+    for b in range(B):
+        m = min(k, lens[b])
+        idx[b, :m] = np.sort(rng.choice(lens[b], m, replace=False))
+    scale = 1 / math.sqrt(d)
+    ws = sa.workspace(sa.sparse_decode_attn_workspace_size(L, B, Hq, Hkv, d, k), dev)
+    o, ml = sa.sparse_decode_attn_partial(bf16_dev(Q, dev), bf16_dev(K, dev), bf16_dev(V, dev),
+                                          torch.from_numpy(seq_off).to(dev),
+                                          torch.tensor(lens, dtype=torch.int32, device=dev),
+                                          torch.from_numpy(idx).to(dev), Hkv, scale,
+                                          idx_count=torch.tensor(counts, dtype=torch.int32, device=dev), ws=ws)
+    got = sa.combine_partials(o.view(1, -1, d), ml.view(1, -1, 2), out_dtype=torch.float32).cpu().numpy()
+    assert_status_ok(ws)
+    cut = idx.copy()
+    for b in range(B):
+        cut[b, counts[b]:] = -1
+    want = oracle.sparse_decode_attn(Q, K, V, seq_off, lens, cut, Hkv, scale).reshape(-1, d)
+    assert np.abs(got - want).max() <= parity.ATOL_F32
+
+
 @pytest.mark.parametrize("P", [1, 3, 8])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_combine_partials_matches_the_oracle(dev, P, out_dtype):
@@ -136,10 +169,12 @@ def test_cp_select_is_bit_exact(dev, N, lens, k, levels):
     g = torch.from_numpy(cand).to(dev)
     s, i = cp.cand_views(g)
     ws = sa.workspace(sa.cp_select_workspace_size(N, len(lens), k), dev)
+    cnt = torch.empty(len(lens), dtype=torch.int32, device=dev)
     for r in range(N):
-        got = sa.cp_select(s, i, r, ws=ws).cpu().numpy()
+        got = sa.cp_select(s, i, r, local_count=cnt, ws=ws).cpu().numpy()
         want = oracle.cp_select(cand[:, 0].view(np.float32), cand[:, 1], r)
         assert np.array_equal(got, want), f"rank {r}"
+        assert np.array_equal(cnt.cpu().numpy(), (want >= 0).sum(1)), f"rank {r} counts"
     assert_status_ok(ws)
 
 
