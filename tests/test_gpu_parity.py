@@ -179,10 +179,12 @@ def test_c5_ragged_group_sampled(dev):
 
 
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("replicas", [1, 10])  # 8 rows: many CTAs per row; 80 rows: one CTA per row
-def test_topk_edge_cases(dev, replicas):
+# 8 rows: many CTAs per row; 80 rows: one CTA per row.  Rows of at most
+# 16384 keys (n = 16384, and a ragged 9001): shorter rows, split over fewer CTAs.
+@pytest.mark.parametrize("n", [100_000, 16384, 9001])
+@pytest.mark.parametrize("replicas", [1, 10])
+def test_topk_edge_cases(dev, replicas, n):
     rng = np.random.default_rng(3)
-    n = 100_000
     rows, nval, ks = [], [], []
     rows.append(np.full(n, 0.75, np.float32)); nval.append(5000)                           # all equal
     rows.append((rng.integers(0, 20, n) / 4).astype(np.float32)); nval.append(n)           # heavy ties at threshold
@@ -193,6 +195,7 @@ def test_topk_edge_cases(dev, replicas):
     big = (1.0 + np.arange(n, dtype=np.float64) * 2 ** -23).astype(np.float32)            # one huge bucket
     rows.append(rng.permutation(big)); nval.append(n)
     rows.append(rng.random(n).astype(np.float32)); nval.append(2048)                       # n_valid == k
+    nval = [min(v, n) for v in nval]
     S = np.concatenate([np.stack(rows)] * replicas)
     nv = np.array(nval * replicas, np.int32)
     rows = rows * replicas
