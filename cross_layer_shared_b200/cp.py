@@ -93,6 +93,12 @@ class CPRank:
     def __init__(self, N: int, rank: int, KI: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                  local_len: Sequence[int], k: int, H_I: int, d_I: int, Hq: int, Hkv: int, d: int, L_g: int,
                  scale: float):
+        if not 0 <= rank < N:
+            raise ValueError(f"rank {rank} outside [0, {N})")
+        if sum(int(x) for x in local_len) == 0:
+            # the attention's tensor maps need at least one cached row
+            raise ValueError(f"rank {rank} holds no token of any sequence: use at most as many ranks as the "
+                             "longest sequence has tokens")
         self.N, self.rank, self.k = N, rank, k
         self.KI, self.K, self.V = KI, K, V
         self.B = len(local_len)

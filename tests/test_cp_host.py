@@ -63,6 +63,14 @@ def test_packed_views():
     assert o[1, 0, 0] == n and ml[1, 0, 0] == n + rows * d
 
 
+def test_rank_state_rejects_empty_slices_and_bad_ranks():
+    x = torch.zeros(0)
+    with pytest.raises(ValueError, match="no token"):
+        cp.CPRank(8, 7, x, x, x, [0, 0], 16, 4, 64, 8, 2, 128, 2, 0.1)
+    with pytest.raises(ValueError, match="outside"):
+        cp.CPRank(2, 2, x, x, x, [5, 5], 16, 4, 64, 8, 2, 128, 2, 0.1)
+
+
 # ---------------------------------------------------------------- two ranks over gloo
 class OracleRank:
     """A rank whose arithmetic is the oracle's (CPU), with CPRank's interface

@@ -82,3 +82,66 @@ def test_index_score_is_monotone_in_each_head_weight(S, H_I, seed):
     assert np.all(up >= base)
     dbl = oracle.index_score(qI, 2 * w, KI, [0, S], [0], [S - 1])[0][:S]
     assert np.array_equal(dbl, 2 * base)
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.lists(st.integers(0, 40), min_size=1, max_size=4), st.integers(1, 6), st.integers(1, 12),
+       st.integers(0, 2**31 - 1))
+def test_slice_candidates_select_the_whole_context_topk(lens, N, k, seed):
+    """Context-parallel selection: for any slicing of each context into N
+    contiguous pieces, the union of every rank's share of the selection over
+    the slices' top-k candidates is the top-k of the whole context (stable
+    sort prefix), and each share is ascending then -1."""
+    rng = np.random.default_rng(seed)
+    B = len(lens)
+    full = [rng.integers(-2, 3, n).astype(np.float32) / 2 for n in lens]
+    cuts = [np.sort(np.concatenate([[0, n], rng.integers(0, n + 1, N - 1)])) for n in lens]
+    cand_s = np.zeros((N, B, k), np.float32)
+    cand_i = np.zeros((N, B, k), np.int32)
+    for r in range(N):
+        w = max(1, max(int(c[r + 1] - c[r]) for c in cuts))
+        sc = np.zeros((B, w), np.float32)
+        nv = []
+        for b in range(B):
+            lo, hi = int(cuts[b][r]), int(cuts[b][r + 1])
+            sc[b, :hi - lo] = full[b][lo:hi]
+            nv.append(hi - lo)
+        cand_i[r], cand_s[r] = oracle.topk(sc, nv, k, with_scores=True)
+    got = [[] for _ in range(B)]
+    for r in range(N):
+        share = oracle.cp_select(cand_s, cand_i, r)
+        for b in range(B):
+            row = [int(t) for t in share[b] if t >= 0]
+            assert row == sorted(row) and all(t < 0 for t in share[b][len(row):])
+            got[b] += [int(cuts[b][r]) + t for t in row]
+    for b in range(B):
+        want = sorted(sorted(range(lens[b]), key=lambda t: (-float(full[b][t]), t))[:k])
+        assert sorted(got[b]) == want
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.integers(1, 6), st.integers(1, 5), st.integers(0, 2**31 - 1))
+def test_combine_is_order_free_and_splits_compose(P, rows, seed):
+    """The log-sum-exp merge does not depend on the order of the parts, and
+    merging two parts first (a part's (m, l, o) after a merge is (M, L, O*L))
+    then the rest gives the same as merging all at once."""
+    rng = np.random.default_rng(seed)
+    d = 4
+    l = rng.uniform(0.5, 4, (P, rows))
+    l[rng.random((P, rows)) < 0.2] = 0.0
+    m = rng.uniform(-6, 6, (P, rows))
+    m[l == 0] = -np.inf
+    o = rng.standard_normal((P, rows, d)) * l[..., None]
+    ml = np.stack([m, l], -1)
+    whole = oracle.combine_partials(o, ml)
+    perm = rng.permutation(P)
+    np.testing.assert_allclose(oracle.combine_partials(o[perm], ml[perm]), whole, rtol=1e-12, atol=1e-12)
+    if P >= 2:
+        first = oracle.combine_partials(o[:2], ml[:2])
+        M = np.max(np.where(ml[:2, :, 1] > 0, ml[:2, :, 0], -np.inf), axis=0)
+        L = np.sum(np.where(ml[:2, :, 1] > 0, np.exp2(ml[:2, :, 0] - np.where(np.isfinite(M), M, 0)) * ml[:2, :, 1],
+                            0), axis=0)
+        merged_ml = np.stack([np.where(L > 0, M, -np.inf), L], -1)[None]
+        merged_o = (first * L[:, None])[None]
+        again = oracle.combine_partials(np.concatenate([merged_o, o[2:]]), np.concatenate([merged_ml, ml[2:]]))
+        np.testing.assert_allclose(again, whole, rtol=1e-10, atol=1e-12)
