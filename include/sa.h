@@ -361,8 +361,9 @@ sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const int32_t* q_po
 
 /* The sparse decode attention of one rank, left unnormalised.  Arguments as
  * sa_sparse_decode_attn, plus idx_count (nullable, device int32 [B]): when
- * set, only the first idx_count[b] entries of idx row b are read (the rest
- * count as padding) and the keys are split over that many, so a rank whose
+ * set, only the first idx_count[b] entries of idx row b (clamped to [0, k])
+ * are read, the rest counting as padding, and the keys are split over that
+ * many, so a rank whose
  * share of the index is small runs on only that share.  For each row
  * (l, b, h), with a reference m (log2
  * units) at most 8 below max_t z_t * log2(e) over its valid selected keys:
