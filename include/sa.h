@@ -382,7 +382,9 @@ sa_status sa_sparse_decode_attn_partial(const void* Q, const void* K, const void
 
 /* Global top-k over the gathered candidates.
  *   cand_scores, cand_idx  rank r's top_scores (fp32 [B, k]) and idx (int32
- *               [B, k], < 0 = padding) from sa_topk over its slice, at
+ *               [B, k]) from sa_topk over its slice: each idx row ascending,
+ *               then -1 padding, as sa_topk writes it (other orders give
+ *               unspecified, in-bounds results), at
  *               element offset r * cand_stride of each (so one all-gathered
  *               buffer of [N][scores | idx] blocks serves both, with
  *               cand_idx = cand_scores + B*k and cand_stride = 2*B*k)
