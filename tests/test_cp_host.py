@@ -169,3 +169,34 @@ def test_gloo_step_equals_the_one_device_step(world):
     for b in range(want_idx.shape[0]):
         got = sorted(t for r in range(world) for t in results[r][1][b])
         assert got == [int(t) for t in want_idx[b] if t >= 0], b
+
+
+def _oracle_ranks(world):
+    lens, H_I, d_I, Hq, Hkv, d, L_g, k, qI, w, KI, K, V, Q = _inputs()
+    bnd = cp.shard_bounds(lens, world)
+    ranks = []
+    for r in range(world):
+        lo, hi = bnd[r, :, 0], bnd[r, :, 1]
+        sl = lambda c, G, dim: cp.shard_cache(torch.from_numpy(c.astype(np.int32)), lens, G, dim, lo, hi).numpy()
+        ranks.append(OracleRank(world, r, sl(KI.reshape(-1), 1, d_I).astype(np.uint16),
+                                sl(K, Hkv, d).astype(np.uint16).reshape(-1), sl(V, Hkv, d).astype(np.uint16).reshape(-1),
+                                hi - lo, k, Hkv, d, L_g, Hq, 0.3))
+    return ranks, qI, w, Q
+
+
+@pytest.mark.parametrize("order", ["rank-major", "reversed"])
+def test_the_exchange_order_matters(order):
+    """All ranks in one process, phase by phase: rank-major gathers give the
+    one-device result; gathering in reverse rank order (a plausible layout
+    slip) breaks the selection's tie rule and the local index mapping."""
+    world = 3
+    ranks, qI, w, Q = _oracle_ranks(world)
+    flip = (lambda t: t.flip(0)) if order == "reversed" else (lambda t: t)
+    cand = flip(torch.stack([r.candidates(qI, w) for r in ranks]))
+    for r in ranks:
+        r.select(cand)
+    parts = torch.stack([r.partial(Q) for r in ranks])
+    O = ranks[0].combine(parts).numpy()
+    want_O, _ = _one_device()
+    same = np.abs(O - want_O).max() <= 1e-5
+    assert same == (order == "rank-major")
