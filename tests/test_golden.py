@@ -41,3 +41,34 @@ def test_golden_block_union():
     c = G["block_union"]
     indptr, indices = oracle.block_union(np.array(c["idx"], np.int32), c["S"], c["block"], c["Hkv"])
     assert indptr.tolist() == c["expected_indptr"] and indices.tolist() == c["expected_indices"]
+
+
+def test_golden_cp_select():
+    c = G["cp_select"]
+    s = np.array(c["scores"], np.float32)
+    k = c["k"]
+    N = len(c["slices"])
+    cand_s = np.zeros((N, 1, k), np.float32)
+    cand_i = np.zeros((N, 1, k), np.int32)
+    for r, (lo, hi) in enumerate(c["slices"]):
+        cand_i[r], cand_s[r] = oracle.topk(s[None, lo:hi], [hi - lo], k, with_scores=True)
+    for r in range(N):
+        assert oracle.cp_select(cand_s, cand_i, r)[0].tolist() == c["expected_local"][r]
+
+
+def test_golden_combine_partials():
+    c = G["combine_partials"]
+    o = np.array([[p["o"]] for p in c["parts"]], np.float64)
+    ml = np.array([[[p["m"], p["l"]]] for p in c["parts"]], np.float64)
+    np.testing.assert_allclose(oracle.combine_partials(o, ml)[0], c["expected"], rtol=0, atol=1e-15)
+
+
+def test_golden_sparse_attention_partial():
+    c = G["sparse_attention_partial"]
+    K, V = np.array(c["K"], np.float32), np.array(c["V"], np.float32)
+    n = K.shape[0]
+    o, ml = oracle.sparse_decode_attn_partial(bf(np.array(c["q"])[None, None, None]), bf(K.ravel()), bf(V.ravel()),
+                                              [0, n], [n], np.array([c["idx"]], np.int32), 1, c["scale"])
+    assert abs(ml[0, 0, 0, 0] - c["expected_m"]) <= 1e-15
+    assert abs(ml[0, 0, 0, 1] - c["expected_l"]) <= 1e-15
+    np.testing.assert_allclose(o[0, 0, 0], c["expected_o"], rtol=0, atol=1e-15)
