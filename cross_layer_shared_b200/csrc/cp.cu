@@ -3,10 +3,11 @@
 // tokens [lo_r(b), hi_r(b)), slices in rank order).
 //
 // A step on rank r: its indexer scores and top-k (with scores) over its
-// slice; the candidates of all ranks exchanged; cp_select_* below keep this
-// rank's share of the global top-k; attention over its selected rows with
-// partial outputs (m, l, o before normalisation); the partials exchanged;
-// combine_partials merges them.  The result equals the single-GPU step: a
+// slice; the candidates of all ranks exchanged; cp_gather_kernel, the top-k
+// and cp_local_kernel below keep this rank's share of the global top-k;
+// attention over its selected rows with partial outputs (m, l, o before
+// normalisation); the partials exchanged; combine_partials_kernel merges
+// them.  The result equals the single-GPU step: a
 // token of the global top-k is in its slice's top-k, ties go to the lower
 // index in both (the gathered candidate order, rank-major then ascending
 // local index, is ascending global index), and softmax attention over a
