@@ -19,6 +19,15 @@ Every rank ends with the whole output.  The arithmetic runs in libsa's
 kernels; this module holds the slicing, the buffer layout and the order of
 the exchanges.  `exchange` is any all-gather: `nccl_exchange()` over
 torch.distributed, or the single-device emulation in `emulate_step`.
+
+One process per GPU (e.g. under torchrun), each holding its slices:
+
+    dist.init_process_group("nccl", device_id=dev)
+    lo, hi = shard_bounds(seq_lens, N)[rank].T
+    me = CPRank(N, rank, KI_slice, K_slice, V_slice, hi - lo, k, H_I, d_I, Hq, Hkv, d, L_g, scale)
+    O = step(me, nccl_exchange(N), qI, w, Q)      # the same O on every rank
+
+Every rank makes the same two collectives in the same order each step.
 """
 from __future__ import annotations
 
