@@ -323,6 +323,9 @@ sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const
  *     larger S returns SA_ERR_UNSUPPORTED before anything is enqueued;
  *   - the first call on each device looks up the array's device address, so
  *     make that first call before any stream capture begins;
+ *   - that address is kept for the life of the process: do not call this
+ *     entry point on a device after a reset of it (cudaDeviceReset or a
+ *     primary-context reset), which would leave the kept address stale;
  *   - every call shares the one array: calls that may overlap on the GPU
  *     (different streams, or different host threads on one device) race and
  *     must be ordered by the caller;

@@ -138,6 +138,18 @@ def decode_group_parity(cfg, g, seqs, dev, out_dtypes=(torch.bfloat16, torch.flo
     scores_h = scores.cpu().numpy()
     idx_h = idx.cpu().numpy()
     outs_h = {dt: o.float().cpu().numpy() for dt, o in outs.items()}
+    check_group(cfg, g, seqs, scores_h, idx_h, outs_h)
+    return idx_h, scores_h
+
+
+def check_group(cfg, g, seqs, scores_h, idx_h, outs_h):
+    """Stage by stage against the oracle for the sequences `seqs` of group g:
+    scores within the fp32 bound; the index bit-exact against the oracle's
+    top-k of the GPU's scores and exact outside the tie band against the
+    oracle's own scores; every layer's output within the dtype's tolerance
+    of the oracle's attention over the GPU's index.  outs_h maps an output
+    dtype to the group's output rows [L_g, B, Hq, d]."""
+    layers = list(cfg.groups[g])
     qI, w, Q = cfg.qI(g), cfg.w(g), cfg.Q()
     for b in seqs:
         S = cfg.seq_lens[b]
@@ -155,7 +167,6 @@ def decode_group_parity(cfg, g, seqs, dev, out_dtypes=(torch.bfloat16, torch.flo
             tol = parity.ATOL_F32 if dt == torch.float32 else parity.ATOL_BF16
             err = np.abs(O[:, b] - O_ora).max()
             assert err <= tol, f"{cfg.name} b={b} {dt}: max-abs {err} > {tol}"
-    return idx_h, scores_h
 
 
 def test_c1_decode_group_with_needles(dev):
@@ -165,17 +176,21 @@ def test_c1_decode_group_with_needles(dev):
     assert set(needles) <= set(idx_h[0].tolist())
 
 
-@pytest.mark.parametrize("name,seqs", [("c2", [0, 5]), ("c3", [0, 3])])
-def test_full_size_decode_group(name, seqs, dev):
+@pytest.mark.parametrize("name,group", [("c2", 0), ("c2", 1), ("c2", 2), ("c3", 0)])
+def test_full_size_decode_group(name, group, dev):
+    """Every sequence of every F group of c2 (8 x 32768 tokens, three groups)
+    and of the c3 group (4 x 131072 tokens, 24 layers): scores, index and
+    both output dtypes against the oracle."""
     cfg = synth.workload(name)
-    decode_group_parity(cfg, len(cfg.groups) - 1, seqs, dev)
+    decode_group_parity(cfg, group, list(range(cfg.B)), dev)
 
 
-def test_c5_ragged_group_sampled(dev):
+@pytest.mark.parametrize("group", [0, 11])
+def test_c5_ragged_group_sampled(dev, group):
     cfg = synth.workload("c5")
     lens = np.array(cfg.seq_lens)
     seqs = [int(np.argmin(lens)), int(np.argmax(lens)), 7]
-    decode_group_parity(cfg, 0, seqs, dev, out_dtypes=(torch.bfloat16,))
+    decode_group_parity(cfg, group, seqs, dev, out_dtypes=(torch.bfloat16,))
 
 
 # --------------------------------------------------------------------------
@@ -299,8 +314,43 @@ def test_decode_step_c1_matches_oracle_walk(dev):
     got_idx = idx.cpu().numpy()
     parity.assert_topk_band(got_idx[0], oracle.index_score(cfg.qI(0), cfg.w(0), KI, cfg.seq_off, [0],
                                                            [cfg.S_max - 1])[0], cfg.S_max, cfg.k)
-    if np.array_equal(got_idx, used[0]):
+    # every layer of the F,S,S,S walk reads the F layer's index
+    assert all(np.array_equal(u, used[0]) for u in used)
+    # the output, always: the oracle's attention over the GPU's (validated) index
+    O_gpu_idx = oracle.sparse_decode_attn(cfg.Q(), K, V, cfg.seq_off, cfg.seq_lens, got_idx, cfg.Hkv, cfg.scale)
+    assert np.abs(O.cpu().numpy() - O_gpu_idx).max() <= parity.ATOL_F32
+    if np.array_equal(got_idx, used[0]):  # no tie inside the band moved the selection: the oracle's own walk too
         assert np.abs(O.cpu().numpy() - O_ora).max() <= parity.ATOL_F32
+
+
+def test_decode_step_plan_c3_matches_oracle(dev):
+    """The call the benchmark times: c3 (4 x 131072 tokens; one indexer pass
+    and top-2048 shared by 24 cross-decoder layers over one KV cache; bf16
+    outputs) through a DecodeStepPlan built as the benchmark builds it, every
+    sequence checked stage by stage against the oracle: the scores the step
+    left behind, its index, and all 24 layers' outputs."""
+    cfg = synth.workload("c3")
+    wl = sgpu.decode_workload(cfg, dev)
+    n = cfg.L
+    grs = wl["groups"]
+    starts = [gr[0] for gr in cfg.groups]
+    qI = [grs[starts.index(l)]["qI"] if l in starts else None for l in range(n)]
+    w = [grs[starts.index(l)]["w"] if l in starts else None for l in range(n)]
+    KI = [grs[starts.index(l)]["KI"] if l in starts else None for l in range(n)]
+    gi = [max(i for i, s0 in enumerate(starts) if s0 <= l) for l in range(n)]
+    K = [grs[gi[l]]["K"] for l in range(n)]
+    V = [grs[gi[l]]["V"] for l in range(n)]
+    plan = sa.DecodeStepPlan(cfg.pattern, qI, w, KI, K, V, wl["seq_off"], wl["seq_len"], cfg.S_max, cfg.k, wl["Q"],
+                             cfg.Hkv, cfg.scale, out_dtype=torch.bfloat16)
+    O, idx = plan.run()
+    torch.cuda.synchronize()
+    assert_status_ok(plan.ws)
+    check_group(cfg, 0, list(range(cfg.B)), plan.scores.cpu().numpy(), idx.cpu().numpy(),
+                {torch.bfloat16: O.float().cpu().numpy()})
+    # a second run of the same plan gives the same bits
+    O2, idx2 = plan.run()
+    torch.cuda.synchronize()
+    assert torch.equal(idx2, idx) and torch.equal(O2.view(torch.int16), O.view(torch.int16))
 
 
 def test_decode_step_append_and_per_layer(dev):
@@ -340,7 +390,10 @@ def test_decode_step_append_and_per_layer(dev):
     for b in range(B):
         ora = oracle.index_score(qI[b:b + 1], w[b:b + 1], KIa, seq_off, [b], [lens[b] - 1])[0][:lens[b]]
         parity.assert_topk_band(got_idx[b], ora, lens[b], k, f"b={b}")
-    if np.array_equal(got_idx, used[0]):
+    # the output, always: the oracle's attention on the appended caches over the GPU's (validated) index
+    O_gpu_idx = oracle.sparse_decode_attn(Q, Ka, Va, seq_off, lens, got_idx, Hkv, scale)
+    assert np.abs(O.cpu().numpy() - O_gpu_idx).max() <= parity.ATOL_F32
+    if np.array_equal(got_idx, used[0]):  # no tie inside the band moved the selection: the oracle's own walk too
         assert np.abs(O.cpu().numpy() - O_ora).max() <= parity.ATOL_F32
     # the caches now hold the new token: per-layer launches against the fused group
     args = (pattern, [dqI] + none, [dw] + none, [dKI] + none, *common)

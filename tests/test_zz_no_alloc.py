@@ -3,13 +3,19 @@
 The no-workspace entry point is for callers that cannot allocate device
 memory around the call (inside a CUDA graph capture, or in a runtime that
 has no device allocator to hand).  Its scratch is a fixed array inside
-libsa, shared by every call, so this test makes two calls in a row with
+libsa, shared by every call, so these tests make two calls in a row with
 different selections: each must match the workspace entry point on the same
 inputs (block table exactly, outputs within the attention tolerance), which
-also shows the second call does not see the first call's leftovers.  It runs
-alone in a fresh process as well as after the rest of the suite.
+also shows the second call does not see the first call's leftovers.  One
+case makes the first call carry an out-of-range entry (recorded in the
+shared array, then skipped) before a valid call; another repeats the two
+calls in a fresh Python process, where the first call on the device is also
+the one that looks up the array's address.
 """
 import ctypes
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -23,6 +29,8 @@ from tests import parity
 
 pytestmark = pytest.mark.gpu
 
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
 
 def _selection(cfg, seed, dev):
     rng = np.random.default_rng(seed)
@@ -33,8 +41,10 @@ def _selection(cfg, seed, dev):
     return torch.from_numpy(idx).to(dev)
 
 
-@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
-def test_noalloc_matches_workspace_entry_point_twice(out_dtype):
+def two_calls(out_dtype, bad_first=False):
+    """Two no-alloc calls in a row, each against the workspace entry point on
+    the same inputs.  With bad_first, the first call's selection holds an
+    entry past the context (skipped by both entry points)."""
     build.build()
     dev = torch.device("cuda")
     cfg = synth.PrefillConfig("noalloc", S=8192, chunk=256, H_I=16, d_I=128, k=192, block=64, Hq=8, Hkv=2, d=128,
@@ -44,6 +54,8 @@ def test_noalloc_matches_workspace_entry_point_twice(out_dtype):
     tol = parity.ATOL_F32 if out_dtype == torch.float32 else parity.ATOL_BF16
     for call, seed in enumerate((5, 6)):
         idx = _selection(cfg, seed, dev)
+        if bad_first and call == 0:
+            idx[3, 0] = cfg.S + 100  # out of range: reported into the scratch's status block and skipped
         want_ptr, want_ind, want_O = sa.block_union_prefill(idx, wl["q_pos"], wl["Q"], wl["K"], wl["V"], cfg.block,
                                                             cfg.scale, out_dtype=out_dtype)
         ptr = torch.full((cfg.Hkv + 1,), -7, dtype=torch.int32, device=dev)
@@ -56,6 +68,21 @@ def test_noalloc_matches_workspace_entry_point_twice(out_dtype):
         assert torch.equal(ind[:n], want_ind[:n]), f"call {call}: kv_indices differ"
         err = (O.float() - want_O.float()).abs().max().item()
         assert err <= tol, f"call {call}: outputs differ by {err}"
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_noalloc_matches_workspace_entry_point_twice(out_dtype):
+    two_calls(out_dtype)
+
+
+def test_noalloc_valid_call_after_one_with_an_out_of_range_entry():
+    two_calls(torch.float32, bad_first=True)
+
+
+def test_noalloc_twice_in_a_fresh_process():
+    code = "import torch; from tests.test_zz_no_alloc import two_calls; two_calls(torch.float32); print('ok')"
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
 
 
 def test_noalloc_rejects_contexts_beyond_its_scratch():
