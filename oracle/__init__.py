@@ -57,6 +57,7 @@ def load(path: str):
     lb.oracle_sparse_decode_attn_partial.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, D, P, P]
     lb.oracle_combine_partials.argtypes = [P, P, I, I64, I, P]
     lb.oracle_cp_select.argtypes = [P, P, I, I, I, I, P]
+    lb.oracle_topk_dynamic.argtypes = [P, I64, P, I, I, D, P, P]
     lb.oracle_num_threads.restype = I
     return lb
 
@@ -104,6 +105,18 @@ def topk(scores, n_valid, k: int, with_scores: bool = False):
     ts = np.empty((Nq, k), dtype=np.float32) if with_scores else None
     lib().oracle_topk(_p(scores), ld, _p(n_valid), Nq, k, _p(idx), _p(ts))
     return (idx, ts) if with_scores else idx
+
+
+def topk_dynamic(scores, n_valid, k_max: int, tau: float):
+    """Dynamic k by routing mass (see oracle_topk_dynamic): (idx [Nq, k_max]
+    ascending then -1, counts [Nq])."""
+    scores = _c(scores, np.float32)
+    Nq, ld = scores.shape
+    n_valid = _c(n_valid, np.int32)
+    idx = np.empty((Nq, k_max), dtype=np.int32)
+    counts = np.empty(Nq, dtype=np.int32)
+    lib().oracle_topk_dynamic(_p(scores), ld, _p(n_valid), Nq, k_max, float(tau), _p(idx), _p(counts))
+    return idx, counts
 
 
 def sparse_decode_attn(Q, K, V, seq_off, seq_len, idx, Hkv: int, scale: float) -> np.ndarray:

@@ -437,6 +437,51 @@ void oracle_cp_select(const float* cand_scores, const int32_t* cand_idx, int N, 
   free(sel);
 }
 
+/*
+ * Dynamic k [CLSA news article, sections "Le cout : limites de
+ * compatibilite" and "Ce que cela signifie pour l'inference sur longs
+ * contextes": the indexer layer could set k per query instead of a fixed k;
+ * the pages leave the rule open].  Reading: the routing mass.  Row q keeps
+ * the smallest number m of its tokens, taken in the top-k order (score
+ * descending, lower index first), whose summed score reaches the fraction
+ * tau of the row's total score (the sum over all n_valid[q] tokens), but at
+ * most k_max; a row that never reaches it keeps min(n, k_max).  Sums are
+ * fp64, the total in index order, the running sum in the top-k order.
+ * idx[q] gets the m indices ascending, then -1 up to k_max; counts[q] = m.
+ */
+void oracle_topk_dynamic(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int k_max, double tau,
+                         int32_t* idx, int32_t* counts) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int q = 0; q < Nq; ++q) {
+    const int n = n_valid[q];
+    double total = 0.0;
+    for (int t = 0; t < n; ++t) total += (double)scores[(int64_t)q * ld + t];
+    scored_t* all = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n > 0 ? n : 1));
+    for (int t = 0; t < n; ++t) {
+      all[t].s = scores[(int64_t)q * ld + t];
+      all[t].i = t;
+    }
+    qsort(all, (size_t)n, sizeof(scored_t), by_score_then_index);
+    const double target = tau * total;
+    int m = n;
+    double run = 0.0;
+    for (int j = 0; j < n; ++j) {
+      run += (double)all[j].s;
+      if (run >= target) {
+        m = j + 1;
+        break;
+      }
+    }
+    if (m > k_max) m = k_max;
+    int32_t* row = idx + (int64_t)q * k_max;
+    for (int j = 0; j < m; ++j) row[j] = all[j].i;
+    qsort(row, (size_t)m, sizeof(int32_t), by_index);
+    for (int j = m; j < k_max; ++j) row[j] = -1;
+    counts[q] = m;
+    free(all);
+  }
+}
+
 /* threads OpenMP will use (reported next to CPU timings) */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

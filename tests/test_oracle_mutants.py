@@ -40,6 +40,13 @@ MUTANTS = {
     "candidates gathered rank-minor": ("rows[(int64_t)b * n + (int64_t)r * k + j] =",
                                        "rows[(int64_t)b * n + (int64_t)j * N + r] ="),
     "selection keeps every rank's share": ("if (pos >= 0 && pos / k == rank) {", "if (pos >= 0) {"),
+    "dynamic k: running sum in index order": ("      run += (double)all[j].s;\n      if (run >= target) {",
+                                              "      run += (double)scores[(int64_t)q * ld + j];\n      if (run >= target) {"),
+    "dynamic k: strict reach": ("      if (run >= target) {", "      if (run > target) {"),
+    "dynamic k: total over the kept tokens only": ("    const double target = tau * total;",
+                                                  "    const double target = tau * (total < 0 ? 0 : (double)all[0].s * 2);"),
+    "dynamic k: cap one short": ("    if (m > k_max) m = k_max;\n    int32_t* row = idx + (int64_t)q * k_max;",
+                                 "    if (m >= k_max) m = k_max - 1;\n    int32_t* row = idx + (int64_t)q * k_max;"),
     "routing drops the last token": ("for (int64_t t = 0; t < seq_len[b]; ++t) {\n      double acc",
                                      "for (int64_t t = 0; t + 1 < seq_len[b]; ++t) {\n      double acc"),
 }

@@ -651,3 +651,76 @@ def _cp_select_case(N):
             got[b] |= {bounds[r][b][0] + t for t in row}
     for b in range(B):
         assert sorted(got[b]) == _python_topk(full[b], k), b
+
+
+# --------------------------------------------------------------------------
+# Dynamic k by routing mass [CLSA news article, "Le cout : limites de
+# compatibilite": k could be set per query; the rule here is a reading]:
+# the smallest m, in the top-k order, whose running score reaches tau of
+# the row's total, at most k_max.
+def _dynamic_brute(row, n, k_max, tau):
+    """Exact rational arithmetic, sorting by (score desc, index asc)."""
+    vals = [Fraction(float(x)) for x in row[:n]]
+    total = sum(vals, Fraction(0))
+    order = sorted(range(n), key=lambda t: (-vals[t], t))
+    target = Fraction(tau) * total
+    m, run = n, Fraction(0)
+    for j, t in enumerate(order):
+        run += vals[t]
+        if run >= target:
+            m = j + 1
+            break
+    m = min(m, k_max)
+    return sorted(order[:m]), m
+
+
+def test_dynamic_k_brute_force_exact_rationals():
+    rng = np.random.default_rng(41)
+    for trial in range(40):
+        n = int(rng.integers(1, 60))
+        # dyadic scores with ties: every sum is exact in fp64
+        row = (rng.integers(0, 12, n) / 8.0).astype(np.float32)
+        k_max = int(rng.integers(1, 70))
+        tau = float(rng.choice([0.125, 0.25, 0.5, 0.75, 0.875, 1.0]))
+        idx, counts = oracle.topk_dynamic(row[None], [n], k_max, tau)
+        want, m = _dynamic_brute(row, n, k_max, tau)
+        assert counts[0] == m, (trial, counts[0], m)
+        assert list(idx[0, :m]) == want and np.all(idx[0, m:] == -1), trial
+
+
+def test_dynamic_k_uniform_scores_closed_form():
+    # n equal scores: the running sum after j tokens is j/n of the total, so
+    # m = ceil(tau * n), the lowest indices
+    n, k_max = 1000, 2048
+    row = np.full((1, n), 0.25, np.float32)
+    for tau, m in ((0.375, 375), (0.5, 500), (0.0625, 63), (1.0, 1000)):
+        idx, counts = oracle.topk_dynamic(row, [n], k_max, tau)
+        assert counts[0] == m, (tau, counts[0])
+        assert np.array_equal(idx[0, :m], np.arange(m)) and np.all(idx[0, m:] == -1)
+
+
+def test_dynamic_k_cap_dominant_token_and_zero_tail():
+    row = np.zeros((1, 300), np.float32)
+    row[0, 7] = 100.0
+    row[0, 50:60] = 1.0
+    # the dominant token alone carries 100/110 of the mass
+    idx, counts = oracle.topk_dynamic(row, [300], 64, 0.9)
+    assert counts[0] == 1 and idx[0, 0] == 7 and np.all(idx[0, 1:] == -1)
+    # the whole mass needs the 11 positive tokens, not the zero tail
+    idx, counts = oracle.topk_dynamic(row, [300], 64, 1.0)
+    assert counts[0] == 11 and list(idx[0, :11]) == [7] + list(range(50, 60))
+    # capped at k_max
+    idx, counts = oracle.topk_dynamic(row, [300], 5, 1.0)
+    assert counts[0] == 5 and list(idx[0, :5]) == [7, 50, 51, 52, 53]
+    # an empty row keeps nothing
+    idx, counts = oracle.topk_dynamic(row, [0], 5, 0.5)
+    assert counts[0] == 0 and np.all(idx[0] == -1)
+
+
+def test_dynamic_k_total_is_over_the_whole_row():
+    # the top-2 carry 2/3 of their own mass but only 2/8 of the row's
+    row = np.array([[1, 1, 1, 1, 1, 1, 1, 1]], np.float32)
+    row[0, 3] = 2.0
+    row[0, 6] = 2.0  # total 10
+    idx, counts = oracle.topk_dynamic(row, [8], 8, 0.5)  # target 5: 2 + 2 + 1
+    assert counts[0] == 3 and list(idx[0, :3]) == [0, 3, 6]
