@@ -20,7 +20,10 @@ MUTANTS = {
     "sequence offset ignored": ("const int64_t base = seq_off[q_seq[q]];", "const int64_t base = 0;"),
     "ties to the higher index": ("return (x->i > y->i) - (x->i < y->i);",
                                  "return (x->i < y->i) - (x->i > y->i);"),
-    "output not in index order": ("qsort(row, (size_t)m, sizeof(int32_t), by_index);", ";"),
+    "output not in index order": ("qsort(row, (size_t)m, sizeof(int32_t), by_index);\n    for (int j = m; j < k; ++j)",
+                                  ";\n    for (int j = m; j < k; ++j)"),
+    "dynamic k: output not in index order": ("qsort(row, (size_t)m, sizeof(int32_t), by_index);\n    for (int j = m; j < k_max;",
+                                             ";\n    for (int j = m; j < k_max;"),
     "scale dropped": ("z[j] = scale * dot;", "z[j] = dot;"),
     "GQA map modulo": ("const int g = h / G;\n    const uint16_t* Kb", "const int g = h % Hkv;\n    const uint16_t* Kb"),
     "ceil block map": ("if (t >= 0) mark[t / block] = 1;", "if (t >= 0) mark[(t + block - 1) / block] = 1;"),
