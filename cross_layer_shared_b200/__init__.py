@@ -32,12 +32,15 @@ SIGNATURES = {
     "sa_abi_version": ([], _I),
     "sa_read_device_status": ([_P, _P, ctypes.POINTER(_I), ctypes.POINTER(_I64)], _I),
     "sa_clear_device_status": ([_P, _P], _I),
+    "sa_wait_probe": ([_P, _SZ, ctypes.c_ulonglong, _P], _I),
     "sa_index_score_workspace_size": ([_I], _SZ),
     "sa_index_score": ([_P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _P, _I64, _P, _SZ, _P], _I),
     "sa_index_score_prefill_workspace_size": ([_I], _SZ),
     "sa_index_score_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P, _SZ, _P], _I),
     "sa_topk_workspace_size": ([_I, _I, _I], _SZ),
     "sa_topk": ([_P, _I64, _P, _I, _I, _I, _P, _P, _P, _SZ, _P], _I),
+    "sa_topk_dynamic_workspace_size": ([_I, _I, _I], _SZ),
+    "sa_topk_dynamic": ([_P, _I64, _P, _I, _I, _I, ctypes.c_double, _P, _P, _P, _SZ, _P], _I),
     "sa_sparse_decode_attn_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "sa_sparse_decode_attn": ([_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _F, _P, _I, _P, _SZ, _P], _I),
     "sa_indexer_layer_attn_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
@@ -159,6 +162,13 @@ def read_status(ws: torch.Tensor, stream=None):
     return code.value, list(det)
 
 
+def wait_probe(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """sa_wait_probe: one CTA whose bounded wait must give up after limit_ns
+    and record SA_ERR_TIMEOUT in ws (a self-test of the kernels' waits)."""
+    _ws(ws)
+    _check(lib().sa_wait_probe(ws.data_ptr(), ws.numel(), int(limit_ns), _stream(stream)))
+
+
 def clear_status(ws: torch.Tensor, stream=None) -> None:
     _check(lib().sa_clear_device_status(_ptr(ws), _stream(stream)))
 
@@ -223,6 +233,28 @@ def topk(scores, n_valid, n_max: int, k: int, idx=None, top_scores=None, want_sc
     _check(lib().sa_topk(_ptr(scores), ld, _ptr(n_valid), Nq, n_max, k, _ptr(idx), _ptr(top_scores), _ptr(ws),
                          ws.numel(), _stream(stream)))
     return (idx, top_scores) if want_scores else idx
+
+
+def topk_dynamic(scores, n_valid, n_max: int, k_max: int, tau: float, idx=None, counts=None, ws=None,
+                 stream=None):
+    """sa_topk_dynamic: per row, the fewest tokens in top-k order whose scores
+    reach tau of the row's total, at most k_max.  Returns (idx [Nq, k_max]
+    ascending then -1, counts [Nq])."""
+    Nq, ld = scores.shape
+    _rows_out(scores, Nq, n_max, "scores")
+    _out(n_valid, (Nq,), (torch.int32,), "n_valid")
+    if idx is None:
+        idx = torch.empty((Nq, k_max), dtype=torch.int32, device=scores.device)
+    _out(idx, (Nq, k_max), (torch.int32,), "idx")
+    if counts is None:
+        counts = torch.empty((Nq,), dtype=torch.int32, device=scores.device)
+    _out(counts, (Nq,), (torch.int32,), "counts")
+    if ws is None:
+        ws = workspace(lib().sa_topk_dynamic_workspace_size(Nq, n_max, k_max), scores.device)
+    _ws(ws)
+    _check(lib().sa_topk_dynamic(_ptr(scores), ld, _ptr(n_valid), Nq, n_max, k_max, float(tau), _ptr(idx),
+                                 _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, counts
 
 
 def sparse_decode_attn_workspace_size(L_g, B, Hq, Hkv, d, k) -> int:
@@ -364,15 +396,20 @@ def indexer_layer_attn(Q, K, V, seq_off, seq_len, S_max: int, Hkv: int, scale: f
 
 def decode_step_attn_route_workspace_size(B, S_max, Hq, Hkv, d, k, L) -> int:
     return max(indexer_layer_attn_workspace_size(B, S_max, Hq, Hkv, d), int(lib().sa_topk_workspace_size(B, S_max, k)),
+               int(lib().sa_topk_dynamic_workspace_size(B, S_max, k)),
                sparse_decode_attn_workspace_size(max(L - 1, 1), B, Hq, Hkv, d, k))
 
 
 def decode_step_attn_route(Q, K, V, seq_off, seq_len, S_max: int, k: int, Hkv: int, scale: float,
-                           out_dtype=torch.bfloat16, O=None, idx=None, scores=None, ws=None, stream=None):
+                           out_dtype=torch.bfloat16, O=None, idx=None, scores=None, ws=None, stream=None,
+                           tau: Optional[float] = None, counts=None):
     """One decode step of a cross-decoder group under the CLSA reading in
     which layer 0 is the indexer layer: it attends densely and its summed
     attention weights give the routing scores; their top-k is the index that
-    layers 1..L-1 share over the same cache.  Q [L, B, Hq, d] -> (O, idx)."""
+    layers 1..L-1 share over the same cache.  Q [L, B, Hq, d] -> (O, idx).
+    With tau, k is dynamic: each sequence keeps the fewest tokens whose
+    routing mass reaches tau of its total, at most k (sa_topk_dynamic); the
+    index is then -1 padded and (O, idx, counts) is returned."""
     L, B, Hq, d = Q.shape
     if O is None:
         O = torch.empty((L, B, Hq, d), dtype=out_dtype, device=Q.device)
@@ -380,10 +417,13 @@ def decode_step_attn_route(Q, K, V, seq_off, seq_len, S_max: int, k: int, Hkv: i
         ws = workspace(decode_step_attn_route_workspace_size(B, S_max, Hq, Hkv, d, k, L), Q.device)
     _, scores = indexer_layer_attn(Q[0], K, V, seq_off, seq_len, S_max, Hkv, scale, O=O[0], scores=scores, ws=ws,
                                    stream=stream)
-    idx = topk(scores, seq_len, S_max, k, idx=idx, ws=ws, stream=stream)
+    if tau is None:
+        idx = topk(scores, seq_len, S_max, k, idx=idx, ws=ws, stream=stream)
+    else:
+        idx, counts = topk_dynamic(scores, seq_len, S_max, k, tau, idx=idx, counts=counts, ws=ws, stream=stream)
     if L > 1:
         sparse_decode_attn(Q[1:], K, V, seq_off, seq_len, idx, Hkv, scale, O=O[1:], ws=ws, stream=stream)
-    return O, idx
+    return (O, idx) if tau is None else (O, idx, counts)
 
 
 def decode_step_workspace_size(n_layers, B, S_max, Hq, Hkv, d, k) -> int:

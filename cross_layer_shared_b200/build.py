@@ -24,8 +24,8 @@ HEADER = os.path.join(ROOT, "include", "sa.h")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVFLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]
-SOURCES = ["api.cu", "indexer.cu", "indexer_prefill.cu", "topk.cu", "topk_split.cu", "attn.cu", "union.cu",
-           "route_attn.cu", "cp.cu"]
+SOURCES = ["api.cu", "indexer.cu", "indexer_prefill.cu", "topk.cu", "topk_split.cu", "topk_dynamic.cu", "attn.cu",
+           "union.cu", "route_attn.cu", "cp.cu"]
 
 
 def nvcc() -> str:

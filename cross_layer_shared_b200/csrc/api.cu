@@ -333,6 +333,38 @@ sa_status sa_clear_device_status(void* ws, void* stream) {
   return SA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+// One CTA waits on an mbarrier that nothing arrives on: the wait routine of
+// every kernel must give up after limit_ns and the give-up must be reported.
+__global__ void wait_probe_kernel(sa::DeviceStatus* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sa::mbar_init(&bar, 1);
+    sa::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !sa::mbar_wait(&bar, 0, limit_ns))
+    sa::report(status, sa::kErrTimeout, sa::kKernWaitProbe, 0, 0, (long long)limit_ns);
+  __syncthreads();
+}
+}  // namespace
+
+extern "C" {
+
+sa_status sa_wait_probe(void* ws, size_t ws_bytes, unsigned long long limit_ns, void* stream) {
+  const char* who = "sa_wait_probe";
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull)
+    return fail(SA_ERR_INVALID_ARG, "%s: limit_ns=%llu outside [1e3, 1e9]", who, limit_ns);
+  sa_status st = check_ws(ws, ws_bytes, SA_WS_HEADER_BYTES, who);
+  if (st != SA_OK) return st;
+  wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(status_of(ws), limit_ns);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("sa_wait_probe launch", e);
+  return SA_OK;
+}
+
 // ---------------------------------------------------------------- indexer
 size_t sa_index_score_workspace_size(int B) {
   (void)B;
@@ -438,6 +470,58 @@ sa_status sa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int N
     e = sa::launch_topk_rows(scores, ld, n_valid, Nq, n_max, k, idx, top_scores, status_of(ws),
                              (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail("sa_topk launch", e);
+  return SA_OK;
+}
+
+// ---------------------------------------------------------------- dynamic k
+namespace {
+struct DynLayout {
+  size_t topk, sel_idx, sel_s, total;  // byte offsets after the header, then the total
+};
+DynLayout dyn_layout(int Nq, int n_max, int k_max) {
+  DynLayout l{};
+  const size_t t = (Nq > 0 && n_max > 0 && sa::topk_use_split(Nq, n_max, num_sms()))
+                       ? sa::topk_split_ws_bytes(Nq, n_max, num_sms())
+                       : 0;
+  l.topk = 0;
+  l.sel_idx = round_up(t, 256);
+  l.sel_s = l.sel_idx + round_up(4 * (size_t)Nq * (size_t)k_max, 256);
+  l.total = SA_WS_HEADER_BYTES + l.sel_s + round_up(4 * (size_t)Nq * (size_t)k_max, 256);
+  return l;
+}
+}  // namespace
+
+size_t sa_topk_dynamic_workspace_size(int Nq, int n_max, int k_max) {
+  if (Nq < 1 || n_max < 1 || k_max < 1) return SA_WS_HEADER_BYTES;
+  return dyn_layout(Nq, n_max, k_max).total;
+}
+
+sa_status sa_topk_dynamic(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max, int k_max,
+                          double tau, int32_t* idx, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  const char* who = "sa_topk_dynamic";
+  if (Nq < 0) return fail(SA_ERR_INVALID_ARG, "%s: Nq=%d < 0", who, Nq);
+  if (k_max < 1 || k_max > 4096) return fail(SA_ERR_UNSUPPORTED, "%s: k_max=%d outside [1, 4096]", who, k_max);
+  if (!(tau > 0.0 && tau <= 1.0)) return fail(SA_ERR_INVALID_ARG, "%s: tau must be in (0, 1]", who);
+  if (n_max < 0 || ld < n_max) return fail(SA_ERR_INVALID_ARG, "%s: need 0 <= n_max <= ld", who);
+  if (Nq > 0 && (!scores || !n_valid || !idx || !counts)) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  sa_status st = check_ws(ws, ws_bytes, sa_topk_dynamic_workspace_size(Nq, n_max, k_max), who);
+  if (st != SA_OK) return st;
+  if (Nq == 0) return SA_OK;
+  const DynLayout l = dyn_layout(Nq, n_max, k_max);
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
+  int32_t* sel_idx = reinterpret_cast<int32_t*>(base + l.sel_idx);
+  float* sel_s = reinterpret_cast<float*>(base + l.sel_s);
+  const cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if (sa::topk_use_split(Nq, n_max, num_sms()))
+    e = sa::launch_topk_split(scores, ld, n_valid, Nq, n_max, k_max, sel_idx, sel_s, status_of(ws), base + l.topk,
+                              num_sms(), s);
+  else
+    e = sa::launch_topk_rows(scores, ld, n_valid, Nq, n_max, k_max, sel_idx, sel_s, status_of(ws), s);
+  if (e != cudaSuccess) return cuda_fail("sa_topk_dynamic top-k launch", e);
+  e = sa::launch_topk_dynamic(scores, ld, n_valid, Nq, n_max, sel_idx, sel_s, k_max, tau, idx, counts, status_of(ws),
+                              s);
+  if (e != cudaSuccess) return cuda_fail("sa_topk_dynamic launch", e);
   return SA_OK;
 }
 

@@ -30,6 +30,7 @@ enum : int {
   kKernUnion = 5,
   kKernIndexerPrefill = 6,
   kKernRoute = 7,
+  kKernWaitProbe = 8,
 };
 
 struct DeviceStatus {

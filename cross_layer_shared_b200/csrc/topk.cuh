@@ -21,4 +21,14 @@ cudaError_t launch_topk_split(const float* scores, int64_t ld, const int32_t* n_
                               int32_t* idx, float* top_scores, DeviceStatus* status, void* scratch, int num_sms,
                               cudaStream_t stream);
 
+// Dynamic k by routing mass (topk_dynamic.cu), one CTA per row, over the
+// row's top k_max (sel_idx ascending then -1, sel_s their scores) from the
+// kernels above: idx [Nq, k_max] keeps the m entries reaching tau of the
+// row's total score in the top-k order, then -1; counts [Nq] = m.
+// k_max <= 4096.
+size_t topk_dynamic_smem_bytes(int k_max);
+cudaError_t launch_topk_dynamic(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max,
+                                const int32_t* sel_idx, const float* sel_s, int k_max, double tau, int32_t* idx,
+                                int32_t* counts, DeviceStatus* status, cudaStream_t stream);
+
 }  // namespace sa

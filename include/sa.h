@@ -96,6 +96,17 @@ sa_status sa_read_device_status(const void* ws, void* stream, int* device_status
 /* Enqueues a reset of the status block to zero on `stream`. */
 sa_status sa_clear_device_status(void* ws, void* stream);
 
+/* Self-test of the bounded waits every kernel of this library uses (not part
+ * of the method; the pages have no counterpart).  Launches one CTA that
+ * waits on an mbarrier nothing ever arrives on, through the same wait
+ * routine the kernels use, with a limit of `limit_ns` nanoseconds instead of
+ * the kernels' 1 s.  The wait gives up and records SA_ERR_TIMEOUT in the
+ * status block of `ws` with detail (kernel id 8, 0, 0, limit_ns); no copy or
+ * tensor-core operation is in flight when it does, and the kernel returns
+ * normally, so the context stays usable.  1e3 <= limit_ns <= 1e9.
+ * ws: at least SA_WS_HEADER_BYTES, 256-byte aligned. */
+sa_status sa_wait_probe(void* ws, size_t ws_bytes, unsigned long long limit_ns, void* stream);
+
 /* ------------------------------------------------------------------------
  * Indexer score, decode form  [IC section 1: the lightning indexer scores
  * every previous token for the current query; CLSA "Comment CLSA
@@ -160,6 +171,32 @@ sa_status sa_index_score_prefill(const void* qI, const float* w, const void* KI,
 size_t sa_topk_workspace_size(int Nq, int n_max, int k);
 sa_status sa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max,
                   int k, int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dynamic k by routing mass  [CLSA news article, sections "Le cout : limites
+ * de compatibilite" and "Ce que cela signifie pour l'inference sur longs
+ * contextes": the indexer layer could choose k per query instead of a fixed
+ * k; the pages leave the rule open.  The reading here: a coverage target on
+ * the routing scores' mass.]
+ *
+ * Row q (n = n_valid[q] scores) keeps the smallest number m of its tokens,
+ * taken in sa_topk's order (score descending, ties to the lower index),
+ * whose summed score reaches tau times the row's total score (the sum over
+ * all n tokens), but at most k_max; a row whose top k_max never reaches it
+ * keeps min(n, k_max).  Sums are fp64.  Meant for non-negative scores (the
+ * routing weights of sa_indexer_layer_attn, or sa_index_score with positive
+ * head weights): the running sum is then non-decreasing.
+ *
+ *   idx     int32 [Nq, k_max]   the m kept indices ascending, then -1
+ *   counts  int32 [Nq]          m per row
+ *   tau     in (0, 1]; 1 <= k_max <= 4096
+ * Other arguments as sa_topk.  Runs sa_topk's kernels for the top k_max
+ * (with their scores, into the workspace), then one CTA per row.
+ * ---------------------------------------------------------------------- */
+size_t sa_topk_dynamic_workspace_size(int Nq, int n_max, int k_max);
+sa_status sa_topk_dynamic(const float* scores, int64_t ld, const int32_t* n_valid, int Nq, int n_max,
+                          int k_max, double tau, int32_t* idx, int32_t* counts, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* ------------------------------------------------------------------------
  * Sparse decode attention for one layer group  [IC section 1: main

@@ -167,3 +167,11 @@ def test_context_parallel_entry_points_reject_bad_requests(lib):
     assert partial(ml=None) == sa.SA_ERR_INVALID_ARG and b"ml" in lib.sa_last_error()
     assert partial(ml=ctypes.c_void_p(0x7F0000001004)) == sa.SA_ERR_INVALID_ARG
     assert partial(d=64) == sa.SA_ERR_UNSUPPORTED
+
+
+def test_wait_probe_checks_its_arguments_before_any_launch(lib):
+    fake = ctypes.c_void_p(0x7F0000001000)
+    assert lib.sa_wait_probe(fake, 256, 10, None) == sa.SA_ERR_INVALID_ARG  # limit below 1 us
+    assert lib.sa_wait_probe(fake, 256, 2_000_000_000, None) == sa.SA_ERR_INVALID_ARG  # above 1 s
+    assert lib.sa_wait_probe(None, 256, 2_000_000, None) == sa.SA_ERR_WORKSPACE
+    assert lib.sa_wait_probe(fake, 64, 2_000_000, None) == sa.SA_ERR_WORKSPACE
