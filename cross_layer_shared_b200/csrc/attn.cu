@@ -79,10 +79,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// two fp32 values rounded to bf16 (nearest even) and packed, lo in bits 0-15,
+// in one conversion instruction
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return l | (h << 16);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
@@ -274,11 +276,17 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   ks.kend = min(n_keys, ks.kbeg + per);
   const int nt = ks.kend > ks.kbeg ? (ks.kend - ks.kbeg + kKT - 1) / kKT : 0;
 
-  // producer lanes: raw entries of tile rows 4*lane .. 4*lane+3, one tile ahead
-  int raw_next[4];
+  // producer lanes: raw entries of tile rows 4*lane .. 4*lane+3 of the next
+  // kPre tiles, all loads in flight at once (a ring in registers, slot = tile
+  // % kPre, statically indexed by the unrolled issue loop below).  One tile
+  // ahead, every tile's issue waited a whole load latency for its entries.
+  constexpr int kPre = 1;
+  int raw[kPre][4];
   if (warp >= kProdWarp0) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) raw_next[i] = key_raw(a, ks, b, ks.kbeg + 4 * lane + i);
+    for (int t = 0; t < kPre; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) raw[t][i] = key_raw(a, ks, b, ks.kbeg + t * kKT + 4 * lane + i);
   }
 
   // softmax state: thread (row r, key half h)
@@ -298,19 +306,23 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     // columns 64-127 on the first tile); V columns 64-127 split between them.
     const int pw = warp - kProdWarp0;
     const int64_t row_base = a.prefill ? (int64_t)g * a.S : a.seq_off[b] * a.Hkv + (int64_t)g * ks.len;
-    for (int j = 0; j < nt; ++j) {
+    bool stop = false;
+    for (int j0 = 0; j0 < nt && !stop; j0 += kPre) {
+#pragma unroll
+    for (int jj = 0; jj < kPre; ++jj) {
+      const int j = j0 + jj;
+      if (j >= nt) break;
       const int s = j % ST;
       int tc[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tc[i] = key_fix(a, ks, b, ks.kbeg + j * kKT + 4 * lane + i, raw_next[i], pw == 0);
-      if (j + 1 < nt) {  // next tile's entries: loads in flight while this tile is issued
+      for (int i = 0; i < 4; ++i) tc[i] = key_fix(a, ks, b, ks.kbeg + j * kKT + 4 * lane + i, raw[jj][i], pw == 0);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) raw_next[i] = key_raw(a, ks, b, ks.kbeg + (j + 1) * kKT + 4 * lane + i);
-      }
+      for (int i = 0; i < 4; ++i) raw[jj][i] = key_raw(a, ks, b, ks.kbeg + (j + kPre) * kKT + 4 * lane + i);
       bool ok = true;
       if (j >= ST && lane == 0) ok = mbar_wait(&kv_empty[s], ((j / ST) & 1) ^ 1, kWaitLimitNs);
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 0, j);
+        stop = true;
         break;
       }
       if (pw == 0) {
@@ -380,6 +392,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         tma_gather4(sbase + Lay::kQOff + (pw - 1) * Lay::kHalf + 4 * lane * 128, &tm_q, &kv_full[0], (pw - 1) * 64,
                     rq);
       }
+    }
     }
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer =======================
@@ -457,15 +470,19 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         tmem_ld32(tmem + sb * 128 + 64 * half + lane_base, sv);
         tmem_ld32(tmem + sb * 128 + 64 * half + 32 + lane_base, sv + 32);
         tmem_wait_ld();
-        float tmax = -INFINITY;
+        // row maximum over the visible keys: eight independent chains
+        float mx[8];
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) mx[c8] = -INFINITY;
         if (all_vis) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) tmax = fmaxf(tmax, __uint_as_float(sv[e]));
+          for (int e = 0; e < 64; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
         } else {
 #pragma unroll
           for (int e = 0; e < 64; ++e)
-            if ((vis[e >> 5] >> (e & 31)) & 1u) tmax = fmaxf(tmax, __uint_as_float(sv[e]));
+            if ((vis[e >> 5] >> (e & 31)) & 1u) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
         }
+        float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         tmax *= a.scale_log2;
         float alpha = 1.f;
         bool rescale = false;
@@ -497,7 +514,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         // p = 2^(s*scale*log2e - m_ref), bf16, over this half of the used K tile
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
         const uint32_t pst = sbase + Lay::kStageOff + s * Lay::kStageBytes + half * Lay::kHalf;
-        float lsum = 0.f;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums: short add chains
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {
           float p[8];
@@ -506,7 +523,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
             const int col = c16 * 8 + e;
             p[e] = ex2_approx(fmaf(__uint_as_float(sv[col]), a.scale_log2, neg_m));
             if (!all_vis && !((vis[col >> 5] >> (col & 31)) & 1u)) p[e] = 0.f;
-            lsum += p[e];
+            ls[e & 3] += p[e];
           }
           const uint32_t off = sw128_offset(r_loc, c16);
           st_shared_v4(pst + off, pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]),
@@ -519,7 +536,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
                          pack_bf16(q[2], q[3]), pack_bf16(q[4], q[5]), pack_bf16(q[6], q[7]));
           }
         }
-        l_run += lsum;
+        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         fence_proxy_async_smem();
       }
       tc_fence_before();
