@@ -353,6 +353,107 @@ def test_decode_step_plan_c3_matches_oracle(dev):
     assert torch.equal(idx2, idx) and torch.equal(O2.view(torch.int16), O.view(torch.int16))
 
 
+def _plan_inputs(cfg, wl):
+    """Per-layer lists of a whole-pattern step, as the benchmark builds them."""
+    n = cfg.L
+    grs = wl["groups"]
+    starts = [gr[0] for gr in cfg.groups]
+    qI = [grs[starts.index(l)]["qI"] if l in starts else None for l in range(n)]
+    w = [grs[starts.index(l)]["w"] if l in starts else None for l in range(n)]
+    KI = [grs[starts.index(l)]["KI"] if l in starts else None for l in range(n)]
+    gi = [max(i for i, s0 in enumerate(starts) if s0 <= l) for l in range(n)]
+    K = [grs[gi[l]]["K"] for l in range(n)]
+    V = [grs[gi[l]]["V"] for l in range(n)]
+    return qI, w, KI, K, V
+
+
+def test_decode_step_plan_c2_matches_oracle(dev):
+    """c2 through a DecodeStepPlan (three F groups of F,S,S,S, B = 8, S =
+    32768), as the benchmark would time it.  Every group's outputs, every
+    sequence, against the oracle over that group's index; the last group's
+    index and scores are also bit-equal to the standalone index-score and
+    top-k calls on the same inputs."""
+    cfg = synth.workload("c2")
+    wl = sgpu.decode_workload(cfg, dev)
+    qI, w, KI, K, V = _plan_inputs(cfg, wl)
+    plan = sa.DecodeStepPlan(cfg.pattern, qI, w, KI, K, V, wl["seq_off"], wl["seq_len"], cfg.S_max, cfg.k, wl["Q"],
+                             cfg.Hkv, cfg.scale, out_dtype=torch.float32)
+    plan.run()
+    O, idx = plan.run()  # a second run on the same workspace
+    torch.cuda.synchronize()
+    assert_status_ok(plan.ws)
+    O_h = O.cpu().numpy()
+    ws = sa.workspace(max(sa.lib().sa_topk_workspace_size(cfg.B, cfg.S_max, cfg.k),
+                          sa.lib().sa_index_score_workspace_size(cfg.B)), dev)
+    for g, layers in enumerate(cfg.groups):
+        gr = wl["groups"][g]
+        scores = sa.index_score(gr["qI"], gr["w"], gr["KI"], wl["seq_off"], wl["seq_len"], cfg.S_max, ws=ws)
+        idx_g = sa.topk(scores, wl["seq_len"], cfg.S_max, cfg.k, ws=ws)
+        if g == len(cfg.groups) - 1:
+            assert torch.equal(idx_g, idx), "the step's index differs from the standalone top-k's"
+            assert torch.equal(scores, plan.scores[:, :cfg.S_max])
+        check_group(cfg, g, list(range(cfg.B)), scores.cpu().numpy(), idx_g.cpu().numpy(),
+                    {torch.float32: O_h[layers[0]:layers[-1] + 1]})
+    assert_status_ok(ws)
+
+
+def test_decode_step_c5_group_matches_oracle(dev):
+    """One c5 group (B = 32, ragged 8192..131072, F,S,S,S) through the step.
+    Sampled sequences (shortest, longest, one more) against the oracle."""
+    cfg = synth.workload("c5")
+    wl = sgpu.decode_workload(cfg, dev, groups=[0])
+    gr = wl["groups"][0]
+    layers = list(cfg.groups[0])
+    n = len(layers)
+    Q = wl["Q"][layers[0]:layers[-1] + 1].contiguous()
+    plan = sa.DecodeStepPlan("F" + "S" * (n - 1), [gr["qI"]] + [None] * (n - 1), [gr["w"]] + [None] * (n - 1),
+                             [gr["KI"]] + [None] * (n - 1), [gr["K"]] * n, [gr["V"]] * n, wl["seq_off"],
+                             wl["seq_len"], cfg.S_max, cfg.k, Q, cfg.Hkv, cfg.scale, out_dtype=torch.bfloat16)
+    plan.run()
+    O, idx = plan.run()
+    torch.cuda.synchronize()
+    assert_status_ok(plan.ws)
+    lens = np.array(cfg.seq_lens)
+    seqs = [int(np.argmin(lens)), int(np.argmax(lens)), 7]
+    check_group(cfg, 0, seqs, plan.scores.cpu().numpy(), idx.cpu().numpy(), {torch.bfloat16: O.float().cpu().numpy()})
+
+
+def test_decode_step_does_not_depend_on_workspace_contents(dev):
+    """The workspace is scratch: a step on a workspace full of garbage (status
+    block clear) gives the same index and outputs, bit for bit, as on a
+    zeroed one, and as the general index-score and top-k calls."""
+    rng = np.random.default_rng(17)
+    lens, H_I, d_I, Hq, Hkv, d, k, pattern = [20000, 9000, 33000], 16, 128, 8, 2, 128, 512, "FSS"
+    B, L = len(lens), len(pattern)
+    seq_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    T = int(seq_off[-1])
+
+    def bf(shape, sd=1.0):
+        return bf16_dev(synth.f32_to_bf16_bits((rng.standard_normal(shape) * sd).astype(np.float32)), dev)
+
+    qI, KI, K, V, Q = bf((B, H_I, d_I), 1 / 8), bf((T, d_I), 1 / 8), bf(T * Hkv * d), bf(T * Hkv * d), bf((L, B, Hq, d))
+    w = torch.from_numpy(rng.uniform(0.1, 1.0, (B, H_I)).astype(np.float32)).to(dev)
+    d_off = torch.from_numpy(seq_off).to(dev)
+    d_len = torch.tensor(lens, dtype=torch.int32, device=dev)
+    S_max = max(lens)
+    none = [None] * (L - 1)
+    args = (pattern, [qI] + none, [w] + none, [KI] + none, [K] * L, [V] * L, d_off, d_len, S_max, k, Q, Hkv,
+            1 / math.sqrt(d))
+    gws = sa.workspace(max(sa.lib().sa_topk_workspace_size(B, S_max, k), sa.lib().sa_index_score_workspace_size(B)),
+                       dev)
+    want = sa.topk(sa.index_score(qI, w, KI, d_off, d_len, S_max, ws=gws), d_len, S_max, k, ws=gws)
+    nbytes = sa.decode_step_workspace_size(L, B, S_max, Hq, Hkv, d, k)
+    O0, idx0 = sa.decode_step(*args, out_dtype=torch.float32, ws=sa.workspace(nbytes, dev))
+    ws = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device=dev)
+    ws[:256] = 0  # a clear status block, garbage everywhere else
+    for trial in range(2):
+        O, idx = sa.decode_step(*args, out_dtype=torch.float32, ws=ws)
+        torch.cuda.synchronize()
+        assert_status_ok(ws)
+        assert torch.equal(idx, want) and torch.equal(idx, idx0), f"trial {trial}: index differs"
+        assert torch.equal(O, O0), f"trial {trial}: outputs differ"
+
+
 def test_decode_step_append_and_per_layer(dev):
     """The new token's rows land in the caches bit-exactly (nothing else
     changes), the step over the appended caches matches the oracle on them,
