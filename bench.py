@@ -43,6 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE = os.path.join(ROOT, "profiles", "indexer_decode_c3.md")
 L2_BYTES = 126 * 1024 * 1024  # B200 L2
 INDEXER_SRC = os.path.join(ROOT, "cross_layer_shared_b200", "csrc", "indexer.cu")
+CSRC_DIR = os.path.join(ROOT, "cross_layer_shared_b200", "csrc")
+STEP_PROFILE = os.path.join(ROOT, "profiles", "step_traffic_c3.md")
 
 
 def parse_args():
@@ -58,6 +60,8 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--out-f32", action="store_true", help="fp32 attention output instead of bf16")
+    p.add_argument("--no-others", action="store_true",
+                   help="skip the one-GPU timings of the other workloads (c1, c2, c5 decode; c4 prefill)")
     p.add_argument("--cp-ranks", type=int, default=8,
                    help="ranks of the emulated context-parallel step (single-group workloads, N=1; 0 = skip)")
     return p.parse_args()
@@ -144,6 +148,25 @@ def profile_traffic(workload: str):
         traffic = float(re.search(r"traffic_bytes_per_launch_full:\s*([0-9.eE+]+)", text).group(1))
         cur = hashlib.sha256(open(INDEXER_SRC, "rb").read()).hexdigest()
         return traffic if cur == sha else None
+    except Exception:
+        return None
+
+
+def step_traffic(workload: str, launches: int):
+    """ncu DRAM bytes (read + write) of one whole step, summed over its
+    launches, recorded in profiles/ for this workload while every kernel
+    source still matches the one profiled; None otherwise."""
+    try:
+        text = open(STEP_PROFILE).read()
+        if re.search(r"workload:\s*(\w+)", text).group(1) != workload:
+            return None
+        if int(re.search(r"launches_per_step:\s*(\d+)", text).group(1)) != launches:
+            return None
+        for name, sha in re.findall(r"source_sha256\[([\w.]+)\]:\s*([0-9a-f]+)", text):
+            cur = hashlib.sha256(open(os.path.join(CSRC_DIR, name), "rb").read()).hexdigest()
+            if cur != sha:
+                return None
+        return float(re.search(r"traffic_bytes_per_step:\s*([0-9.eE+]+)", text).group(1))
     except Exception:
         return None
 
@@ -321,20 +344,15 @@ def prefill_oracle_sample(cfg: synth.PrefillConfig, budget_s: float):
     return 1e3 * t_total / n * cfg.chunk, t_total, n, oracle.num_threads()
 
 
-def run_prefill(args):
+def prefill_device_timing(args, dev, cap):
+    """One c4 chunk (indexer, per-query top-k, block union + paged attention)
+    replayed from CUDA graphs: chunk and per-stage device times, FLOPs and
+    the tensors and calls the end-to-end leg reuses."""
     import torch
 
     import cross_layer_shared_b200 as sa
-    from cross_layer_shared_b200 import build
     from synth import gpu as sgpu
 
-    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
-        print(json.dumps({"workload": "c4", "error": "the prefill chunk runs on one GPU"}), flush=True)
-        return 0
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    build.build()
-    sa.lib()
     cfg = synth.workload("c4")
     wl = sgpu.prefill_workload(cfg, dev)
     out_dtype = torch.float32 if args.out_f32 else torch.bfloat16
@@ -369,7 +387,6 @@ def run_prefill(args):
         code, det = sa.read_status(w_)
         if code != 0:
             raise RuntimeError(f"device status {code} {det}")
-    cap = torch.cuda.Stream()
     graphs = {}
     for name, fn in (("chunk", chunk), ("indexer", run_index), ("topk", run_topk), ("attention", run_attn)):
         g = torch.cuda.CUDAGraph()
@@ -392,7 +409,7 @@ def run_prefill(args):
     warm = max(3, min(args.warmup, 10))
     for _ in range(warm):
         graphs["chunk"].replay()
-    with ClockSampler(0) as clocks:
+    with ClockSampler(dev.index or 0) as clocks:
         ms = timed(graphs["chunk"], steps)
     stage_ms = {name: timed(graphs[name], steps) for name in ("indexer", "topk", "attention")}
     ptr_h, ind_h = kv_indptr.cpu().numpy(), kv_indices.cpu().numpy()
@@ -405,6 +422,35 @@ def run_prefill(args):
     except Exception:
         peak, peak_kind = 1590.0, "fallback"
     attn_tf = attn_flops / (stage_ms["attention"] / 1e3) / 1e12
+
+    return {"cfg": cfg, "wl": wl, "O": O, "run_index": run_index, "run_topk": run_topk, "run_attn": run_attn,
+            "ms": ms, "stage_ms": stage_ms, "attn_flops": attn_flops, "idx_flops": idx_flops, "peak": peak,
+            "peak_kind": peak_kind, "attn_tf": attn_tf, "clocks": clocks, "union_blocks": int(ptr_h[1]),
+            "steps": steps, "warm": warm, "graphs": graphs}
+
+
+def run_prefill(args):
+    import torch
+
+    import cross_layer_shared_b200 as sa
+    from cross_layer_shared_b200 import build
+    from synth import gpu as sgpu
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        print(json.dumps({"workload": "c4", "error": "the prefill chunk runs on one GPU"}), flush=True)
+        return 0
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    build.build()
+    sa.lib()
+    cap = torch.cuda.Stream()
+    pt = prefill_device_timing(args, dev, cap)
+    cfg, wl, O = pt["cfg"], pt["wl"], pt["O"]
+    run_index, run_topk, run_attn = pt["run_index"], pt["run_topk"], pt["run_attn"]
+    ms, stage_ms, steps, warm = pt["ms"], pt["stage_ms"], pt["steps"], pt["warm"]
+    attn_flops, idx_flops, peak, peak_kind, attn_tf = (pt["attn_flops"], pt["idx_flops"], pt["peak"],
+                                                        pt["peak_kind"], pt["attn_tf"])
+    clocks = pt["clocks"]
 
     # end to end through the public API: host Q, qI, w in, host O out
     Q_h, qI_h, w_h = (wl["Q"].cpu().pin_memory(), wl["qI"].cpu().pin_memory(), wl["w"].cpu().pin_memory())
@@ -442,7 +488,7 @@ def run_prefill(args):
         "data": "synthetic (seeded counter-based generator, random init)",
         "config": {"workload": "c4: " + synth.DESCRIPTIONS["c4"], "queries": cfg.chunk, "context": cfg.S,
                    "top_k": cfg.k, "block": cfg.block, "heads": f"{cfg.Hq}q/{cfg.Hkv}kv", "head_dim": cfg.d,
-                   "union_blocks": int(ptr_h[1]), "l2": "scores (1.07 GB) and K/V (537 MB) exceed L2",
+                   "union_blocks": pt["union_blocks"], "l2": "scores (1.07 GB) and K/V (537 MB) exceed L2",
                    "parallelism": "single"},
         "roofline": {"kernel": "sparse_attn_kernel (paged prefill, with the block-union kernels)", "bound": "tensor",
                      "achieved": attn_tf, "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak, "traffic": None,
@@ -500,6 +546,91 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def build_decode_sets(cfg, dev, n_sets: int, out_dtype):
+    """n_sets independent device copies of a decode workload, each with the
+    per-layer lists a step takes and its own outputs and workspace."""
+    import torch
+
+    import cross_layer_shared_b200 as sa
+    from synth import gpu as sgpu
+
+    n = cfg.L
+    sets = []
+    for _ in range(n_sets):
+        wl = sgpu.decode_workload(cfg, dev)
+        grs = wl["groups"]
+        starts = [gr[0] for gr in cfg.groups]
+        qI = [grs[starts.index(l)]["qI"] if l in starts else None for l in range(n)]
+        w = [grs[starts.index(l)]["w"] if l in starts else None for l in range(n)]
+        KI = [grs[starts.index(l)]["KI"] if l in starts else None for l in range(n)]
+        gi = [max(i for i, s0 in enumerate(starts) if s0 <= l) for l in range(n)]
+        K = [grs[gi[l]]["K"] for l in range(n)]
+        V = [grs[gi[l]]["V"] for l in range(n)]
+        sets.append({"wl": wl, "qI": qI, "w": w, "KI": KI, "K": K, "V": V,
+                     "O": torch.empty((n, cfg.B, cfg.Hq, cfg.d), dtype=out_dtype, device=dev),
+                     "idx": torch.empty((cfg.B, cfg.k), dtype=torch.int32, device=dev),
+                     "scores": torch.empty((cfg.B, cfg.S_max), dtype=torch.float32, device=dev),
+                     "ws": sa.workspace(sa.decode_step_workspace_size(n, cfg.B, cfg.S_max, cfg.Hq, cfg.Hkv, cfg.d,
+                                                                      cfg.k), dev)})
+    return sets
+
+
+def decode_step_fn(cfg):
+    import cross_layer_shared_b200 as sa
+
+    def step(st, stream=None):
+        sa.decode_step(cfg.pattern, st["qI"], st["w"], st["KI"], st["K"], st["V"], st["wl"]["seq_off"],
+                       st["wl"]["seq_len"], cfg.S_max, cfg.k, st["wl"]["Q"], cfg.Hkv, cfg.scale, O=st["O"],
+                       idx=st["idx"], scores=st["scores"], ws=st["ws"], stream=stream)
+    return step
+
+
+def time_decode_workload(name: str, args, dev, cap, peak: float) -> dict:
+    """Device time of whole decode steps of another workload (one GPU):
+    CUDA graphs of 8 steps over alternating input sets, after warm-up."""
+    import torch
+
+    import cross_layer_shared_b200 as sa
+
+    cfg = synth.workload(name)
+    out_dtype = torch.float32 if args.out_f32 else torch.bfloat16
+    n_sets = 2 if 2 * set_bytes(cfg) < 0.5 * torch.cuda.mem_get_info()[0] else 1
+    sets = build_decode_sets(cfg, dev, n_sets, out_dtype)
+    step = decode_step_fn(cfg)
+    for st in sets:
+        step(st)
+    torch.cuda.synchronize()
+    for st in sets:
+        code, det = sa.read_status(st["ws"])
+        if code != 0:
+            raise RuntimeError(f"{name}: device status {code} {det}")
+    per_graph = 8
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for j in range(per_graph):
+            step(sets[j % len(sets)])
+    for _ in range(max(1, args.warmup // per_graph)):
+        g.replay()
+    torch.cuda.synchronize()
+    n_rep = max(3, min(200, args.steps // (4 * per_graph)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_rep):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (n_rep * per_graph)
+    nb = algorithmic_bytes(cfg, 4 if args.out_f32 else 2)
+    gbs = nb["total"] / (ms / 1e3) / 1e9
+    del g
+    out = {"value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms, "hbm_gbs": gbs, "hbm_frac": gbs / peak,
+           "algorithmic_bytes_per_step": nb["total"], "steps_timed": n_rep * per_graph, "input_sets": n_sets,
+           "workload": name + ": " + synth.DESCRIPTIONS[name]}
+    sets.clear()
+    torch.cuda.empty_cache()
+    return out
 
 
 def set_bytes(cfg) -> int:
@@ -641,29 +772,8 @@ def run_ours(args):
     nb = algorithmic_bytes(cfg, 4 if args.out_f32 else 2)
 
     args.sets = input_sets(cfg, args)
-    sets = []
-    for si in range(args.sets):
-        wl = sgpu.decode_workload(cfg, dev)
-        grs = wl["groups"]
-        starts = [gr[0] for gr in cfg.groups]
-        qI = [grs[starts.index(l)]["qI"] if l in starts else None for l in range(n)]
-        w = [grs[starts.index(l)]["w"] if l in starts else None for l in range(n)]
-        KI = [grs[starts.index(l)]["KI"] if l in starts else None for l in range(n)]
-        gi = [max(i for i, s0 in enumerate(starts) if s0 <= l) for l in range(n)]
-        K = [grs[gi[l]]["K"] for l in range(n)]
-        V = [grs[gi[l]]["V"] for l in range(n)]
-        st = {"wl": wl, "qI": qI, "w": w, "KI": KI, "K": K, "V": V,
-              "O": torch.empty((n, cfg.B, cfg.Hq, cfg.d), dtype=out_dtype, device=dev),
-              "idx": torch.empty((cfg.B, cfg.k), dtype=torch.int32, device=dev),
-              "scores": torch.empty((cfg.B, cfg.S_max), dtype=torch.float32, device=dev),
-              "ws": sa.workspace(sa.decode_step_workspace_size(n, cfg.B, cfg.S_max, cfg.Hq, cfg.Hkv, cfg.d, cfg.k),
-                                 dev)}
-        sets.append(st)
-
-    def step(st, stream=None):
-        sa.decode_step(cfg.pattern, st["qI"], st["w"], st["KI"], st["K"], st["V"], st["wl"]["seq_off"],
-                       st["wl"]["seq_len"], cfg.S_max, cfg.k, st["wl"]["Q"], cfg.Hkv, cfg.scale, O=st["O"],
-                       idx=st["idx"], scores=st["scores"], ws=st["ws"], stream=stream)
+    sets = build_decode_sets(cfg, dev, args.sets, out_dtype)
+    step = decode_step_fn(cfg)
 
     # eager run first (sets kernel attributes, checks status), then capture
     for st in sets:
@@ -936,6 +1046,30 @@ def run_ours(args):
                "sample": f"{nseq} whole sequences of this workload ({secs:.1f} s of CPU work: index score over every "
                          f"key, top-{cfg.k}, attention of all {cfg.L} layers); steps/s = sequences/{cfg.B}/s"}
 
+    peak, peak_kind = measured_peaks()
+    # ---- the other workloads on this GPU (N = 1): each decode workload's
+    # whole step and the c4 prefill chunk, device-timed from CUDA graphs ----
+    others = None
+    if world == 1 and not args.no_others:
+        e2e.clear()
+        graphs.clear()
+        sets.clear()
+        del multi, g_idx, g_topk, g_attn, g_seq
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        others = {}
+        for name in ("c1", "c2", "c5"):
+            if name != cfg.name:
+                others[name] = time_decode_workload(name, args, dev, cap, peak)
+        pt = prefill_device_timing(args, dev, cap)
+        others["c4"] = {"value": pt["ms"], "unit": "ms per chunk", "stage_ms": pt["stage_ms"],
+                        "attention_tflops": pt["attn_tf"], "attention_frac": pt["attn_tf"] / pt["peak"],
+                        "indexer_tflops": pt["idx_flops"] / (pt["stage_ms"]["indexer"] / 1e3) / 1e12,
+                        "peak_tflops": pt["peak"], "peak_kind": pt["peak_kind"],
+                        "workload": "c4: " + synth.DESCRIPTIONS["c4"]}
+        del pt
+        torch.cuda.empty_cache()
+
     if world > 1:
         graphs.clear()
         del multi, g_idx, g_topk, g_attn, g_seq
@@ -944,7 +1078,6 @@ def run_ours(args):
     if rank != 0:
         return 0
 
-    peak, peak_kind = measured_peaks()
     if route is not None:
         route["hbm_frac"] = route["hbm_gbs"] / world / peak
     step_gbs = nb["total"] / (ms_per_step / 1e3) / 1e9
@@ -959,10 +1092,17 @@ def run_ours(args):
         "config": workload_config(cfg, args),
         "hbm_gbs": step_gbs * world, "hbm_frac": step_gbs / peak, "hbm_peak_gbs": peak, "hbm_peak_kind": peak_kind,
         "algorithmic_bytes_per_step": nb,
-        "roofline": {"kernel": "indexer_decode_kernel", "bound": "hbm", "achieved": idx_gbs, "peak": peak,
-                     "unit": "GB/s", "frac": idx_gbs / peak, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": idx_bytes, "launch_ms": ms_idx,
-                     "peak_kind": f"{peak_kind} (burst copy, kernel timed alone)"},
+        # the metric's own roofline: one whole step (indexer, top-k and the
+        # group's attention, replayed from CUDA graphs) against the measured
+        # copy peak; the dominant HBM kernel's own figure sits beside it
+        "roofline": {"kernel": "decode step (indexer + top-k + one attention launch per fused group)",
+                     "bound": "hbm", "achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
+                     "traffic": step_traffic(cfg.name, launches_per_step),
+                     "algorithmic_bytes_per_launch": nb["total"], "launch_ms": ms_per_step,
+                     "peak_kind": f"{peak_kind} (burst copy)",
+                     "indexer": {"kernel": "indexer_decode_kernel", "bound": "hbm", "achieved": idx_gbs,
+                                 "peak": peak, "unit": "GB/s", "frac": idx_gbs / peak, "traffic": traffic,
+                                 "algorithmic_bytes_per_launch": idx_bytes, "launch_ms": ms_idx}},
         "kernels_ms": {"indexer": ms_idx, "topk": ms_topk, "attention_group": ms_attn},
         "per_layer_with_append": {"value": aggregate_rate(1, world, ms_seq), "unit": "steps/s", "ms_per_step": ms_seq,
                                   "launches_per_step": seq_launches,
@@ -971,6 +1111,7 @@ def run_ours(args):
                                           "decoder that computes layer l+1's queries from layer l runs it"},
         "attn_route": route,
         "context_parallel": cpar,
+        "other_workloads": others,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "per step: one pinned host -> device copy of that step's queries, indexer queries and "
