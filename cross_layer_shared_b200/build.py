@@ -55,24 +55,39 @@ def _compile(src: str, obj: str, extra=()) -> None:
     os.replace(obj + ".tmp", obj)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+TIMELINE_LIB = os.path.join(PKG, "libsa_timeline.so")
+
+
+def _build_lib(out: str, objdir: str, extra, force: bool) -> None:
+    os.makedirs(objdir, exist_ok=True)
     deps = _deps()
     jobs = []
     objs = []
     for s in SOURCES:
         src = os.path.join(CSRC, s)
-        obj = os.path.join(BUILD, s.replace(".cu", ".o"))
+        obj = os.path.join(objdir, s.replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, [src] + deps):
             jobs.append((src, obj))
     with cf.ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
-        for f in [ex.submit(_compile, s, o) for s, o in jobs]:
+        for f in [ex.submit(_compile, s, o, extra) for s, o in jobs]:
             f.result()
-    if force or _stale(LIB, objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB + ".tmp", *objs]
+    if force or _stale(out, objs):
+        cmd = [nvcc(), *ARCH, "-shared", "-o", out + ".tmp", *objs]
         subprocess.check_call(cmd)
-        os.replace(LIB + ".tmp", LIB)
+        os.replace(out + ".tmp", out)
+
+
+def build_timeline(force: bool = False) -> str:
+    """The tracing build (-DSA_TIMELINE, see csrc/timeline.cuh) as a library
+    of its own; the library proper is not touched."""
+    _build_lib(TIMELINE_LIB, os.path.join(BUILD, "timeline"), ("-DSA_TIMELINE",), force)
+    return TIMELINE_LIB
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    os.makedirs(BUILD, exist_ok=True)
+    _build_lib(LIB, BUILD, (), force)
     if force or _stale(SYNTH_LIB, [SYNTH_SRC]):
         cmd = [nvcc(), *NVFLAGS, "-shared", "-o", SYNTH_LIB + ".tmp", SYNTH_SRC]
         subprocess.check_call(cmd)

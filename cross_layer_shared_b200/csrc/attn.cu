@@ -40,6 +40,7 @@
 
 #include "attn.cuh"
 #include "sm100.cuh"
+#include "timeline.cuh"
 
 namespace sa {
 namespace {
@@ -226,6 +227,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   const int g = a.prefill ? bg : bg % a.Hkv;
 
   pdl_trigger();
+  if (tid == 0) SA_TL(kTlAttn, 0);
   if (warp == kMmaWarp) tmem_alloc(slot, 512);
   if (tid == 0) {
     tma_prefetch_desc(&tm_q);
@@ -248,9 +250,11 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
+  if (tid == 0) SA_TL(kTlAttn, 1);
 
   // everything below reads what earlier kernels of the stream wrote
   pdl_wait();
+  if (tid == 0) SA_TL(kTlAttn, 2);
   KeySrc ks;
   int n_keys;
   if (!a.prefill) {
@@ -352,6 +356,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
       const uint32_t tx = (a.prefill ? (pw == 0 ? 2 * Lay::kTile : 0) : Lay::kHalf + (uint32_t)(vhi - vlo) * 512u) +
                           (j == 0 && pw > 0 ? Lay::kHalf : 0);
       if (lane == 0) mbar_arrive_expect_tx(&kv_full[s], tx);
+      if (pw == 0 && lane == 0 && j < 8) SA_TL(kTlAttn, 3 + j);  // tile j issued
       __syncwarp();
       const uint32_t kst0 = sbase + Lay::kStageOff + s * Lay::kStageBytes;
       if (a.prefill) {
@@ -448,6 +453,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     for (int j = 0; j < nt; ++j) {
       const int s = j % ST, sb = j & 1;
       if (!warp_wait(&s_full[sb], (j >> 1) & 1)) { failed = true; break; }
+      if (tid == 0 && j < 8) SA_TL(kTlAttn, 12 + j);  // S of tile j ready
       tc_fence_after();
       if (warp_active) {
         if (!warp_wait(&kv_full[s], (j / ST) & 1)) { failed = true; break; }
@@ -537,6 +543,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
           }
         }
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        if (tid == 0 && j < 8) SA_TL(kTlAttn, 20 + j);  // P of tile j written
         fence_proxy_async_smem();
       }
       tc_fence_before();
@@ -560,6 +567,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   // ======================= output: all threads =======================
   tc_fence_before();
   __syncthreads();  // every MMA has completed (o_done) and no stage is in use
+  if (tid == 0) SA_TL(kTlAttn, 30);
   tc_fence_after();
   if (a.n_split > 1) {
     // this CTA's stages are free for its peers' slices: arm the receive
@@ -628,7 +636,9 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     const uint32_t recv = sbase + Lay::kStageOff;                      // [ns] slots, slot s from CTA s
     const uint32_t send = recv + ((ns * slot_bytes + 1023u) & ~1023u);  // [ns] slots, slot t for CTA t
     // every CTA is done with its stages and has armed its receive barrier
+    if (tid == 0) SA_TL(kTlAttn, 31);
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (tid == 0) SA_TL(kTlAttn, 32);
     if (warp_active) {
       const bool live = have_o && me.valid;
       if (half == 0)
@@ -663,7 +673,9 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     if (warp == kMmaWarp && lane < ns && lane != rank)
       bulk_copy_to_peer(recv + rank * slot_bytes, send + lane * slot_bytes, slot_bytes, recv_bar, lane);
     bool got = true;
+    if (tid == 0) SA_TL(kTlAttn, 33);
     if (warp < kSoftWarps) got = warp_wait(recv_bar, 0);
+    if (tid == 0) SA_TL(kTlAttn, 34);
     if (!got && lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 4, warp);
     // all that was sent to this CTA has landed; its own send slots are still
     // read by its peers' copies until every CTA of the cluster arrives here
@@ -710,12 +722,14 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         store_out(a, me.qoff + (rank * cw + ci) * 4, f, 4);
       }
     }
+    if (tid == 0) SA_TL(kTlAttn, 35);
     // every bulk copy out of this CTA has been consumed before it exits
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   }
 
   tc_fence_before();
   __syncthreads();
+  if (tid == 0) SA_TL(kTlAttn, 36);
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -757,3 +771,5 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& tm_q, const
 }
 
 }  // namespace sa
+
+SA_TL_SETTER(sa_timeline_set_attn)

@@ -23,6 +23,7 @@
 
 #include "indexer.cuh"
 #include "sm100.cuh"
+#include "timeline.cuh"
 
 namespace sa {
 namespace {
@@ -142,6 +143,7 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
 
   // ---- set-up: barriers and TMEM (overlaps the previous kernel's tail) ----
   pdl_trigger();
+  if (threadIdx.x == 0) SA_TL(kTlIndexer, 0);
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < kAcc; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
@@ -183,6 +185,7 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = prefix[B];
+  if (threadIdx.x == 0) SA_TL(kTlIndexer, 1);
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -279,6 +282,7 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
       // the new token's row, when this call appends it, is scored below from
       // its fresh key (the tile may hold the stale cache row)
       const int t_new = APPEND ? len - 1 : -1;
+      if (warp == 2 && lane == 0) SA_TL(kTlIndexer, 2 + (b < 12 ? b : 12));  // this CTA's last tile of b
       if (t < len && t != t_new) {
         float acc = 0.f;
 #pragma unroll
@@ -295,6 +299,7 @@ indexer_decode_kernel(const __grid_constant__ CUtensorMap tm_ki, const __grid_co
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) SA_TL(kTlIndexer, 15);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Lay::kTmemCols);
@@ -345,3 +350,5 @@ cudaError_t launch_indexer_decode(const IndexerArgs& a, const CUtensorMap& tm_ki
 }
 
 }  // namespace sa
+
+SA_TL_SETTER(sa_timeline_set_indexer)

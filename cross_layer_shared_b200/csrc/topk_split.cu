@@ -28,6 +28,7 @@
 #include <stdint.h>
 
 #include "sm100.cuh"
+#include "timeline.cuh"
 #include "status.cuh"
 #include "topk.cuh"
 
@@ -179,7 +180,9 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
     sm.cand_ctr = 0;
     sm.above_ctr = 0;
   }
+  if (tid == 0) SA_TL(kTlTopk, 0);
   pdl_wait();  // the scores come from the previous kernel of the stream
+  if (tid == 0) SA_TL(kTlTopk, 1);
   int n = n_valid[q];
   if (n < 0 || n > n_max) {
     if (c == 0 && tid == 0) report(status, kErrDevice, kKernTopk, q, n, n_max);
@@ -239,7 +242,9 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
     }
     if (tid == 0) sm.nlist = tot;
   }
+  if (tid == 0) SA_TL(kTlTopk, 2);
   cluster.sync();
+  if (tid == 0) SA_TL(kTlTopk, 3);
 
   // ---- phase A: row histogram, threshold bucket, this chunk's candidates ----
   for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
@@ -261,6 +266,7 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
   }
   __syncthreads();
   find_bin_desc(sm.hist, kBins1, k, sm.ws, &sm.bin, &sm.before);
+  if (tid == 0) SA_TL(kTlTopk, 4);
   const int beta = sm.bin, above = sm.before;
   uint2* my_spill = spill + (int64_t)blockIdx.x * chunk;
   const bool use_bits = chunk <= kBitWords * 32;
@@ -316,7 +322,9 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
       peer->peer_spill[c] = spilled;
     }
   }
+  if (tid == 0) SA_TL(kTlTopk, 5);
   cluster.sync();
+  if (tid == 0) SA_TL(kTlTopk, 6);
 
   // ---- phase B: exact k-th key, then this chunk's part of the output ----
   if (warp == 0) {  // candidate prefix over the chunks, keys above the bucket before this chunk
@@ -367,12 +375,14 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
     }
     __syncthreads();
   }
+  if (tid == 0) SA_TL(kTlTopk, 7);
   auto ckey = [&](int j) { return fast ? sm.row_cand[j].x : cand_at(j).x; };
   auto cidx = [&](int j) { return fast ? sm.row_cand[j].y : cand_at(j).y; };
   int need = k - above, n_eq = 0;
   const int ks[2] = {10, 0}, kw[2] = {10, 10};
   const uint32_t T = radix_desc(nc, ckey, [](int) { return true; }, (uint32_t)beta << 20, 0xFFF00000u, ks, kw, 2,
                                 &need, &n_eq, sm);
+  if (tid == 0) SA_TL(kTlTopk, 8);
   uint32_t cut = 0xFFFFFFFFu;
   if (need < n_eq) {
     // the `need` lowest indices among keys == T: largest values of ~index
@@ -392,6 +402,7 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
   int tot_sel_before;
   block_scan_excl(sel_before, sm.ws, &tot_sel_before);
   int written = above_before + tot_sel_before;
+  if (tid == 0) SA_TL(kTlTopk, 9);
   // The next kernel of the stream may start launching now, a few us before
   // this one ends, so its set-up overlaps the emission below.  Letting it
   // launch at entry put its waiting CTAs on the free SMs for the whole
@@ -438,7 +449,9 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(const float* __r
         ++pos;
       }
     }
+    if (tid == 0) SA_TL(kTlTopk, 10);
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    if (tid == 0) SA_TL(kTlTopk, 11);
     return;
   }
   for (int base0 = 0; base0 < len; base0 += kPass) {
@@ -562,3 +575,5 @@ cudaError_t launch_topk_split(const float* scores, int64_t ld, const int32_t* n_
 }
 
 }  // namespace sa
+
+SA_TL_SETTER(sa_timeline_set_topk)
