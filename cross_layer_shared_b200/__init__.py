@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libsa.so")
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, SA_ERR_TIMEOUT, SA_ERR_DEVICE = range(7)
 SA_BF16, SA_F32 = 0, 1
-WS_HEADER_BYTES = 256
+WS_HEADER_BYTES = 4096
 
 # every symbol include/sa.h declares, with its ctypes signature
 _P, _I, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float

@@ -526,9 +526,21 @@ sa_status sa_topk_dynamic(const float* scores, int64_t ld, const int32_t* n_vali
 }
 
 // ---------------------------------------------------------------- attention
+// The CUDA-core path (few rows per (b, g)): its per-(b, g) counters sit in the
+// workspace header after the status block, the slices' partials after it.
+constexpr size_t kSmallCounterOffset = 256;
+constexpr int kSmallMaxCounters = (int)((SA_WS_HEADER_BYTES - kSmallCounterOffset) / 4);
+
+bool small_attn_path(int L_g, int Hq, int Hkv) { return (int64_t)L_g * (Hq / Hkv) <= sa::kSmallMaxRows; }
+
+int small_attn_plan(int B, int Hkv, int k) { return sa::small_attn_splits(B * Hkv, k, num_sms(), kSmallMaxCounters); }
+
 size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int d, int k) {
   (void)d;
   if (L_g < 1 || B < 1 || Hkv < 1 || Hq < Hkv || k < 1) return SA_WS_HEADER_BYTES;
+  if (small_attn_path(L_g, Hq, Hkv))
+    return SA_WS_HEADER_BYTES +
+           sa::small_attn_scratch_bytes(B * Hkv, small_attn_plan(B, Hkv, k), L_g * (Hq / Hkv));
   return attn_ws_bytes(plan_decode_attn(L_g, B, Hq, Hkv, k));
 }
 
@@ -549,6 +561,42 @@ static sa_status run_decode_attn(const void* Q, const void* K, const void* V, co
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
     return fail(SA_ERR_INVALID_ARG, "%s: Q, K, V, O must be 16-byte aligned", who);
   if (!(scale > 0.f)) return fail(SA_ERR_INVALID_ARG, "%s: scale must be > 0", who);
+  if (!ml && !idx_count && small_attn_path(L_g, Hq, Hkv)) {
+    // few query rows per (b, g): the warp-level MMA kernel
+    const int ns = small_attn_plan(B, Hkv, k);
+    const size_t scratch = sa::small_attn_scratch_bytes(B * Hkv, ns, L_g * (Hq / Hkv));
+    sa_status st = check_ws(ws, ws_bytes, SA_WS_HEADER_BYTES + scratch, who);
+    if (st != SA_OK) return st;
+    sa::AttnArgs a{};
+    a.Q = reinterpret_cast<const uint16_t*>(Q);
+    a.K = reinterpret_cast<const uint16_t*>(K);
+    a.V = reinterpret_cast<const uint16_t*>(V);
+    a.seq_off = seq_off;
+    a.seq_len = seq_len;
+    a.idx = idx;
+    a.k = k;
+    a.L = L_g;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = Hq / Hkv;
+    a.R = L_g * a.G;
+    a.n_split = ns;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.O = O;
+    a.out_f32 = out_dtype == SA_F32;
+    a.status = status_of(ws);
+    if (ns > 1) {
+      uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+      const size_t n = (size_t)B * Hkv * ns * sa::small_attn_rows(a.R);
+      a.small_cnt = reinterpret_cast<uint32_t*>(base + kSmallCounterOffset);
+      a.small_po = reinterpret_cast<float*>(base + SA_WS_HEADER_BYTES);
+      a.small_pml = reinterpret_cast<float2*>(base + SA_WS_HEADER_BYTES + round_up(n * 128 * 4, 256));
+    }
+    cudaError_t e = sa::launch_sparse_attn_small(a, stream);
+    if (e != cudaSuccess) return cuda_fail("sa_sparse_decode_attn launch", e);
+    return SA_OK;
+  }
   const AttnPlan p = plan_decode_attn(L_g, B, Hq, Hkv, k);
   sa_status st = check_ws(ws, ws_bytes, attn_ws_bytes(p), who);
   if (st != SA_OK) return st;

@@ -49,6 +49,12 @@ struct AttnArgs {
   // decode, optional: idx_count[b] entries of idx row b are real, the rest
   // padding; the key splits then cover only those entries
   const int32_t* idx_count = nullptr;
+  // CUDA-core path with n_split > 1 key slices: per-(b, g) counters (zero
+  // between launches) and the slices' partials [B*Hkv][n_split][rows][d],
+  // (m, l) [B*Hkv][n_split][rows]
+  uint32_t* small_cnt = nullptr;
+  float* small_po = nullptr;
+  float2* small_pml = nullptr;
   DeviceStatus* status;
 };
 
@@ -58,5 +64,17 @@ int attn_num_units(const AttnArgs& a);
 // a time).  tm_k / tm_v in prefill: box 64 x 64 (one KV block per load).
 cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                const CUtensorMap& tm_v, bool precise_p, cudaStream_t stream);
+
+// Path for at most kSmallMaxRows query rows per (b, g) (decode, neither
+// partial outputs nor idx_count): warp-level MMA, one CTA per (b, g, key
+// slice).  small_attn_splits gives n_split for `units` = B*Hkv (1 when units
+// exceeds the counters available); with n_split > 1 the call needs
+// small_attn_scratch_bytes of workspace scratch and the counters.
+constexpr int kSmallMaxRows = 8;
+constexpr int kSmallMaxSplits = 16;
+int small_attn_rows(int R);
+int small_attn_splits(int units, int k, int sms, int max_counters);
+size_t small_attn_scratch_bytes(int units, int ns, int R);
+cudaError_t launch_sparse_attn_small(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace sa

@@ -15,7 +15,7 @@
 namespace sa {
 constexpr int kTimelineCtas = 4096;
 constexpr int kTimelineSlots = 64;
-enum : int { kTlIndexer = 0, kTlTopk = 1, kTlAttn = 2 };
+enum : int { kTlIndexer = 0, kTlTopk = 1, kTlAttn = 2, kTlAttnSmall = 3 };
 }  // namespace sa
 
 #ifdef SA_TIMELINE

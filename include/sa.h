@@ -39,11 +39,15 @@
  *   of touching memory outside the buffers.
  * - Workspace: `ws` must be 256-byte aligned and at least the size returned
  *   by the matching *_workspace_size() function.  Its first
- *   SA_WS_HEADER_BYTES bytes are the status block; zero them once when the
- *   workspace is allocated (the library only ever writes a non-zero code
- *   there, so the status is sticky until sa_clear_device_status()).  The
- *   rest is scratch owned by the call while it runs on `stream`: calls that
- *   overlap on the GPU must not share one workspace.
+ *   SA_WS_HEADER_BYTES bytes are the header: the status block (the first
+ *   256 bytes) and the slice counters of sa_sparse_decode_attn's path for
+ *   few rows per KV head.  Zero the header once when the workspace is
+ *   allocated: the library only ever writes a non-zero code into the status
+ *   block (so the status is sticky until sa_clear_device_status(), which
+ *   zeroes the whole header), and every launch leaves the counters it used
+ *   at zero when it ends.  The rest is scratch owned by the call while it
+ *   runs on `stream`: calls that overlap on the GPU must not share one
+ *   workspace.
  * - Between calls the library keeps only per-device facts it looks up once
  *   (the driver's tensor-map entry point, the SM count, the largest cluster
  *   the top-k kernel can be scheduled with, which kernels have had their
@@ -74,7 +78,7 @@ typedef int sa_status;
 
 typedef enum { SA_BF16 = 0, SA_F32 = 1 } sa_dtype;
 
-#define SA_WS_HEADER_BYTES 256
+#define SA_WS_HEADER_BYTES 4096
 
 /* Human-readable name of a status code (static string). */
 const char* sa_status_string(sa_status status);
@@ -221,7 +225,15 @@ sa_status sa_topk_dynamic(const float* scores, int64_t ld, const int32_t* n_vali
  *   O        [L_g, B, Hq, d], bf16 or fp32 per out_dtype
  * Each selected K/V row is brought from HBM once per (sequence, KV head)
  * for the whole group.  Supported: d = 128, Hq % Hkv == 0, Hq/Hkv <= 128.
- * Device errors: idx entry >= seq_len[b] -> SA_ERR_DEVICE, entry skipped.
+ * Two kernels: with L_g * Hq/Hkv > 8 rows per (sequence, KV head), 128-row
+ * tensor-core tiles (tcgen05; P rounded to bf16 for bf16 outputs, split in
+ * two bf16 parts for fp32 outputs); with at most 8 (one layer of a
+ * per-layer decoder), warp-level 16-row MMA tiles with P always split in
+ * two bf16 parts.  The second kernel splits the index entries of a
+ * (sequence, KV head) over several CTAs whose partials meet in the
+ * workspace scratch, counted on counters in the workspace header.
+ * Device errors: idx entry >= seq_len[b] -> SA_ERR_DEVICE, entry skipped;
+ * a bounded wait that gave up -> SA_ERR_TIMEOUT.
  * ---------------------------------------------------------------------- */
 size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int d, int k);
 sa_status sa_sparse_decode_attn(const void* Q, const void* K, const void* V, const int64_t* seq_off,

@@ -445,7 +445,7 @@ def test_decode_step_does_not_depend_on_workspace_contents(dev):
     nbytes = sa.decode_step_workspace_size(L, B, S_max, Hq, Hkv, d, k)
     O0, idx0 = sa.decode_step(*args, out_dtype=torch.float32, ws=sa.workspace(nbytes, dev))
     ws = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device=dev)
-    ws[:256] = 0  # a clear status block, garbage everywhere else
+    ws[:sa.WS_HEADER_BYTES] = 0  # a clear header (status block, counters), garbage everywhere else
     for trial in range(2):
         O, idx = sa.decode_step(*args, out_dtype=torch.float32, ws=ws)
         torch.cuda.synchronize()
@@ -496,12 +496,15 @@ def test_decode_step_append_and_per_layer(dev):
     assert np.abs(O.cpu().numpy() - O_gpu_idx).max() <= parity.ATOL_F32
     if np.array_equal(got_idx, used[0]):  # no tie inside the band moved the selection: the oracle's own walk too
         assert np.abs(O.cpu().numpy() - O_ora).max() <= parity.ATOL_F32
-    # the caches now hold the new token: per-layer launches against the fused group
+    # the caches now hold the new token: per-layer launches (R = G = 4 rows per
+    # (b, g): the CUDA-core kernel) against the fused group (R = 16: the
+    # tensor-core kernel) and against the oracle over the same index
     args = (pattern, [dqI] + none, [dw] + none, [dKI] + none, *common)
     O_fused, i_fused = sa.decode_step(*args, out_dtype=torch.float32)
     O_layer, i_layer = sa.decode_step(*args, out_dtype=torch.float32, per_layer=True)
     assert torch.equal(i_fused, i_layer)
-    assert torch.equal(O_fused, O_layer)
+    assert (O_fused - O_layer).abs().max().item() <= parity.ATOL_F32
+    assert np.abs(O_layer.cpu().numpy() - O_gpu_idx).max() <= parity.ATOL_F32
 
 
 def test_shared_index_equals_per_layer_recompute(dev):
@@ -514,7 +517,9 @@ def test_shared_index_equals_per_layer_recompute(dev):
     O1, i1 = sa.decode_step("FFFF", [gr["qI"]] * n, [gr["w"]] * n, [gr["KI"]] * n, *common, out_dtype=torch.float32)
     O2, i2 = sa.decode_step("FSSS", [gr["qI"]] * n, [gr["w"]] * n, [gr["KI"]] * n, *common, out_dtype=torch.float32)
     assert torch.equal(i1, i2)
-    assert torch.allclose(O1, O2, rtol=0, atol=1e-6)
+    # FFFF runs one layer per launch (8 rows per (b, g): the CUDA-core kernel),
+    # FSSS one launch of 32 rows (the tensor-core kernel)
+    assert (O1 - O2).abs().max().item() <= parity.ATOL_F32
 
 
 def test_step_is_deterministic(dev):
