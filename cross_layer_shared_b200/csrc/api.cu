@@ -548,7 +548,7 @@ static sa_status run_decode_attn(const void* Q, const void* K, const void* V, co
                                  const int32_t* seq_len, const int32_t* idx, int L_g, int B, int64_t n_tokens, int Hq,
                                  int Hkv, int d, int k, float scale, void* O, sa_dtype out_dtype, void* ws,
                                  size_t ws_bytes, cudaStream_t stream, float* ml = nullptr,
-                                 const int32_t* idx_count = nullptr) {
+                                 const int32_t* idx_count = nullptr, bool early = false) {
   const char* who = ml ? "sa_sparse_decode_attn_partial" : "sa_sparse_decode_attn";
   if (ml && (out_dtype != SA_F32 || !aligned(ml, 8)))
     return fail(SA_ERR_INVALID_ARG, "%s: partial outputs are fp32 and ml 8-byte aligned", who);
@@ -586,6 +586,7 @@ static sa_status run_decode_attn(const void* Q, const void* K, const void* V, co
     a.O = O;
     a.out_f32 = out_dtype == SA_F32;
     a.status = status_of(ws);
+    a.early = early ? 1 : 0;
     if (ns > 1) {
       uint8_t* base = reinterpret_cast<uint8_t*>(ws);
       const size_t n = (size_t)B * Hkv * ns * sa::small_attn_rows(a.R);
@@ -854,8 +855,10 @@ sa_status sa_decode_step_ex(const char* pattern, int n_layers, const void* const
   const size_t esize = out_dtype == SA_F32 ? 4 : 2;
   const size_t layer_elems = (size_t)B * Hq * d;
   int l = 0;
+  bool prev_small = false;  // the previous launch of this call was the few-rows attention kernel
   while (l < n_layers) {
     if (pattern[l] == 'F') {
+      prev_small = false;
       sa::AppendArgs ap{};
       if (new_KI) {
         ap.qI = static_cast<const uint16_t*>(qI[l]);
@@ -881,11 +884,15 @@ sa_status sa_decode_step_ex(const char* pattern, int n_layers, const void* const
     int m = l;
     if (!(flags & SA_STEP_PER_LAYER))
       while (m + 1 < n_layers && pattern[m + 1] == 'S' && K[m + 1] == K[l] && V[m + 1] == V[l]) ++m;
+    // after another launch of the few-rows kernel (which writes neither the
+    // index nor the caches), this one may start its loads before the wait
+    const bool small = small_attn_path(m - l + 1, Hq, Hkv);
     st = run_decode_attn(reinterpret_cast<const uint8_t*>(Q) + (size_t)l * layer_elems * 2, K[l], V[l], seq_off,
                          seq_len, idx, m - l + 1, B, n_tokens, Hq, Hkv, d, k, scale,
                          reinterpret_cast<uint8_t*>(O) + (size_t)l * layer_elems * esize, out_dtype, ws, ws_bytes,
-                         (cudaStream_t)stream);
+                         (cudaStream_t)stream, nullptr, nullptr, prev_small && small);
     if (st != SA_OK) return st;
+    prev_small = small;
     l = m + 1;
   }
   return SA_OK;

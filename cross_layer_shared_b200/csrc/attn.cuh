@@ -53,6 +53,11 @@ struct AttnArgs {
   // between launches) and the slices' partials [B*Hkv][n_split][rows][d],
   // (m, l) [B*Hkv][n_split][rows]
   uint32_t* small_cnt = nullptr;
+  // few-rows path: read idx, seq_off, seq_len, K and V (and start the first
+  // loads) before griddepcontrol.wait.  Only when the stream's previous
+  // kernel writes none of them and triggers its dependents after its own
+  // wait (a launch of this same path).
+  int early = 0;
   float* small_po = nullptr;
   float2* small_pml = nullptr;
   DeviceStatus* status;

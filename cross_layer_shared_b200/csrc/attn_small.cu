@@ -130,9 +130,6 @@ __global__ void __launch_bounds__(kThreadsS, 3) sparse_attn_small_kernel(const A
     g_sa_timeline[((size_t)kTlAttnSmall * kTimelineCtas + blockIdx.x) * kTimelineSlots + 16] = smid + 1;
   }
 #endif
-  pdl_trigger();
-  pdl_wait();  // the index comes from the top-k before this kernel
-  if (tid == 0) SA_TL(kTlAttnSmall, 1);
   // this CTA's entries: [rank*per, min(k, (rank+1)*per)), kSliceKeys at a time;
   // this warp's passes: entries e_beg + warp*16 + p*kSliceKeys + [0, 16)
   const int per = ((a.k + ns - 1) / ns + kKeysW - 1) / kKeysW * kKeysW;
@@ -144,41 +141,11 @@ __global__ void __launch_bounds__(kThreadsS, 3) sparse_attn_small_kernel(const A
   auto entry_raw = [&](int p) -> int {
     const int e = e_w + p * kSliceKeys + lane;
     if (lane >= kKeysW || p >= n_slice_pass || e >= e_end) return -1;
-    return __ldg(&a.idx[(int64_t)b * a.k + e]);
+    return __ldcg(&a.idx[(int64_t)b * a.k + e]);
   };
-  // the first two passes' entries travel with the sequence's length and
-  // offset and with the query
-  const int r0 = entry_raw(0), r1 = entry_raw(1);
-  const int len = a.seq_len[b];
-  const int64_t kv_base = (a.seq_off[b] * a.Hkv + (int64_t)g * len) * kD;
-  const uint16_t* Kb = a.K + kv_base;
-  const uint16_t* Vb = a.V + kv_base;
-  // query row gq (layer gq / G, head g*G + gq % G) as B fragments of Q^T:
-  // for k-step 2i + h, b0 = dims 32i + 8tq + 4h + {0, 1}, b1 = .. + {2, 3};
-  // rows gq >= R are zero.  Kept in shared memory, read back each pass.
-  if (warp == 0) {
-    uint4 q4[4] = {};
-    if (gq < a.R) {
-      const int h = g * a.G + gq % a.G, l = gq / a.G;
-      const uint4* qp = reinterpret_cast<const uint4*>(a.Q + (((int64_t)l * a.B + b) * a.Hq + h) * kD + 8 * tq);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) q4[i] = __ldg(qp + 4 * i);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sm.qb[lane][i] = q4[i];
-  }
-  if (tid < R) {
-    const int h = g * a.G + tid % a.G, l = tid / a.G;
-    sm.out_off[tid] = (((int64_t)l * a.B + b) * a.Hq + h) * kD;
-  }
-  __syncthreads();
-  if (tid == 0) SA_TL(kTlAttnSmall, 2);
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // rows 2tq, 2tq + 1
-  float o[8][4];  // O^T: dims 16mt + gq (+8 for [2], [3]) at rows 2tq ([0], [2]) and 2tq + 1
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-  // (no pass when the sequence is empty: padding entries stage row 0)
-  const int n_pass = len > 0 ? n_slice_pass : 0;
+  int len = 0, n_pass = 0, t0 = -1, t1 = -1, r1 = -1;
+  const uint16_t* Kb = nullptr;
+  const uint16_t* Vb = nullptr;
   auto entry_check = [&](int p, int raw) -> int {
     if (raw >= len) {
       report(a.status, kErrDevice, kKernAttn, (int64_t)b * a.k + e_w + p * kSliceKeys + lane, raw, len);
@@ -206,16 +173,59 @@ __global__ void __launch_bounds__(kThreadsS, 3) sparse_attn_small_kernel(const A
       const int tk = max(__shfl_sync(0xffffffffu, tt, 8 * nt + gq), 0);
       const uint4* kp = reinterpret_cast<const uint4*>(Kb + (int64_t)tk * kD + 8 * tq);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) kb[nt][i] = __ldg(kp + 4 * i);
+      for (int i = 0; i < 4; ++i) kb[nt][i] = __ldcg(kp + 4 * i);
     }
   };
-  // pipeline: pass p computes while pass p+1's K and V loads and pass p+2's
-  // entries are in flight
-  int t0 = entry_check(0, r0), t1 = entry_check(1, r1);
-  if (n_pass > 0) {
-    stage_v(t0, 0);
-    load_k(t0);
+  // the first two passes' entries, the sequence's place in the cache, and
+  // pass 0's K and V loads (pass p computes while pass p+1's loads and pass
+  // p+2's entries are in flight)
+  auto prologue = [&]() {
+    const int r0 = entry_raw(0);
+    r1 = entry_raw(1);
+    len = __ldcg(&a.seq_len[b]);
+    const int64_t kv_base = (__ldcg(&a.seq_off[b]) * a.Hkv + (int64_t)g * len) * kD;
+    Kb = a.K + kv_base;
+    Vb = a.V + kv_base;
+    n_pass = len > 0 ? n_slice_pass : 0;  // none for an empty sequence: padding stages row 0
+    t0 = entry_check(0, r0);
+    if (n_pass > 0) {
+      stage_v(t0, 0);
+      load_k(t0);
+    }
+  };
+  // early: the stream's previous kernel writes none of idx, seq_off,
+  // seq_len, K and V, and lets this one start only after its own wait, so
+  // they are complete: the first loads overlap that kernel's tail
+  if (a.early) prologue();
+  pdl_wait();     // the previous kernel of the stream is complete
+  pdl_trigger();  // after the wait: a following early launch relies on it
+  if (tid == 0) SA_TL(kTlAttnSmall, 1);
+  if (!a.early) prologue();
+  // query row gq (layer gq / G, head g*G + gq % G) as B fragments of Q^T:
+  // for k-step 2i + h, b0 = dims 32i + 8tq + 4h + {0, 1}, b1 = .. + {2, 3};
+  // rows gq >= R are zero.  Kept in shared memory, read back each pass.
+  if (warp == 0) {
+    uint4 q4[4] = {};
+    if (gq < a.R) {
+      const int h = g * a.G + gq % a.G, l = gq / a.G;
+      const uint4* qp = reinterpret_cast<const uint4*>(a.Q + (((int64_t)l * a.B + b) * a.Hq + h) * kD + 8 * tq);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) q4[i] = __ldcg(qp + 4 * i);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sm.qb[lane][i] = q4[i];
   }
+  if (tid < R) {
+    const int h = g * a.G + tid % a.G, l = tid / a.G;
+    sm.out_off[tid] = (((int64_t)l * a.B + b) * a.Hq + h) * kD;
+  }
+  __syncthreads();
+  if (tid == 0) SA_TL(kTlAttnSmall, 2);
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // rows 2tq, 2tq + 1
+  float o[8][4];  // O^T: dims 16mt + gq (+8 for [2], [3]) at rows 2tq ([0], [2]) and 2tq + 1
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  t1 = entry_check(1, r1);
   if (tid == 0) SA_TL(kTlAttnSmall, 3);
   for (int p = 0; p < n_pass; ++p) {
     const uint32_t live = __ballot_sync(0xffffffffu, t0 >= 0);
