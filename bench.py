@@ -699,11 +699,19 @@ def context_parallel_section(cfg, st, N, cap, dev, reps: int = 16, iters: int = 
         same_idx &= got == [int(t) for t in idx_h[b] if t >= 0]
     max_abs = (O_cp.float() - O1.float()).abs().max().item()
     for r in ranks:
-        for ws in (r.ws_index, r.ws_topk, r.ws_sel, r.ws_attn):
+        for ws in (r.ws_index, r.ws_radix, r.ws_attn):
             code, det = sa.read_status(ws)
             if code != 0:
                 raise RuntimeError(f"context-parallel device status {code} {det}")
-    cand = torch.stack([r.cand for r in ranks])
+    # every rank's histograms of each exchange level, and its partials, as
+    # the all-gathers of that step delivered them
+    for r in ranks:
+        r.scores_local(qI, w)
+    gathered = [torch.stack([r.radix_level(0) for r in ranks])]
+    gathered.append(torch.stack([r.radix_level(1, gathered[0]) for r in ranks]))
+    gathered.append(torch.stack([r.radix_level(2, gathered[1]) for r in ranks]))
+    for r in ranks:
+        r.radix_select(gathered[2])
     parts = torch.stack([r.part for r in ranks])
     O = torch.empty_like(O1)
 
@@ -722,27 +730,35 @@ def context_parallel_section(cfg, st, N, cap, dev, reps: int = 16, iters: int = 
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / (iters * reps)
 
+    def select(r):
+        r.radix_level(0)
+        r.radix_level(1, gathered[0])
+        r.radix_level(2, gathered[1])
+        r.radix_select(gathered[2])
+
     def chain(r):
-        r.candidates(qI, w)
-        r.select(cand)
+        r.scores_local(qI, w)
+        select(r)
         r.partial(Q)
         r.combine(parts, O)
 
     per_rank = [graph_ms(lambda r=r: chain(r)) for r in ranks]
     slow = ranks[max(range(N), key=lambda i: per_rank[i])]
-    phases = {"candidates": graph_ms(lambda: slow.candidates(qI, w)), "select": graph_ms(lambda: slow.select(cand)),
+    phases = {"scores": graph_ms(lambda: slow.scores_local(qI, w)), "select": graph_ms(lambda: select(slow)),
               "partial_attention": graph_ms(lambda: slow.partial(Q)),
               "combine": graph_ms(lambda: slow.combine(parts, O))}
-    cand_b, part_b = ranks[0].cand.numel() * 4, ranks[0].part.numel() * 4
+    hist_b = sum(h.numel() * 4 for h in ranks[0].hist)
+    part_b = ranks[0].part.numel() * 4
     return {"ranks": N, "context_per_rank": [int(x) for x in (bnd[:, :, 1] - bnd[:, :, 0]).max(1)],
             "ms_per_rank_step_max": max(per_rank), "ms_per_rank_step": per_rank, "phases_ms_slowest_rank": phases,
             "selected_per_rank": [int((x >= 0).sum().item()) for x in local],
-            "allgather_bytes_per_rank": {"candidates": cand_b, "partials": part_b},
-            "allgather_bytes_received_per_rank": (N - 1) * (cand_b + part_b),
-            "launches_per_rank_step": 7, "same_index_as_one_device": bool(same_idx),
+            "allgather_bytes_per_rank": {"histograms": hist_b, "partials": part_b},
+            "allgather_bytes_received_per_rank": (N - 1) * (hist_b + part_b),
+            "launches_per_rank_step": 7, "collectives_per_rank_step": 4, "same_index_as_one_device": bool(same_idx),
             "max_abs_vs_one_device": max_abs,
-            "note": "every rank emulated on one GPU; the two all-gathers are not timed (one GPU): add their "
-                    "NVLink time for the received bytes; one group of all layers shares the index"}
+            "note": "every rank emulated on one GPU; the four all-gathers (three histogram levels, the partials) "
+                    "are not timed (one GPU): add their NVLink time for the received bytes; one group of all "
+                    "layers shares the index"}
 
 
 def run_ours(args):
@@ -912,9 +928,9 @@ def run_ours(args):
 
     # ---- context-parallel decode, every rank emulated on this GPU: each
     # sequence's context sharded over cp_ranks ranks; a rank's step is its
-    # indexer + top-k over its slice, the global selection over all ranks'
-    # candidates, attention over its share, and the merge of all partials.
-    # The two all-gathers between the phases are not run (one GPU): their
+    # indexer over its slice, the global selection by three histogram
+    # levels, attention over its share, and the merge of all partials.
+    # The four all-gathers between the phases are not run (one GPU): their
     # bytes per rank are reported instead ----
     cpar = None
     if world == 1 and len(cfg.groups) == 1 and args.cp_ranks > 1:

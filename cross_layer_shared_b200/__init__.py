@@ -60,6 +60,9 @@ SIGNATURES = {
     "sa_cp_select_workspace_size": ([_I, _I, _I], _SZ),
     "sa_cp_select": ([_P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "sa_combine_partials": ([_P, _I64, _P, _I64, _I, _I64, _I, _P, _I, _P], _I),
+    "sa_cp_radix_workspace_size": ([_I], _SZ),
+    "sa_cp_radix_level": ([_P, _I64, _P, _I, _I, _I, _I, _P, _I64, _P, _P, _SZ, _P], _I),
+    "sa_cp_radix_select": ([_P, _I64, _P, _I, _I, _I, _I, _P, _I64, _P, _P, _P, _SZ, _P], _I),
 }
 
 
@@ -342,6 +345,73 @@ def cp_select(cand_scores, cand_idx, rank: int, local_idx=None, local_count=None
     _ws(ws)
     _check(lib().sa_cp_select(_ptr(cand_scores), _ptr(cand_idx), stride, N, B, k, int(rank), _ptr(local_idx),
                               _ptr(local_count), _ptr(ws), ws.numel(), _stream(stream)))
+    return local_idx
+
+
+RADIX_BINS = (4096, 4096, 256)  # histogram bins of the exchange's levels 0, 1, 2
+
+
+def cp_radix_workspace_size(B: int) -> int:
+    return int(lib().sa_cp_radix_workspace_size(B))
+
+
+def _gathered(gathered, N: int, B: int, bins: int, what: str):
+    if gathered is None:
+        return None, 0
+    if not (gathered.is_cuda and gathered.dtype == torch.int32 and gathered.dim() == 3
+            and tuple(gathered.shape) == (N, B, bins) and gathered.stride()[1:] == (bins, 1)):
+        raise ValueError(f"{what}: gathered histograms must be int32 CUDA [N, B, {bins}] with [B, {bins}] blocks")
+    return gathered, (gathered.stride(0) if N > 1 else B * bins)
+
+
+def cp_radix_level(scores, n_local, k: int, N: int, level: int, gathered=None, hist_out=None, ws=None,
+                   stream=None) -> torch.Tensor:
+    """One level of the histogram exchange (levels 0, 1, 2): the previous
+    level's threshold from `gathered` (every rank's histograms of it, int32
+    [N, B, bins]; None at level 0), then this rank's histogram of the level's
+    digit over its scores fp32 [B, ld] (entries [0, n_local[b])).  Returns
+    hist_out int32 [B, 4096] (levels 0, 1) or [B, 256] (level 2).  `ws`
+    (cp_radix_workspace_size) carries the state across the step's calls."""
+    B = n_local.shape[0]
+    _rows_out(scores, B, 1, "scores")
+    _dev(n_local, torch.int32, "n_local")
+    if level not in (0, 1, 2):
+        raise ValueError("level must be 0, 1 or 2")
+    if (gathered is None) != (level == 0):
+        raise ValueError("gathered histograms are needed at levels 1 and 2 only")
+    g, stride = _gathered(gathered, N, B, RADIX_BINS[level - 1], "cp_radix_level") if level else (None, 0)
+    if hist_out is None:
+        hist_out = torch.empty((B, RADIX_BINS[level]), dtype=torch.int32, device=scores.device)
+    _out(hist_out, (B, RADIX_BINS[level]), (torch.int32,), "hist_out")
+    if ws is None:
+        raise ValueError("cp_radix_level needs the step's workspace (it carries the state across levels)")
+    _ws(ws)
+    _check(lib().sa_cp_radix_level(_ptr(scores), scores.stride(0), _ptr(n_local), B, int(k), int(N), int(level),
+                                   _ptr(g), stride, _ptr(hist_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return hist_out
+
+
+def cp_radix_select(scores, n_local, k: int, N: int, rank: int, gathered, local_idx=None, local_count=None, ws=None,
+                    stream=None) -> torch.Tensor:
+    """The exchange's last call: the level-2 threshold from `gathered`
+    (int32 [N, B, 256]), then this rank's entries of the global top-k as
+    local indices [B, k] (ascending, -1 padded; their number into
+    local_count int32 [B] if given)."""
+    B = n_local.shape[0]
+    _rows_out(scores, B, 1, "scores")
+    _dev(n_local, torch.int32, "n_local")
+    g, stride = _gathered(gathered, N, B, RADIX_BINS[2], "cp_radix_select")
+    if local_idx is None:
+        local_idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+    _out(local_idx, (B, k), (torch.int32,), "local_idx")
+    if local_count is not None:
+        _out(local_count, (B,), (torch.int32,), "local_count")
+    if ws is None:
+        raise ValueError("cp_radix_select needs the step's workspace (it carries the state across levels)")
+    _ws(ws)
+    _check(lib().sa_cp_radix_select(_ptr(scores), scores.stride(0), _ptr(n_local), B, int(k), int(N), int(rank),
+                                    _ptr(g), stride, _ptr(local_idx), _ptr(local_count), _ptr(ws), ws.numel(),
+                                    _stream(stream)))
     return local_idx
 
 

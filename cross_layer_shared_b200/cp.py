@@ -5,15 +5,20 @@ que cela signifie pour l'inference sur longs contextes").  This is the
 plainest sharding that gives the one-GPU result: rank r keeps the contiguous
 slice [lo_r(b), hi_r(b)) of every sequence b in its own packed caches, and a
 decode step over one layer group (one index shared by the group's layers)
-takes two all-gathers:
+takes four all-gathers:
 
-1. indexer scores + top-k (with scores) over the local slice -> candidates;
-2. all-gather of the candidates ([N][scores | idx], k x 8 bytes per sequence
-   and rank);
-3. sa_cp_select: the global top-k of the N*k candidates, mapped back to
-   this rank's local indices;
-4. sparse attention over the local selected rows, left unnormalised (o, m, l);
-5. all-gather of the partials; sa_combine_partials (log-sum-exp merge).
+1. indexer scores over the local slice;
+2. the global top-k by a radix select whose histograms are summed over the
+   ranks: three levels (key bits [31:20], [19:8], [7:0]), each this rank's
+   histogram of the level's digit (sa_cp_radix_level) all-gathered, the
+   next level finding the previous threshold from the gathered histograms;
+   sa_cp_radix_select then keeps this rank's share as local indices;
+3. sparse attention over the local selected rows, left unnormalised (o, m, l);
+4. all-gather of the partials; sa_combine_partials (log-sum-exp merge).
+
+A histogram exchange carries 16 KB per sequence and level (1 KB at the last
+level) whatever k is; sa_cp_select (still exported) is the earlier design:
+every rank's top-k candidates gathered and selected again.
 
 Every rank ends with the whole output.  The arithmetic runs in libsa's
 kernels; this module holds the slicing, the buffer layout and the order of
@@ -27,7 +32,7 @@ One process per GPU (e.g. under torchrun), each holding its slices:
     me = CPRank(N, rank, KI_slice, K_slice, V_slice, hi - lo, k, H_I, d_I, Hq, Hkv, d, L_g, scale)
     O = step(me, nccl_exchange(N), qI, w, Q)      # the same O on every rank
 
-Every rank makes the same two collectives in the same order each step.
+Every rank makes the same four collectives in the same order each step.
 """
 from __future__ import annotations
 
@@ -37,8 +42,8 @@ import numpy as np
 import torch
 import torch.distributed as dist
 
-from . import (combine_partials, cp_select, cp_select_workspace_size, index_score, sparse_decode_attn_partial,
-               sparse_decode_attn_workspace_size, topk, workspace)
+from . import (RADIX_BINS, combine_partials, cp_radix_level, cp_radix_select, cp_radix_workspace_size, index_score,
+               sparse_decode_attn_partial, sparse_decode_attn_workspace_size, workspace)
 from . import lib
 
 
@@ -91,7 +96,8 @@ def part_views(buf: torch.Tensor, rows: int, d: int) -> Tuple[torch.Tensor, torc
 
 def cand_views(buf: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
     """(scores fp32, idx int32) views of packed candidate blocks buf int32
-    [..., 2, B, k]: the scores are bit-cast in [..., 0, :, :]."""
+    [..., 2, B, k] (sa_cp_select's input): the scores are bit-cast in
+    [..., 0, :, :]."""
     return buf[..., 0, :, :].view(torch.float32), buf[..., 1, :, :]
 
 
@@ -118,33 +124,37 @@ class CPRank:
         self.seq_off, self.seq_len = seq_tables(local_len, dev)
         B = self.B
         self.scores = torch.empty((B, max(self.S_max, 1)), dtype=torch.float32, device=dev)
-        # candidates: [scores | idx] as one int32 block, all-gathered as is
-        self.cand = torch.empty((2, B, k), dtype=torch.int32, device=dev)
+        # this rank's histogram of each exchange level, all-gathered as is
+        self.hist = [torch.empty((B, bins), dtype=torch.int32, device=dev) for bins in RADIX_BINS]
         self.rows = L_g * B * Hq
         self.part_floats = part_floats(self.rows, d)
         self.part = torch.empty(self.part_floats, dtype=torch.float32, device=dev)
         self.local_idx = torch.empty((B, k), dtype=torch.int32, device=dev)
         self.local_count = torch.empty(B, dtype=torch.int32, device=dev)
         self.ws_index = workspace(int(lib().sa_index_score_workspace_size(B)), dev)
-        self.ws_topk = workspace(int(lib().sa_topk_workspace_size(B, self.S_max, k)), dev)
-        self.ws_sel = workspace(cp_select_workspace_size(N, B, k), dev)
+        self.ws_radix = workspace(cp_radix_workspace_size(B), dev)
         self.ws_attn = workspace(sparse_decode_attn_workspace_size(L_g, B, Hq, Hkv, d, k), dev)
 
-    def candidates(self, qI: torch.Tensor, w: torch.Tensor, stream=None) -> torch.Tensor:
-        """Indexer scores and top-k over the local slice, into self.cand."""
+    def scores_local(self, qI: torch.Tensor, w: torch.Tensor, stream=None) -> torch.Tensor:
+        """Indexer scores over the local slice, into self.scores."""
         if self.S_max > 0:
             index_score(qI, w, self.KI, self.seq_off, self.seq_len, self.S_max, scores=self.scores,
                         ws=self.ws_index, stream=stream)
-        scores, idx = cand_views(self.cand)
-        topk(self.scores, self.seq_len, self.S_max, self.k, idx=idx, top_scores=scores, ws=self.ws_topk,
-             stream=stream)
-        return self.cand
+        return self.scores
 
-    def select(self, gathered: torch.Tensor, stream=None) -> torch.Tensor:
-        """gathered int32 [N, 2, B, k] -> this rank's share of the global top-k."""
-        scores, idx = cand_views(gathered)
-        return cp_select(scores, idx, self.rank, local_idx=self.local_idx, local_count=self.local_count,
-                         ws=self.ws_sel, stream=stream)
+    def radix_level(self, level: int, gathered: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Exchange level 0, 1 or 2: the previous level's threshold from every
+        rank's histograms `gathered` int32 [N, B, bins] (levels 1, 2), then
+        this rank's histogram of the level, into self.hist[level]."""
+        return cp_radix_level(self.scores, self.seq_len, self.k, self.N, level, gathered, hist_out=self.hist[level],
+                              ws=self.ws_radix, stream=stream)
+
+    def radix_select(self, gathered: torch.Tensor, stream=None) -> torch.Tensor:
+        """gathered int32 [N, B, 256] (level 2) -> this rank's share of the
+        global top-k, into self.local_idx and self.local_count."""
+        return cp_radix_select(self.scores, self.seq_len, self.k, self.N, self.rank, gathered,
+                               local_idx=self.local_idx, local_count=self.local_count, ws=self.ws_radix,
+                               stream=stream)
 
     def partial(self, Q: torch.Tensor, stream=None) -> torch.Tensor:
         """Unnormalised attention over the local selected rows, into self.part."""
@@ -178,6 +188,15 @@ def nccl_exchange(N: int, group=None) -> Exchange:
     return exchange
 
 
+def select(rank_state: CPRank, exchange: Exchange, stream=None) -> torch.Tensor:
+    """This rank's share of the global top-k from its scores: three histogram
+    levels, each all-gathered, then the selection."""
+    h = rank_state.radix_level(0, None, stream)
+    h = rank_state.radix_level(1, exchange(h), stream)
+    h = rank_state.radix_level(2, exchange(h), stream)
+    return rank_state.radix_select(exchange(h), stream)
+
+
 def step(rank_state: CPRank, exchange: Exchange, qI: torch.Tensor, w: torch.Tensor, Q: torch.Tensor,
          O: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
     """One context-parallel decode step of a layer group on this rank.
@@ -185,8 +204,8 @@ def step(rank_state: CPRank, exchange: Exchange, qI: torch.Tensor, w: torch.Tens
     qI bf16 [B, H_I, d_I], w fp32 [B, H_I]: the group's indexer query (the
     same on every rank); Q bf16 [L_g, B, Hq, d]: the group's queries.  Every
     rank returns the whole O [L_g, B, Hq, d]."""
-    cand = rank_state.candidates(qI, w, stream)
-    rank_state.select(exchange(cand), stream)
+    rank_state.scores_local(qI, w, stream)
+    select(rank_state, exchange, stream)
     part = rank_state.partial(Q, stream)
     return rank_state.combine(exchange(part), O, out_dtype, stream)
 
@@ -195,9 +214,13 @@ def emulate_step(ranks: Sequence[CPRank], qI: torch.Tensor, w: torch.Tensor, Q: 
                  out_dtype=torch.bfloat16, stream=None) -> Tuple[torch.Tensor, List[torch.Tensor]]:
     """All N ranks of a step on one device, phase by phase (no kernel waits on
     another rank's): returns rank 0's O and every rank's local index."""
-    cand = torch.stack([r.candidates(qI, w, stream) for r in ranks])
     for r in ranks:
-        r.select(cand, stream)
+        r.scores_local(qI, w, stream)
+    h = torch.stack([r.radix_level(0, None, stream) for r in ranks])
+    h = torch.stack([r.radix_level(1, h, stream) for r in ranks])
+    h = torch.stack([r.radix_level(2, h, stream) for r in ranks])
+    for r in ranks:
+        r.radix_select(h, stream)
     parts = torch.stack([r.partial(Q, stream) for r in ranks])
     return ranks[0].combine(parts, None, out_dtype, stream), [r.local_idx for r in ranks]
 

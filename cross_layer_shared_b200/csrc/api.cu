@@ -773,6 +773,58 @@ sa_status sa_cp_select(const float* cand_scores, const int32_t* cand_idx, int64_
   return SA_OK;
 }
 
+size_t sa_cp_radix_workspace_size(int B) {
+  if (B < 1) return SA_WS_HEADER_BYTES;
+  return SA_WS_HEADER_BYTES + round_up((size_t)B * sizeof(sa::CpRadixState), 256);
+}
+
+static sa_status cp_radix_check(const float* scores, int64_t ld, const int32_t* n_local, int B, int k, int N,
+                                int level, const int32_t* gathered, int64_t rank_stride, void* ws, size_t ws_bytes,
+                                const char* who) {
+  if (B < 1 || k < 1 || N < 1) return fail(SA_ERR_INVALID_ARG, "%s: B, k, N must be >= 1", who);
+  if (N > 1024) return fail(SA_ERR_UNSUPPORTED, "%s: N=%d above 1024 ranks", who, N);
+  if (!scores || !n_local) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (ld < 1) return fail(SA_ERR_INVALID_ARG, "%s: ld must be >= 1", who);
+  if (level > 0) {
+    const int64_t prev = level == 3 ? 256 : 4096;  // bins of the level whose histograms are gathered
+    if (!gathered) return fail(SA_ERR_INVALID_ARG, "%s: NULL gathered histograms", who);
+    if (N > 1 && rank_stride < (int64_t)B * prev)
+      return fail(SA_ERR_INVALID_ARG, "%s: rank_stride=%lld below B*%lld", who, (long long)rank_stride,
+                  (long long)prev);
+  }
+  return check_ws(ws, ws_bytes, sa_cp_radix_workspace_size(B), who);
+}
+
+sa_status sa_cp_radix_level(const float* scores, int64_t ld, const int32_t* n_local, int B, int k, int N, int level,
+                            const int32_t* gathered, int64_t rank_stride, int32_t* hist_out, void* ws,
+                            size_t ws_bytes, void* stream) {
+  const char* who = "sa_cp_radix_level";
+  if (level < 0 || level > 2) return fail(SA_ERR_INVALID_ARG, "%s: level=%d outside [0, 2]", who, level);
+  if (!hist_out) return fail(SA_ERR_INVALID_ARG, "%s: NULL hist_out", who);
+  sa_status st = cp_radix_check(scores, ld, n_local, B, k, N, level, gathered, rank_stride, ws, ws_bytes, who);
+  if (st != SA_OK) return st;
+  auto* state = reinterpret_cast<sa::CpRadixState*>(reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES);
+  cudaError_t e = sa::launch_cp_radix_level(scores, ld, n_local, B, k, N, level, gathered, rank_stride, state,
+                                            hist_out, status_of(ws), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail("sa_cp_radix_level launch", e);
+  return SA_OK;
+}
+
+sa_status sa_cp_radix_select(const float* scores, int64_t ld, const int32_t* n_local, int B, int k, int N, int rank,
+                             const int32_t* gathered, int64_t rank_stride, int32_t* local_idx, int32_t* local_count,
+                             void* ws, size_t ws_bytes, void* stream) {
+  const char* who = "sa_cp_radix_select";
+  if (N >= 1 && (rank < 0 || rank >= N)) return fail(SA_ERR_INVALID_ARG, "%s: rank=%d outside [0, %d)", who, rank, N);
+  if (!local_idx) return fail(SA_ERR_INVALID_ARG, "%s: NULL local_idx", who);
+  sa_status st = cp_radix_check(scores, ld, n_local, B, k, N, 3, gathered, rank_stride, ws, ws_bytes, who);
+  if (st != SA_OK) return st;
+  auto* state = reinterpret_cast<const sa::CpRadixState*>(reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES);
+  cudaError_t e = sa::launch_cp_radix_finish(scores, ld, n_local, B, k, N, rank, gathered, rank_stride, state,
+                                             local_idx, local_count, status_of(ws), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail("sa_cp_radix_select launch", e);
+  return SA_OK;
+}
+
 sa_status sa_combine_partials(const float* O_part, int64_t o_stride, const float* ml, int64_t ml_stride, int P,
                               int64_t rows, int d, void* O, sa_dtype out_dtype, void* stream) {
   const char* who = "sa_combine_partials";

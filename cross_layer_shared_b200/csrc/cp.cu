@@ -18,6 +18,8 @@
 #include <stdint.h>
 
 #include "cp.cuh"
+#include "sm100.cuh"
+#include "status.cuh"
 
 namespace sa {
 namespace {
@@ -129,7 +131,340 @@ __global__ void combine_partials_kernel(const float* __restrict__ parts, int64_t
   }
 }
 
+
+// ---------------------------------------------------------------- radix exchange
+// The global top-k by exchanging histograms instead of candidates.  Scores
+// map to 32-bit keys that order like the floats (-0 == +0); the k-th largest
+// key T is found digit by digit, 12 + 12 + 8 bits, from the histograms of
+// every rank (summed on every rank alike):
+//   level 0: digit key[31:20] of every local key;
+//   level 1: digit key[19:8] of the local keys whose key[31:20] is the
+//            level-0 threshold digit;
+//   level 2: digit key[7:0] of the keys matching the 24-bit prefix.
+// The threshold digit of a level is the one where the count of larger keys,
+// summed over the ranks, first reaches the number still needed.  After
+// level 2 the prefix is T itself: a rank keeps its keys above T, and of its
+// keys equal to T the ones the lower-index rule gives it: ties go to lower
+// global indices, that is, to lower ranks first (slices are in rank order),
+// then to lower local indices.  When all ranks together hold no more than k
+// valid keys, every one is kept.
+
+constexpr int kRadixThreads = 1024;
+constexpr int kRadixBins = 4096;
+constexpr int kPer = 16;  // entries per thread per round
+
+__device__ __forceinline__ uint32_t cp_order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;  // -0 == +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ int level_bins(int level) { return level == 2 ? 256 : kRadixBins; }
+
+// digit of `key` at `level`, or -1 if key does not match the prefix found so far
+__device__ __forceinline__ int level_digit(uint32_t key, int level, uint32_t prefix) {
+  if (level == 0) return (int)(key >> 20);
+  if (level == 1) return (key >> 20) == prefix ? (int)((key >> 8) & 0xFFFu) : -1;
+  return (key >> 8) == prefix ? (int)(key & 0xFFu) : -1;
+}
+
+struct RadixSmem {
+  int hist[kRadixBins];
+  int wsum[kRadixThreads / 32 + 1];
+  CpRadixState st;
+};
+
+// Block-wide: exclusive prefix sum of v over the CTA's threads in thread order.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* wsum, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = lane < kRadixThreads / 32 ? wsum[lane] : 0;
+    int z = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, z, o);
+      if (lane >= o) z += y;
+    }
+    wsum[lane] = z - w;
+    if (lane == 31) wsum[kRadixThreads / 32] = z;
+  }
+  __syncthreads();
+  total = wsum[kRadixThreads / 32];
+  return wsum[warp] + x - v;
+}
+
+// The threshold digit of the previous level from every rank's histogram of
+// it (gathered [N] blocks of [B][bins] ints, rank_stride ints apart): the
+// digit where the keys above, summed over the ranks, are fewer than the
+// number needed and the keys above and at it are not; st.prefix grows by
+// that digit and st.need drops by the count above it.  Fewer keys than
+// needed in all: st.all = 1.  Also returns, through *at_digit, the digit.
+__device__ void radix_threshold(const int32_t* __restrict__ gathered, int64_t rank_stride, int N, int b, int bins,
+                                RadixSmem& sm, int* at_digit) {
+  {
+    // this thread's (up to) 4 digits of every rank: all loads independent
+    int acc[4] = {0, 0, 0, 0};
+#pragma unroll 4
+    for (int r = 0; r < N; ++r) {
+      const int32_t* g = gathered + r * rank_stride + (int64_t)b * bins;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = threadIdx.x + u * kRadixThreads;
+        if (i < bins) acc[u] += __ldcg(&g[i]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = threadIdx.x + u * kRadixThreads;
+      if (i < bins) sm.hist[i] = acc[u];
+    }
+  }
+  __syncthreads();
+  // thread j owns the digits bins-1-per*j .. bins-per*(j+1) (descending)
+  const int per = bins / kRadixThreads > 0 ? bins / kRadixThreads : 1;
+  const int j0 = threadIdx.x * per;
+  int mine = 0;
+  for (int u = 0; u < per; ++u)
+    if (j0 + u < bins) mine += sm.hist[bins - 1 - (j0 + u)];
+  int total = 0;
+  int above = block_exclusive_scan(mine, sm.wsum, total);
+  const int need = sm.st.need;
+  __syncthreads();
+  if (total < need) {
+    if (threadIdx.x == 0) {
+      sm.st.all = 1;
+      *at_digit = -1;
+    }
+  } else {
+    for (int u = 0; u < per && j0 + u < bins; ++u) {
+      const int dgt = bins - 1 - (j0 + u);
+      const int c = sm.hist[dgt];
+      if (above < need && above + c >= need) {  // exactly one thread, one digit
+        sm.st.prefix = (sm.st.prefix << (bins == 256 ? 8 : 12)) | (uint32_t)dgt;
+        sm.st.need = need - above;
+        *at_digit = dgt;
+      }
+      above += c;
+    }
+  }
+  __syncthreads();
+}
+
+// One CTA per sequence: the threshold of level-1 (if level > 0), then this
+// rank's histogram of level `level` into hist_out [B][bins].
+__global__ void __launch_bounds__(kRadixThreads) cp_radix_level_kernel(
+    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_local, int k, int N, int level,
+    const int32_t* __restrict__ gathered, int64_t rank_stride, CpRadixState* __restrict__ state,
+    int32_t* __restrict__ hist_out, DeviceStatus* status) {
+  __shared__ RadixSmem sm;
+  __shared__ int digit;
+  const int b = blockIdx.x, lane = threadIdx.x & 31;
+  pdl_wait();
+  const int n_raw = __ldcg(&n_local[b]);
+  const int n = n_raw > 0 ? n_raw : 0;
+  const float* row = scores + (int64_t)b * ld;
+  // the first round's scores travel while the threshold is found
+  float v[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = u * kRadixThreads + threadIdx.x;
+    v[u] = i < n ? __ldcg(&row[i]) : 0.f;
+  }
+  if (threadIdx.x == 0) {
+    if (level == 0) {
+      sm.st.prefix = 0;
+      sm.st.need = k;
+      sm.st.all = 0;
+      sm.st.pad = 0;
+    } else {
+      sm.st = state[b];
+    }
+  }
+  __syncthreads();
+  if (level > 0 && !sm.st.all) radix_threshold(gathered, rank_stride, N, b, kRadixBins, sm, &digit);
+  const int bins = level_bins(level);
+  for (int i = threadIdx.x; i < bins; i += kRadixThreads) sm.hist[i] = 0;
+  __syncthreads();
+  pdl_trigger();
+  if (n_raw < 0 && threadIdx.x == 0) report(status, kErrDevice, kKernCp, b, n_raw, 0);
+  if (!sm.st.all) {
+    const uint32_t prefix = sm.st.prefix;
+    for (int base = 0; base < n; base += kRadixThreads * kPer) {
+      if (base > 0) {
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+          const int i = base + u * kRadixThreads + threadIdx.x;
+          v[u] = i < n ? __ldcg(&row[i]) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = base + u * kRadixThreads + threadIdx.x;
+        const int dgt = i < n ? level_digit(cp_order_key(v[u]), level, prefix) : -1;
+        // scores of one row share their top digits: when the whole warp
+        // holds one digit, one atomic adds it (same-address atomics
+        // serialise); otherwise each lane adds its own
+        const int d0 = __shfl_sync(0xffffffffu, dgt, 0);
+        if (__all_sync(0xffffffffu, dgt == d0)) {
+          if (lane == 0 && d0 >= 0) atomicAdd(&sm.hist[d0], 32);
+        } else if (dgt >= 0) {
+          atomicAdd(&sm.hist[dgt], 1);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < bins; i += kRadixThreads) hist_out[(int64_t)b * bins + i] = sm.hist[i];
+  if (threadIdx.x == 0) state[b] = sm.st;
+}
+
+// One CTA per sequence: the level-2 threshold, then this rank's entries of
+// the global top-k as ascending local indices (then -1) and their count.
+__global__ void __launch_bounds__(kRadixThreads) cp_radix_finish_kernel(
+    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_local, int k, int N, int rank,
+    const int32_t* __restrict__ gathered, int64_t rank_stride, const CpRadixState* __restrict__ state,
+    int32_t* __restrict__ local_idx, int32_t* __restrict__ count, DeviceStatus* status) {
+  __shared__ RadixSmem sm;
+  __shared__ int digit;
+  __shared__ int take;
+  const int b = blockIdx.x;
+  pdl_wait();
+  const int n_raw = __ldcg(&n_local[b]);
+  const int n = n_raw > 0 ? n_raw : 0;
+  const float* row = scores + (int64_t)b * ld;
+  // a round: warp w owns the 32*kPer consecutive entries base + w*32*kPer ..,
+  // entry u*32 + lane of them in lane `lane` (coalesced loads; (u, lane)
+  // order within a warp, warp order across, is index order).  The first
+  // round's scores travel while the threshold is found.
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  float v[kPer];
+  {
+    const int w0 = warp * 32 * kPer + lane;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) v[u] = w0 + u * 32 < n ? __ldcg(&row[w0 + u * 32]) : 0.f;
+  }
+  if (threadIdx.x == 0) {
+    sm.st = state[b];
+    digit = -1;
+    take = 0;
+  }
+  __syncthreads();
+  if (!sm.st.all) radix_threshold(gathered, rank_stride, N, b, 256, sm, &digit);
+  const bool all = sm.st.all != 0;
+  const uint32_t T = sm.st.prefix;  // the k-th largest key (when not all)
+  if (!all) {
+    // ties at T: the ranks before this one take theirs first (every rank's
+    // count at the digit, loaded in parallel)
+    if (threadIdx.x < N) sm.hist[threadIdx.x] = __ldcg(&gathered[threadIdx.x * rank_stride + (int64_t)b * 256 + digit]);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int before = 0;
+      for (int r = 0; r < rank; ++r) before += sm.hist[r];
+      const int t = sm.st.need - before, mine = sm.hist[rank];
+      take = t < 0 ? 0 : (t > mine ? mine : t);
+    }
+  }
+  __syncthreads();
+  pdl_trigger();
+  if (n_raw < 0 && threadIdx.x == 0) report(status, kErrDevice, kKernCp, b, n_raw, 0);
+  int32_t* out = local_idx + (int64_t)b * k;
+  int kept = 0, ties = 0;  // before this round
+  const int take_t = take;
+  for (int base = 0; base < n; base += kRadixThreads * kPer) {
+    const int w0 = base + warp * 32 * kPer + lane;
+    if (base > 0) {
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) v[u] = w0 + u * 32 < n ? __ldcg(&row[w0 + u * 32]) : 0.f;
+    }
+    uint32_t gtb[kPer], eqb[kPer];  // warp-uniform masks per u
+    int weq = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      bool g = false, e = false;
+      if (w0 + u * 32 < n) {
+        const uint32_t key = cp_order_key(v[u]);
+        g = all || key > T;
+        e = !all && key == T;
+      }
+      gtb[u] = __ballot_sync(0xffffffffu, g);
+      eqb[u] = __ballot_sync(0xffffffffu, e);
+      weq += __popc(eqb[u]);
+    }
+    // ties before this warp (this round), then each lane's tie ordinal
+    int tot_eq = 0;
+    const int eq_scan = block_exclusive_scan(lane == 0 ? weq : 0, sm.wsum, tot_eq);
+    int tie = ties + __shfl_sync(0xffffffffu, eq_scan, 0);
+    uint32_t keepb[kPer];
+    int wkeep = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const bool mine_eq = (eqb[u] >> lane) & 1u;
+      const bool k_lane = ((gtb[u] >> lane) & 1u) || (mine_eq && tie + __popc(eqb[u] & lt) < take_t);
+      keepb[u] = __ballot_sync(0xffffffffu, k_lane);
+      tie += __popc(eqb[u]);
+      wkeep += __popc(keepb[u]);
+    }
+    int tot_keep = 0;
+    const int keep_scan = block_exclusive_scan(lane == 0 ? wkeep : 0, sm.wsum, tot_keep);
+    int pos = kept + __shfl_sync(0xffffffffu, keep_scan, 0);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if ((keepb[u] >> lane) & 1u) {
+        const int p = pos + __popc(keepb[u] & lt);
+        if (p < k) out[p] = w0 + u * 32;
+      }
+      pos += __popc(keepb[u]);
+    }
+    kept += tot_keep;
+    ties += tot_eq;
+  }
+  const int cnt = kept < k ? kept : k;
+  for (int j = cnt + threadIdx.x; j < k; j += kRadixThreads) out[j] = -1;
+  if (threadIdx.x == 0 && count != nullptr) count[b] = cnt;
+}
 }  // namespace
+
+cudaError_t launch_cp_radix_level(const float* scores, int64_t ld, const int32_t* n_local, int B, int k, int N,
+                                  int level, const int32_t* gathered, int64_t rank_stride, CpRadixState* state,
+                                  int32_t* hist_out, DeviceStatus* status, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)B);
+  cfg.blockDim = dim3(kRadixThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, cp_radix_level_kernel, scores, ld, n_local, k, N, level, gathered,
+                                     rank_stride, state, hist_out, status);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cp_radix_finish(const float* scores, int64_t ld, const int32_t* n_local, int B, int k, int N,
+                                   int rank, const int32_t* gathered, int64_t rank_stride, const CpRadixState* state,
+                                   int32_t* local_idx, int32_t* count, DeviceStatus* status, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)B);
+  cfg.blockDim = dim3(kRadixThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, cp_radix_finish_kernel, scores, ld, n_local, k, N, rank, gathered,
+                                     rank_stride, state, local_idx, count, status);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_cp_gather(const float* cand_scores, const int32_t* cand_idx, int64_t stride, int N, int B, int k,
                              float* rows, int32_t* n_valid, cudaStream_t stream) {

@@ -31,6 +31,7 @@ enum : int {
   kKernIndexerPrefill = 6,
   kKernRoute = 7,
   kKernWaitProbe = 8,
+  kKernCp = 9,
 };
 
 struct DeviceStatus {

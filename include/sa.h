@@ -432,6 +432,46 @@ sa_status sa_sparse_decode_attn_partial(const void* Q, const void* K, const void
                                         float* O_part, float* ml, void* ws, size_t ws_bytes,
                                         void* stream);
 
+/* The global top-k by exchanging histograms (the context-parallel step's
+ * selection; replaces steps 1-3 above after the local sa_index_score).
+ * Scores map to 32-bit keys ordered like the floats (-0 == +0); the k-th
+ * largest key T over all ranks is found digit by digit, key bits [31:20],
+ * [19:8], [7:0], each digit the one where the count of larger keys summed
+ * over the ranks' histograms first reaches the number still needed (the
+ * radix select of sa_topk, with the ranks' histograms summed).  A rank then
+ * keeps its keys above T and, of its keys equal to T, those the lower-index
+ * rule gives it: slices are in rank order, so ties go to the lower ranks,
+ * then to the lower local indices.  The union over ranks is exactly
+ * sa_topk's selection over the whole context (all valid keys when there
+ * are at most k).  A step, every rank alike:
+ *   sa_cp_radix_level(level 0) -> hist [B][4096]; all-gather (rank-major);
+ *   sa_cp_radix_level(level 1, the gathered level-0 histograms) -> [B][4096];
+ *   all-gather; sa_cp_radix_level(level 2, gathered level 1) -> [B][256];
+ *   all-gather; sa_cp_radix_select(the gathered level-2 histograms).
+ *   scores     fp32 [B, ld]: this rank's indexer scores over its slice,
+ *              entries [0, n_local[b]) of row b
+ *   n_local    int32 [B] (device): this rank's slice length per sequence
+ *   gathered   every rank's histograms of the previous level, rank r's
+ *              [B][bins] block at element offset r * rank_stride (bins 4096
+ *              for levels 0 and 1, 256 for level 2); NULL at level 0
+ *   hist_out   int32 [B][4096] (levels 0, 1) or [B][256] (level 2)
+ *   local_idx  int32 [B, k] out: this rank's entries of the global top-k,
+ *              as local indices, ascending, then -1
+ *   local_count int32 [B] out (nullable): their number (the idx_count of
+ *              sa_sparse_decode_attn_partial)
+ * The workspace (sa_cp_radix_workspace_size, one per rank) carries the
+ * per-sequence state from each call to the next: keep it for the step's
+ * four calls.  1 <= N <= 1024.  Device errors: n_local[b] < 0 ->
+ * SA_ERR_DEVICE, the row counts as empty.  One CTA of 1024 threads per
+ * sequence per call. */
+size_t sa_cp_radix_workspace_size(int B);
+sa_status sa_cp_radix_level(const float* scores, int64_t ld, const int32_t* n_local, int B, int k, int N,
+                            int level, const int32_t* gathered, int64_t rank_stride, int32_t* hist_out,
+                            void* ws, size_t ws_bytes, void* stream);
+sa_status sa_cp_radix_select(const float* scores, int64_t ld, const int32_t* n_local, int B, int k, int N,
+                             int rank, const int32_t* gathered, int64_t rank_stride, int32_t* local_idx,
+                             int32_t* local_count, void* ws, size_t ws_bytes, void* stream);
+
 /* Global top-k over the gathered candidates.
  *   cand_scores, cand_idx  rank r's top_scores (fp32 [B, k]) and idx (int32
  *               [B, k]) from sa_topk over its slice: each idx row ascending,

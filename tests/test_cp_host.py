@@ -72,9 +72,32 @@ def test_rank_state_rejects_empty_slices_and_bad_ranks():
 
 
 # ---------------------------------------------------------------- two ranks over gloo
+def _order_keys(sc):
+    """fp32 scores -> the 32-bit keys the kernels order them by (-0 == +0)."""
+    u = np.ascontiguousarray(sc, dtype=np.float32).view(np.uint32).copy()
+    u[u == 0x80000000] = 0
+    return np.where(u & 0x80000000, ~u, u | 0x80000000).astype(np.uint32)
+
+
+def _threshold(g, prefix, need, all_, bits):
+    """The previous level's threshold digit from every rank's histograms g
+    [N, bins]: where the keys above, summed over the ranks, first reach
+    `need`.  Returns (prefix, need, all, digit)."""
+    if all_:
+        return prefix, need, True, -1
+    tot = g.sum(0)
+    above = 0
+    for dgt in range(len(tot) - 1, -1, -1):
+        if above + int(tot[dgt]) >= need:
+            return (prefix << bits) | dgt, need - above, False, dgt
+        above += int(tot[dgt])
+    return prefix, need, True, -1
+
+
 class OracleRank:
-    """A rank whose arithmetic is the oracle's (CPU), with CPRank's interface
-    and exchange layouts."""
+    """A rank whose arithmetic runs on the CPU (the oracle's scores and
+    attention; the exchange's histograms and thresholds in numpy), with
+    CPRank's interface and exchange layouts."""
 
     def __init__(self, N, rank, KI, K, V, local_len, k, Hkv, d, L_g, Hq, scale):
         self.N, self.rank, self.k = N, rank, k
@@ -85,19 +108,48 @@ class OracleRank:
         self.B = len(local_len)
         self.rows = L_g * self.B * Hq
 
-    def candidates(self, qI, w, stream=None):
-        B = self.B
-        sc = oracle.index_score(qI, w, self.KI, self.off, np.arange(B), self.len - 1, ld=int(self.len.max()))
-        idx, ts = oracle.topk(sc, self.len, self.k, with_scores=True)
-        buf = torch.empty((2, B, self.k), dtype=torch.int32)
-        s, i = cp.cand_views(buf)
-        s.copy_(torch.from_numpy(ts))
-        i.copy_(torch.from_numpy(idx))
-        return buf
+    def scores_local(self, qI, w, stream=None):
+        self.sc = oracle.index_score(qI, w, self.KI, self.off, np.arange(self.B), self.len - 1,
+                                     ld=max(int(self.len.max()), 1))
+        return self.sc
 
-    def select(self, gathered, stream=None):
-        s, i = cp.cand_views(gathered)
-        self.local_idx = oracle.cp_select(s.numpy(), i.numpy(), self.rank)
+    def radix_level(self, level, gathered=None, stream=None):
+        bins = (4096, 4096, 256)[level]
+        if level == 0:
+            self.state = [(0, self.k, False)] * self.B
+        else:
+            g = gathered.numpy()
+            self.state = [_threshold(g[:, b], *self.state[b], 12)[:3] for b in range(self.B)]
+        hist = np.zeros((self.B, bins), np.int32)
+        for b in range(self.B):
+            prefix, need, all_ = self.state[b]
+            if all_:
+                continue
+            key = _order_keys(self.sc[b, :self.len[b]])
+            if level == 0:
+                dg = key >> 20
+            elif level == 1:
+                dg = (key[key >> 20 == prefix] >> 8) & 0xFFF
+            else:
+                dg = key[key >> 8 == prefix] & 0xFF
+            hist[b] = np.bincount(dg.astype(np.int64), minlength=bins)
+        return torch.from_numpy(hist)
+
+    def radix_select(self, gathered, stream=None):
+        g = gathered.numpy()
+        self.local_idx = np.full((self.B, self.k), -1, np.int32)
+        for b in range(self.B):
+            T, need, all_, dgt = _threshold(g[:, b], *self.state[b], 8)
+            key = _order_keys(self.sc[b, :self.len[b]])
+            if all_:
+                keep = np.ones(len(key), bool)
+            else:
+                before = int(g[:self.rank, b, dgt].sum())
+                take = min(max(need - before, 0), int(g[self.rank, b, dgt]))
+                eq = key == T
+                keep = (key > T) | (eq & (np.cumsum(eq) - 1 < take))
+            sel = np.nonzero(keep)[0]
+            self.local_idx[b, :len(sel)] = sel
         return self.local_idx
 
     def partial(self, Q, stream=None):
@@ -188,13 +240,18 @@ def _oracle_ranks(world):
 def test_the_exchange_order_matters(order):
     """All ranks in one process, phase by phase: rank-major gathers give the
     one-device result; gathering in reverse rank order (a plausible layout
-    slip) breaks the selection's tie rule and the local index mapping."""
+    slip) breaks the selection's tie rule: the ties at the threshold go to
+    the wrong ranks."""
     world = 3
     ranks, qI, w, Q = _oracle_ranks(world)
     flip = (lambda t: t.flip(0)) if order == "reversed" else (lambda t: t)
-    cand = flip(torch.stack([r.candidates(qI, w) for r in ranks]))
     for r in ranks:
-        r.select(cand)
+        r.scores_local(qI, w)
+    h = flip(torch.stack([r.radix_level(0) for r in ranks]))
+    h = flip(torch.stack([r.radix_level(1, h) for r in ranks]))
+    h = flip(torch.stack([r.radix_level(2, h) for r in ranks]))
+    for r in ranks:
+        r.radix_select(h)
     parts = torch.stack([r.partial(Q) for r in ranks])
     O = ranks[0].combine(parts).numpy()
     want_O, _ = _one_device()

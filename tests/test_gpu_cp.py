@@ -1,7 +1,8 @@
 """Context-parallel decode on the GPU against the oracle: the unnormalised
-attention, the log-sum-exp combine, the global selection over gathered
-candidates, and whole sharded steps (all ranks emulated on one device, phase
-by phase) against the one-device step.  Every call goes through the C ABI."""
+attention, the log-sum-exp combine, the global selection (by histogram
+exchange, and over gathered candidates), and whole sharded steps (all ranks
+emulated on one device, phase by phase) against the one-device step.  Every
+call goes through the C ABI."""
 import math
 
 import numpy as np
@@ -178,6 +179,84 @@ def test_cp_select_is_bit_exact(dev, N, lens, k, levels):
     assert_status_ok(ws)
 
 
+def _radix_exchange(dev, full, lens, N, k):
+    """Every rank's share of the global top-k by the histogram exchange, all
+    ranks on this device: [N] local index arrays [B, k] and counts [B]."""
+    B = len(lens)
+    bnd = cp.shard_bounds(lens, N)
+    ranks = []
+    for r in range(N):
+        n = (bnd[r, :, 1] - bnd[r, :, 0]).astype(np.int32)
+        sc = np.zeros((B, max(1, int(n.max()))), np.float32)
+        for b in range(B):
+            sc[b, :n[b]] = full[b][bnd[r, b, 0]:bnd[r, b, 1]]
+        ranks.append((torch.from_numpy(sc).to(dev), torch.from_numpy(n).to(dev),
+                      sa.workspace(sa.cp_radix_workspace_size(B), dev)))
+    h = torch.stack([sa.cp_radix_level(sc, n, k, N, 0, ws=ws) for sc, n, ws in ranks])
+    h = torch.stack([sa.cp_radix_level(sc, n, k, N, 1, h, ws=ws) for sc, n, ws in ranks])
+    h = torch.stack([sa.cp_radix_level(sc, n, k, N, 2, h, ws=ws) for sc, n, ws in ranks])
+    out = []
+    for r, (sc, n, ws) in enumerate(ranks):
+        cnt = torch.empty(B, dtype=torch.int32, device=dev)
+        idx = sa.cp_radix_select(sc, n, k, N, r, h, local_count=cnt, ws=ws)
+        assert_status_ok(ws)
+        out.append((idx.cpu().numpy(), cnt.cpu().numpy()))
+    return out, bnd
+
+
+@pytest.mark.parametrize("N,lens,k,kind", [
+    (1, [3000, 100], 256, "levels"),            # one rank: the plain top-k
+    (2, [20000, 5000, 300, 9000], 2048, "levels"),
+    (3, [4096, 50, 7000], 512, "normal"),       # distinct scores, ragged slices
+    (8, [131072, 4000], 2048, "levels"),        # c3's sharding
+    (8, [7, 5000, 64], 64, "levels"),           # empty slices (7 tokens over 8 ranks), k above a sequence
+    (4, [6000, 6000], 700, "one_value"),        # every score equal: ties decided by index alone
+    (4, [3000, 3000], 300, "signed"),           # negative scores, -0 and +0
+    (5, [40, 30], 128, "normal"),               # fewer tokens than k in all: every one selected
+])
+def test_radix_exchange_selects_the_global_top_k(dev, N, lens, k, kind):
+    """The union of the ranks' shares, in global positions, is the oracle's
+    top-k of the whole row (the lower index first among ties); each share
+    is ascending, -1 padded, and counted."""
+    rng = np.random.default_rng(N * 31 + k)
+    if kind == "levels":      # few distinct values: ties across slice edges
+        full = [(rng.integers(0, 300, S) * 0.125).astype(np.float32) for S in lens]
+    elif kind == "one_value":
+        full = [np.full(S, 0.5, np.float32) for S in lens]
+    elif kind == "signed":
+        full = [(rng.integers(-40, 40, S) * 0.25).astype(np.float32) for S in lens]
+        for f in full:
+            f[rng.random(len(f)) < 0.1] = -0.0
+    else:
+        full = [rng.standard_normal(S).astype(np.float32) for S in lens]
+    shares, bnd = _radix_exchange(dev, full, lens, N, k)
+    W = max(lens)
+    rows = np.zeros((len(lens), W), np.float32)
+    for b, f in enumerate(full):
+        rows[b, :len(f)] = f
+    want = oracle.topk(rows, lens, k)
+    for b in range(len(lens)):
+        got = []
+        for r in range(N):
+            idx, cnt = shares[r]
+            row = idx[b]
+            assert np.all(row[:cnt[b]] >= 0) and np.all(row[cnt[b]:] == -1), f"rank {r} b={b} padding"
+            assert np.all(np.diff(row[:cnt[b]]) > 0), f"rank {r} b={b} order"
+            assert np.all(row[:cnt[b]] < bnd[r, b, 1] - bnd[r, b, 0]), f"rank {r} b={b} range"
+            got += [int(bnd[r, b, 0] + t) for t in row[:cnt[b]]]
+        assert sorted(got) == [int(t) for t in want[b] if t >= 0], f"b={b}"
+
+
+def test_radix_exchange_reports_a_negative_length(dev):
+    sc = torch.zeros((2, 8), dtype=torch.float32, device=dev)
+    n = torch.tensor([8, -3], dtype=torch.int32, device=dev)
+    ws = sa.workspace(sa.cp_radix_workspace_size(2), dev)
+    h = sa.cp_radix_level(sc, n, 4, 1, 0, ws=ws)
+    code, det = sa.read_status(ws)
+    assert code == sa.SA_ERR_DEVICE and det[0] == 9 and det[1] == 1 and det[2] == -3
+    assert int(h[1].sum()) == 0 and int(h[0].sum()) == 8
+
+
 # --------------------------------------------------------------------------
 def _step_inputs(seed, lens, H_I=32, d_I=128, Hq=32, Hkv=8, d=128, L_g=3):
     rng = np.random.default_rng(seed)
@@ -204,7 +283,7 @@ def test_emulated_context_parallel_step_matches_one_device(dev, N, lens, k):
                                Hkv, d, L_g, scale))
     O_cp, local = cp.emulate_step(ranks, qI, w, Q, out_dtype=torch.float32)
     for r in ranks:
-        for ws in (r.ws_index, r.ws_topk, r.ws_sel, r.ws_attn):
+        for ws in (r.ws_index, r.ws_radix, r.ws_attn):
             assert_status_ok(ws)
     # the one-device step on the whole context
     seq_off, seq_len = cp.seq_tables(lens, dev)
