@@ -60,6 +60,8 @@ SIGNATURES = {
     "sa_cp_select_workspace_size": ([_I, _I, _I], _SZ),
     "sa_cp_select": ([_P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "sa_combine_partials": ([_P, _I64, _P, _I64, _I, _I64, _I, _P, _I, _P], _I),
+    "sa_index_topk_prefill_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
+    "sa_index_topk_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P], _I),
     "sa_cp_radix_workspace_size": ([_I], _SZ),
     "sa_cp_radix_level": ([_P, _I64, _P, _I, _I, _I, _I, _P, _I64, _P, _P, _SZ, _P], _I),
     "sa_cp_radix_select": ([_P, _I64, _P, _I, _I, _I, _I, _P, _I64, _P, _P, _P, _SZ, _P], _I),
@@ -217,6 +219,29 @@ def index_score_prefill(qI, w, KI, q_pos, max_pos: int, scores=None, ld: Optiona
     _check(lib().sa_index_score_prefill(_ptr(qI), _ptr(w), _ptr(KI), _ptr(q_pos), Nq, KI.shape[0], max_pos, H_I,
                                         d_I, _ptr(scores), ld, _ptr(ws), ws.numel(), _stream(stream)))
     return scores
+
+
+def index_topk_prefill_workspace_size(Nq: int, S: int, max_pos: int, k: int, rows_per_block: int = 0) -> int:
+    return int(lib().sa_index_topk_prefill_workspace_size(Nq, S, max_pos, k, rows_per_block))
+
+
+def index_topk_prefill(qI, w, KI, q_pos, max_pos: int, k: int, idx=None, rows_per_block: int = 0, ws=None,
+                       stream=None) -> torch.Tensor:
+    """Prefill indexer scores and per-query top-k, block of queries by block
+    (no score matrix for the whole chunk): idx int32 [Nq, k]."""
+    Nq, H_I, d_I = qI.shape
+    _dev(qI, torch.bfloat16, "qI"), _dev(w, torch.float32, "w"), _dev(KI, torch.bfloat16, "KI")
+    _out(q_pos, (Nq,), (torch.int32,), "q_pos")
+    if idx is None:
+        idx = torch.empty((Nq, k), dtype=torch.int32, device=qI.device)
+    _out(idx, (Nq, k), (torch.int32,), "idx")
+    S = KI.shape[0]
+    if ws is None:
+        ws = workspace(index_topk_prefill_workspace_size(Nq, S, max_pos, k, rows_per_block), qI.device)
+    _ws(ws)
+    _check(lib().sa_index_topk_prefill(_ptr(qI), _ptr(w), _ptr(KI), _ptr(q_pos), Nq, S, max_pos, H_I, d_I, k,
+                                       int(rows_per_block), _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx
 
 
 def topk(scores, n_valid, n_max: int, k: int, idx=None, top_scores=None, want_scores=False, ws=None, stream=None):

@@ -444,6 +444,108 @@ sa_status sa_index_score_prefill(const void* qI, const float* w, const void* KI,
   return run_index_decode(qI, w, KI, soff, slen, Nq, S, max_pos + 1, H_I, d_I, scores, ld, ws, s);
 }
 
+// ---------------------------------------------------------------- prefill indexer + top-k, blocked
+namespace {
+// Queries per block: all of them by default.  The indexer streams every key
+// tile once per block of queries, so smaller blocks trade time for
+// workspace (c4, S = 131072: 1.93 ms for one block of 2048 queries, 3.0 ms
+// in blocks of 1024, 5.4 ms of 512, 9.9 ms of 256, 18.9 ms of 128).
+int index_topk_rows(int Nq, int S, int rows_per_block) {
+  (void)S;
+  int nb = rows_per_block > 0 ? rows_per_block : Nq;
+  if (nb < 1) nb = 1;
+  if (nb > Nq) nb = Nq;
+  return nb;
+}
+
+struct IndexTopkLayout {
+  size_t soff, slen, scores, topk, total;  // byte offsets after the header, then the total
+  int rows;
+};
+
+IndexTopkLayout index_topk_layout(int Nq, int S, int max_pos, int k, int rows_per_block) {
+  IndexTopkLayout l{};
+  l.rows = index_topk_rows(Nq, S, rows_per_block);
+  l.soff = 0;
+  l.slen = round_up(8 * ((size_t)Nq + 1), 256);
+  l.scores = l.slen + round_up(4 * (size_t)Nq, 256);
+  l.topk = l.scores + round_up((size_t)l.rows * S * 4, 256);
+  const size_t t = sa::topk_use_split(l.rows, max_pos + 1, num_sms())
+                       ? sa::topk_split_ws_bytes(l.rows, max_pos + 1, num_sms())
+                       : 0;
+  (void)k;
+  l.total = SA_WS_HEADER_BYTES + l.topk + round_up(t, 256);
+  return l;
+}
+}  // namespace
+
+size_t sa_index_topk_prefill_workspace_size(int Nq, int S, int max_pos, int k, int rows_per_block) {
+  if (Nq < 1 || S < 1 || max_pos < 0 || max_pos >= S || k < 1) return SA_WS_HEADER_BYTES;
+  return index_topk_layout(Nq, S, max_pos, k, rows_per_block).total;
+}
+
+sa_status sa_index_topk_prefill(const void* qI, const float* w, const void* KI, const int32_t* q_pos, int Nq, int S,
+                                int max_pos, int H_I, int d_I, int k, int rows_per_block, int32_t* idx, void* ws,
+                                size_t ws_bytes, void* stream) {
+  const char* who = "sa_index_topk_prefill";
+  if (Nq < 0 || Nq > 4096) return fail(SA_ERR_INVALID_ARG, "%s: Nq=%d outside [0, 4096]", who, Nq);
+  if (S < 1 || max_pos < 0 || max_pos >= S) return fail(SA_ERR_INVALID_ARG, "%s: need 0 <= max_pos < S", who);
+  if (k < 1) return fail(SA_ERR_INVALID_ARG, "%s: k=%d < 1", who, k);
+  if (rows_per_block < 0) return fail(SA_ERR_INVALID_ARG, "%s: rows_per_block < 0", who);
+  sa_status st = validate_index(qI, w, KI, H_I, d_I, who);
+  if (st != SA_OK) return st;
+  if (!q_pos || !idx) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if ((st = check_ws(ws, ws_bytes, sa_index_topk_prefill_workspace_size(Nq, S, max_pos, k, rows_per_block), who)) !=
+      SA_OK)
+    return st;
+  if (Nq == 0) return SA_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  const IndexTopkLayout l = index_topk_layout(Nq, S, max_pos, k, rows_per_block);
+  uint8_t* p = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
+  int64_t* soff = reinterpret_cast<int64_t*>(p + l.soff);
+  int32_t* slen = reinterpret_cast<int32_t*>(p + l.slen);  // q_pos + 1: each row's valid length
+  float* blk = reinterpret_cast<float*>(p + l.scores);
+  const int64_t ld = S;
+  const int n_max = max_pos + 1;
+  prefill_rows_kernel<<<(Nq + 256) / 256, 256, 0, s>>>(q_pos, Nq, max_pos, soff, slen, status_of(ws));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail("sa_index_topk_prefill rows", e);
+  const bool tc = sa::indexer_prefill_supported(H_I, d_I);
+  CUtensorMap tm_ki;
+  if (tc) {
+    const uint64_t kd[2] = {(uint64_t)d_I, (uint64_t)S};
+    const uint64_t ks[1] = {(uint64_t)d_I * 2};
+    const uint32_t kb[2] = {64, 128};
+    if ((st = make_tmap(&tm_ki, KI, 2, kd, ks, kb)) != SA_OK) return st;
+  }
+  // one block of queries at a time: its scores (in the workspace), then its top-k
+  for (int j0 = 0; j0 < Nq; j0 += l.rows) {
+    const int nb = Nq - j0 < l.rows ? Nq - j0 : l.rows;
+    const void* qI_b = reinterpret_cast<const uint8_t*>(qI) + (size_t)j0 * H_I * d_I * 2;
+    if (tc) {
+      CUtensorMap tm_qi;
+      const uint64_t qd[2] = {(uint64_t)d_I, (uint64_t)nb * H_I};
+      const uint64_t qs[1] = {(uint64_t)d_I * 2};
+      const uint32_t qb[2] = {64, 256};
+      if ((st = make_tmap(&tm_qi, qI_b, 2, qd, qs, qb)) != SA_OK) return st;
+      sa::PrefillIndexerArgs a{w + (size_t)j0 * H_I, q_pos + j0, nb, S, max_pos, H_I, d_I, blk, ld, status_of(ws)};
+      e = sa::launch_indexer_prefill(a, tm_ki, tm_qi, num_sms(), s);
+      if (e != cudaSuccess) return cuda_fail("sa_index_topk_prefill indexer launch", e);
+    } else {
+      st = run_index_decode(qI_b, w + (size_t)j0 * H_I, KI, soff + j0, slen + j0, nb, S, n_max, H_I, d_I, blk, ld, ws,
+                            s);
+      if (st != SA_OK) return st;
+    }
+    if (sa::topk_use_split(nb, n_max, num_sms()))
+      e = sa::launch_topk_split(blk, ld, slen + j0, nb, n_max, k, idx + (size_t)j0 * k, nullptr, status_of(ws),
+                                p + l.topk, num_sms(), s);
+    else
+      e = sa::launch_topk_rows(blk, ld, slen + j0, nb, n_max, k, idx + (size_t)j0 * k, nullptr, status_of(ws), s);
+    if (e != cudaSuccess) return cuda_fail("sa_index_topk_prefill top-k launch", e);
+  }
+  return SA_OK;
+}
+
 // ---------------------------------------------------------------- top-k
 size_t sa_topk_workspace_size(int Nq, int n_max, int k) {
   (void)k;

@@ -160,6 +160,24 @@ sa_status sa_index_score_prefill(const void* qI, const float* w, const void* KI,
                                  int d_I, float* scores, int64_t ld, void* ws, size_t ws_bytes,
                                  void* stream);
 
+/* The prefill indexer followed by the per-query top-k, with the same result
+ * as sa_index_score_prefill then sa_topk (n_valid = q_pos + 1, n_max =
+ * max_pos + 1), writing no scores for the caller: the queries run in blocks
+ * of rows_per_block (0: all Nq in one block), each block's scores written to
+ * the workspace and selected before the next block is scored.  The
+ * workspace then holds rows_per_block x S fp32 scores.  Every block streams
+ * all key tiles again, so smaller blocks trade time for workspace (c4,
+ * S = 131072, 2048 queries: 1.93 ms in one block, 3.0 ms in blocks of 1024,
+ * 5.4 ms of 512, 18.9 ms of 128).
+ *   idx  int32 [Nq, k] out, as sa_topk writes it (ascending, -1 padded)
+ * Other arguments and device errors as sa_index_score_prefill and sa_topk.
+ * Workspace: sa_index_topk_prefill_workspace_size (the same rows_per_block). */
+size_t sa_index_topk_prefill_workspace_size(int Nq, int S, int max_pos, int k, int rows_per_block);
+sa_status sa_index_topk_prefill(const void* qI, const float* w, const void* KI, const int32_t* q_pos,
+                                int Nq, int S, int max_pos, int H_I, int d_I, int k,
+                                int rows_per_block, int32_t* idx, void* ws, size_t ws_bytes,
+                                void* stream);
+
 /* ------------------------------------------------------------------------
  * Top-k  [IC section 1: keep the k most relevant tokens; CLSA: the top-k
  * selection runs once and its index is reused].

@@ -609,6 +609,38 @@ def test_prefill_indexer_shapes(dev, H_I, d_I, Nq, S):
         parity.assert_scores_close(got[p, :n], ora, parity.index_error_bound(qI[p], w[p], KI[:n]), f"p={p}")
 
 
+@pytest.mark.parametrize("H_I,d_I,Nq,S,k,rows", [
+    (16, 128, 300, 6000, 256, 37),    # tensor-core indexer; blocks of 37 queries, a ragged last block
+    (16, 128, 64, 3000, 128, 0),      # one block (the default block size)
+    (12, 64, 50, 2000, 64, 16),       # the one-query-per-row indexer path
+    (16, 128, 129, 131072, 2048, 64), # the c4 context: two full blocks and a one-query block
+])
+def test_index_topk_prefill_blocked(dev, H_I, d_I, Nq, S, k, rows):
+    """The blocked indexer + top-k selects exactly what the indexer over the
+    whole chunk followed by the top-k selects (the same kernels, the same
+    scores), and that index holds against the oracle's scores outside the
+    tie band."""
+    rng = np.random.default_rng(Nq + S)
+    qI = synth.f32_to_bf16_bits((rng.standard_normal((Nq, H_I, d_I)) / 8).astype(np.float32))
+    KI = synth.f32_to_bf16_bits((rng.standard_normal((S, d_I)) / 8).astype(np.float32))
+    w = rng.uniform(0.1, 1.0, (Nq, H_I)).astype(np.float32)
+    q_pos = (S - Nq + np.arange(Nq)).astype(np.int32)
+    q_pos[::5] = rng.integers(0, S - Nq, len(q_pos[::5]))  # some queries see a short prefix
+    q_pos[3] = 10  # a prefix shorter than k
+    dq, dw, dK, dp = bf16_dev(qI, dev), torch.from_numpy(w).to(dev), bf16_dev(KI, dev), torch.from_numpy(q_pos).to(dev)
+    ws = sa.workspace(sa.index_topk_prefill_workspace_size(Nq, S, S - 1, k, rows), dev)
+    idx = sa.index_topk_prefill(dq, dw, dK, dp, S - 1, k, rows_per_block=rows, ws=ws)
+    assert_status_ok(ws)
+    scores = sa.index_score_prefill(dq, dw, dK, dp, S - 1)
+    want = sa.topk(scores, dp + 1, S, k)
+    assert torch.equal(idx, want)
+    got = idx.cpu().numpy()
+    for p in list(range(0, Nq, max(1, Nq // 6))) + [3]:
+        n = int(q_pos[p]) + 1
+        ora = oracle.index_score(qI[p:p + 1], w[p:p + 1], KI, [0, S], [0], [n - 1])[0][:n]
+        parity.assert_topk_band(got[p], ora, n, k, f"p={p}")
+
+
 def test_prefill_ragged_last_block(dev):
     """A context that is not a whole number of 64-token blocks: the last
     block is partial (its tile load reaches past the head's keys), every
