@@ -637,12 +637,32 @@ bool small_attn_path(int L_g, int Hq, int Hkv) { return (int64_t)L_g * (Hq / Hkv
 
 int small_attn_plan(int B, int Hkv, int k) { return sa::small_attn_splits(B * Hkv, k, num_sms(), kSmallMaxCounters); }
 
+// 9 to 128 rows per (b, g) on too few units to fill the GPU (the tcgen05
+// plan has fewer CTAs than half the SMs, e.g. one sequence with one KV
+// head): the warp-level MMA kernel with one warp per 16 rows, whose key
+// slices spread the few units over many CTAs.  With more units the tcgen05
+// kernel is faster (c2: 154 against 165 us per step; c3: 63 against 75).
+bool mid_attn_path(int L_g, int B, int Hq, int Hkv, int k) {
+  const int64_t R = (int64_t)L_g * (Hq / Hkv);
+  if (R <= sa::kSmallMaxRows || R > sa::kMidMaxRows) return false;
+  if ((int64_t)k > (int64_t)sa::kMidMaxSplits * sa::kMidMaxSlice) return false;
+  return plan_decode_attn(L_g, B, Hq, Hkv, k).units * 2 < num_sms();
+}
+
+int mid_attn_plan(int B, int Hkv, int R, int k) { return sa::mid_attn_splits(B * Hkv, R, k, num_sms()); }
+
 size_t sa_sparse_decode_attn_workspace_size(int L_g, int B, int Hq, int Hkv, int d, int k) {
   (void)d;
   if (L_g < 1 || B < 1 || Hkv < 1 || Hq < Hkv || k < 1) return SA_WS_HEADER_BYTES;
   if (small_attn_path(L_g, Hq, Hkv))
     return SA_WS_HEADER_BYTES +
            sa::small_attn_scratch_bytes(B * Hkv, small_attn_plan(B, Hkv, k), L_g * (Hq / Hkv));
+  if (mid_attn_path(L_g, B, Hq, Hkv, k)) {
+    const int R = L_g * (Hq / Hkv);
+    const size_t mid = SA_WS_HEADER_BYTES + sa::mid_attn_scratch_bytes(B * Hkv, mid_attn_plan(B, Hkv, R, k), R);
+    const size_t big = attn_ws_bytes(plan_decode_attn(L_g, B, Hq, Hkv, k));
+    return mid > big ? mid : big;  // the partial-output mode still takes the tcgen05 kernel
+  }
   return attn_ws_bytes(plan_decode_attn(L_g, B, Hq, Hkv, k));
 }
 
@@ -697,6 +717,41 @@ static sa_status run_decode_attn(const void* Q, const void* K, const void* V, co
       a.small_pml = reinterpret_cast<float2*>(base + SA_WS_HEADER_BYTES + round_up(n * 128 * 4, 256));
     }
     cudaError_t e = sa::launch_sparse_attn_small(a, stream);
+    if (e != cudaSuccess) return cuda_fail("sa_sparse_decode_attn launch", e);
+    return SA_OK;
+  }
+  if (!ml && !idx_count && mid_attn_path(L_g, B, Hq, Hkv, k)) {
+    // 9 to 128 rows per (b, g): the warp-level MMA kernel, one warp per 16 rows
+    const int R = L_g * (Hq / Hkv);
+    const int ns = mid_attn_plan(B, Hkv, R, k);
+    sa_status st = check_ws(ws, ws_bytes, SA_WS_HEADER_BYTES + sa::mid_attn_scratch_bytes(B * Hkv, ns, R), who);
+    if (st != SA_OK) return st;
+    sa::AttnArgs a{};
+    a.Q = reinterpret_cast<const uint16_t*>(Q);
+    a.K = reinterpret_cast<const uint16_t*>(K);
+    a.V = reinterpret_cast<const uint16_t*>(V);
+    a.seq_off = seq_off;
+    a.seq_len = seq_len;
+    a.idx = idx;
+    a.k = k;
+    a.L = L_g;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = Hq / Hkv;
+    a.R = R;
+    a.n_split = ns;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.O = O;
+    a.out_f32 = out_dtype == SA_F32;
+    a.status = status_of(ws);
+    if (ns > 1) {
+      uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+      const size_t n = (size_t)B * Hkv * ns * R;
+      a.small_po = reinterpret_cast<float*>(base + SA_WS_HEADER_BYTES);
+      a.small_pml = reinterpret_cast<float2*>(base + SA_WS_HEADER_BYTES + round_up(n * 128 * 4, 256));
+    }
+    cudaError_t e = sa::launch_sparse_attn_mid(a, stream);
     if (e != cudaSuccess) return cuda_fail("sa_sparse_decode_attn launch", e);
     return SA_OK;
   }

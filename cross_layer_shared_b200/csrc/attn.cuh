@@ -82,4 +82,16 @@ int small_attn_splits(int units, int k, int sms, int max_counters);
 size_t small_attn_scratch_bytes(int units, int ns, int R);
 cudaError_t launch_sparse_attn_small(const AttnArgs& a, cudaStream_t stream);
 
+// Path for 9 to kMidMaxRows query rows per (b, g) (decode, neither partial
+// outputs nor idx_count): warp-level MMA, one warp per 16 rows, one CTA per
+// (b, g, key slice), then (n_split > 1) a merge kernel.  mid_attn_splits
+// gives n_split; with n_split > 1 the call needs mid_attn_scratch_bytes of
+// workspace scratch for the partials (small_po, small_pml, [B*Hkv][n_split][R]).
+constexpr int kMidMaxRows = 128;  // the kernel supports up to this many
+constexpr int kMidMaxSplits = 16;
+constexpr int kMidMaxSlice = 4096;  // index entries per slice: k <= kMidMaxSplits * kMidMaxSlice
+int mid_attn_splits(int units, int R, int k, int sms);
+size_t mid_attn_scratch_bytes(int units, int ns, int R);
+cudaError_t launch_sparse_attn_mid(const AttnArgs& a, cudaStream_t stream);
+
 }  // namespace sa

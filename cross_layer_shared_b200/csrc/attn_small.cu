@@ -47,12 +47,14 @@
 #include <stdint.h>
 
 #include "attn.cuh"
+#include "attn_warp.cuh"
 #include "sm100.cuh"
 #include "status.cuh"
 #include "timeline.cuh"
 
 namespace sa {
 namespace {
+using namespace wm;
 
 constexpr int kD = 128;
 constexpr int kWarpsS = 4;
@@ -80,36 +82,7 @@ struct SmallSmem {
   int64_t out_off[R];                    // each row's first element in O
 };
 
-__device__ __forceinline__ float ex2f(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
-// 16 bytes global -> shared, asynchronous; src_bytes = 0 writes zeros
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src), "r"(src_bytes)
-               : "memory");
-}
-
-// D = A B + D, m16n8k16, bf16 in, fp32 accumulate
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 template <int R>
 __global__ void __launch_bounds__(kThreadsS, 3) sparse_attn_small_kernel(const AttnArgs a) {

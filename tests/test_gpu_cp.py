@@ -78,8 +78,9 @@ def test_partial_attention_matches_the_oracle(dev, L, B, Hq, Hkv, lens, k, empty
     assert np.abs(lse - lse_ora).max() <= 1e-4
     norm = o[live] / ml[live][:, 1:2]
     assert np.abs(norm - o_ora[live] / ml_ora[live][:, 1:2]).max() <= parity.ATOL_F32
-    # one part merged alone is the normalised output
-    assert (one.view_as(full) - full).abs().max().item() <= 1e-6
+    # one part merged alone is the normalised output (within fp32 rounding:
+    # with few units the full call takes the warp-level MMA kernel)
+    assert (one.view_as(full) - full).abs().max().item() <= parity.ATOL_F32
 
 
 @pytest.mark.parametrize("B,lens,k,counts", [
