@@ -20,7 +20,8 @@
 //   * each warp computes S^T = K Q^T for its 16 rows (keys on M, rows on
 //     N: two n-tiles), the online softmax of its rows (lazy reference: it
 //     moves only when the running max passes it by more than 8 in log2
-//     units), and O^T += V^T P^T with V^T and K from ldmatrix (the K tile
+//     units, which a warp vote detects; row sums stay per lane until the
+//     end), and O^T += V^T P^T with V^T and K from ldmatrix (the K tile
 //     and the V tile of a pass are shared by all warps);
 //   * P is rounded to bf16 for bf16 outputs (as the tcgen05 kernel does)
 //     and split into two bf16 parts (hi + lo) for fp32 outputs.
@@ -147,43 +148,59 @@ __global__ void __launch_bounds__(kMaxWarpsM * 32) sparse_attn_mid_kernel(const 
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) mma_bf16(sc[nt], k0, k1, k2, k3, qb[nt][s2][0], qb[nt][s2][1]);
     }
-    // ---- online softmax of each row over the pass (log2 units) ----
-    float pw[2][4];
+    // ---- online softmax of each row over the pass (log2 units).  The
+    // row's reference only moves when some key passes it by more than 8,
+    // which after a row's first pass is rare: a warp vote decides whether
+    // the row maxima are reduced at all.  Row sums stay per lane (each lane
+    // adds its own keys' weights) until the end. ----
+    float z[2][4];
+    bool over = false;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      float alpha[2] = {1.f, 1.f};
-      bool moved = false;
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float z0 = live0 ? sc[nt][e] * a.scale_log2 : -INFINITY;
-        const float z1 = live1 ? sc[nt][2 + e] * a.scale_log2 : -INFINITY;
-        float mx = fmaxf(z0, z1);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        if (mx > m_run[nt][e] + 8.f) {  // also when the row has no reference yet
-          alpha[e] = m_run[nt][e] == -INFINITY ? 0.f : ex2f(m_run[nt][e] - mx);
-          m_run[nt][e] = mx;
-          moved = true;
-        }
-        pw[nt][e] = z0 == -INFINITY ? 0.f : ex2f(z0 - m_run[nt][e]);
-        pw[nt][2 + e] = z1 == -INFINITY ? 0.f : ex2f(z1 - m_run[nt][e]);
-        float ps = pw[nt][e] + pw[nt][2 + e];
-        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-        l_run[nt][e] = l_run[nt][e] * alpha[e] + ps;
+        z[nt][e] = live0 ? sc[nt][e] * a.scale_log2 : -INFINITY;
+        z[nt][2 + e] = live1 ? sc[nt][2 + e] * a.scale_log2 : -INFINITY;
+        over |= fmaxf(z[nt][e], z[nt][2 + e]) > m_run[nt][e] + 8.f;
       }
-      if (moved) {
+    if (__any_sync(0xffffffffu, over)) {
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          o[mt][nt][0] *= alpha[0];
-          o[mt][nt][1] *= alpha[1];
-          o[mt][nt][2] *= alpha[0];
-          o[mt][nt][3] *= alpha[1];
+      for (int nt = 0; nt < 2; ++nt) {
+        float alpha[2] = {1.f, 1.f};
+        bool moved = false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float mx = fmaxf(z[nt][e], z[nt][2 + e]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          if (mx > m_run[nt][e] + 8.f) {  // also when the row has no reference yet
+            alpha[e] = m_run[nt][e] == -INFINITY ? 0.f : ex2f(m_run[nt][e] - mx);
+            m_run[nt][e] = mx;
+            l_run[nt][e] *= alpha[e];
+            moved = true;
+          }
+        }
+        if (moved) {
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            o[mt][nt][0] *= alpha[0];
+            o[mt][nt][1] *= alpha[1];
+            o[mt][nt][2] *= alpha[0];
+            o[mt][nt][3] *= alpha[1];
+          }
         }
       }
     }
+    float pw[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        pw[nt][e] = z[nt][e] == -INFINITY ? 0.f : ex2f(z[nt][e] - m_run[nt][e]);
+        pw[nt][2 + e] = z[nt][2 + e] == -INFINITY ? 0.f : ex2f(z[nt][2 + e] - m_run[nt][e]);
+        l_run[nt][e] += pw[nt][e] + pw[nt][2 + e];  // this lane's keys only
+      }
     // ---- P^T's B fragments per n-tile: b0 = row gq at keys 2tq, 2tq + 1,
     // b1 = at 2tq + 8, 2tq + 9.  Row gq at key j sits in lane 4 (j mod 8) +
     // gq / 2, half gq % 2 of its (rows 2tq', 2tq' + 1) pair. ----
@@ -219,6 +236,17 @@ __global__ void __launch_bounds__(kMaxWarpsM * 32) sparse_attn_mid_kernel(const 
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+  // the row sums over the 8 lanes that share each row
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float v = l_run[nt][e];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      l_run[nt][e] = v;
+    }
   // ---- this warp's rows: the output (one slice) or the slice's partial ----
   const bool single = ns == 1;
 #pragma unroll

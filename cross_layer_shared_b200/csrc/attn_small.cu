@@ -38,8 +38,9 @@
 // the workspace's zero-once header; the slice that finds itself last merges
 // all slices, normalises and stores the rows, and puts the counter back to
 // zero.  Softmax references are lazy: a row's reference logit m only moves
-// when the running max passes it by more than 8 (log2 units), so the weights
-// stay below 2^8 and the accumulators are rescaled only then.  Entries < 0
+// when the running max passes it by more than 8 (log2 units, detected by a
+// warp vote), so the weights stay below 2^8 and the accumulators are
+// rescaled only then; row sums stay per lane until the end.  Entries < 0
 // are padding; entries >= seq_len[b] are reported and skipped.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -222,39 +223,44 @@ __global__ void __launch_bounds__(kThreadsS, 3) sparse_attn_small_kernel(const A
       z[e] = (live >> gq) & 1u ? sc[e] * a.scale_log2 : -INFINITY;
       z[2 + e] = (live >> (gq + 8)) & 1u ? sc[2 + e] * a.scale_log2 : -INFINITY;
     }
-    float pw[4], alpha0 = 1.f, alpha1 = 1.f;
-    bool moved = false;
+    // the reference only moves when some key passes it by more than 8 (rare
+    // after a row's first pass: a warp vote decides whether the maxima are
+    // reduced); row sums stay per lane (this lane's keys) until the end
+    bool over = false;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) over |= fmaxf(z[e], z[2 + e]) > m_run[e] + 8.f;
+    if (__any_sync(0xffffffffu, over)) {
+      float alpha[2] = {1.f, 1.f};
+      bool moved = false;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float mx = fmaxf(z[e], z[2 + e]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        if (mx > m_run[e] + 8.f) {  // also when the row has no reference yet
+          alpha[e] = m_run[e] == -INFINITY ? 0.f : ex2f(m_run[e] - mx);
+          m_run[e] = mx;
+          l_run[e] *= alpha[e];
+          moved = true;
+        }
+      }
+      if (moved) {  // this lane's rows (lanes of one tq agree)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          o[mt][0] *= alpha[0];
+          o[mt][1] *= alpha[1];
+          o[mt][2] *= alpha[0];
+          o[mt][3] *= alpha[1];
+        }
+      }
+    }
+    float pw[4];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      float mx = fmaxf(z[e], z[2 + e]);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      // lazy reference: moves only when the max passes it by more than 8
-      float alpha = 1.f;
-      if (mx > m_run[e] + 8.f) {  // also when the row has no reference yet
-        alpha = m_run[e] == -INFINITY ? 0.f : ex2f(m_run[e] - mx);
-        m_run[e] = mx;
-        moved = true;
-      }
       pw[e] = z[e] == -INFINITY ? 0.f : ex2f(z[e] - m_run[e]);
       pw[2 + e] = z[2 + e] == -INFINITY ? 0.f : ex2f(z[2 + e] - m_run[e]);
-      float ps = pw[e] + pw[2 + e];
-      ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-      ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-      ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-      l_run[e] = l_run[e] * alpha + ps;
-      if (e == 0) alpha0 = alpha;
-      else alpha1 = alpha;
-    }
-    if (moved) {  // this lane's rows (lanes of one tq agree)
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        o[mt][0] *= alpha0;
-        o[mt][1] *= alpha1;
-        o[mt][2] *= alpha0;
-        o[mt][3] *= alpha1;
-      }
+      l_run[e] += pw[e] + pw[2 + e];
     }
     // ---- P^T's B fragments: b0 = row gq at keys 2tq, 2tq + 1, b1 = at keys
     // 2tq + 8, 2tq + 9.  Row gq at key j sits in lane 4 (j mod 8) + gq / 2,
@@ -294,6 +300,15 @@ __global__ void __launch_bounds__(kThreadsS, 3) sparse_attn_small_kernel(const A
     t1 = entry_check(p + 2, rn);
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+  // the row sums over the 8 lanes that share each row
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    float v = l_run[e];
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    l_run[e] = v;
+  }
   // ---- the warps' partials into this CTA's (m, l, o) ----
   __syncthreads();  // every warp is done with its V rows (wo shares their space)
   if (tid == 0) SA_TL(kTlAttnSmall, 12);
