@@ -58,6 +58,8 @@ def load(path: str):
     lb.oracle_combine_partials.argtypes = [P, P, I, I64, I, P]
     lb.oracle_cp_select.argtypes = [P, P, I, I, I, I, P]
     lb.oracle_topk_dynamic.argtypes = [P, I64, P, I, I, D, P, P]
+    lb.oracle_kap_order.argtypes = [P, I, I, I, I, I, P, I, P, I64]
+    lb.oracle_osk_prefill_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, P, I64, I, I, D, D, I, P, I, P, P, P, I64]
     lb.oracle_num_threads.restype = I
     return lb
 
@@ -226,6 +228,51 @@ def paged_prefill_attn(Q, q_pos, K, V, block: int, kv_indptr, kv_indices, scale:
                                     block, _p(_c(kv_indptr, np.int32)), _p(ind), float(scale),
                                     _p(out))
     return out
+
+
+def kap_order(idx, S: int, block: int, q_block: int, T) -> np.ndarray:
+    """CoSA's proxy read as a priority list per query block of q_block
+    queries: the union table T ordered by hit count (entries of the block's
+    index rows falling in each table block), larger first, ties by
+    ascending block id.  Returns int32 [ceil(Nq/q_block), len(T)]."""
+    idx = _c(idx, np.int32)
+    Nq, k = idx.shape
+    T = _c(T, np.int32)
+    nT = int(T.size)
+    n_qb = (Nq + q_block - 1) // q_block
+    order = np.zeros((n_qb, max(1, nT)), dtype=np.int32)
+    lib().oracle_kap_order(_p(idx), Nq, k, S, block, q_block, _p(T if nT else np.zeros(1, np.int32)), nT,
+                           _p(order), order.shape[1])
+    return order[:, :nT].copy()
+
+
+def osk_prefill_attn(Q, q_pos, K, V, block: int, order, q_block: int, scale: float, tau: float,
+                     lag: int = 2, units=None):
+    """CoSA's ordered-skipping kernel under the reading in oracle/sa_oracle.c:
+    unit (query block i, KV group g) runs the blocks of order[i] two per
+    step and stops lag steps after the first step whose largest row share
+    of the running softmax mass is below tau.  Returns (O [Nq,Hq,d] fp64,
+    NaN outside the computed units; steps [n_units] int32, -1 where not
+    computed; crit [n_units, n_steps] fp64, NaN where not computed)."""
+    Q = _c(Q, np.uint16)
+    Nq, Hq, d = Q.shape
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    Hkv, S, _ = K.shape
+    order = _c(order, np.int32)
+    n_qb, nT = order.shape
+    assert n_qb == (Nq + q_block - 1) // q_block
+    n_steps = (nT + 1) // 2
+    O = np.full((Nq, Hq, d), np.nan, dtype=np.float64)
+    steps = np.full(n_qb * Hkv, -1, dtype=np.int32)
+    crit = np.full((n_qb * Hkv, max(1, n_steps)), np.nan, dtype=np.float64)
+    u = None if units is None else _c(units, np.int32)
+    ordp = order if order.size else np.zeros(1, np.int32)
+    lib().oracle_osk_prefill_attn(_p(Q), _p(_c(q_pos, np.int32)), _p(K), _p(V), S, Nq, Hq, Hkv, d, block,
+                                  _p(ordp), max(1, nT), nT, q_block, float(scale), float(tau), int(lag),
+                                  _p(u), 0 if u is None else int(u.size), _p(O), _p(steps), _p(crit),
+                                  crit.shape[1])
+    return O, steps, crit[:, :n_steps]
 
 
 def kv_append(KI, K, V, seq_off, seq_len, new_KI, new_K, new_V, Hkv: int, d: int):

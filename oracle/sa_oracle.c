@@ -21,6 +21,9 @@
  *            Block-Union KV Selection", technical summary, section
  *            "Methodologie : CompactAttention" (selection step, execution
  *            step).
+ *   [CoSA]   "CoSA: Accelerating Long-Context Inference via Proxy-Kernel
+ *            Co-Designed Sparse Attention", lay summary (the kernel-aware
+ *            proxy's priority list, the ordered-skipping kernel).
  *
  * The pages name the DSA "lightning indexer" but print no formula for its
  * score; the oracle uses the DSA form score_t = sum_j w_j * ReLU(q_j . k_t)
@@ -479,6 +482,171 @@ void oracle_topk_dynamic(const float* scores, int64_t ld, const int32_t* n_valid
     for (int j = m; j < k_max; ++j) row[j] = -1;
     counts[q] = m;
     free(all);
+  }
+}
+
+/*
+ * CoSA's kernel-aware proxy, read as one priority list per query block
+ * [CoSA lay summary: the proxy no longer hands the kernel a yes/no list of
+ * blocks but a priority list, most important block first].  The pages
+ * give no formula for the priority.  The reading used here takes it from
+ * the selection the indexer already made: for query block i (queries
+ * i*q_block .. i*q_block + q_block - 1, the last block possibly shorter),
+ * block B's hit count is the number of entries (p, e) of those queries'
+ * index rows with 0 <= idx[p,e] < S and idx[p,e] / block == B.  The list
+ * is the union table T (nT distinct block ids) ordered by hit count,
+ * larger first, equal counts by ascending block id.
+ * idx [Nq, k]; order [ceil(Nq/q_block), ld], row i's first nT entries.
+ */
+typedef struct {
+  int64_t hits;
+  int32_t id;
+} kap_t;
+
+static int by_hits_then_id(const void* a, const void* b) {
+  const kap_t* x = (const kap_t*)a;
+  const kap_t* y = (const kap_t*)b;
+  if (x->hits != y->hits) return x->hits > y->hits ? -1 : 1;
+  return (x->id > y->id) - (x->id < y->id);
+}
+
+void oracle_kap_order(const int32_t* idx, int Nq, int k, int S, int block, int q_block,
+                      const int32_t* T, int nT, int32_t* order, int64_t ld) {
+  const int nb = (S + block - 1) / block;
+  const int n_qb = (Nq + q_block - 1) / q_block;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int i = 0; i < n_qb; ++i) {
+    int64_t* hits = (int64_t*)calloc((size_t)(nb > 0 ? nb : 1), sizeof(int64_t));
+    for (int p = i * q_block; p < Nq && p < (i + 1) * q_block; ++p)
+      for (int e = 0; e < k; ++e) {
+        const int32_t t = idx[(int64_t)p * k + e];
+        if (t >= 0 && t < S) hits[t / block] += 1;
+      }
+    kap_t* list = (kap_t*)malloc(sizeof(kap_t) * (size_t)(nT > 0 ? nT : 1));
+    for (int j = 0; j < nT; ++j) {
+      list[j].id = T[j];
+      list[j].hits = hits[T[j]];
+    }
+    qsort(list, (size_t)nT, sizeof(kap_t), by_hits_then_id);
+    for (int j = 0; j < nT; ++j) order[(int64_t)i * ld + j] = list[j].id;
+    free(list);
+    free(hits);
+  }
+}
+
+/*
+ * CoSA's ordered-skipping kernel over the union blocks of a prefill chunk
+ * [CoSA lay summary: the kernel reads the blocks in the proxy's priority
+ * order, so that a progressive score of what matters is built early, and
+ * then skips the later blocks with confidence].  The pages give no skip
+ * rule.  The reading used here:
+ *   unit (i, g): the rows (p, h) of the queries p of query block i and the
+ *     G = Hq/Hkv query heads h of KV group g;
+ *   step n: the keys of blocks order[i][2n] and order[i][2n+1] (the last
+ *     step may hold one block); row (p, h) sees key t when t <= q_pos[p]
+ *     and t < S, with logit z = scale * (Q[p,h] . K[g,t]);
+ *   after step n, for each row: M = the largest logit the row has seen in
+ *     steps 0..n, a = sum over the row's visible keys of step n of
+ *     exp(z - M), L = the same sum over steps 0..n; the step's share
+ *     is a / L, and +inf for a row that has seen no key yet;
+ *   c_n = the largest share over the unit's rows (the progressive score:
+ *     the most any row still gained from step n);
+ *   the first step n* with c_n < tau ends the unit after step n* + lag
+ *     (the steps already in flight finish), so the unit runs
+ *     N = min(n_steps, n* + 1 + lag) steps; N = n_steps when no step
+ *     qualifies.  n_steps = ceil(nT / 2).
+ *   O[p,h] = softmax attention of row (p, h) over its visible keys of
+ *   steps 0..N-1.
+ * Only the units listed in units[0..n_units) are computed (all of them
+ * when units is NULL); unit id u = g * n_qb + i.  steps[u] = N; crit, when
+ * given, gets c_n at crit[u * ld_crit + n] for n < n_steps (the running
+ * sums are kept in fp64 over the whole list so that every c_n is known).
+ * Q [Nq,Hq,d]; K, V [Hkv,S,d]; O [Nq,Hq,d] fp64 (rows of other units
+ * untouched).
+ */
+void oracle_osk_prefill_attn(const uint16_t* Q, const int32_t* q_pos, const uint16_t* K,
+                             const uint16_t* V, int S, int Nq, int Hq, int Hkv, int d, int block,
+                             const int32_t* order, int64_t ld, int nT, int q_block, double scale,
+                             double tau, int lag, const int32_t* units, int n_units, double* O,
+                             int32_t* steps, double* crit, int64_t ld_crit) {
+  const int G = Hq / Hkv;
+  const int n_qb = (Nq + q_block - 1) / q_block;
+  const int n_steps = (nT + 1) / 2;
+  const int n_all = n_qb * Hkv;
+  const int nu = units ? n_units : n_all;
+  for (int ui = 0; ui < nu; ++ui) {
+    const int u = units ? units[ui] : ui;
+    const int g = u / n_qb, i = u % n_qb;
+    const int p0 = i * q_block;
+    const int p1 = (p0 + q_block < Nq) ? p0 + q_block : Nq;
+    const int rows = (p1 - p0) * G;
+    const int32_t* list = order + (int64_t)i * ld;
+    const uint16_t* Kg = K + (int64_t)g * S * d;
+    const uint16_t* Vg = V + (int64_t)g * S * d;
+    /* share[r * n_steps + n]: row r's a / L after step n */
+    double* share = (double*)malloc(sizeof(double) * (size_t)(rows > 0 ? rows : 1) *
+                                    (size_t)(n_steps > 0 ? n_steps : 1));
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < rows; ++r) {
+      const int p = p0 + r / G;
+      const int h = g * G + r % G;
+      const uint16_t* q = Q + ((int64_t)p * Hq + h) * d;
+      double M = -INFINITY, L = 0.0;
+      double* z = (double*)malloc(sizeof(double) * (size_t)(2 * block));
+      for (int n = 0; n < n_steps; ++n) {
+        int nz = 0;
+        for (int b2 = 2 * n; b2 < 2 * n + 2 && b2 < nT; ++b2) {
+          const int64_t t0 = (int64_t)list[b2] * block;
+          for (int64_t t = t0; t < t0 + block; ++t) {
+            if (t > q_pos[p] || t >= S) continue;
+            const uint16_t* kr = Kg + t * d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) dot += bf(q[c]) * bf(kr[c]);
+            z[nz++] = scale * dot;
+          }
+        }
+        double m_step = -INFINITY;
+        for (int j = 0; j < nz; ++j)
+          if (z[j] > m_step) m_step = z[j];
+        const double M_new = m_step > M ? m_step : M;
+        double a = 0.0;
+        for (int j = 0; j < nz; ++j) a += exp(z[j] - M_new);
+        if (M_new != -INFINITY) L = (M == -INFINITY ? 0.0 : L * exp(M - M_new)) + a;
+        M = M_new;
+        share[(int64_t)r * n_steps + n] = L > 0.0 ? a / L : INFINITY;
+      }
+      free(z);
+    }
+    int N = n_steps;
+    for (int n = 0; n < n_steps; ++n) {
+      double c = -INFINITY;
+      for (int r = 0; r < rows; ++r) {
+        const double s = share[(int64_t)r * n_steps + n];
+        if (s > c) c = s;
+      }
+      if (crit) crit[(int64_t)u * ld_crit + n] = c;
+      if (c < tau && N == n_steps) N = (n + 1 + lag < n_steps) ? n + 1 + lag : n_steps;
+    }
+    steps[u] = N;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < rows; ++r) {
+      const int p = p0 + r / G;
+      const int h = g * G + r % G;
+      const int64_t cap = (int64_t)2 * N * block + 1;
+      int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap);
+      double* z = (double*)malloc(sizeof(double) * (size_t)cap);
+      int64_t n = 0;
+      for (int b2 = 0; b2 < 2 * N && b2 < nT; ++b2) {
+        const int64_t t0 = (int64_t)list[b2] * block;
+        for (int64_t t = t0; t < t0 + block; ++t)
+          if (t <= q_pos[p] && t < S) keys[n++] = t;
+      }
+      attend_row(Q + ((int64_t)p * Hq + h) * d, Kg, Vg, keys, n, d, scale, z,
+                 O + ((int64_t)p * Hq + h) * d);
+      free(keys);
+      free(z);
+    }
+    free(share);
   }
 }
 

@@ -27,7 +27,13 @@ MUTANTS = {
     "scale dropped": ("z[j] = scale * dot;", "z[j] = dot;"),
     "GQA map modulo": ("const int g = h / G;\n    const uint16_t* Kb", "const int g = h % Hkv;\n    const uint16_t* Kb"),
     "ceil block map": ("if (t >= 0) mark[t / block] = 1;", "if (t >= 0) mark[(t + block - 1) / block] = 1;"),
-    "causal strict": ("if (t <= q_pos[p] && t < S) keys[n++] = t;", "if (t < q_pos[p] && t < S) keys[n++] = t;"),
+    "causal strict": ("for (int64_t t = b0; t < b0 + block; ++t)\n        if (t <= q_pos[p] && t < S) keys[n++] = t;",
+                      "for (int64_t t = b0; t < b0 + block; ++t)\n        if (t < q_pos[p] && t < S) keys[n++] = t;"),
+    "ordered skipping: causal strict in the output": (
+        "for (int64_t t = t0; t < t0 + block; ++t)\n          if (t <= q_pos[p] && t < S) keys[n++] = t;",
+        "for (int64_t t = t0; t < t0 + block; ++t)\n          if (t < q_pos[p] && t < S) keys[n++] = t;"),
+    "ordered skipping: causal strict in the shares": ("if (t > q_pos[p] || t >= S) continue;",
+                                                       "if (t >= q_pos[p] || t >= S) continue;"),
     "value row of the wrong token": ("const uint16_t* vr = Vb + keys[j] * d;", "const uint16_t* vr = Vb + keys[0] * d;"),
     "routing weights not normalised": ("p[t] = exp(p[t] - m) / den;", "p[t] = exp(p[t] - m);"),
     "routing GQA map modulo": ("const int g = h / G;\n    const int64_t S = seq_len[b];",
@@ -50,6 +56,25 @@ MUTANTS = {
                                                   "    const double target = tau * (total < 0 ? 0 : (double)all[0].s * 2);"),
     "dynamic k: cap one short": ("    if (m > k_max) m = k_max;\n    int32_t* row = idx + (int64_t)q * k_max;",
                                  "    if (m >= k_max) m = k_max - 1;\n    int32_t* row = idx + (int64_t)q * k_max;"),
+    "proxy order ascending": ("if (x->hits != y->hits) return x->hits > y->hits ? -1 : 1;",
+                              "if (x->hits != y->hits) return x->hits < y->hits ? -1 : 1;"),
+    "proxy ties to the higher block": ("return (x->id > y->id) - (x->id < y->id);",
+                                       "return (x->id < y->id) - (x->id > y->id);"),
+    "proxy counts padding entries": ("if (t >= 0 && t < S) hits[t / block] += 1;",
+                                     "if (t >= -1 && t < S) hits[t / block] += 1;"),
+    "skip rule not strict": ("if (c < tau && N == n_steps)", "if (c <= tau && N == n_steps)"),
+    "skip without the steps in flight": ("N = (n + 1 + lag < n_steps) ? n + 1 + lag : n_steps;",
+                                         "N = (n + 1 < n_steps) ? n + 1 : n_steps;"),
+    "progressive score of the first row only": ("for (int r = 0; r < rows; ++r) {\n        const double s = share",
+                                                "for (int r = 0; r < 1; ++r) {\n        const double s = share"),
+    "share against the mass before the step": ("share[(int64_t)r * n_steps + n] = L > 0.0 ? a / L : INFINITY;",
+                                               "share[(int64_t)r * n_steps + n] = L > a ? a / (L - a) : INFINITY;"),
+    "unseen row counts as no gain": ("share[(int64_t)r * n_steps + n] = L > 0.0 ? a / L : INFINITY;",
+                                     "share[(int64_t)r * n_steps + n] = L > 0.0 ? a / L : 0.0;"),
+    "steps of one block": ("for (int b2 = 2 * n; b2 < 2 * n + 2 && b2 < nT; ++b2) {",
+                           "for (int b2 = 2 * n; b2 < 2 * n + 1 && b2 < nT; ++b2) {"),
+    "output over N blocks instead of N steps": ("for (int b2 = 0; b2 < 2 * N && b2 < nT; ++b2) {",
+                                                "for (int b2 = 0; b2 < N && b2 < nT; ++b2) {"),
     "routing drops the last token": ("for (int64_t t = 0; t < seq_len[b]; ++t) {\n      double acc",
                                      "for (int64_t t = 0; t + 1 < seq_len[b]; ++t) {\n      double acc"),
 }

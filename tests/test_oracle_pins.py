@@ -724,3 +724,173 @@ def test_dynamic_k_total_is_over_the_whole_row():
     row[0, 6] = 2.0  # total 10
     idx, counts = oracle.topk_dynamic(row, [8], 8, 0.5)  # target 5: 2 + 2 + 1
     assert counts[0] == 3 and list(idx[0, :3]) == [0, 3, 6]
+
+
+# ----------------------------------------------------------------------------
+# CoSA: the proxy's priority list and the ordered-skipping kernel (reading in
+# oracle/sa_oracle.c: hit counts order the union table per query block; the
+# kernel runs two blocks per step and stops `lag` steps after the first step
+# whose largest row share of the running softmax mass is below tau)
+# ----------------------------------------------------------------------------
+def _kap_brute(idx, S, block, q_block, T):
+    out = []
+    Nq = len(idx)
+    for i in range(0, Nq, q_block):
+        hits = {int(b): 0 for b in T}
+        for p in range(i, min(Nq, i + q_block)):
+            for t in idx[p]:
+                t = int(t)
+                if 0 <= t < S and t // block in hits:
+                    hits[t // block] += 1
+        out.append(sorted(hits, key=lambda b: (-hits[b], b)))
+    return out
+
+
+def test_kap_order_hand_example():
+    # S = 512, 64-token blocks; query block 0 = queries 0, 1; block 1 = query 2
+    idx = np.array([[5, 70, 71, 300],      # blocks 0, 1, 1, 4
+                    [72, 301, -1, 600],    # blocks 1, 4; -1 and 600 >= S not counted
+                    [130, 131, 450, 0]],   # blocks 2, 2, 7, 0
+                   np.int32)
+    T = [0, 1, 2, 4, 7]
+    order = oracle.kap_order(idx, 512, 64, 2, T)
+    # block 0: hits 0:1, 1:3, 2:0, 4:2, 7:0; block 1: 0:1, 1:0, 2:2, 4:0, 7:1
+    assert order.tolist() == [[1, 4, 0, 2, 7], [2, 0, 7, 1, 4]]
+
+
+def test_kap_order_brute_force():
+    rng = np.random.default_rng(51)
+    for trial in range(20):
+        S = int(rng.integers(64, 2000))
+        block = int(rng.choice([16, 64]))
+        Nq, k, q_block = int(rng.integers(1, 12)), int(rng.integers(1, 40)), int(rng.integers(1, 5))
+        idx = rng.integers(-3, S + 40, (Nq, k)).astype(np.int32)      # padding, past-S entries, duplicates
+        nb = (S + block - 1) // block
+        T = sorted(set(rng.choice(nb, int(rng.integers(0, nb + 1)), replace=False).tolist()) |
+                   {int(t) // block for t in idx.ravel() if 0 <= t < S})
+        got = oracle.kap_order(idx, S, block, q_block, T)
+        want = _kap_brute(idx, S, block, q_block, T)
+        assert got.tolist() == want, trial
+        assert all(sorted(r) == T for r in got.tolist())
+
+
+def _osk_case(seed, Nq=6, Hq=4, Hkv=2, S=700, d=16, block=64, chunk_end=True):
+    rng = np.random.default_rng(seed)
+    q_pos = (np.arange(S - Nq, S) if chunk_end else np.sort(rng.choice(S, Nq, replace=False))).astype(np.int32)
+    Q = bf(rng.standard_normal((Nq, Hq, d)))
+    K = bf(rng.standard_normal((Hkv, S, d)))
+    V = bf(rng.standard_normal((Hkv, S, d)))
+    idx = np.full((Nq, 40), -1, np.int32)
+    for i, p in enumerate(q_pos):
+        n = min(40, int(p) + 1)
+        idx[i, :n] = rng.choice(int(p) + 1, n, replace=False)
+    return rng, q_pos, Q, K, V, idx
+
+
+def test_osk_without_skipping_is_the_paged_attention():
+    # tau = 0: no share is below it, every unit runs every step, and the
+    # order of the blocks does not change a softmax over the same keys
+    for seed, chunk_end in ((52, True), (53, False)):
+        rng, q_pos, Q, K, V, idx = _osk_case(seed, chunk_end=chunk_end)
+        S, block, Hkv, q_block = K.shape[1], 64, K.shape[0], 2
+        indptr, indices = oracle.block_union(idx, S, block, Hkv)
+        T = indices[:indptr[1]]
+        order = oracle.kap_order(idx, S, block, q_block, T)
+        O, steps, crit = oracle.osk_prefill_attn(Q, q_pos, K, V, block, order, q_block, 0.25, tau=0.0)
+        want = oracle.paged_prefill_attn(Q, q_pos, K, V, block, indptr, indices, 0.25)
+        np.testing.assert_allclose(O, want, rtol=0, atol=1e-12)
+        assert np.all(steps == (len(T) + 1) // 2)
+        assert np.all((crit >= 0) & ((crit <= 1 + 1e-12) | np.isinf(crit)))  # 0: a step no row sees
+
+
+def test_osk_stopping_at_once_reads_the_first_blocks_only():
+    # tau > 1: every step's share is at most 1, so each unit stops after
+    # step 0 and runs 1 + lag steps: attention over its first 2 (1 + lag)
+    # blocks of the order, the paged attention over that table
+    rng, q_pos, Q, K, V, idx = _osk_case(54)
+    S, block, Hkv, G, q_block = K.shape[1], 64, K.shape[0], 2, 3
+    T = list(range((S + block - 1) // block))
+    order = np.stack([rng.permutation(T) for _ in range(2)]).astype(np.int32)
+    for lag in (0, 1, 2):
+        O, steps, _ = oracle.osk_prefill_attn(Q, q_pos, K, V, block, order, q_block, 0.25, tau=1.5, lag=lag)
+        assert np.all(steps == 1 + lag)
+        for i in range(2):
+            sub = np.sort(order[i, :2 * (1 + lag)]).astype(np.int32)
+            want = oracle.paged_prefill_attn(Q, q_pos, K, V, block, [g * len(sub) for g in range(Hkv + 1)],
+                                             np.tile(sub, Hkv), 0.25)
+            rows = slice(i * q_block, (i + 1) * q_block)
+            np.testing.assert_allclose(O[rows], want[rows], rtol=0, atol=1e-12)
+
+
+def _osk_pow2_case():
+    # one query (position 15, sees every key), two heads of one KV group,
+    # 2-token blocks run in the order 3 1 6 0 2 7 4 5: steps (3,1) (6,0) (2,7) (4,5).
+    # scale = ln 2 and integer dots make every weight a power of two:
+    #   head 0 dots 3, 1, 0, -1 per step -> masses 32, 8, 4, 2
+    #   head 1 dots 0, 1, 0, -2 per step -> masses 4, 8, 4, 1
+    # shares per step: head 0  1, 8/40, 4/44, 2/46;  head 1  1, 8/12, 4/16, 1/17
+    # largest share c = 1, 2/3, 1/4, 1/17
+    order = np.array([[3, 1, 6, 0, 2, 7, 4, 5]], np.int32)
+    step_of = {}
+    for n in range(4):
+        for b in order[0, 2 * n:2 * n + 2]:
+            step_of[2 * int(b)] = n
+            step_of[2 * int(b) + 1] = n
+    dots = {0: (3, 1, 0, -1), 1: (0, 1, 0, -2)}
+    K = np.zeros((1, 16, 2), np.float32)
+    V = np.zeros((1, 16, 2), np.float32)
+    for t in range(16):
+        K[0, t] = (dots[0][step_of[t]], dots[1][step_of[t]])
+        V[0, t] = (step_of[t], 1.0)
+    Q = np.array([[[1.0, 0.0], [0.0, 1.0]]], np.float32)
+    return bf(Q), bf(K), bf(V), order
+
+
+def test_osk_powers_of_two_closed_form():
+    Q, K, V, order = _osk_pow2_case()
+    mass = {0: (32, 8, 4, 2), 1: (4, 8, 4, 1)}
+    for tau, lag, N in ((0.7, 0, 2), (0.7, 1, 3), (0.7, 2, 4), (0.3, 0, 3), (0.3, 1, 4), (0.1, 0, 4),
+                        (0.05, 0, 4), (1.5, 0, 1)):
+        O, steps, crit = oracle.osk_prefill_attn(Q, [15], K, V, 2, order, 1, math.log(2.0), tau=tau, lag=lag)
+        np.testing.assert_allclose(crit[0], [1.0, 2 / 3, 1 / 4, 1 / 17], rtol=1e-13)
+        assert steps[0] == N, (tau, lag)
+        for h in range(2):
+            w = [Fraction(4 * 0 + m) for m in mass[h][:N]]
+            want = float(sum(n * w[n] for n in range(N)) / sum(w))
+            np.testing.assert_allclose(O[0, h], [want, 1.0], rtol=0, atol=1e-13)
+
+
+def test_osk_equal_logits_strict_threshold():
+    # K = 0: every logit is 0 and every weight exp(0) = 1 exactly, so after
+    # step n (4 keys per step) the share is exactly 4 / (4 (n + 1)).
+    # tau = 1/4: step 3's share equals tau and does not stop (strict), step 4's does.
+    d, S = 4, 48
+    Q = bf(np.ones((1, 1, d)))
+    K = bf(np.zeros((1, S, d)))
+    V = bf(np.arange(S * d, dtype=np.float32).reshape(1, S, d) % 7)
+    order = np.arange(12, dtype=np.int32)[None]
+    for tau, N in ((0.25, 5), (0.2, 6), (0.5, 3), (0.49, 3)):
+        O, steps, crit = oracle.osk_prefill_attn(Q, [S - 1], K, V, 4, order, 1, 1.0, tau=tau, lag=0)
+        assert crit[0].tolist() == [1 / (n + 1) for n in range(6)]
+        assert steps[0] == N, tau
+        want = bf16_bits_to_f32(V[0, :8 * N]).astype(np.float64).mean(axis=0)
+        np.testing.assert_allclose(O[0, 0], want, rtol=0, atol=1e-12)
+
+
+def test_osk_a_row_with_nothing_visible_keeps_the_unit_running():
+    # query 0 (position 3) sees only block 0, which comes last in the order;
+    # query 1 (position 47) sees everything.  With tau = 0.9 query 1 alone
+    # would stop after step 1, but query 0 has seen no key until the last
+    # step (share +inf), so the unit runs all of them.
+    d, S = 4, 48
+    Q = bf(np.ones((2, 1, d)))
+    K = bf(np.zeros((1, S, d)))
+    V = bf(np.arange(S * d, dtype=np.float32).reshape(1, S, d) % 5)
+    order = np.array([[11, 10, 9, 8, 7, 6, 5, 4, 3, 2, 1, 0]], np.int32)
+    O, steps, crit = oracle.osk_prefill_attn(Q, [3, 47], K, V, 4, order, 2, 1.0, tau=0.9, lag=0)
+    assert steps[0] == 6 and np.all(np.isinf(crit[0, :5])) and crit[0, 5] == 1.0
+    # the same query 1 in a unit of its own stops after step 1 (share 1/2)
+    O1, steps1, _ = oracle.osk_prefill_attn(Q[1:], [47], K, V, 4, order, 1, 1.0, tau=0.9, lag=0)
+    assert steps1[0] == 2
+    np.testing.assert_allclose(O1[0, 0], bf16_bits_to_f32(V[0, 32:48]).astype(np.float64).mean(axis=0),
+                               rtol=0, atol=1e-12)
