@@ -62,6 +62,8 @@ def parse_args():
     p.add_argument("--out-f32", action="store_true", help="fp32 attention output instead of bf16")
     p.add_argument("--no-others", action="store_true",
                    help="skip the one-GPU timings of the other workloads (c1, c2, c5 decode; c4 prefill)")
+    p.add_argument("--osk-only", action="store_true",
+                   help="with --workload c4: time only the ordered-skipping prefill path against the full one")
     p.add_argument("--cp-ranks", type=int, default=8,
                    help="ranks of the emulated context-parallel step (single-group workloads, N=1; 0 = skip)")
     return p.parse_args()
@@ -423,10 +425,100 @@ def prefill_device_timing(args, dev, cap):
         peak, peak_kind = 1590.0, "fallback"
     attn_tf = attn_flops / (stage_ms["attention"] / 1e3) / 1e12
 
-    return {"cfg": cfg, "wl": wl, "O": O, "run_index": run_index, "run_topk": run_topk, "run_attn": run_attn,
+    return {"cfg": cfg, "wl": wl, "O": O, "idx": idx, "run_index": run_index, "run_topk": run_topk,
+            "run_attn": run_attn,
             "ms": ms, "stage_ms": stage_ms, "attn_flops": attn_flops, "idx_flops": idx_flops, "peak": peak,
             "peak_kind": peak_kind, "attn_tf": attn_tf, "clocks": clocks, "union_blocks": int(ptr_h[1]),
             "steps": steps, "warm": warm, "graphs": graphs}
+
+
+OSK_TAU = 2.0 ** -10
+
+
+def osk_device_timing(args, dev, cap, idx, tau: float = OSK_TAU, names=("c4-concentrated", "c4")) -> dict:
+    """Priority-ordered block execution with early skipping on the c4 chunk's
+    own selection (idx from its indexer and top-k): sa_osk_prefill (union,
+    priority lists, ordered-skipping attention) against sa_block_union_prefill
+    (union, attention over every union block), both replayed from CUDA graphs,
+    on the plain chunk and on the chunk whose attention is drawn to the hot
+    regions.  Times are taken with bf16 outputs (the chunk's own); the
+    share of tiles run and how far the skipped output is from the full one
+    come from one untimed call of each with fp32 outputs."""
+    import torch
+
+    import cross_layer_shared_b200 as sa
+    from synth import gpu as sgpu
+
+    out = {"tau": tau}
+    steps = max(1, min(args.steps, 50))
+    for name in names:
+        cfg = synth.workload(name)
+        wl = sgpu.prefill_workload(cfg, dev)
+        G = cfg.Hq // cfg.Hkv
+        n_qb = (cfg.chunk * G + 127) // 128
+        nb = (cfg.S + cfg.block - 1) // cfg.block
+        ws = sa.workspace(sa.osk_prefill_workspace_size(cfg.S, cfg.chunk, cfg.Hq, cfg.Hkv, cfg.d, cfg.k, cfg.block),
+                          dev)
+        uws = sa.workspace(sa.lib().sa_block_union_prefill_workspace_size(cfg.S, cfg.chunk, cfg.Hq, cfg.Hkv, cfg.d,
+                                                                            cfg.k, cfg.block), dev)
+        kws = sa.workspace(sa.kap_order_workspace_size(), dev)
+        ptr = torch.empty(cfg.Hkv + 1, dtype=torch.int32, device=dev)
+        ind = torch.empty(cfg.Hkv * nb, dtype=torch.int32, device=dev)
+        order = torch.empty((n_qb, nb), dtype=torch.int32, device=dev)
+        st = torch.empty(cfg.Hkv * n_qb, dtype=torch.int32, device=dev)
+        O_osk = torch.empty((cfg.chunk, cfg.Hq, cfg.d), dtype=torch.float32, device=dev)
+        O_full = torch.empty_like(O_osk)
+        O_b16 = torch.empty((cfg.chunk, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=dev)
+
+        def run_osk(O=O_b16):
+            sa.osk_prefill(idx, wl["q_pos"], wl["Q"], wl["K"], wl["V"], cfg.block, cfg.scale, tau, O=O,
+                           kv_indptr=ptr, kv_indices=ind, order=order, steps=st, ws=ws)
+
+        def run_full(O=O_b16):
+            sa.block_union_prefill(idx, wl["q_pos"], wl["Q"], wl["K"], wl["V"], cfg.block, cfg.scale, O=O,
+                                   kv_indptr=ptr, kv_indices=ind, ws=uws)
+
+        def run_order():
+            sa.kap_order(idx, cfg.S, cfg.block, 128 // G, ptr, ind, order=order, ws=kws)
+
+        run_full(O_full)
+        run_osk(O_osk)
+        torch.cuda.synchronize()
+        for w_ in (ws, uws, kws):
+            code, det = sa.read_status(w_)
+            if code != 0:
+                raise RuntimeError(f"device status {code} {det}")
+        res = {}
+        for key, fn in (("osk", run_osk), ("full", run_full), ("order", run_order)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                fn()
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            res[key] = e0.elapsed_time(e1) / steps
+            del g
+        n_t = int(ptr[1].item())
+        n_steps = (n_t + 1) // 2
+        st_h = st.cpu().numpy()
+        diff = (O_osk - O_full).abs()
+        out[name] = {"osk_ms": res["osk"], "full_ms": res["full"], "order_ms": res["order"],
+                     "speedup": res["full"] / res["osk"], "union_blocks": n_t,
+                     "tiles_run_frac": float(st_h.sum()) / (len(st_h) * max(1, n_steps)),
+                     "tiles_per_unit_min_max": [int(st_h.min()), int(st_h.max())],
+                     "max_abs_diff_vs_full": float(diff.max().item()),
+                     "mean_abs_diff_vs_full": float(diff.mean().item()),
+                     "workload": name + ": " + synth.DESCRIPTIONS.get(name, synth.DESCRIPTIONS["c4"])}
+        del wl, O_osk, O_full, O_b16, ws, uws, kws
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_prefill(args):
@@ -501,6 +593,47 @@ def run_prefill(args):
         "clocks": clocks.summary(),
     }
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_osk_only(args):
+    """--workload c4 --osk-only: the chunk's selection (indexer and top-k,
+    untimed), then only the ordered-skipping comparison, on the chunk whose
+    attention is drawn to its hot regions.  Prints one JSON line."""
+    import torch
+
+    import cross_layer_shared_b200 as sa
+    from cross_layer_shared_b200 import build
+    from synth import gpu as sgpu
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        print(json.dumps({"workload": "c4", "error": "the prefill chunk runs on one GPU"}), flush=True)
+        return 0
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    build.build()
+    sa.lib()
+    cap = torch.cuda.Stream()
+    cfg = synth.workload("c4")
+    wl = sgpu.prefill_workload(cfg, dev)
+    ws = sa.workspace(max(sa.lib().sa_index_score_prefill_workspace_size(cfg.chunk),
+                          sa.lib().sa_topk_workspace_size(cfg.chunk, cfg.S, cfg.k)), dev)
+    scores = torch.empty((cfg.chunk, cfg.S), dtype=torch.float32, device=dev)
+    idx = torch.empty((cfg.chunk, cfg.k), dtype=torch.int32, device=dev)
+    sa.index_score_prefill(wl["qI"], wl["w"], wl["KI"], wl["q_pos"], cfg.S - 1, scores=scores, ld=cfg.S, ws=ws)
+    sa.topk(scores, (wl["q_pos"] + 1).to(torch.int32), cfg.S, cfg.k, idx=idx, ws=ws)
+    torch.cuda.synchronize()
+    code, det = sa.read_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} {det}")
+    del scores, wl
+    torch.cuda.empty_cache()
+    res = osk_device_timing(args, dev, cap, idx, names=("c4-concentrated",))
+    r = res["c4-concentrated"]
+    print(json.dumps({"metric": "ordered-skipping prefill chunk (union + priority lists + attention), 1xB200",
+                      "value": r["osk_ms"], "unit": "ms per chunk", "higher_is_better": False,
+                      "config": {"workload": r["workload"], "tau": res["tau"]}, "ordered_skipping": res}),
+          flush=True)
     return 0
 
 
@@ -1083,6 +1216,7 @@ def run_ours(args):
                         "indexer_tflops": pt["idx_flops"] / (pt["stage_ms"]["indexer"] / 1e3) / 1e12,
                         "peak_tflops": pt["peak"], "peak_kind": pt["peak_kind"],
                         "workload": "c4: " + synth.DESCRIPTIONS["c4"]}
+        others["c4_ordered_skipping"] = osk_device_timing(args, dev, cap, pt["idx"])
         del pt
         torch.cuda.empty_cache()
 
@@ -1158,6 +1292,8 @@ def main():
                               "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
                   flush=True)
             return 0
+        if args.osk_only:
+            return run_osk_only(args)
         return run_prefill(args)
     if args.impl == "reference":
         return run_reference(args)

@@ -65,6 +65,11 @@ SIGNATURES = {
     "sa_cp_radix_workspace_size": ([_I], _SZ),
     "sa_cp_radix_level": ([_P, _I64, _P, _I, _I, _I, _I, _P, _I64, _P, _P, _SZ, _P], _I),
     "sa_cp_radix_select": ([_P, _I64, _P, _I, _I, _I, _I, _P, _I64, _P, _P, _P, _SZ, _P], _I),
+    "sa_kap_order_workspace_size": ([], _SZ),
+    "sa_kap_order": ([_P, _I, _I, _I, _I, _I, _P, _P, _P, _I64, _P, _SZ, _P], _I),
+    "sa_osk_prefill_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
+    "sa_osk_prefill": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P, _P, _I, _P, _SZ,
+                        _P], _I),
 }
 
 
@@ -675,6 +680,77 @@ def block_union_prefill(idx, q_pos, Q, K, V, block: int, scale: float, out_dtype
                                         block, float(scale), _ptr(kv_indptr), _ptr(kv_indices), _ptr(O), code,
                                         _ptr(ws), ws.numel(), _stream(stream)))
     return kv_indptr, kv_indices, O
+
+
+def kap_order_workspace_size() -> int:
+    return int(lib().sa_kap_order_workspace_size())
+
+
+def osk_prefill_workspace_size(S, Nq, Hq, Hkv, d, k, block) -> int:
+    return int(lib().sa_osk_prefill_workspace_size(S, Nq, Hq, Hkv, d, k, block))
+
+
+def kap_order(idx, S: int, block: int, q_block: int, kv_indptr, kv_indices, order=None, ws=None, stream=None):
+    """sa_kap_order: the union table ordered per query block of q_block
+    queries by hit count (larger first, ties by ascending block id).
+    Returns order [ceil(Nq/q_block), ceil(S/block)] int32; row i's first
+    kv_indptr[1] - kv_indptr[0] entries are written."""
+    Nq, k = idx.shape
+    _out(idx, (Nq, k), (torch.int32,), "idx")
+    nb = (S + block - 1) // block
+    n_qb = (Nq + q_block - 1) // q_block
+    _out(kv_indptr, (kv_indptr.numel(),), (torch.int32,), "kv_indptr")
+    _out(kv_indices, (kv_indices.numel(),), (torch.int32,), "kv_indices")
+    if order is None:
+        order = torch.empty((n_qb, nb), dtype=torch.int32, device=idx.device)
+    _out(order, (n_qb, nb), (torch.int32,), "order")
+    if ws is None:
+        ws = workspace(lib().sa_kap_order_workspace_size(), idx.device)
+    _ws(ws)
+    _check(lib().sa_kap_order(_ptr(idx), Nq, k, S, block, q_block, _ptr(kv_indptr), _ptr(kv_indices), _ptr(order),
+                              nb, _ptr(ws), ws.numel(), _stream(stream)))
+    return order
+
+
+def osk_prefill(idx, q_pos, Q, K, V, block: int, scale: float, tau: float, out_dtype=torch.bfloat16, O=None,
+                kv_indptr=None, kv_indices=None, order=None, steps=None, ws=None, stream=None):
+    """sa_osk_prefill: block union, priority lists (one per query block of
+    128 / (Hq/Hkv) queries) and ordered-skipping attention with threshold
+    tau.  Returns (kv_indptr, kv_indices, order [n_qb, ceil(S/block)],
+    steps [Hkv * n_qb] (tiles of two blocks run per unit g * n_qb + i),
+    O [Nq,Hq,d])."""
+    Nq, Hq, d = Q.shape
+    Hkv, S, _ = K.shape
+    k = idx.shape[1]
+    _out(idx, (Nq, k), (torch.int32,), "idx"), _out(q_pos, (Nq,), (torch.int32,), "q_pos")
+    _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V")
+    nb = (S + block - 1) // block
+    G = Hq // Hkv
+    n_qb = (Nq * G + 127) // 128
+    dev = Q.device
+    if kv_indptr is None:
+        kv_indptr = torch.empty(Hkv + 1, dtype=torch.int32, device=dev)
+    _out(kv_indptr, (Hkv + 1,), (torch.int32,), "kv_indptr")
+    if kv_indices is None:
+        kv_indices = torch.empty(Hkv * nb, dtype=torch.int32, device=dev)
+    _out(kv_indices, (Hkv * nb,), (torch.int32,), "kv_indices")
+    if order is None:
+        order = torch.empty((n_qb, nb), dtype=torch.int32, device=dev)
+    _out(order, (n_qb, nb), (torch.int32,), "order")
+    if steps is None:
+        steps = torch.empty(Hkv * n_qb, dtype=torch.int32, device=dev)
+    _out(steps, (Hkv * n_qb,), (torch.int32,), "steps")
+    if O is None:
+        O = torch.empty((Nq, Hq, d), dtype=out_dtype, device=dev)
+    _out(O, (Nq, Hq, d), (torch.bfloat16, torch.float32), "O")
+    if ws is None:
+        ws = workspace(lib().sa_osk_prefill_workspace_size(S, Nq, Hq, Hkv, d, k, block), dev)
+    _ws(ws)
+    code = SA_F32 if O.dtype == torch.float32 else SA_BF16
+    _check(lib().sa_osk_prefill(_ptr(idx), _ptr(q_pos), _ptr(Q), _ptr(K), _ptr(V), S, Nq, Hq, Hkv, d, k, block,
+                                float(scale), float(tau), _ptr(kv_indptr), _ptr(kv_indices), _ptr(order), _ptr(steps),
+                                _ptr(O), code, _ptr(ws), ws.numel(), _stream(stream)))
+    return kv_indptr, kv_indices, order, steps, O
 
 
 def block_union_prefill_noalloc(idx, q_pos, Q, K, V, block: int, scale: float, kv_indptr, kv_indices, O,

@@ -25,7 +25,7 @@ HEADER = os.path.join(ROOT, "include", "sa.h")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVFLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]
 SOURCES = ["api.cu", "indexer.cu", "indexer_prefill.cu", "topk.cu", "topk_split.cu", "topk_dynamic.cu", "attn.cu",
-           "attn_small.cu", "attn_mid.cu", "union.cu", "route_attn.cu", "cp.cu"]
+           "attn_small.cu", "attn_mid.cu", "union.cu", "kap.cu", "route_attn.cu", "cp.cu"]
 
 
 def nvcc() -> str:

@@ -1108,6 +1108,57 @@ sa_status sa_decode_step_ex(const char* pattern, int n_layers, const void* const
 }
 
 // ---------------------------------------------------------------- prefill union
+}  // extern "C"
+
+// Paged causal attention of a prefill chunk over the group tables
+// (kv_indptr, kv_indices) written by the union kernels, or, with osk_order,
+// over each row tile's ordered list with ordered skipping (one CTA per row
+// tile, no key splits).
+static sa_status prefill_attn(const void* Q, const void* K, const void* V, const int32_t* q_pos,
+                              const int32_t* kv_indptr, const int32_t* kv_indices, int S, int Nq, int Hq, int Hkv,
+                              int block, float scale, void* O, sa_dtype out_dtype, sa::DeviceStatus* status,
+                              const int32_t* osk_order, int64_t osk_ld, float osk_tau, int32_t* osk_steps,
+                              cudaStream_t s, const char* who) {
+  sa::AttnArgs a{};
+  a.Q = reinterpret_cast<const uint16_t*>(Q);
+  a.K = reinterpret_cast<const uint16_t*>(K);
+  a.V = reinterpret_cast<const uint16_t*>(V);
+  a.prefill = 1;
+  a.q_pos = q_pos;
+  a.kv_indptr = kv_indptr;
+  a.kv_indices = kv_indices;
+  a.S = S;
+  a.block = block;
+  a.Nq = Nq;
+  a.L = 1;
+  a.B = 1;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.R = Nq * a.G;
+  a.n_mtiles = (a.R + 127) / 128;
+  a.n_split = osk_order != nullptr ? 1 : prefill_split(Hkv * a.n_mtiles);
+  a.keys_per_split = (int)round_up((size_t)((S + block - 1) / block) * block, 128);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.O = O;
+  a.out_f32 = out_dtype == SA_F32;
+  a.status = status;
+  a.osk_order = osk_order;
+  a.osk_ld = osk_ld;
+  a.osk_tau = osk_tau;
+  a.osk_steps = osk_steps;
+  CUtensorMap tm_q, tm_k, tm_v;
+  sa_status st2;
+  if ((st2 = make_rows_tmap(&tm_q, Q, (int64_t)Nq * Hq)) != SA_OK) return st2;
+  if ((st2 = make_block_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
+  if ((st2 = make_block_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
+  const cudaError_t e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, s);
+  if (e != cudaSuccess) return cuda_fail(who, e);
+  return SA_OK;
+}
+
+extern "C" {
+
 size_t sa_block_union_prefill_workspace_size(int S, int Nq, int Hq, int Hkv, int d, int k, int block) {
   (void)Nq;
   (void)Hq;
@@ -1140,40 +1191,67 @@ sa_status sa_block_union_prefill(const int32_t* idx, const int32_t* q_pos, const
   uint8_t* mark = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
   cudaError_t e = sa::launch_block_union(idx, Nq, k, S, block, Hkv, mark, kv_indptr, kv_indices, status_of(ws), s);
   if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill union", e);
-  sa::AttnArgs a{};
-  a.Q = reinterpret_cast<const uint16_t*>(Q);
-  a.K = reinterpret_cast<const uint16_t*>(K);
-  a.V = reinterpret_cast<const uint16_t*>(V);
-  a.prefill = 1;
-  a.q_pos = q_pos;
-  a.kv_indptr = kv_indptr;
-  a.kv_indices = kv_indices;
-  a.S = S;
-  a.block = block;
-  a.Nq = Nq;
-  a.L = 1;
-  a.B = 1;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.G = Hq / Hkv;
-  a.R = Nq * a.G;
-  a.n_mtiles = (a.R + 127) / 128;
-  a.n_split = prefill_split(Hkv * a.n_mtiles);
-  a.keys_per_split = (int)round_up((size_t)((S + block - 1) / block) * block, 128);
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.O = O;
-  a.out_f32 = out_dtype == SA_F32;
-  a.status = status_of(ws);
-  {
-    CUtensorMap tm_q, tm_k, tm_v;
-    sa_status st2;
-    if ((st2 = make_rows_tmap(&tm_q, Q, (int64_t)Nq * Hq)) != SA_OK) return st2;
-    if ((st2 = make_block_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
-    if ((st2 = make_block_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
-    e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, s);
-  }
-  if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill attention", e);
+  return prefill_attn(Q, K, V, q_pos, kv_indptr, kv_indices, S, Nq, Hq, Hkv, block, scale, O, out_dtype,
+                      status_of(ws), nullptr, 0, 0.f, nullptr, s, "sa_block_union_prefill attention");
+}
+
+// ---------------------------------------------------------------- ordered skipping
+size_t sa_kap_order_workspace_size(void) { return SA_WS_HEADER_BYTES; }
+
+sa_status sa_kap_order(const int32_t* idx, int Nq, int k, int S, int block, int q_block, const int32_t* kv_indptr,
+                       const int32_t* kv_indices, int32_t* order, int64_t ld, void* ws, size_t ws_bytes,
+                       void* stream) {
+  const char* who = "sa_kap_order";
+  if (Nq < 1 || k < 1 || S < 1 || block < 1 || q_block < 1) return fail(SA_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+  const int64_t nb = ((int64_t)S + block - 1) / block;
+  if (nb > sa::kKapMaxBlocks)
+    return fail(SA_ERR_UNSUPPORTED, "%s: %lld KV blocks (at most %d are built)", who, (long long)nb, sa::kKapMaxBlocks);
+  if (ld < nb) return fail(SA_ERR_INVALID_ARG, "%s: ld=%lld is below ceil(S/block)=%lld", who, (long long)ld, (long long)nb);
+  if (!idx || !kv_indptr || !kv_indices || !order) return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  sa_status st = check_ws(ws, ws_bytes, sa_kap_order_workspace_size(), who);
+  if (st != SA_OK) return st;
+  cudaError_t e = sa::launch_kap_order(idx, Nq, k, S, block, q_block, kv_indptr, kv_indices, order, ld,
+                                       status_of(ws), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(who, e);
   return SA_OK;
+}
+
+size_t sa_osk_prefill_workspace_size(int S, int Nq, int Hq, int Hkv, int d, int k, int block) {
+  return sa_block_union_prefill_workspace_size(S, Nq, Hq, Hkv, d, k, block);
+}
+
+sa_status sa_osk_prefill(const int32_t* idx, const int32_t* q_pos, const void* Q, const void* K, const void* V, int S,
+                         int Nq, int Hq, int Hkv, int d, int k, int block, float scale, float tau, int32_t* kv_indptr,
+                         int32_t* kv_indices, int32_t* order, int32_t* steps, void* O, sa_dtype out_dtype, void* ws,
+                         size_t ws_bytes, void* stream) {
+  const char* who = "sa_osk_prefill";
+  if (S < 1 || Nq < 1 || Hq < 1 || Hkv < 1 || k < 1) return fail(SA_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+  if (d != 128) return fail(SA_ERR_UNSUPPORTED, "%s: d=%d (only 128 is built)", who, d);
+  if (block != 64) return fail(SA_ERR_UNSUPPORTED, "%s: block=%d (only 64 is built)", who, block);
+  if (Hq % Hkv != 0) return fail(SA_ERR_INVALID_ARG, "%s: Hq not a multiple of Hkv", who);
+  const int G = Hq / Hkv;
+  if (128 % G != 0) return fail(SA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d does not divide 128", who, G);
+  if ((int64_t)Nq * G > (1 << 30)) return fail(SA_ERR_INVALID_ARG, "%s: too many query rows", who);
+  const int64_t nb = ((int64_t)S + block - 1) / block;
+  if (nb > sa::kKapMaxBlocks)
+    return fail(SA_ERR_UNSUPPORTED, "%s: %lld KV blocks (at most %d are built)", who, (long long)nb, sa::kKapMaxBlocks);
+  if (out_dtype != SA_BF16 && out_dtype != SA_F32) return fail(SA_ERR_INVALID_ARG, "%s: bad out_dtype", who);
+  if (!idx || !q_pos || !Q || !K || !V || !kv_indptr || !kv_indices || !order || !steps || !O)
+    return fail(SA_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
+    return fail(SA_ERR_INVALID_ARG, "%s: Q, K, V, O must be 16-byte aligned", who);
+  if (!(scale > 0.f)) return fail(SA_ERR_INVALID_ARG, "%s: scale must be > 0", who);
+  if (!(tau >= 0.f) || tau > 3.0e38f) return fail(SA_ERR_INVALID_ARG, "%s: tau must be finite and >= 0", who);
+  sa_status st = check_ws(ws, ws_bytes, sa_osk_prefill_workspace_size(S, Nq, Hq, Hkv, d, k, block), who);
+  if (st != SA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* mark = reinterpret_cast<uint8_t*>(ws) + SA_WS_HEADER_BYTES;
+  cudaError_t e = sa::launch_block_union(idx, Nq, k, S, block, Hkv, mark, kv_indptr, kv_indices, status_of(ws), s);
+  if (e != cudaSuccess) return cuda_fail("sa_osk_prefill union", e);
+  e = sa::launch_kap_order(idx, Nq, k, S, block, 128 / G, kv_indptr, kv_indices, order, nb, status_of(ws), s);
+  if (e != cudaSuccess) return cuda_fail("sa_osk_prefill order", e);
+  return prefill_attn(Q, K, V, q_pos, kv_indptr, kv_indices, S, Nq, Hq, Hkv, block, scale, O, out_dtype,
+                      status_of(ws), order, nb, tau, steps, s, "sa_osk_prefill attention");
 }
 
 }  // extern "C"
@@ -1239,38 +1317,6 @@ extern "C" sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const in
   uint8_t* mark = reinterpret_cast<uint8_t*>(scratch) + SA_WS_HEADER_BYTES;
   e = sa::launch_block_union(idx, Nq, k, S, block, Hkv, mark, kv_indptr, kv_indices, status_of(scratch), s);
   if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc union", e);
-  sa::AttnArgs a{};
-  a.Q = reinterpret_cast<const uint16_t*>(Q);
-  a.K = reinterpret_cast<const uint16_t*>(K);
-  a.V = reinterpret_cast<const uint16_t*>(V);
-  a.prefill = 1;
-  a.q_pos = q_pos;
-  a.kv_indptr = kv_indptr;
-  a.kv_indices = kv_indices;
-  a.S = S;
-  a.block = block;
-  a.Nq = Nq;
-  a.L = 1;
-  a.B = 1;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.G = Hq / Hkv;
-  a.R = Nq * a.G;
-  a.n_mtiles = (a.R + 127) / 128;
-  a.n_split = prefill_split(Hkv * a.n_mtiles);
-  a.keys_per_split = (int)round_up((size_t)nb * block, 128);
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.O = O;
-  a.out_f32 = out_dtype == SA_F32;
-  a.status = status_of(scratch);
-  {
-    CUtensorMap tm_q, tm_k, tm_v;
-    sa_status st2;
-    if ((st2 = make_rows_tmap(&tm_q, Q, (int64_t)Nq * Hq)) != SA_OK) return st2;
-    if ((st2 = make_block_tmap(&tm_k, K, (int64_t)Hkv * S)) != SA_OK) return st2;
-    if ((st2 = make_block_tmap(&tm_v, V, (int64_t)Hkv * S)) != SA_OK) return st2;
-    e = sa::launch_sparse_attn(a, tm_q, tm_k, tm_v, out_dtype == SA_F32, s);
-  }
-  if (e != cudaSuccess) return cuda_fail("sa_block_union_prefill_noalloc attention", e);
-  return SA_OK;
+  return prefill_attn(Q, K, V, q_pos, kv_indptr, kv_indices, S, Nq, Hq, Hkv, block, scale, O, out_dtype,
+                      status_of(scratch), nullptr, 0, 0.f, nullptr, s, "sa_block_union_prefill_noalloc attention");
 }

@@ -71,6 +71,18 @@ struct AttnLayout {
   static constexpr int kSlotOff = kBarOff + 8 * kNBar;
   static constexpr size_t kSmem = 1024 + kSlotOff + 16;
   static_assert(kSmem <= 232448, "shared memory budget");
+  // ordered skipping: half 1's (log2 tile mass, log2 running mass) per row
+  // [128] float2, the votes [kOskSlots tiles][4 warps], then the mbarriers
+  // xfull, xfree and dec[kOskSlots].  The producer reads the vote on tile
+  // j - kOskSlots before it issues tile j (the softmax and MMA warps read
+  // the vote on tile j - 3), so a vote's slot is free again once tile
+  // j + kOskSlots can be issued.
+  static constexpr int kOskSlots = 3 + kStages;
+  static constexpr int kOskOff = (kSlotOff + 16 + 15) & ~15;
+  static constexpr int kOskVoteOff = kOskOff + 128 * 8;
+  static constexpr int kOskBarOff = kOskVoteOff + kOskSlots * 4 * 4;
+  static constexpr size_t kSmemOsk = 1024 + kOskBarOff + (2 + kOskSlots) * 8;
+  static_assert(kSmemOsk <= 232448, "shared memory budget (ordered skipping)");
 };
 
 // 2^x on the special-function unit (ex2.approx.ftz.f32; 2^-inf = +0)
@@ -163,6 +175,7 @@ __device__ __forceinline__ int q_row(const AttnArgs& a, int b, int g, int r) {
 struct KeySrc {
   int len;   // decode: seq_len[b]
   int base;  // prefill: kv_indptr[g]
+  const int32_t* list;  // prefill: the blocks in the order they are read
   int kbeg, kend;
 };
 
@@ -172,7 +185,7 @@ struct KeySrc {
 // padding / invalid (an index past the sequence is reported and skipped).
 __device__ __forceinline__ int key_raw(const AttnArgs& a, const KeySrc& ks, int b, int jj) {
   if (jj >= ks.kend) return -1;
-  return a.prefill ? __ldg(&a.kv_indices[ks.base + jj / a.block]) : __ldg(&a.idx[(int64_t)b * a.k + jj]);
+  return a.prefill ? __ldg(&ks.list[jj / a.block]) : __ldg(&a.idx[(int64_t)b * a.k + jj]);
 }
 
 __device__ __forceinline__ int key_fix(const AttnArgs& a, const KeySrc& ks, int b, int jj, int raw, bool rep) {
@@ -199,7 +212,7 @@ __device__ __forceinline__ void store_out(const AttnArgs& a, int64_t off, const 
   }
 }
 
-template <bool PRECISE>
+template <bool PRECISE, bool OSK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v) {
@@ -217,6 +230,15 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   uint64_t* o_done = p_full + 2;  // [4]: completion of PV_i on o_done[i % 4]
   uint64_t* recv_bar = o_done + 4;
   uint32_t* slot = reinterpret_cast<uint32_t*>(smem + Lay::kSlotOff);
+  // ordered skipping: the row exchange between key halves, the votes, and
+  // their barriers (xfull: half 1 wrote, xfree: half 0 read, dec[t % slots]:
+  // the four row warps voted on tile t)
+  constexpr int kSlots = Lay::kOskSlots;
+  float2* osk_x = reinterpret_cast<float2*>(smem + Lay::kOskOff);
+  volatile uint32_t* osk_vote = reinterpret_cast<volatile uint32_t*>(smem + Lay::kOskVoteOff);
+  uint64_t* osk_xfull = reinterpret_cast<uint64_t*>(smem + Lay::kOskBarOff);
+  uint64_t* osk_xfree = osk_xfull + 1;
+  uint64_t* osk_dec = osk_xfull + 2;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int u = blockIdx.x;
@@ -244,6 +266,11 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     }
     for (int i = 0; i < 4; ++i) mbar_init(&o_done[i], 1);
     mbar_init(recv_bar, 1);
+    if constexpr (OSK) {
+      mbar_init(osk_xfull, 4);
+      mbar_init(osk_xfree, 4);
+      for (int i = 0; i < kSlots; ++i) mbar_init(&osk_dec[i], 4);
+    }
     fence_mbar_init();
   }
   tc_fence_before();
@@ -260,6 +287,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   if (!a.prefill) {
     ks.len = a.seq_len[b];
     ks.base = 0;
+    ks.list = nullptr;
     n_keys = a.k;
     if (a.idx_count != nullptr) {
       const int c = a.idx_count[b];
@@ -268,6 +296,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   } else {
     ks.len = a.S;
     ks.base = a.kv_indptr[g];
+    ks.list = OSK ? a.osk_order + (int64_t)mt * a.osk_ld : a.kv_indices + ks.base;
     n_keys = (a.kv_indptr[g + 1] - ks.base) * a.block;
   }
   // decode: the host's even split of k; prefill, and decode with a count of
@@ -279,6 +308,44 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
   ks.kbeg = split * per;
   ks.kend = min(n_keys, ks.kbeg + per);
   const int nt = ks.kend > ks.kbeg ? (ks.kend - ks.kbeg + kKT - 1) / kKT : 0;
+  int n_run = nt;  // tiles this role runs: nt, or fewer once ordered skipping stops
+
+  // Ordered skipping: whether the vote on tile t says stop (every row's
+  // share below tau); the tiles then end after tile t + 2 (the two tiles
+  // after it were already in flight), so the softmax and MMA warps read the
+  // vote on tile j - 3 before tile j.  ok = false when the wait gave up.
+  // One thread, then a whole warp.
+  auto osk_vote_stop = [&](int t, bool& ok) -> bool {
+    const int sl = t % kSlots;
+    ok = mbar_wait(&osk_dec[sl], (t / kSlots) & 1, kWaitLimitNs);
+    if (!ok) return false;
+    uint32_t any = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) any |= osk_vote[sl * 4 + w] & 1u;
+    return any == 0;
+  };
+  auto osk_vote_stop_warp = [&](int t, bool& ok) -> bool {
+    bool st = false, k2 = true;
+    if (lane == 0) st = osk_vote_stop(t, k2);
+    ok = __shfl_sync(0xffffffffu, k2, 0);
+    return __shfl_sync(0xffffffffu, st, 0);
+  };
+  // The softmax warps read the vote on tile j - 3 at the top of tile j
+  // without waiting on its barrier: a half-1 warp there has passed xfree of
+  // tile j - 2, and a half-0 warp xfull of tile j - 1, which the half-0
+  // warps reach only after voting on tile j - 3 (each barrier wait is an
+  // acquire of every earlier write of the arriving threads).
+  auto osk_vote_read_warp = [&](int t) -> bool {
+    uint32_t any = 0;
+    if (lane == 0) {
+      uint32_t v0, v1, v2, v3;
+      asm volatile("ld.volatile.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                   : "r"(smem_u32(const_cast<uint32_t*>(osk_vote + (t % kSlots) * 4))));
+      any = (v0 | v1 | v2 | v3) & 1u;
+    }
+    return __shfl_sync(0xffffffffu, any, 0) == 0;
+  };
 
   // producer lanes: raw entries of tile rows 4*lane .. 4*lane+3 of the next
   // kPre tiles, all loads in flight at once (a ring in registers, slot = tile
@@ -311,11 +378,38 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     const int pw = warp - kProdWarp0;
     const int64_t row_base = a.prefill ? (int64_t)g * a.S : a.seq_off[b] * a.Hkv + (int64_t)g * ks.len;
     bool stop = false;
+    // ordered skipping: the producer reads the vote on tile j - kSlots before
+    // issuing tile j, far enough back that the vote is in long before the
+    // stage is free; tiles issued past the end are drained below
+    int issued = nt;       // tiles issued
+    int osk_read = 0;      // votes read so far (tiles 0 .. osk_read-1 said continue)
+    int osk_n = nt;        // tiles the other roles run, once a stop vote is read
+    bool osk_failed = false;
     for (int j0 = 0; j0 < nt && !stop; j0 += kPre) {
 #pragma unroll
     for (int jj = 0; jj < kPre; ++jj) {
       const int j = j0 + jj;
       if (j >= nt) break;
+      if constexpr (OSK) {
+        if (j >= kSlots) {
+          bool ok3;
+          const bool st3 = osk_vote_stop_warp(j - kSlots, ok3);
+          osk_read = j - kSlots + 1;
+          if (!ok3) {
+            if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 5, j);
+            osk_failed = true;
+            issued = j;
+            stop = true;
+            break;
+          }
+          if (st3) {
+            osk_n = j - kSlots + 3;
+            issued = j;
+            stop = true;
+            break;
+          }
+        }
+      }
       const int s = j % ST;
       int tc[4];
 #pragma unroll
@@ -326,6 +420,8 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
       if (j >= ST && lane == 0) ok = mbar_wait(&kv_empty[s], ((j / ST) & 1) ^ 1, kWaitLimitNs);
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 0, j);
+        issued = j;
+        osk_failed = true;
         stop = true;
         break;
       }
@@ -364,7 +460,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
 #pragma unroll
           for (int b2 = 0; b2 < 2; ++b2) {
             const int jj = ks.kbeg + j * kKT + b2 * 64;  // first entry of the block
-            const int row = jj < ks.kend ? (int)(row_base + (int64_t)a.kv_indices[ks.base + jj / 64] * 64)
+            const int row = jj < ks.kend ? (int)(row_base + (int64_t)ks.list[jj / 64] * 64)
                                          : a.Hkv * a.S;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -398,6 +494,32 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
                     rq);
       }
     }
+    }
+    if constexpr (OSK) {
+      // the rest of the votes that can end the tiles before the last issued
+      // one, then wait for the issued tiles nobody will consume (their TMA
+      // writes land in this CTA's shared memory)
+      if (!osk_failed && osk_n == nt) {
+        for (int t = osk_read; t + 3 < issued; ++t) {
+          bool ok3;
+          const bool st3 = osk_vote_stop_warp(t, ok3);
+          if (!ok3) {
+            if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 6, t);
+            osk_failed = true;
+            break;
+          }
+          if (st3) {
+            osk_n = t + 3;
+            break;
+          }
+        }
+      }
+      if (!osk_failed)
+        for (int t = osk_n; t < issued; ++t)
+          if (!warp_wait(&kv_full[t % ST], (t / ST) & 1)) {
+            if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 7, t);
+            break;
+          }
     }
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer =======================
@@ -433,6 +555,21 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         ok = mbar_wait(&kv_full[s], (j / ST) & 1, kWaitLimitNs) &&
              mbar_wait(&s_free[sb], ((j >> 1) & 1) ^ 1, kWaitLimitNs);
         if (!ok) break;
+        if constexpr (OSK) {
+          // S buffer sb free again means every softmax warp is done with
+          // tile j - 2, and the half-0 warps voted on tile j - 3 before
+          // that: the vote is read without a wait.  A tile the producer
+          // issued and this warp does not consume is drained there.
+          if (j >= 3) {
+            uint32_t any = 0;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) any |= osk_vote[((j - 3) % kSlots) * 4 + w] & 1u;
+            if (any == 0) {
+              n_run = j;
+              break;
+            }
+          }
+        }
         tc_fence_after();
         const uint32_t kst = sbase + Lay::kStageOff + s * Lay::kStageBytes;
 #pragma unroll
@@ -444,13 +581,20 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         umma_commit(&s_full[sb]);
         if (j >= 1) ok = pv(j - 1);
       }
-      if (ok && nt >= 1) ok = pv(nt - 1);
+      if (ok && n_run >= 1) ok = pv(n_run - 1);
       if (!ok) report(a.status, kErrTimeout, kKernAttn, u, 1, 0);
     }
   } else {
     // ======================= softmax (warps 0-7) =======================
     bool failed = false;
     for (int j = 0; j < nt; ++j) {
+      if constexpr (OSK) {
+        if (j >= 3 && osk_vote_read_warp(j - 3)) {
+          n_run = j;
+          break;
+        }
+      }
+      float tile_sum = 0.f;  // this thread's weights of the tile (relative to m_ref)
       const int s = j % ST, sb = j & 1;
       if (!warp_wait(&s_full[sb], (j >> 1) & 1)) { failed = true; break; }
       if (tid == 0 && j < 8) SA_TL(kTlAttn, 12 + j);  // S of tile j ready
@@ -542,7 +686,8 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
                          pack_bf16(q[2], q[3]), pack_bf16(q[4], q[5]), pack_bf16(q[6], q[7]));
           }
         }
-        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tile_sum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        l_run += tile_sum;
         if (tid == 0 && j < 8) SA_TL(kTlAttn, 20 + j);  // P of tile j written
         fence_proxy_async_smem();
       }
@@ -552,11 +697,48 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
         mbar_arrive(&s_free[sb]);
         mbar_arrive(&p_full[sb]);
       }
+      if constexpr (OSK) {
+        // the tile's share of each row's running softmax mass over both key
+        // halves: half 1 passes its (log2 tile mass, log2 running mass) to
+        // half 0, which votes to continue while some row's share is at
+        // least osk_tau (a row that has seen no key yet always continues)
+        const float lA = (warp_active && tile_sum > 0.f) ? m_ref + __log2f(tile_sum) : -INFINITY;
+        const float lB = (warp_active && l_run > 0.f) ? m_ref + __log2f(l_run) : -INFINITY;
+        if (half == 1) {
+          if (j >= 1 && !warp_wait(osk_xfree, (j - 1) & 1)) { failed = true; break; }
+          __syncwarp();
+          osk_x[r_loc] = make_float2(lA, lB);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(osk_xfull);
+        } else {
+          if (!warp_wait(osk_xfull, j & 1)) { failed = true; break; }
+          __syncwarp();
+          const float2 o = osk_x[r_loc];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(osk_xfree);
+          bool cont = false;
+          if (warp_active && me.valid) {
+            const float mm = fmaxf(lB, o.y);
+            if (mm == -INFINITY) {
+              cont = true;
+            } else {
+              const float num = ex2_approx(lA - mm) + ex2_approx(o.x - mm);
+              const float den = ex2_approx(lB - mm) + ex2_approx(o.y - mm);
+              cont = !(num < a.osk_tau * den);
+            }
+          }
+          const bool any = __any_sync(0xffffffffu, cont);
+          if (lane == 0) {
+            osk_vote[(j % kSlots) * 4 + (warp & 3)] = ((uint32_t)j << 1) | (any ? 1u : 0u);
+            mbar_arrive(&osk_dec[j % kSlots]);
+          }
+        }
+      }
     }
     if (failed) {
       if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 2, warp);
     } else if (warp_active) {
-      if (nt > 0 && !warp_wait(&o_done[(nt - 1) & 3], ((nt - 1) >> 2) & 1)) {
+      if (n_run > 0 && !warp_wait(&o_done[(n_run - 1) & 3], ((n_run - 1) >> 2) & 1)) {
         if (lane == 0) report(a.status, kErrTimeout, kKernAttn, u, 3, warp);
       } else {
         have_o = true;
@@ -609,7 +791,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
         float f[32];
-        if (nt > 0) {
+        if (n_run > 0) {
           row_out(c2, f);
         } else {
 #pragma unroll
@@ -648,7 +830,7 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {
         float f[32];
-        if (have_o && nt > 0) {  // warp-uniform: TMEM loads are warp-collective
+        if (have_o && n_run > 0) {  // warp-uniform: TMEM loads are warp-collective
           row_out(c2, f);
         } else {
 #pragma unroll
@@ -727,6 +909,9 @@ sparse_attn_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tm_q, c
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   }
 
+  if constexpr (OSK) {
+    if (tid == 0 && a.osk_steps != nullptr) a.osk_steps[u] = n_run;
+  }
   tc_fence_before();
   __syncthreads();
   if (tid == 0) SA_TL(kTlAttn, 36);
@@ -748,8 +933,12 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, const CUtensorMap& tm_q, const
   const int units = attn_num_units(a);
   if (units == 0) return cudaSuccess;
   if (a.n_split != 1 && a.n_split != 2 && a.n_split != 4 && a.n_split != 8) return cudaErrorInvalidValue;
-  auto kern = precise_p ? sparse_attn_kernel<true> : sparse_attn_kernel<false>;
-  const size_t smem = precise_p ? AttnLayout<true>::kSmem : AttnLayout<false>::kSmem;
+  const bool osk = a.osk_order != nullptr;
+  if (osk && (!a.prefill || a.n_split != 1)) return cudaErrorInvalidValue;
+  auto kern = osk ? (precise_p ? sparse_attn_kernel<true, true> : sparse_attn_kernel<false, true>)
+                  : (precise_p ? sparse_attn_kernel<true, false> : sparse_attn_kernel<false, false>);
+  const size_t smem = osk ? (precise_p ? AttnLayout<true>::kSmemOsk : AttnLayout<false>::kSmemOsk)
+                          : (precise_p ? AttnLayout<true>::kSmem : AttnLayout<false>::kSmem);
   cudaError_t e = ensure_smem(kern, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

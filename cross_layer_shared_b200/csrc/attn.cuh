@@ -60,6 +60,16 @@ struct AttnArgs {
   int early = 0;
   float* small_po = nullptr;
   float2* small_pml = nullptr;
+  // prefill with ordered skipping (osk_order set, n_split 1): row tile mt
+  // reads the blocks osk_order[mt*osk_ld + 0 : |T|] in that order, 128 keys
+  // (two 64-token blocks) per tile.  After each tile every row's share of
+  // its running softmax mass that the tile added is checked; the first tile
+  // where every row's share is below osk_tau is followed by the two tiles
+  // already in flight and nothing more.  osk_steps[unit] = tiles run.
+  const int32_t* osk_order = nullptr;
+  int64_t osk_ld = 0;
+  float osk_tau = 0.f;
+  int32_t* osk_steps = nullptr;
   DeviceStatus* status;
 };
 

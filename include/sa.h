@@ -407,6 +407,63 @@ sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const int32_t* q_po
                                          int32_t* kv_indices, void* O, sa_dtype out_dtype, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Priority-ordered block execution with early skipping for a prefill chunk
+ * [CoSA lay summary: a kernel-aware proxy hands the attention kernel a
+ * priority list of blocks instead of a yes/no list; the ordered-skipping
+ * kernel reads the blocks in that order, builds a progressive score from
+ * the most important ones first and then skips the rest].  The pages give
+ * neither the proxy's formula nor the skip rule; the readings built here:
+ *
+ * sa_kap_order (the proxy): for query block i (queries i*q_block ..
+ * i*q_block + q_block - 1; the last block may be shorter), block B's hit
+ * count is the number of entries idx[p, e] of those queries with
+ * 0 <= idx[p,e] < S and idx[p,e] / block == B.  order[i, 0 : nT] is the
+ * union table kv_indices[kv_indptr[0] : kv_indptr[1]] (nT blocks, the
+ * table of group 0; every group's table is the same set) ordered by hit
+ * count, larger first, equal counts by ascending block id.
+ *   idx        int32 [Nq, k]
+ *   order      int32 [ceil(Nq / q_block), ld], ld >= ceil(S / block);
+ *              entries past nT of each row are not written
+ * Supported: ceil(S / block) <= 16384.  A table entry outside
+ * [0, ceil(S/block)) is reported (SA_ERR_DEVICE, kernel id 5) and ranked
+ * with count 0.  Workspace: sa_kap_order_workspace_size() bytes (the
+ * status block).
+ *
+ * sa_osk_prefill (union, proxy and ordered-skipping attention in one
+ * call): the block union of sa_block_union_prefill (kv_indptr,
+ * kv_indices), then sa_kap_order with q_block = 128 / (Hq / Hkv) (one
+ * query block fills the 128 rows of an attention tile), then attention
+ * per unit (query block i, KV group g) - the rows (p, h) of the block's
+ * queries and the group's heads:
+ *   step n = blocks order[i][2n] and order[i][2n+1] (128 keys);
+ *   after step n, a row's share is the weight its visible keys in the
+ *   step add to its softmax, relative to its running sum over steps
+ *   0..n (+inf while it has seen no key); the first step where every row
+ *   of the unit has a share below tau ends the unit two steps later (the
+ *   steps already in flight finish); N = min(steps in the list, that
+ *   step + 3), or all steps when no step qualifies;
+ *   O[p, h] = softmax attention of row (p, h) over its visible keys
+ *   (t <= q_pos[p], t < S) of steps 0..N-1.
+ * tau = 0 never skips: O equals sa_block_union_prefill's output.
+ *   order      int32 [ceil(Nq*G/128), ceil(S/block)] (output, G = Hq/Hkv)
+ *   steps      int32 [Hkv * ceil(Nq*G/128)] (output): N of unit
+ *              g * ceil(Nq*G/128) + i
+ * Other arguments and outputs as in sa_block_union_prefill.  Supported:
+ * d = 128, block = 64, G dividing 128, ceil(S/block) <= 16384.
+ * Workspace: sa_osk_prefill_workspace_size bytes.
+ * ---------------------------------------------------------------------- */
+size_t sa_kap_order_workspace_size(void);
+sa_status sa_kap_order(const int32_t* idx, int Nq, int k, int S, int block, int q_block,
+                       const int32_t* kv_indptr, const int32_t* kv_indices, int32_t* order,
+                       int64_t ld, void* ws, size_t ws_bytes, void* stream);
+size_t sa_osk_prefill_workspace_size(int S, int Nq, int Hq, int Hkv, int d, int k, int block);
+sa_status sa_osk_prefill(const int32_t* idx, const int32_t* q_pos, const void* Q, const void* K,
+                         const void* V, int S, int Nq, int Hq, int Hkv, int d, int k, int block,
+                         float scale, float tau, int32_t* kv_indptr, int32_t* kv_indices,
+                         int32_t* order, int32_t* steps, void* O, sa_dtype out_dtype, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Context-parallel decode: one sequence's context sharded over N ranks
  * [CLSA news article, section "Ce que cela signifie pour l'inference sur
  * longs contextes": how the method behaves past 128K tokens is left open.

@@ -59,7 +59,7 @@ def load(path: str):
     lb.oracle_cp_select.argtypes = [P, P, I, I, I, I, P]
     lb.oracle_topk_dynamic.argtypes = [P, I64, P, I, I, D, P, P]
     lb.oracle_kap_order.argtypes = [P, I, I, I, I, I, P, I, P, I64]
-    lb.oracle_osk_prefill_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, P, I64, I, I, D, D, I, P, I, P, P, P, I64]
+    lb.oracle_osk_prefill_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, P, I64, I, I, D, D, I, P, I, P, P, P, P, I64]
     lb.oracle_num_threads.restype = I
     return lb
 
@@ -247,13 +247,15 @@ def kap_order(idx, S: int, block: int, q_block: int, T) -> np.ndarray:
 
 
 def osk_prefill_attn(Q, q_pos, K, V, block: int, order, q_block: int, scale: float, tau: float,
-                     lag: int = 2, units=None):
+                     lag: int = 2, units=None, steps_in=None):
     """CoSA's ordered-skipping kernel under the reading in oracle/sa_oracle.c:
     unit (query block i, KV group g) runs the blocks of order[i] two per
     step and stops lag steps after the first step whose largest row share
     of the running softmax mass is below tau.  Returns (O [Nq,Hq,d] fp64,
     NaN outside the computed units; steps [n_units] int32, -1 where not
-    computed; crit [n_units, n_steps] fp64, NaN where not computed)."""
+    computed; crit [n_units, n_steps] fp64, NaN where not computed).  With
+    steps_in [n_units], unit u runs steps_in[u] steps instead (the attention
+    over a given prefix of its order; crit is still the rule's)."""
     Q = _c(Q, np.uint16)
     Nq, Hq, d = Q.shape
     K = _c(K, np.uint16)
@@ -270,7 +272,8 @@ def osk_prefill_attn(Q, q_pos, K, V, block: int, order, q_block: int, scale: flo
     ordp = order if order.size else np.zeros(1, np.int32)
     lib().oracle_osk_prefill_attn(_p(Q), _p(_c(q_pos, np.int32)), _p(K), _p(V), S, Nq, Hq, Hkv, d, block,
                                   _p(ordp), max(1, nT), nT, q_block, float(scale), float(tau), int(lag),
-                                  _p(u), 0 if u is None else int(u.size), _p(O), _p(steps), _p(crit),
+                                  _p(u), 0 if u is None else int(u.size),
+                                  _p(None if steps_in is None else _c(steps_in, np.int32)), _p(O), _p(steps), _p(crit),
                                   crit.shape[1])
     return O, steps, crit[:, :n_steps]
 

@@ -557,6 +557,9 @@ void oracle_kap_order(const int32_t* idx, int Nq, int k, int S, int block, int q
  *     qualifies.  n_steps = ceil(nT / 2).
  *   O[p,h] = softmax attention of row (p, h) over its visible keys of
  *   steps 0..N-1.
+ * With steps_in given, unit u runs N = steps_in[u] steps (clamped to
+ * [0, n_steps]) whatever the rule says: attention over a prefix of the
+ * order fixed by the caller.
  * Only the units listed in units[0..n_units) are computed (all of them
  * when units is NULL); unit id u = g * n_qb + i.  steps[u] = N; crit, when
  * given, gets c_n at crit[u * ld_crit + n] for n < n_steps (the running
@@ -567,8 +570,9 @@ void oracle_kap_order(const int32_t* idx, int Nq, int k, int S, int block, int q
 void oracle_osk_prefill_attn(const uint16_t* Q, const int32_t* q_pos, const uint16_t* K,
                              const uint16_t* V, int S, int Nq, int Hq, int Hkv, int d, int block,
                              const int32_t* order, int64_t ld, int nT, int q_block, double scale,
-                             double tau, int lag, const int32_t* units, int n_units, double* O,
-                             int32_t* steps, double* crit, int64_t ld_crit) {
+                             double tau, int lag, const int32_t* units, int n_units,
+                             const int32_t* steps_in, double* O, int32_t* steps, double* crit,
+                             int64_t ld_crit) {
   const int G = Hq / Hkv;
   const int n_qb = (Nq + q_block - 1) / q_block;
   const int n_steps = (nT + 1) / 2;
@@ -627,6 +631,7 @@ void oracle_osk_prefill_attn(const uint16_t* Q, const int32_t* q_pos, const uint
       if (crit) crit[(int64_t)u * ld_crit + n] = c;
       if (c < tau && N == n_steps) N = (n + 1 + lag < n_steps) ? n + 1 + lag : n_steps;
     }
+    if (steps_in) N = steps_in[u] < 0 ? 0 : (steps_in[u] > n_steps ? n_steps : steps_in[u]);
     steps[u] = N;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < rows; ++r) {

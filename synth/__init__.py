@@ -330,6 +330,10 @@ class PrefillConfig:
     seed: int
     hot_regions: int = 16
     region_len: int = 256
+    # attention queries drawn toward the hot regions: Q[p,h] gets q_gain * v_hat(h's KV head)
+    # added, and the hot K rows carry hot_k_gain * v_hat (0 and 2 in the plain chunk)
+    q_gain: float = 0.0
+    hot_k_gain: float = 2.0
 
     @property
     def q_pos(self) -> np.ndarray:
@@ -363,7 +367,13 @@ class PrefillConfig:
 
     def Q(self) -> np.ndarray:
         n = self.chunk * self.Hq * self.d
-        return normal_bf16(self.seed, TID_Q, n).reshape(self.chunk, self.Hq, self.d)
+        if self.q_gain == 0.0:
+            return normal_bf16(self.seed, TID_Q, n).reshape(self.chunk, self.Hq, self.d)
+        x = normal_at(self.seed, TID_Q, np.arange(n)).reshape(self.chunk, self.Hq, self.d)
+        G = self.Hq // self.Hkv
+        for h in range(self.Hq):
+            x[:, h, :] += (self.q_gain * self.v_hat(h // G)).astype(np.float32)
+        return f32_to_bf16_bits(x.astype(np.float32))
 
     def ki_stream(self):
         return TID_KI, 0.125
@@ -388,7 +398,7 @@ class PrefillConfig:
         if pos.size == 0:
             return pos, np.zeros((0, self.d), np.uint16)
         flat = ((h * self.S + pos)[:, None] * self.d + np.arange(self.d)[None, :]).astype(np.uint64)
-        x = normal_at(self.seed, TID_K, flat) + (2.0 * self.v_hat(h)).astype(np.float32)
+        x = normal_at(self.seed, TID_K, flat) + (self.hot_k_gain * self.v_hat(h)).astype(np.float32)
         return pos, f32_to_bf16_bits(x.astype(np.float32))
 
     def KI_full(self) -> np.ndarray:
@@ -441,6 +451,12 @@ def workload(name: str):
                             q_rho=0.9)
     if name == "c4":
         return PrefillConfig("c4", 131072, 2048, 16, 128, 2048, 64, 32, 8, 128, seed=1238)
+    if name == "c4-concentrated":
+        # the c4 chunk with the attention drawn to the hot regions the indexer
+        # finds: same indexer inputs, queries biased along each group's
+        # direction, hot K rows four times further along it
+        return PrefillConfig("c4-concentrated", 131072, 2048, 16, 128, 2048, 64, 32, 8, 128, seed=1238,
+                             q_gain=16.0, hot_k_gain=8.0)
     if name == "c5":
         return DecodeConfig("c5", c5_seq_lens(1239), 16, 128, 2048, "FSSS" * 12, 32, 8, 128, seed=1239)
     raise KeyError(name)
@@ -454,4 +470,6 @@ DESCRIPTIONS = {
     "c3": "decode B=4 S=131072, one indexer pass 16x128, k=2048, shared by 24 cross-decoder layers, 32q/8kv d=128",
     "c4": "chunked prefill 2048 queries vs 131072-token cache, indexer 16x128 k=2048, 64-token blocks, 32q/8kv d=128",
     "c5": "decode B=32 ragged S in [8192,131072], indexer 16x128, k=2048, 48 layers F,S,S,S, 32q/8kv d=128",
+    "c4-concentrated": "the c4 chunk with its attention queries biased along each KV group's hot-region "
+                       "direction (gain 16) and the hot K rows at gain 8 instead of 2",
 }

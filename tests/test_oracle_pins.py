@@ -894,3 +894,24 @@ def test_osk_a_row_with_nothing_visible_keeps_the_unit_running():
     assert steps1[0] == 2
     np.testing.assert_allclose(O1[0, 0], bf16_bits_to_f32(V[0, 32:48]).astype(np.float64).mean(axis=0),
                                rtol=0, atol=1e-12)
+
+
+def test_osk_given_steps_is_the_attention_over_that_prefix():
+    # steps_in fixes N per unit: the output is the paged attention over the
+    # first 2N blocks of the unit's order, whatever tau says
+    rng, q_pos, Q, K, V, idx = _osk_case(55)
+    S, block, Hkv, q_block = K.shape[1], 64, K.shape[0], 3
+    T = list(range((S + block - 1) // block))
+    order = np.stack([rng.permutation(T) for _ in range(2)]).astype(np.int32)
+    steps_in = np.array([2, 0, 5, 1], np.int32)   # unit u = g * 2 + i
+    O, steps, _ = oracle.osk_prefill_attn(Q, q_pos, K, V, block, order, q_block, 0.25, tau=0.5, steps_in=steps_in)
+    assert steps.tolist() == [2, 0, 5, 1]
+    G = Q.shape[1] // Hkv
+    for u, N in enumerate(steps_in):
+        g, i = divmod(u, 2)
+        sub = np.sort(order[i, :2 * N]).astype(np.int32)
+        want = oracle.paged_prefill_attn(Q, q_pos, K, V, block, [j * len(sub) for j in range(Hkv + 1)],
+                                         np.tile(sub, Hkv), 0.25)
+        rows = slice(i * q_block, (i + 1) * q_block)
+        heads = slice(g * G, (g + 1) * G)
+        np.testing.assert_allclose(O[rows, heads], want[rows, heads], rtol=0, atol=1e-12)
