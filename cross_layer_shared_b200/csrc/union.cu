@@ -14,27 +14,16 @@
 namespace sa {
 namespace {
 
-// A block already marked is not stored again: many selected tokens fall in
-// the same few blocks, and stores of one byte address from many threads
-// serialise in L2, while loads of it do not.  Four entries per thread are
-// loaded before any is looked at.
 __global__ void union_mark_kernel(const int32_t* __restrict__ idx, int64_t n, int S, int block,
                                   uint8_t* __restrict__ mark, DeviceStatus* status) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n; i0 += 4 * stride) {
-    int t[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) t[u] = i0 + u * stride < n ? __ldg(&idx[i0 + u * stride]) : -1;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (t[u] < 0) continue;
-      if (t[u] >= S) {
-        report(status, kErrDevice, kKernUnion, i0 + u * stride, t[u], S);
-        continue;
-      }
-      uint8_t* m = &mark[t[u] / block];
-      if (*reinterpret_cast<volatile uint8_t*>(m) == 0) *m = 1;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int t = idx[i];
+    if (t < 0) continue;
+    if (t >= S) {
+      report(status, kErrDevice, kKernUnion, i, t, S);
+      continue;
     }
+    mark[t / block] = 1;
   }
 }
 
