@@ -145,3 +145,59 @@ def test_combine_is_order_free_and_splits_compose(P, rows, seed):
         merged_o = (first * L[:, None])[None]
         again = oracle.combine_partials(np.concatenate([merged_o, o[2:]]), np.concatenate([merged_ml, ml[2:]]))
         np.testing.assert_allclose(again, whole, rtol=1e-10, atol=1e-12)
+
+
+def _osk_inputs(rng, Nq, Hq, Hkv, S, d, block):
+    q_pos = np.sort(rng.choice(S, Nq, replace=False)).astype(np.int32)
+    Q = bf16(rng.standard_normal((Nq, Hq, d)) * 2)
+    K = bf16(rng.standard_normal((Hkv, S, d)))
+    V = bf16(rng.standard_normal((Hkv, S, d)))
+    return q_pos, Q, K, V
+
+
+@settings(max_examples=30, deadline=None)
+@given(st.integers(1, 6), st.sampled_from([(2, 1), (4, 2), (2, 2)]), st.integers(40, 400), st.integers(1, 3),
+       st.integers(0, 2**31 - 1))
+def test_osk_steps_fall_as_tau_rises_and_the_rule_holds(Nq, heads, S, q_block, seed):
+    """Ordered skipping: the step count of every unit is non-increasing in
+    tau (the first step below a larger tau comes no later), tau = 0 runs
+    every step, and each count satisfies the rule against the unit's
+    per-step scores."""
+    Hq, Hkv = heads
+    block, d, lag = 8, 4, 2
+    rng = np.random.default_rng(seed)
+    q_pos, Q, K, V = _osk_inputs(rng, Nq, Hq, Hkv, S, d, block)
+    nb = (S + block - 1) // block
+    n_qb = (Nq + q_block - 1) // q_block
+    order = np.stack([rng.permutation(nb) for _ in range(n_qb)]).astype(np.int32)
+    n_steps = (nb + 1) // 2
+    prev = None
+    for tau in (0.0, 0.01, 0.1, 0.3, 0.7, 1.5):
+        _, steps, crit = oracle.osk_prefill_attn(Q, q_pos, K, V, block, order, q_block, 0.5, tau, lag=lag)
+        if tau == 0.0:
+            assert np.all(steps == n_steps)
+        for u, N in enumerate(steps):
+            below = np.nonzero(crit[u] < tau)[0]
+            want = n_steps if below.size == 0 else min(n_steps, int(below[0]) + 1 + lag)
+            assert N == want
+        if prev is not None:
+            assert np.all(steps <= prev)
+        prev = steps
+
+
+@settings(max_examples=25, deadline=None)
+@given(st.integers(1, 5), st.integers(30, 300), st.integers(0, 2**31 - 1))
+def test_osk_without_skipping_ignores_the_order(Nq, S, seed):
+    """tau = 0 runs every step, so any two orders of the same table give the
+    same softmax over the same keys."""
+    rng = np.random.default_rng(seed)
+    block, d, Hq, Hkv, q_block = 8, 4, 2, 1, 2
+    q_pos, Q, K, V = _osk_inputs(rng, Nq, Hq, Hkv, S, d, block)
+    nb = (S + block - 1) // block
+    n_qb = (Nq + q_block - 1) // q_block
+    T = np.sort(rng.choice(nb, max(1, nb // 2), replace=False)).astype(np.int32)
+    o1 = np.stack([rng.permutation(T) for _ in range(n_qb)]).astype(np.int32)
+    o2 = np.stack([rng.permutation(T) for _ in range(n_qb)]).astype(np.int32)
+    A, _, _ = oracle.osk_prefill_attn(Q, q_pos, K, V, block, o1, q_block, 0.5, 0.0)
+    B, _, _ = oracle.osk_prefill_attn(Q, q_pos, K, V, block, o2, q_block, 0.5, 0.0)
+    np.testing.assert_allclose(A, B, rtol=0, atol=1e-12)
