@@ -41,9 +41,18 @@ kap_order_kernel(const int32_t* __restrict__ idx, int Nq, int k, int S, int bloc
   const int p1 = min(Nq, p0 + q_block);
   const int64_t n = (int64_t)(p1 - p0) * k;
   const int32_t* rows = idx + (int64_t)p0 * k;
-  for (int64_t e = tid; e < n; e += kKapThreads) {
-    const int t = __ldg(&rows[e]);
-    if (t >= 0 && t < S) atomicAdd(&cnt[t / block], 1u);
+  // eight coalesced loads in flight per thread before the atomics
+  constexpr int kBatch = 8;
+  for (int64_t e0 = tid; e0 < n; e0 += (int64_t)kBatch * kKapThreads) {
+    int t[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int64_t e = e0 + (int64_t)u * kKapThreads;
+      t[u] = e < n ? __ldg(&rows[e]) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (t[u] >= 0 && t[u] < S) atomicAdd(&cnt[t[u] / block], 1u);
   }
   __syncthreads();
   for (int j = tid; j < np; j += kKapThreads) {
