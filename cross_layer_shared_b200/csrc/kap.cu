@@ -29,7 +29,13 @@ kap_order_kernel(const int32_t* __restrict__ idx, int Nq, int k, int S, int bloc
   extern __shared__ uint64_t kap_smem[];
   const int tid = threadIdx.x;
   const int i = blockIdx.x;
-  const int nT = kv_indptr[1] - kv_indptr[0];
+  // a table longer than the KV blocks (or negative) is reported and clamped:
+  // the shared-memory key array is sized for at most nb entries
+  int nT = kv_indptr[1] - kv_indptr[0];
+  if (nT < 0 || nT > nb) {
+    if (tid == 0) report(status, kErrDevice, kKernUnion, -1, nT, nb);
+    nT = nT < 0 ? 0 : nb;
+  }
   const int32_t* T = kv_indices + kv_indptr[0];
   int np = 1;
   while (np < nT) np <<= 1;

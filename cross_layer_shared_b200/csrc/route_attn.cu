@@ -67,7 +67,7 @@ struct PartLayout {
 
 __device__ __forceinline__ void comp_bar() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kCompWarps) : "memory"); }
 
-// lane 0 waits, the verdict is the warp's
+// lane 0 waits, the outcome is the warp's
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, kWaitLimitNs);

@@ -426,7 +426,8 @@ sa_status sa_block_union_prefill_noalloc(const int32_t* idx, const int32_t* q_po
  *              entries past nT of each row are not written
  * Supported: ceil(S / block) <= 16384.  A table entry outside
  * [0, ceil(S/block)) is reported (SA_ERR_DEVICE, kernel id 5) and ranked
- * with count 0.  Workspace: sa_kap_order_workspace_size() bytes (the
+ * with count 0; a table longer than ceil(S/block) entries is reported the
+ * same way (entry -1) and only its first ceil(S/block) entries are ordered.  Workspace: sa_kap_order_workspace_size() bytes (the
  * status block).
  *
  * sa_osk_prefill (union, proxy and ordered-skipping attention in one
