@@ -175,3 +175,36 @@ def test_wait_probe_checks_its_arguments_before_any_launch(lib):
     assert lib.sa_wait_probe(fake, 256, 2_000_000_000, None) == sa.SA_ERR_INVALID_ARG  # above 1 s
     assert lib.sa_wait_probe(None, 256, 2_000_000, None) == sa.SA_ERR_WORKSPACE
     assert lib.sa_wait_probe(fake, 64, 2_000_000, None) == sa.SA_ERR_WORKSPACE
+
+
+def test_ordered_skipping_entry_points_reject_bad_requests(lib):
+    """sa_kap_order / sa_osk_prefill check their arguments before any launch."""
+    # the proxy: query blocks of at least one query, ld covering every KV block,
+    # and at most 16384 KV blocks
+    ws = lib.sa_kap_order_workspace_size()
+    assert ws == sa.WS_HEADER_BYTES
+    assert lib.sa_kap_order(FAKE, 64, 32, 4096, 64, 0, FAKE, FAKE, FAKE, 64, FAKE_WS, ws, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_kap_order(FAKE, 64, 32, 4096, 64, 32, FAKE, FAKE, FAKE, 63, FAKE_WS, ws, None) == sa.SA_ERR_INVALID_ARG
+    assert b"ld=63" in lib.sa_last_error()
+    assert lib.sa_kap_order(FAKE, 64, 32, 64 * 16385, 64, 32, FAKE, FAKE, FAKE, 16385, FAKE_WS, ws,
+                            None) == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_kap_order(FAKE, 64, 32, 4096, 64, 32, None, FAKE, FAKE, 64, FAKE_WS, ws, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_kap_order(FAKE, 64, 32, 4096, 64, 32, FAKE, FAKE, FAKE, 64, None, ws, None) == sa.SA_ERR_WORKSPACE
+
+    wsz = lib.sa_osk_prefill_workspace_size(4096, 64, 32, 8, 128, 32, 64)
+    assert wsz == lib.sa_block_union_prefill_workspace_size(4096, 64, 32, 8, 128, 32, 64)
+
+    def osk(S=4096, Hq=32, Hkv=8, d=128, block=64, tau=1e-3, steps=FAKE, ws_=FAKE_WS):
+        return lib.sa_osk_prefill(FAKE, FAKE, FAKE, FAKE, FAKE, S, 64, Hq, Hkv, d, 32, block, 0.088, tau, FAKE, FAKE,
+                                  FAKE, steps, FAKE, 0, ws_, 1 << 20, None)
+
+    assert osk(d=64) == sa.SA_ERR_UNSUPPORTED
+    assert osk(block=32) == sa.SA_ERR_UNSUPPORTED
+    assert osk(Hq=24, Hkv=8) == sa.SA_ERR_UNSUPPORTED and b"divide 128" in lib.sa_last_error()  # G = 3
+    assert osk(Hq=30, Hkv=8) == sa.SA_ERR_INVALID_ARG  # Hq not a multiple of Hkv
+    assert osk(S=64 * 16385) == sa.SA_ERR_UNSUPPORTED
+    assert osk(tau=-0.5) == sa.SA_ERR_INVALID_ARG and b"tau" in lib.sa_last_error()
+    assert osk(tau=float("nan")) == sa.SA_ERR_INVALID_ARG
+    assert osk(tau=float("inf")) == sa.SA_ERR_INVALID_ARG
+    assert osk(steps=None) == sa.SA_ERR_INVALID_ARG
+    assert osk(ws_=None) == sa.SA_ERR_WORKSPACE
