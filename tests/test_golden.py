@@ -72,3 +72,20 @@ def test_golden_sparse_attention_partial():
     assert abs(ml[0, 0, 0, 0] - c["expected_m"]) <= 1e-15
     assert abs(ml[0, 0, 0, 1] - c["expected_l"]) <= 1e-15
     np.testing.assert_allclose(o[0, 0, 0], c["expected_o"], rtol=0, atol=1e-15)
+
+
+def test_golden_ordered_skipping():
+    c = G["ordered_skipping"]
+    idx = np.array(c["idx"], np.int32)
+    order = oracle.kap_order(idx, c["S"], c["block"], c["q_block"], c["table"])
+    assert order.tolist() == c["expected_order"]
+    S = c["S"]
+    K = np.array([[[x, 0.0] for x in c["K_x"]]], np.float32)
+    V = np.array([[[float(t), 1.0] for t in range(S)]], np.float32)
+    Q = np.array([[c["q"]]], np.float32)
+    for case in c["cases"]:
+        O, steps, crit = oracle.osk_prefill_attn(bf(Q), c["q_pos"], bf(K), bf(V), c["block"], order, c["q_block"],
+                                                 float(np.log(2.0)), case["tau"], lag=case["lag"])
+        np.testing.assert_allclose(crit[0], c["expected_crit"], rtol=1e-13)
+        assert steps[0] == case["expected_steps"], case
+        np.testing.assert_allclose(O[0, 0], case["expected_o"], rtol=0, atol=1e-13)
