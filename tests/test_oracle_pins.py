@@ -915,3 +915,81 @@ def test_osk_given_steps_is_the_attention_over_that_prefix():
         rows = slice(i * q_block, (i + 1) * q_block)
         heads = slice(g * G, (g + 1) * G)
         np.testing.assert_allclose(O[rows, heads], want[rows, heads], rtol=0, atol=1e-12)
+
+
+def _osk_brute(Q, q_pos, K, V, block, order, q_block, scale, tau, lag):
+    """The ordered-skipping rule written out directly on tiny inputs: after
+    each step the shares are recomputed from every logit seen so far (no
+    running update), then the output over the steps run."""
+    Qf, Kf, Vf = (bf16_bits_to_f32(x).astype(np.float64) for x in (Q, K, V))
+    Nq, Hq, d = Qf.shape
+    Hkv, S, _ = Kf.shape
+    G = Hq // Hkv
+    n_qb, nT = order.shape
+    n_steps = (nT + 1) // 2
+    O = np.zeros((Nq, Hq, d))
+    steps = np.zeros(n_qb * Hkv, np.int64)
+    crit = np.zeros((n_qb * Hkv, n_steps))
+    for g in range(Hkv):
+        for i in range(n_qb):
+            rows = [(p, g * G + h) for p in range(i * q_block, min(Nq, (i + 1) * q_block)) for h in range(G)]
+            step_keys = []
+            for n in range(n_steps):
+                ks = []
+                for b in order[i, 2 * n:2 * n + 2]:
+                    ks += [t for t in range(int(b) * block, int(b) * block + block) if t < S]
+                step_keys.append(ks)
+            N = n_steps
+            for n in range(n_steps):
+                c = -math.inf
+                for (p, h) in rows:
+                    seen = [t for m in range(n + 1) for t in step_keys[m] if t <= q_pos[p]]
+                    if not seen:
+                        share = math.inf
+                    else:
+                        z = {t: scale * float(Qf[p, h] @ Kf[g, t]) for t in seen}
+                        M = max(z.values())
+                        L = sum(math.exp(v - M) for v in z.values())
+                        a = sum(math.exp(z[t] - M) for t in step_keys[n] if t <= q_pos[p])
+                        share = a / L
+                    c = max(c, share)
+                crit[g * n_qb + i, n] = c
+                if c < tau and N == n_steps:
+                    N = min(n_steps, n + 1 + lag)
+            steps[g * n_qb + i] = N
+            for (p, h) in rows:
+                ks = [t for m in range(N) for t in step_keys[m] if t <= q_pos[p]]
+                if ks:
+                    z = np.array([scale * float(Qf[p, h] @ Kf[g, t]) for t in ks])
+                    w = np.exp(z - z.max())
+                    O[p, h] = (w[:, None] * Vf[g, ks]).sum(0) / w.sum()
+    return O, steps, crit
+
+
+def test_osk_brute_force_on_tiny_chunks():
+    rng = np.random.default_rng(57)
+    for trial in range(8):
+        Nq = int(rng.integers(1, 5))
+        Hkv = int(rng.choice([1, 2]))
+        G = int(rng.choice([1, 2, 3]))
+        S = int(rng.integers(10, 48))
+        block = int(rng.choice([3, 4, 8]))
+        d = 4
+        q_block = int(rng.integers(1, 4))
+        q_pos = np.sort(rng.choice(S, Nq, replace=False)).astype(np.int32)
+        Q = bf(rng.standard_normal((Nq, Hkv * G, d)) * 1.5)
+        K = bf(rng.standard_normal((Hkv, S, d)))
+        V = bf(rng.standard_normal((Hkv, S, d)))
+        nb = (S + block - 1) // block
+        T = np.sort(rng.choice(nb, int(rng.integers(1, nb + 1)), replace=False))
+        n_qb = (Nq + q_block - 1) // q_block
+        order = np.stack([rng.permutation(T) for _ in range(n_qb)]).astype(np.int32)
+        tau = float(rng.choice([0.0, 0.05, 0.2, 0.5]))
+        lag = int(rng.integers(0, 3))
+        O, steps, crit = oracle.osk_prefill_attn(Q, q_pos, K, V, block, order, q_block, 0.7, tau, lag=lag)
+        Ob, sb, cb = _osk_brute(Q, q_pos, K, V, block, order, q_block, 0.7, tau, lag)
+        finite = np.isfinite(cb)
+        assert np.array_equal(np.isfinite(crit), finite), trial
+        np.testing.assert_allclose(crit[finite], cb[finite], rtol=1e-12, atol=0)
+        assert np.array_equal(steps, sb), (trial, steps, sb)
+        np.testing.assert_allclose(O, Ob, rtol=0, atol=1e-12)
