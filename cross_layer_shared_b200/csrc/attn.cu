@@ -118,10 +118,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // Bulk copy of `bytes` from this CTA's shared memory to the same-offset
 // layout in CTA `rank` of the cluster, completion counted on that CTA's
 // mbarrier (both given as this CTA's addresses, mapped with mapa).
