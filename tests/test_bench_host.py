@@ -72,3 +72,17 @@ def test_byte_counts_and_profile_lookup():
     assert bench.set_bytes(synth.workload("c1")) < bench.L2_BYTES < bench.set_bytes(cfg)
     # ncu traffic is reported only for the workload it was captured on
     assert bench.profile_traffic("c1") is None
+
+
+def test_prefill_flop_counts_match_a_brute_force_count():
+    """The prefill roofline's flops: 4 d flops per (query, head, visible key
+    of the union blocks); the indexer's 2 H_I d_I per (query, key <= its
+    position).  Checked on a small chunk by counting pairs one by one."""
+    import numpy as np
+    cfg = synth.PrefillConfig("t", 300, 7, 2, 8, 5, 64, 4, 2, 16, seed=5)
+    ind = np.array([0, 2, 4], np.int32)     # blocks 0, 2 and the partial last block 4 (256..299)
+    ptr = np.array([0, 3, 6], np.int32)
+    visible = sum(1 for p in cfg.q_pos for b in ind for t in range(b * 64, b * 64 + 64) if t < cfg.S and t <= p)
+    assert bench.prefill_attention_flops(cfg, ptr, np.concatenate([ind, ind])) == 4 * cfg.d * cfg.Hq * visible
+    pairs = sum(int(p) + 1 for p in cfg.q_pos)
+    assert bench.prefill_indexer_flops(cfg) == 2 * cfg.H_I * cfg.d_I * pairs
